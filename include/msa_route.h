@@ -1,0 +1,75 @@
+/* Step 2 of the MSA hot path: online routing of queries over the pooled routing keys
+ * with fused top-k document selection.
+ *
+ * Defined by: "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", section 架构 (cosine
+ * similarity of router query Q_r and pooled router key K-bar_r, mean over attention heads
+ * first, then max over query tokens, Top-k documents) and section 推理流水线 step 2 (the
+ * query is projected to Q_r and matched against K-bar_r); MSA paper reading notes, section
+ * 路由投影器 + Top-k 稀疏注意力 (Top-16 documents, cosine against every document) and
+ * section KV 缓存压缩 + Memory Parallel (routing keys stay in GPU memory and every query
+ * scans them all).
+ *
+ * For query b, layer l, query token t, query head h (G = n_q_heads / n_kv_heads):
+ *   s[t][c]  = (1/Hq) sum_h cos(Q_r[t][h], K-bar_r[c][h / G])
+ *   m[c]     = max over the query's tokens of s[t][c]
+ *   S[doc]   = max over the document's blocks of m[c]     (a document with no block: -inf)
+ *   ids      = the top_k documents by S, descending, equal scores -> smaller id first;
+ *              fewer than top_k documents -> id -1, score -inf.
+ * The [T x C] score matrix is never stored.  Computed as
+ *   s[t][c] = < (1/Hq) sum_{h: h/G = g} Q_r[t][h] / max(||Q_r[t][h]||, 1e-8) , kr_hat[c][g] >
+ * summed over key heads g, with kr_hat the unit routing keys written by msa_pool_blocks,
+ * in fp32 accumulation (bf16 operands on the tensor-core path).
+ */
+#ifndef MSA_ROUTE_H
+#define MSA_ROUTE_H
+
+#include "msa_common.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Path selection for msa_route_topk (flags argument). */
+#define MSA_ROUTE_AUTO 0    /* pick by query length                                  */
+#define MSA_ROUTE_SCAN 1    /* CUDA-core streaming scan (few query tokens)           */
+#define MSA_ROUTE_TENSOR 2  /* tcgen05 tensor-core GEMM with fused token-max epilogue */
+
+/* Workspace bytes for one msa_route_topk call with these sizes. */
+msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, int32_t total_q_tokens,
+                                         int32_t n_kv_heads, int64_t n_chunks, int32_t n_docs, int32_t top_k,
+                                         size_t* bytes);
+
+/* Routes n_queries queries over n_layers routing layers (each layer selects its own
+ * top_k documents).
+ *   qr               DEVICE [n_layers][total_q_tokens][n_q_heads][head_dim], q_dtype
+ *                    (MSA_F32 or MSA_BF16); the tokens of query b are rows
+ *                    [q_offsets_host[b], q_offsets_host[b+1]).
+ *   q_offsets_host   HOST int32 [n_queries + 1], q_offsets_host[0] = 0, strictly increasing
+ *                    (every query has at least one token); read during the call only.
+ *   kr_hat           DEVICE bf16 [n_layers][n_chunks][n_kv_heads][head_dim], unit-norm
+ *                    routing keys (msa_pool_blocks), 16-byte aligned.
+ *   doc_chunk_offsets DEVICE int64 [n_docs + 1], doc_chunk_offsets[n_docs] = n_chunks.
+ *   head_dim = 128; n_kv_heads = 8 on the tensor-core path; n_q_heads % n_kv_heads = 0;
+ *   1 <= top_k <= 64; 1 <= n_queries <= 256; n_kv_heads in {2, 4, 8, 16}; n_q_heads <= 64.
+ *   out_ids, out_scores DEVICE [n_queries][n_layers][top_k] int32 / fp32.
+ *   workspace        DEVICE, >= msa_route_topk_workspace_size bytes, 256-byte aligned.
+ *   flags            MSA_ROUTE_AUTO / _SCAN / _TENSOR.
+ * Asynchronous on stream; no host synchronisation. */
+msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
+                          int32_t n_queries, const void* kr_hat, const int64_t* doc_chunk_offsets,
+                          int32_t n_docs, int64_t n_chunks, int32_t n_layers, int32_t n_q_heads,
+                          int32_t n_kv_heads, int32_t head_dim, int32_t top_k, int32_t* out_ids,
+                          float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,
+                          int32_t* dev_err, msa_stream_t stream);
+
+/* Number of kernel launches the last successful msa_route_topk on this thread enqueued
+ * (for launch accounting). */
+int32_t msa_route_last_launch_count(void);
+
+const char* msa_route_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_ROUTE_H */

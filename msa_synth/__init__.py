@@ -310,3 +310,42 @@ def pooled_content(bank: BankSpec, layer: int, c0: int, n_c: int, dtype: str = "
     k = fill(bank.seed, STREAM_KBAR, layer, 0, c0, n_c, rl, sigma=POOLED_NOISE, dtype=dtype)
     v = fill(bank.seed, STREAM_VBAR, layer, 0, c0, n_c, rl, sigma=POOLED_NOISE, dtype=dtype)
     return np.stack([k, v], axis=1).reshape(n_c, 2, bank.n_heads, bank.head_dim)
+
+
+# ----------------------------------------------------------------------------- device fill
+
+_dev_lib = None
+
+
+def _device_lib():
+    import ctypes
+    import os
+    global _dev_lib
+    if _dev_lib is None:
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa_synth.so")
+        if not os.path.exists(path):
+            raise ImportError(f"{path} missing: run python -m top_kv_routing_b200.build")
+        lib = ctypes.CDLL(path)
+        lib.msa_synth_fill.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_uint32,
+                                       ctypes.c_uint32, ctypes.c_uint32, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p]
+        lib.msa_synth_fill.restype = ctypes.c_int32
+        _dev_lib = lib
+    return _dev_lib
+
+
+def device_fill(dst, seed: int, stream: int, layer: int, sub: int, row0: int, n_rows: int, row_len: int,
+                sigma: float = 1.0, topic=None, row_topic=None, cuda_stream=None) -> None:
+    """Same values as ``fill`` written by a GPU kernel into the torch tensor ``dst``
+    (fp32 or bf16, contiguous, >= n_rows*row_len elements).  topic / row_topic are
+    device tensors (fp32 [n][tlen], int32 [n_rows]) or None."""
+    import torch
+    dtype = 1 if dst.dtype == torch.bfloat16 else 0
+    s = torch.cuda.current_stream().cuda_stream if cuda_stream is None else cuda_stream
+    tl = 0 if topic is None else int(topic.shape[-1])
+    r = _device_lib().msa_synth_fill(dst.data_ptr(), dtype, seed, stream, layer, sub, row0, n_rows, row_len,
+                                     sigma, None if topic is None else topic.data_ptr(), tl,
+                                     None if row_topic is None else row_topic.data_ptr(), s)
+    if r != 0:
+        raise RuntimeError(f"msa_synth_fill failed ({r})")

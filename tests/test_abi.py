@@ -1,0 +1,80 @@
+"""The C-ABI libraries load without a GPU, export every symbol their headers declare, and
+reject bad arguments before touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = {"pool": "msa_pool.h", "route": "msa_route.h", "gather": "msa_gather.h", "decode": "msa_decode.h"}
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def msa():
+    import top_kv_routing_b200 as m
+    return m
+
+
+@pytest.mark.parametrize("lib", sorted(HEADERS))
+def test_library_exports_declared_symbols(msa, lib):
+    path = os.path.join(msa.LIB_DIR, f"libmsa_{lib}.so")
+    names = _declared(HEADERS[lib])
+    assert names, lib
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    dll = ctypes.CDLL(path)
+    for n in names:
+        assert getattr(dll, n) is not None
+
+
+def test_common_header_constants_match_binding(msa):
+    text = open(os.path.join(ROOT, "include", "msa_common.h")).read()
+    for name in ("MSA_DEVERR_CAPACITY", "MSA_DEVERR_BAD_DOC", "MSA_DEVERR_LOCAL_FULL", "MSA_DEVERR_BAD_OFFSETS"):
+        v = int(re.search(rf"#define {name} (\d+)u", text).group(1))
+        assert getattr(msa, name) == v
+    text = open(os.path.join(ROOT, "include", "msa_route.h")).read()
+    for name in ("MSA_ROUTE_AUTO", "MSA_ROUTE_SCAN", "MSA_ROUTE_TENSOR"):
+        assert getattr(msa, name) == int(re.search(rf"#define {name} (\d+)", text).group(1))
+
+
+def test_count_chunks_host(msa):
+    n, offs = msa.msa_count_chunks(np.array([0, 64, 65, 65, 200]), 64)
+    assert n == 1 + 1 + 0 + 3 and offs.tolist() == [0, 1, 2, 2, 5]
+    with pytest.raises(msa.MsaError):
+        msa.msa_count_chunks(np.array([0, 5, 3]), 64)
+
+
+def test_invalid_arguments_rejected_without_gpu(msa):
+    with pytest.raises(msa.MsaError) as e:   # head_dim 64
+        msa.msa_pool_blocks(None, None, np.zeros(8, np.float32), np.zeros(2, np.int64), np.zeros(2, np.int64), 1, 1,
+                            8, 64, 64, 1e6, None, None, np.zeros(8, np.uint16), None, None, in_dtype=0, stream=0)
+    assert e.value.status == msa.MSA_ERR_INVALID_ARG
+    with pytest.raises(msa.MsaError) as e:   # top_k 65
+        msa.msa_route_topk_workspace_size(1, 1, 1, 8, 10, 10, 65)
+    assert e.value.status == msa.MSA_ERR_INVALID_ARG
+    with pytest.raises(msa.MsaError) as e:   # null ids
+        msa.msa_gather_kv(np.zeros(16, np.uint16), 1, np.zeros(2, np.int64), None, 1, None, 1, 1, 1, 8, 128, 8,
+                          np.zeros(16, np.uint16), np.zeros(1, np.int32), stream=0)
+    assert e.value.status == msa.MSA_ERR_INVALID_ARG
+    with pytest.raises(msa.MsaError) as e:   # 32 query heads over 5 key heads
+        z = np.zeros(16, np.uint16)
+        msa.msa_sparse_decode(z, z, z, 1, 1, 32, 5, 128, z, z, np.zeros(1, np.int32), 4, z, np.zeros(1, np.int32),
+                              4, 16, 1e6, 0.1, z, stream=0)
+    assert e.value.status == msa.MSA_ERR_INVALID_ARG
+
+
+def test_workspace_size_grows_with_bank(msa):
+    a = msa.msa_route_topk_workspace_size(18, 1, 256, 8, 1000, 100, 16)
+    b = msa.msa_route_topk_workspace_size(18, 1, 256, 8, 2000, 100, 16)
+    assert b - a >= 18 * 1000 * 4 - 256
