@@ -51,6 +51,9 @@ typedef struct CUstream_st* msa_stream_t;
 #define MSA_DEVERR_BAD_DOC 2u     /* a document id outside [0, n_docs) (skipped)         */
 #define MSA_DEVERR_LOCAL_FULL 4u  /* local cache has no room for the new token (skipped) */
 #define MSA_DEVERR_BAD_OFFSETS 8u /* offsets disagree with the declared counts           */
+#define MSA_DEVERR_TIMEOUT 16u    /* a bounded in-kernel wait ran out (work abandoned)    */
+#define MSA_DEVERR_UNCERTIFIED 32u /* tensor-core routing: the exactly rescored candidates do
+                                      not provably contain the exact top-k (see msa_route.h) */
 
 /* Bytes of one memory block of one layer in a bf16 bank:
  * routing key H*d*2; content key + value 2*H*d*2. */

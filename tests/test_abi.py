@@ -40,7 +40,8 @@ def test_library_exports_declared_symbols(msa, lib):
 
 def test_common_header_constants_match_binding(msa):
     text = open(os.path.join(ROOT, "include", "msa_common.h")).read()
-    for name in ("MSA_DEVERR_CAPACITY", "MSA_DEVERR_BAD_DOC", "MSA_DEVERR_LOCAL_FULL", "MSA_DEVERR_BAD_OFFSETS"):
+    for name in ("MSA_DEVERR_CAPACITY", "MSA_DEVERR_BAD_DOC", "MSA_DEVERR_LOCAL_FULL", "MSA_DEVERR_BAD_OFFSETS",
+                 "MSA_DEVERR_TIMEOUT", "MSA_DEVERR_UNCERTIFIED"):
         v = int(re.search(rf"#define {name} (\d+)u", text).group(1))
         assert getattr(msa, name) == v
     text = open(os.path.join(ROOT, "include", "msa_route.h")).read()

@@ -129,18 +129,18 @@ def test_pool_rejects_bad_arguments(msa):
 
 # ----------------------------------------------------------------------------- step 2
 
-def _normalised_bank(msa, bank, layers):
-    """Pooled-level router keys for each layer (bf16 bits [L][C][H][D]) and the GPU's unit
-    keys made from them by msa_pool_blocks with chunk = 1."""
+def _route_bank(bank, layers):
+    """Stored routing keys for each layer, bf16 bits [L][C][H][D]: pooled-level keys drawn
+    by the generator, made unit-norm per head by the oracle (chunk = 1 pass-through) and
+    rounded to bf16.  The same bits feed the GPU route and the oracle route."""
     C = bank.n_chunks
-    bits = np.stack([syn.pooled_router_keys(bank, l, 0, C) for l in range(layers)])
-    kr_hat = torch.empty((layers, C, H, D), dtype=torch.bfloat16, device="cuda")
-    ones = _dev_i64(np.arange(C + 1))
-    coffs = _dev_i64(bank.doc_chunk_offsets)
+    out = []
     for l in range(layers):
-        msa.msa_pool_blocks(None, None, bf16_tensor(bits[l]), ones, ones, C, C, H, D, 1, 0.0, None, None,
-                            kr_hat[l], None, None, in_dtype=msa.MSA_BF16)
-    return bits, kr_hat, coffs
+        raw = syn.bf16_bits_to_f32(syn.pooled_router_keys(bank, l, 0, C))
+        unit = oracle.pool(None, None, raw, np.arange(C + 1), H, D, 1, 1e6, rope_k=False)["kr_unit"]
+        out.append(syn.f32_to_bf16_bits(unit.astype(np.float32)))
+    bits = np.stack(out)
+    return bits, bf16_tensor(bits), _dev_i64(bank.doc_chunk_offsets)
 
 
 def _route_gpu(msa, qr, q_offsets, kr_hat, coffs, n_docs, C, L, k, flags):
@@ -149,15 +149,16 @@ def _route_gpu(msa, qr, q_offsets, kr_hat, coffs, n_docs, C, L, k, flags):
     ws = torch.empty(msa.msa_route_topk_workspace_size(L, B, T, H, C, n_docs, k), dtype=torch.uint8, device="cuda")
     ids = torch.full((B, L, k), -7, dtype=torch.int32, device="cuda")
     sc = torch.full((B, L, k), float("nan"), device="cuda")
+    err = _err()
     msa.msa_route_topk(torch.from_numpy(np.ascontiguousarray(qr, dtype=np.float32)).cuda(), q_offsets, kr_hat,
-                       coffs, n_docs, C, L, HQ, H, D, k, ids, sc, ws, flags=flags)
+                       coffs, n_docs, C, L, HQ, H, D, k, ids, sc, ws, flags=flags, dev_err=err)
     torch.cuda.synchronize()
-    return ids.cpu().numpy(), sc.cpu().numpy()
+    return ids.cpu().numpy(), sc.cpu().numpy(), int(err.item())
 
 
 def _route_case(msa, seed, lens, L, Ts, k, flags, n_targets=2):
     bank = syn.make_bank(seed, len(lens), lens, L)
-    bits, kr_hat, coffs = _normalised_bank(msa, bank, L)
+    bits, kr_hat, coffs = _route_bank(bank, L)
     q_off = syn.offsets(np.asarray(Ts)).astype(np.int32)
     nonempty = [d for d in range(len(lens)) if lens[d] > 0]
     qr = np.zeros((L, int(q_off[-1]), HQ, D), dtype=np.float32)
@@ -167,7 +168,8 @@ def _route_case(msa, seed, lens, L, Ts, k, flags, n_targets=2):
         targets[b] = tg
         for l in range(L):
             qr[l, q_off[b]:q_off[b + 1]] = syn.query_router(seed, l, b, T, HQ, D, bank.topic, tg)
-    ids, sc = _route_gpu(msa, qr, q_off, kr_hat, coffs, len(lens), bank.n_chunks, L, k, flags)
+    ids, sc, err = _route_gpu(msa, qr, q_off, kr_hat, coffs, len(lens), bank.n_chunks, L, k, flags)
+    assert err & ~msa.MSA_DEVERR_UNCERTIFIED == 0
     for b in range(len(Ts)):
         for l in range(L):
             keys = syn.bf16_bits_to_f32(bits[l])
@@ -177,25 +179,56 @@ def _route_case(msa, seed, lens, L, Ts, k, flags, n_targets=2):
             planted = targets[b][:min(Ts[b], len(targets[b]))]   # token t carries target t mod n
             if k >= len(planted):
                 assert set(planted.tolist()) <= set(ids[b, l].tolist())
-    return ids, sc
+    return ids, sc, err
 
 
-@pytest.mark.parametrize("flags", [1])
+@pytest.mark.parametrize("flags", [1, 2])
 def test_route_multi_query_multi_layer(msa, flags):
     lens = syn.doc_lengths_lognormal(1, 200)
     _route_case(msa, 1, lens, 2, [1, 5, 2], 16, flags)
 
 
-@pytest.mark.parametrize("flags", [1])
+@pytest.mark.parametrize("flags", [1, 2])
 def test_route_fewer_docs_than_k_and_empty_docs(msa, flags):
     lens = np.array([100, 0, 64, 0, 1, 300])
-    ids, sc = _route_case(msa, 2, lens, 1, [3], 8, flags)
+    ids, sc, _ = _route_case(msa, 2, lens, 1, [3], 8, flags)
     assert list(ids[0, 0, 6:]) == [-1, -1] and np.all(np.isneginf(sc[0, 0, 4:]))
 
 
-@pytest.mark.parametrize("flags", [1])
+@pytest.mark.parametrize("flags", [1, 2])
 def test_route_single_document(msa, flags):
     _route_case(msa, 3, np.array([65]), 1, [2], 4, flags, n_targets=1)
+
+
+@pytest.mark.parametrize("Ts", [[300, 40, 257], [64], [129], [33, 31, 1, 64]])
+def test_route_tensor_long_queries_span_tiles(msa, Ts):
+    # several N tiles per block tile (queries crossing tile edges), ragged last M tile,
+    # two layers (tiles at the layer boundary)
+    lens = syn.doc_lengths_lognormal(7, 150)
+    _route_case(msa, 7, lens, 2, Ts, 64, 2, n_targets=4)
+
+
+def test_route_tensor_selection_is_certified_for_planted_needles(msa):
+    # k = number of planted documents: the k-th exact score sits far above the filter's
+    # margin over the best document left out, so the certification bit stays clear
+    lens = syn.doc_lengths_lognormal(9, 400)
+    _, _, err = _route_case(msa, 9, lens, 1, [64], 4, 2, n_targets=4)
+    assert err == 0
+
+
+def test_route_auto_picks_tensor_for_long_query_and_scan_for_short(msa):
+    lens = syn.doc_lengths_lognormal(8, 60)
+    bank = syn.make_bank(8, 60, lens, 1)
+    _, kr_hat, coffs = _route_bank(bank, 1)
+    C = bank.n_chunks
+    # scan: qprep + scan + 2 top-k; tensor: zero-pad + qprep + GEMM + 2 top-k + rescore + final
+    for T, expect in ((4, 4), (40, 7)):
+        ws = torch.empty(msa.msa_route_topk_workspace_size(1, 1, T, H, C, 60, 16), dtype=torch.uint8, device="cuda")
+        ids = torch.empty((1, 1, 16), dtype=torch.int32, device="cuda")
+        sc = torch.empty((1, 1, 16), device="cuda")
+        n = msa.msa_route_topk(torch.randn((1, T, HQ, D), device="cuda"), [0, T], kr_hat, coffs, 60, C, 1, HQ, H, D,
+                               16, ids, sc, ws)
+        assert n == expect
 
 
 # ----------------------------------------------------------------------------- step 3

@@ -18,7 +18,8 @@ LIB_DIR = os.path.join(_HERE, "lib")
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY, MSA_ERR_TIMEOUT = range(6)
 MSA_F32, MSA_BF16 = 0, 1
 MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR = 0, 1, 2
-MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS = 1, 2, 4, 8
+(MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS, MSA_DEVERR_TIMEOUT,
+ MSA_DEVERR_UNCERTIFIED) = 1, 2, 4, 8, 16, 32
 
 _STATUS = {1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA", 4: "MSA_ERR_CAPACITY",
            5: "MSA_ERR_TIMEOUT"}

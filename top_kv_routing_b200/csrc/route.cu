@@ -6,10 +6,17 @@
 //
 // Launch sequence of one call:
 //   1. qprep    Q_r -> qt[l][t][g][:] = (1/Hq) sum_{h: h/G = g} Q_r[t][h] / max(||Q_r[t][h]||,1e-8)
-//               (fp32 for the scan, bf16 rows padded to the tile for the tensor-core path)
-//   2. score    m[b][l][c] = max_{t in b} <qt[l][t], kr_hat[l][c]>   (scan or tcgen05 GEMM)
-//   3. docmax   S[doc] = max of m over the document's blocks; per-CTA top-k candidates
-//   4. merge    one CTA per (b, l) merges the candidates into the final top-k
+//               (fp32 for the exact kernels, bf16 rows padded per query for the GEMM)
+//   2. score    m[b][l][c] = max_{t in b} cos-score(t, c)
+//               scan path (few tokens): exact fp32 on CUDA cores, keys normalised per head
+//               tensor path: tcgen05 GEMM on bf16 operands (a filter; also the runner-up
+//               score and the argmax token of each block)
+//   3. docmax   S[doc] = max of m over the document's blocks; per-CTA best candidates
+//   4. merge    the per-CTA candidates -> top_k (scan) or the K2 filter candidates (tensor)
+//   tensor path only:
+//   5. rescore  exact fp32 scores of the K2 candidates, evaluating only the (block, token)
+//               pairs whose filter score lies within the filter's error window of the max
+//   6. final    top_k of the exact scores; certification of the selection
 // The score matrix s[t][c] only ever lives in registers / TMEM.
 #include "common.cuh"
 #include "msa_route.h"
@@ -22,34 +29,65 @@ namespace {
 constexpr int kD = 128;
 constexpr int kMaxQueries = 256;
 constexpr int kMaxTopK = 64;
-constexpr int kTopkThreads = 256;
+constexpr int kMaxCandidates = 128;  // documents rescored exactly after the tensor-core filter
+constexpr int kTopkThreads = 512;
+constexpr int kMaxDocs = 1 << 20;    // documents per bank
+constexpr int kMaxBlocks = 64;       // docmax CTAs per (query, layer)
+// Error bound assumed for the tensor-core filter scores (bf16 operands, fp32 accumulate):
+// the observed error is ~1e-4 (3e-4 worst seen), this is ~10 standard deviations.  Pairs
+// within 2x of it from a block's best are rescored; a selection is certified when the
+// k-th exact score beats the best filter score left out by more than it.
+constexpr float kFilterErr = 1e-3f;
+
+// Candidates rescored exactly on the tensor-core path.
+int rescore_count(int32_t n_docs, int32_t k) {
+  int k2 = 2 * k > k + 32 ? 2 * k : k + 32;
+  if (k2 > kMaxCandidates) k2 = kMaxCandidates;
+  return n_docs < k2 ? n_docs : k2;
+}
 
 static thread_local int32_t g_launches = 0;
 
 struct QueryOffsets {
   int32_t n;
-  int32_t off[kMaxQueries + 1];
+  int32_t off[kMaxQueries + 1];   // token offsets of the queries in qr
+  int32_t row0[kMaxQueries + 1];  // first row of each query in the padded bf16 operand
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int topk_blocks(int32_t n_docs) {
-  int nb = (n_docs + 511) / 512;
+  int nb = (n_docs + 2047) / 2048;
   if (nb < 1) nb = 1;
-  if (nb > 256) nb = 256;
+  if (nb > kMaxBlocks) nb = kMaxBlocks;
   return nb;
 }
 
+int pow2_at_least(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
 struct WsLayout {
-  size_t qt_f32, qt_bf16, m, cand, total;
+  size_t qt_f32, qt_bf16, m, aux, cand, apx, exact, total;
   int n_pad;
   int nblk;
+  int k2;
 };
+
+// Upper bound of the padded operand rows for B queries of T_total tokens in all.
+int operand_rows_bound(int32_t T_total, int32_t B) {
+  const int r = T_total + (route_tc::kQueryAlign - 1) * B;
+  return (r + route_tc::kMaxTileN - 1) / route_tc::kMaxTileN * route_tc::kMaxTileN;
+}
 
 WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, int32_t n_docs, int32_t k) {
   WsLayout w;
-  w.n_pad = route_tc::padded_tokens(T_total);
+  w.n_pad = operand_rows_bound(T_total, B);
   w.nblk = topk_blocks(n_docs);
+  w.k2 = rescore_count(n_docs, k);
+  const int ksel = w.k2 > k ? w.k2 : k;
   size_t o = 0;
   w.qt_f32 = o;
   o += align256((size_t)L * T_total * H * kD * sizeof(float));
@@ -57,19 +95,36 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   o += align256((size_t)L * w.n_pad * H * kD * 2);
   w.m = o;
   o += align256((size_t)B * L * (size_t)C * sizeof(float));
+  w.aux = o;
+  o += align256((size_t)B * L * (size_t)C * sizeof(int2));
   w.cand = o;
-  o += align256((size_t)B * L * w.nblk * k * sizeof(unsigned long long));
+  o += align256((size_t)B * L * w.nblk * ksel * sizeof(unsigned long long));
+  w.apx = o;
+  o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(unsigned long long));
+  w.exact = o;
+  o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(float));
   w.total = o;
   return w;
 }
 
 // ---------------------------------------------------------------------------- 1. q prep
-// grid (T_total, L); block 128 threads.  Hq <= 64.
+// grid (T_total, L); block 128 threads.  Hq <= 64.  The bf16 copy of token t of query b
+// goes to operand row row0[b] + (t - off[b]) of layer l (n_rows rows per layer).
 __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr, int q_is_bf16, int T_total,
-                                                    int Hq, int H, int n_pad, float* __restrict__ qt_f32,
-                                                    __nv_bfloat16* __restrict__ qt_bf16) {
+                                                    int Hq, int H, int n_rows, QueryOffsets qo,
+                                                    float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16) {
   __shared__ float qhat[64][kD];
   const int t = blockIdx.x, l = blockIdx.y;
+  int qb = 0;
+  {
+    int lo = 0, hi = qo.n;  // largest b with off[b] <= t
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (qo.off[mid] <= t) lo = mid; else hi = mid;
+    }
+    qb = lo;
+  }
+  const int orow = qo.row0[qb] + (t - qo.off[qb]);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t row0 = ((int64_t)l * T_total + t) * Hq * kD;
   for (int h = warp; h < Hq; h += 4) {
@@ -100,29 +155,91 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
     for (int u = 0; u < G; ++u) acc += qhat[g * G + u][j];
     acc *= inv_hq;
     qt_f32[((int64_t)l * T_total + t) * H * kD + e] = acc;
-    qt_bf16[((int64_t)l * n_pad + t) * H * kD + e] = __float2bfloat16_rn(acc);
+    if (qt_bf16 != nullptr) qt_bf16[((int64_t)l * n_rows + orow) * H * kD + e] = __float2bfloat16_rn(acc);
   }
 }
 
-// Zero the padding rows [T_total, n_pad) of the bf16 operand of every layer.
-__global__ void zero_pad_kernel(__nv_bfloat16* __restrict__ qt_bf16, int T_total, int n_pad, int row, int L) {
-  const int64_t per_layer = (int64_t)(n_pad - T_total) * row;
-  const int64_t total = per_layer * L;
+// Zero every operand row that holds no query token (per-query alignment gaps and the
+// tail up to n_rows), in 16-byte words.
+__global__ void zero_pad_kernel(uint4* __restrict__ qt_bf16, int n_rows, int words_per_row, int L, QueryOffsets qo) {
+  const int64_t total = (int64_t)L * n_rows * words_per_row;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t l = i / per_layer, r = i % per_layer;
-    qt_bf16[(l * n_pad + T_total) * row + r] = __float2bfloat16_rn(0.f);
+    const int r = (int)((i / words_per_row) % n_rows);
+    int lo = 0, hi = qo.n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (qo.row0[mid] <= r) lo = mid; else hi = mid;
+    }
+    const bool token_row = r < qo.row0[qo.n] && (r - qo.row0[lo]) < (qo.off[lo + 1] - qo.off[lo]);
+    if (!token_row) qt_bf16[i] = make_uint4(0u, 0u, 0u, 0u);
   }
+}
+
+// ---------------------------------------------------------------------------- key rows
+// A warp holds one key row of R = 2*NV*128 elements: lane owns the 8-element vectors
+// v = lane + 32 i (i < NV), i.e. head (v >> 4) = 2 i + (lane >> 4).  The row is widened
+// to fp32 and every head is scaled by 1 / max(||k_head||, 1e-8) computed from the stored
+// bf16 values, so dots with the unit query sums are exact cosines (fp32).
+template <int NV>
+__device__ __forceinline__ void load_unit_row(const __nv_bfloat16* __restrict__ row, int lane, float (&kx)[NV][8]) {
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + lane + 32 * i);
+    float2 f;
+    f = msa::bf16x2_to_float2(w.x); kx[i][0] = f.x; kx[i][1] = f.y;
+    f = msa::bf16x2_to_float2(w.y); kx[i][2] = f.x; kx[i][3] = f.y;
+    f = msa::bf16x2_to_float2(w.z); kx[i][4] = f.x; kx[i][5] = f.y;
+    f = msa::bf16x2_to_float2(w.w); kx[i][6] = f.x; kx[i][7] = f.y;
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) ss = fmaf(kx[i][u], kx[i][u], ss);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);   // the 16 lanes of a head half-warp
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+    const float rho = 1.0f / fmaxf(sqrtf(ss), 1e-8f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) kx[i][u] *= rho;
+  }
+}
+
+// <qt[t], unit row> for the lane's slice (before the warp reduction).
+template <int NV>
+__device__ __forceinline__ float lane_dot(const float4* __restrict__ qv, int lane, const float (&kx)[NV][8]) {
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const float4 a = __ldg(qv + 2 * (lane + 32 * i));
+    const float4 b = __ldg(qv + 2 * (lane + 32 * i) + 1);
+    acc = fmaf(kx[i][0], a.x, acc);
+    acc = fmaf(kx[i][1], a.y, acc);
+    acc = fmaf(kx[i][2], a.z, acc);
+    acc = fmaf(kx[i][3], a.w, acc);
+    acc = fmaf(kx[i][4], b.x, acc);
+    acc = fmaf(kx[i][5], b.y, acc);
+    acc = fmaf(kx[i][6], b.z, acc);
+    acc = fmaf(kx[i][7], b.w, acc);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // ---------------------------------------------------------------------------- 2a. scan
-// One warp per (layer, block) task.  Lane holds NV 8-element vectors of the key row
-// (vectors lane, lane+32, ...), dots them against every query token, reduces across the
-// warp and keeps the running max per query.
+// One warp per (layer, block) task: exact cosine scores of the block against every
+// query token, running max per query.
 template <int NV>
 __global__ void __launch_bounds__(256) scan_kernel(const __nv_bfloat16* __restrict__ kr_hat,
                                                    const float* __restrict__ qt, int L, int64_t C,
                                                    int T_total, QueryOffsets qo, float* __restrict__ m) {
-  constexpr int R = NV * 256;  // elements per key row = H * 128
+  constexpr int R = NV * 256;
   const int lane = threadIdx.x % 32;
   const int64_t warp_global = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
   const int64_t n_warps = (int64_t)gridDim.x * blockDim.x / 32;
@@ -130,40 +247,13 @@ __global__ void __launch_bounds__(256) scan_kernel(const __nv_bfloat16* __restri
   for (int64_t task = warp_global; task < tasks; task += n_warps) {
     const int l = (int)(task / C);
     const int64_t c = task % C;
-    const __nv_bfloat16* row = kr_hat + ((int64_t)l * C + c) * R;
     float kx[NV][8];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + lane + 32 * i);
-      float2 f;
-      f = msa::bf16x2_to_float2(w.x); kx[i][0] = f.x; kx[i][1] = f.y;
-      f = msa::bf16x2_to_float2(w.y); kx[i][2] = f.x; kx[i][3] = f.y;
-      f = msa::bf16x2_to_float2(w.z); kx[i][4] = f.x; kx[i][5] = f.y;
-      f = msa::bf16x2_to_float2(w.w); kx[i][6] = f.x; kx[i][7] = f.y;
-    }
+    load_unit_row<NV>(kr_hat + ((int64_t)l * C + c) * R, lane, kx);
     const float* qbase = qt + (int64_t)l * T_total * R;
     for (int b = 0; b < qo.n; ++b) {
       float best = -INFINITY;
-      for (int t = qo.off[b]; t < qo.off[b + 1]; ++t) {
-        const float4* qv = reinterpret_cast<const float4*>(qbase + (int64_t)t * R);
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-          const float4 a = __ldg(qv + 2 * (lane + 32 * i));
-          const float4 bq = __ldg(qv + 2 * (lane + 32 * i) + 1);
-          acc = fmaf(kx[i][0], a.x, acc);
-          acc = fmaf(kx[i][1], a.y, acc);
-          acc = fmaf(kx[i][2], a.z, acc);
-          acc = fmaf(kx[i][3], a.w, acc);
-          acc = fmaf(kx[i][4], bq.x, acc);
-          acc = fmaf(kx[i][5], bq.y, acc);
-          acc = fmaf(kx[i][6], bq.z, acc);
-          acc = fmaf(kx[i][7], bq.w, acc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        best = fmaxf(best, acc);
-      }
+      for (int t = qo.off[b]; t < qo.off[b + 1]; ++t)
+        best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
       if (lane == 0) m[((int64_t)b * L + l) * C + c] = best;
     }
   }
@@ -189,49 +279,32 @@ __device__ __forceinline__ void split_key(unsigned long long key, int* doc, floa
   *doc = (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
 }
 
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w > v ? w : v;
-  }
-  return v;
-}
-
-// Block-wide max of v (all threads get it).
-__device__ unsigned long long block_max_u64(unsigned long long v, unsigned long long* red) {
-  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  v = warp_max_u64(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  unsigned long long r = 0ull;
-  for (int i = 0; i < (int)(blockDim.x / 32); ++i) r = red[i] > r ? red[i] : r;
-  return r;
-}
-
-// Selects the k largest keys of keys[0..n) (smem, destroyed) into out[0..k).
-__device__ void block_select_topk(unsigned long long* keys, int n, int k, unsigned long long* out,
-                                  unsigned long long* red) {
-  for (int r = 0; r < k; ++r) {
-    unsigned long long mine = 0ull;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) mine = keys[i] > mine ? keys[i] : mine;
-    const unsigned long long best = block_max_u64(mine, red);
-    if (threadIdx.x == 0) out[r] = best;
-    if (best != 0ull)
-      for (int i = threadIdx.x; i < n; i += blockDim.x)
-        if (keys[i] == best) keys[i] = 0ull;
-    __syncthreads();
+// Sorts keys[0..n) (smem, n a power of two) in descending order (bitonic network).
+__device__ void block_sort_desc(unsigned long long* keys, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], b = keys[ixj];
+          const bool desc = (i & k) == 0;
+          if (desc ? (a < b) : (a > b)) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
   }
 }
 
-// grid (nblk, L, B): documents [blk*per, (blk+1)*per) of (b, l).
+// grid (nblk, L, B): documents [blk*per, (blk+1)*per) of (b, l); writes its k_sel best keys.
 __global__ void __launch_bounds__(kTopkThreads) docmax_topk_kernel(const float* __restrict__ m,
                                                                    const int64_t* __restrict__ doc_chunk_off,
-                                                                   int n_docs, int64_t C, int L, int k,
-                                                                   unsigned long long* __restrict__ cand) {
+                                                                   int n_docs, int64_t C, int L, int k_sel,
+                                                                   int n_pow2, unsigned long long* __restrict__ cand) {
   extern __shared__ unsigned long long tk_smem[];
-  __shared__ unsigned long long red[kTopkThreads / 32];
   const int blk = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
   const int nblk = gridDim.x;
   const int per = (n_docs + nblk - 1) / nblk;
@@ -239,38 +312,139 @@ __global__ void __launch_bounds__(kTopkThreads) docmax_topk_kernel(const float* 
   const int d1 = min(n_docs, d0 + per);
   const int n = max(0, d1 - d0);
   const float* mb = m + ((int64_t)b * L + l) * C;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int doc = d0 + i;
-    const int64_t c0 = __ldg(doc_chunk_off + doc), c1 = __ldg(doc_chunk_off + doc + 1);
-    float s = -INFINITY;
-    for (int64_t c = c0; c < c1; ++c) s = fmaxf(s, __ldg(mb + c));
-    tk_smem[i] = make_key(s, doc);
+  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+    unsigned long long key = 0ull;
+    if (i < n) {
+      const int doc = d0 + i;
+      const int64_t c0 = __ldg(doc_chunk_off + doc), c1 = __ldg(doc_chunk_off + doc + 1);
+      float s = -INFINITY;
+      for (int64_t c = c0; c < c1; ++c) s = fmaxf(s, __ldg(mb + c));
+      key = make_key(s, doc);
+    }
+    tk_smem[i] = key;
   }
   __syncthreads();
-  unsigned long long* out = cand + (((int64_t)b * L + l) * nblk + blk) * k;
-  block_select_topk(tk_smem, n, k, out, red);
+  block_sort_desc(tk_smem, n_pow2);
+  unsigned long long* out = cand + (((int64_t)b * L + l) * nblk + blk) * k_sel;
+  for (int r = threadIdx.x; r < k_sel; r += blockDim.x) out[r] = r < n_pow2 ? tk_smem[r] : 0ull;
 }
 
-// grid (L, B): merges nblk * k candidates.
+// grid (L, B): merges nblk * k_sel candidates into the k_sel best.  Writes keys_out
+// [B][L][k_sel] when given, else ids / scores [B][L][k_sel].
 __global__ void __launch_bounds__(kTopkThreads) merge_topk_kernel(const unsigned long long* __restrict__ cand,
-                                                                  int nblk, int L, int k,
+                                                                  int nblk, int L, int k_sel, int n_pow2,
+                                                                  unsigned long long* __restrict__ keys_out,
                                                                   int32_t* __restrict__ out_ids,
                                                                   float* __restrict__ out_scores) {
   extern __shared__ unsigned long long tk_smem[];
-  __shared__ unsigned long long red[kTopkThreads / 32];
-  __shared__ unsigned long long best[kMaxTopK];
   const int l = blockIdx.x, b = blockIdx.y;
-  const int n = nblk * k;
+  const int n = nblk * k_sel;
   const unsigned long long* src = cand + ((int64_t)b * L + l) * n;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) tk_smem[i] = src[i];
+  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) tk_smem[i] = i < n ? src[i] : 0ull;
   __syncthreads();
-  block_select_topk(tk_smem, n, k, best, red);
+  block_sort_desc(tk_smem, n_pow2);
+  for (int r = threadIdx.x; r < k_sel; r += blockDim.x) {
+    const int64_t o = ((int64_t)b * L + l) * k_sel + r;
+    const unsigned long long key = r < n_pow2 ? tk_smem[r] : 0ull;
+    if (keys_out != nullptr) {
+      keys_out[o] = key;
+    } else {
+      int doc;
+      float s;
+      split_key(key, &doc, &s);
+      out_ids[o] = doc;
+      out_scores[o] = s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- 2c. exact rescoring
+// grid (K2, L, B), 128 threads: exact fp32 score of filter candidate r of (b, l).  The
+// document's exact best (block, token) pair has a filter score within 2 E of the
+// document's filter maximum, and within 2 E of its block's filter maximum; so only
+// blocks with m >= max - 2E are visited, and in those only the argmax token unless the
+// runner-up is also within 2E (then every token of the query).
+template <int NV>
+__global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __restrict__ kr_hat,
+                                                      const float* __restrict__ qt, int L, int64_t C, int T_total,
+                                                      QueryOffsets qo, const int64_t* __restrict__ doc_chunk_off,
+                                                      const float* __restrict__ m, const int2* __restrict__ aux,
+                                                      const unsigned long long* __restrict__ apx, int K2, float err,
+                                                      float* __restrict__ exact) {
+  constexpr int R = NV * 256;
+  __shared__ float red[4];
+  const int r = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t o = ((int64_t)b * L + l) * K2 + r;
+  int doc;
+  float doc_apx;
+  split_key(apx[o], &doc, &doc_apx);
+  if (doc < 0) {
+    if (threadIdx.x == 0) exact[o] = -INFINITY;
+    return;
+  }
+  const int64_t c0 = doc_chunk_off[doc], c1 = doc_chunk_off[doc + 1];
+  const int64_t mrow = ((int64_t)b * L + l) * C;
+  const float* qbase = qt + (int64_t)l * T_total * R;
+  const float window = 2.0f * err;
+  float best = -INFINITY;
+  for (int64_t c = c0 + warp; c < c1; c += 4) {
+    const float m1 = m[mrow + c];
+    if (!(m1 >= doc_apx - window)) continue;
+    const int2 ax = aux[mrow + c];
+    const float m2 = __int_as_float(ax.x);
+    float kx[NV][8];
+    load_unit_row<NV>(kr_hat + ((int64_t)l * C + c) * R, lane, kx);
+    if (m2 < m1 - window) {
+      const int t = qo.off[b] + ax.y;
+      best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
+    } else {
+      for (int t = qo.off[b]; t < qo.off[b + 1]; ++t)
+        best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
+    }
+  }
+  if (lane == 0) red[warp] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) exact[o] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+}
+
+// grid (L, B), 128 threads: final top-k of the K2 exactly rescored candidates.  The
+// selection is certified when the k-th exact score beats the best filter score left out
+// (the K2-th) by more than the filter's error bound; otherwise MSA_DEVERR_UNCERTIFIED.
+__global__ void __launch_bounds__(128) select_final_kernel(const unsigned long long* __restrict__ apx,
+                                                           const float* __restrict__ exact, int K2, int k,
+                                                           int n_docs, int L, float err,
+                                                           int32_t* __restrict__ out_ids,
+                                                           float* __restrict__ out_scores, int32_t* dev_err) {
+  __shared__ unsigned long long keys[kMaxCandidates];
+  const int l = blockIdx.x, b = blockIdx.y;
+  const int64_t base = ((int64_t)b * L + l) * K2;
+  const int n_pow2 = K2 <= 1 ? 1 : (1 << (32 - __clz(K2 - 1)));
+  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+    unsigned long long key = 0ull;
+    if (i < K2) {
+      int doc;
+      float s;
+      split_key(apx[base + i], &doc, &s);
+      if (doc >= 0) key = make_key(exact[base + i], doc);
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  block_sort_desc(keys, n_pow2);
   for (int r = threadIdx.x; r < k; r += blockDim.x) {
     int doc;
     float s;
-    split_key(best[r], &doc, &s);
+    split_key(r < n_pow2 ? keys[r] : 0ull, &doc, &s);
     out_ids[((int64_t)b * L + l) * k + r] = doc;
     out_scores[((int64_t)b * L + l) * k + r] = s;
+  }
+  if (threadIdx.x == 0 && n_docs > K2 && K2 >= k) {
+    int d_left, d_kth;
+    float s_left, s_kth;
+    split_key(apx[base + K2 - 1], &d_left, &s_left);
+    split_key(keys[k - 1], &d_kth, &s_kth);
+    if (!(s_kth > s_left + err)) msa::set_err(dev_err, MSA_DEVERR_UNCERTIFIED);
   }
 }
 
@@ -304,7 +478,8 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     return msa_fail(MSA_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads, <= 64");
   if (n_queries < 1 || n_queries > kMaxQueries) return msa_fail(MSA_ERR_INVALID_ARG, "n_queries in [1,256]");
   if (top_k < 1 || top_k > kMaxTopK) return msa_fail(MSA_ERR_INVALID_ARG, "top_k in [1,64]");
-  if (n_layers < 1 || n_chunks < 0 || n_docs < 0) return msa_fail(MSA_ERR_INVALID_ARG, "bad counts");
+  if (n_layers < 1 || n_chunks < 0 || n_docs < 0 || n_docs > kMaxDocs)
+    return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_docs <= 2^20)");
   if (q_dtype != MSA_F32 && q_dtype != MSA_BF16) return msa_fail(MSA_ERR_UNSUPPORTED, "q_dtype");
   if (flags < MSA_ROUTE_AUTO || flags > MSA_ROUTE_TENSOR) return msa_fail(MSA_ERR_INVALID_ARG, "flags");
   if (!msa::aligned16(qr) || !msa::aligned16(kr_hat) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -317,9 +492,12 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     if (b > 0 && qo.off[b] <= qo.off[b - 1]) return msa_fail(MSA_ERR_INVALID_ARG, "every query needs >= 1 token");
   }
   const int T_total = qo.off[n_queries];
+  route_tc::padded_rows(qo.off, n_queries, qo.row0);
+  const int n_rows = route_tc::operand_rows(qo.off, n_queries);
   const WsLayout w = ws_layout(n_layers, n_queries, T_total, n_kv_heads, n_chunks, n_docs, top_k);
   if (workspace_bytes < w.total) return msa_fail(MSA_ERR_CAPACITY, "workspace too small (%zu < %zu)",
                                                  workspace_bytes, w.total);
+  if (n_rows > w.n_pad) return msa_fail(MSA_ERR_INVALID_ARG, "internal: operand rows exceed bound");
   const int arch = msa::current_device_is_sm100(nullptr);
   if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
   if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
@@ -339,13 +517,20 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     if (flags == MSA_ROUTE_TENSOR) return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
     path = MSA_ROUTE_SCAN;
   }
+  const bool tensor = path == MSA_ROUTE_TENSOR && n_chunks > 0;
 
-  qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, w.n_pad,
-                                                      qt_f32, qt_bf16);
+  if (tensor) {
+    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(reinterpret_cast<uint4*>(qt_bf16), n_rows, H * kD / 8,
+                                                         n_layers, qo);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+  }
+  qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
+                                                      qt_f32, tensor ? qt_bf16 : nullptr);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
   if (n_chunks > 0) {
-    if (path == MSA_ROUTE_SCAN) {
+    if (!tensor) {
       int64_t warps = (int64_t)n_layers * n_chunks;
       int64_t blocks = (warps + 7) / 8;
       const int64_t cap = (int64_t)msa::sm_count() * 8;
@@ -359,20 +544,18 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
       ++g_launches;
       MSA_CUDA_TRY(cudaGetLastError());
     } else {
-      if (w.n_pad > T_total) {
-        zero_pad_kernel<<<64, 256, 0, s>>>(qt_bf16, T_total, w.n_pad, H * kD, n_layers);
-        ++g_launches;
-        MSA_CUDA_TRY(cudaGetLastError());
-      }
       route_tc::LaunchArgs a;
       a.kr_hat = kr_hat;
       a.qt = qt_bf16;
       a.L = n_layers;
       a.C = n_chunks;
-      a.n_pad = w.n_pad;
-      a.n_queries = n_queries;
-      for (int b = 0; b <= n_queries; ++b) a.q_off[b] = qo.off[b];
+      a.n_rows = n_rows;
+      a.ql.n_queries = n_queries;
+      for (int b = 0; b <= n_queries; ++b) a.ql.row0[b] = qo.row0[b];
+      for (int b = 0; b < n_queries; ++b) a.ql.len[b] = qo.off[b + 1] - qo.off[b];
       a.m = m;
+      a.aux = reinterpret_cast<int2*>(ws + w.aux);
+      a.dev_err = dev_err;
       int launches = 0;
       const char* why = nullptr;
       if (route_tc::launch(a, s, &launches, &why) != 0)
@@ -380,22 +563,52 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
       g_launches += launches;
     }
   }
-  const size_t tk_smem = (size_t)((n_docs + w.nblk - 1) / w.nblk) * sizeof(unsigned long long);
-  const size_t mg_smem = (size_t)w.nblk * top_k * sizeof(unsigned long long);
-  if (tk_smem > 48 * 1024) {
+  const int per = (n_docs + w.nblk - 1) / w.nblk;
+  const int doc_pow2 = pow2_at_least(per > 0 ? per : 1);
+  const size_t tk_smem = (size_t)doc_pow2 * sizeof(unsigned long long);
+  if (tk_smem > 48 * 1024)
     MSA_CUDA_TRY(cudaFuncSetAttribute(docmax_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tk_smem));
+  if (!tensor || n_docs == 0) {
+    // scan path (exact scores): per-block top-k, then one merge straight to the outputs
+    const int mg_pow2 = pow2_at_least(w.nblk * top_k);
+    const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
+    if (mg_smem > 48 * 1024)
+      MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
+    docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
+        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, top_k, doc_pow2, cand);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, top_k, mg_pow2,
+                                                                            nullptr, out_ids, out_scores);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    return msa_ok();
   }
-  if (mg_smem > 48 * 1024) {
+  // tensor path: the GEMM scores are a filter; the K2 best documents by those scores are
+  // rescored exactly (fp32 cosines) and the final top-k is taken from the exact scores
+  const int K2 = w.k2;
+  unsigned long long* apx = reinterpret_cast<unsigned long long*>(ws + w.apx);
+  float* exact = reinterpret_cast<float*>(ws + w.exact);
+  const int mg_pow2 = pow2_at_least(w.nblk * K2);
+  const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
+  if (mg_smem > 48 * 1024)
     MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
-  }
-  docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(m, doc_chunk_offsets, n_docs,
-                                                                                   n_chunks, n_layers, top_k, cand);
+  docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
+      m, doc_chunk_offsets, n_docs, n_chunks, n_layers, K2, doc_pow2, cand);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
-  merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, top_k, out_ids,
-                                                                          out_scores);
+  merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, K2, mg_pow2, apx,
+                                                                          nullptr, nullptr);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
-  (void)dev_err;
+  rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, 0, s>>>(
+      (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks, T_total, qo, doc_chunk_offsets, m,
+      reinterpret_cast<const int2*>(ws + w.aux), apx, K2, kFilterErr, exact);
+  ++g_launches;
+  MSA_CUDA_TRY(cudaGetLastError());
+  select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, kFilterErr,
+                                                               out_ids, out_scores, dev_err);
+  ++g_launches;
+  MSA_CUDA_TRY(cudaGetLastError());
   return msa_ok();
 }

@@ -1,15 +1,493 @@
-// Tensor-core (tcgen05) routing score path.
+// Tensor-core (tcgen05) routing scores with a fused token-max epilogue.
+//
+// Per layer l the scores of every memory block c against every query token t are
+//   D[c][t] = < kr_hat[l][c][:], qt[l][t][:] >      (K = 8 heads x 128 = 1024)
+// a dense bf16 GEMM with fp32 accumulation (M = blocks, N = query tokens).  The
+// epilogue reduces each row over the columns of every query and writes, per (query,
+// layer, block), the largest score m, the second largest and the argmax token; D itself
+// never leaves TMEM.  These bf16-operand scores are a filter: the caller rescores the
+// pairs that can hold the maximum exactly.
+//
+// Warp roles of the persistent kernel (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile [128 blocks x 64] + B tile [BN tokens x 64] per
+//               K-block into a ring of shared-memory stages (128-byte swizzle)
+//   warp 1      one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
+//               accumulators and commits stage / accumulator completion to mbarriers
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max over each query's
+//               columns, store; then release the accumulator
+// Every wait is bounded (2 s on the global timer); on a timeout the kernel sets
+// MSA_DEVERR_TIMEOUT, drains its own copies and MMAs (bounded) and frees TMEM.
+#include <cuda.h>
+
+#include "common.cuh"
 #include "route_tc.cuh"
 
 namespace route_tc {
+namespace {
 
-bool supported(int n_kv_heads) { (void)n_kv_heads; return false; }
+constexpr int kBM = 128;
+constexpr int kBK = 64;                  // bf16 elements per 128-byte row
+constexpr int kKDim = 1024;              // 8 key heads x 128
+constexpr int kKBlocks = kKDim / kBK;    // 16
+constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+constexpr int kThreads = 192;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+template <int BN>
+struct Cfg {
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kTmemCols = 2 * BN;  // two accumulators: 128, 256 or 512 columns
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmem = kStages * kStage + 1024 + kBarBytes;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  False on timeout or when
+// another role has aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer() - t0 > kTimeoutNs) return false;
+    }
+  }
+}
+
+// Bounded wait used while draining after an abort (ignores the abort flag).
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer() - t0 > kTimeoutNs) return;
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 2D tiled TMA load (no multicast) completing on an mbarrier of this CTA.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_slot), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the 128-byte
+// swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte offset), leading
+// byte offset unused for swizzled K-major layouts, descriptor version 1, swizzle mode 2.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int L,
+                    long long C, int n_rows, int m_tiles, const __grid_constant__ QueryLayout ql,
+                    float* __restrict__ m_out, int2* __restrict__ aux_out, int32_t* dev_err) {
+  using K = Cfg<BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::kStages * K::kStage);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + K::kStages;
+  uint64_t* accf = empty + K::kStages;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tiles = n_rows / BN;
+  const int units = L * m_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < K::kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&accf[b]), 1);
+      mbar_init(smem_u32(&acce[b]), 4);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), K::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b)) : "memory");
+      const uint64_t pol_a = policy_evict_first(), pol_b = policy_evict_last();
+      int armed[K::kStages];
+#pragma unroll
+      for (int s = 0; s < K::kStages; ++s) armed[s] = -1;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int l = u / m_tiles, mt = u % m_tiles;
+        const int row_a = (int)((long long)l * C) + mt * kBM;
+        for (int nt = 0; nt < n_tiles && ok; ++nt) {
+          const int row_b = l * n_rows + nt * BN;
+          for (int kb = 0; kb < kKBlocks; ++kb) {
+            if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(&full[stage]);
+            const uint32_t sa = smem_u32(smem + stage * K::kStage);
+            mbar_arrive_expect_tx(fb, K::kStage);
+            tma_load_2d(sa, &tm_a, fb, kb * kBK, row_a, pol_a);
+            tma_load_2d(sa + kABytes, &tm_b, fb, kb * kBK, row_b, pol_b);
+            armed[stage] = (int)phase;
+            if (++stage == K::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+        // let every copy this thread issued land before the CTA can exit
+        for (int s = 0; s < K::kStages; ++s)
+          if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16(kBM, BN);
+      int stage = 0, buf = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, issued = false;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        for (int nt = 0; nt < n_tiles && ok; ++nt) {
+          if (!mbar_wait(smem_u32(&acce[buf]), acc_phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+          for (int kb = 0; kb < kKBlocks; ++kb) {
+            if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * K::kStage);
+            const uint64_t da = sw128_desc(sa), db = sw128_desc(sa + kABytes);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc, (kb | k) != 0 ? 1u : 0u);
+            issued = true;
+            umma_commit(smem_u32(&empty[stage]));
+            if (++stage == K::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(&accf[buf]));
+          if (++buf == 2) {
+            buf = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+        if (issued) {
+          umma_commit(smem_u32(drain));  // arrives once every MMA issued so far has finished
+          mbar_drain(smem_u32(drain), 0u);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 -> TMEM lane quarters 2, 3, 0, 1)
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int l = u / m_tiles, mt = u % m_tiles;
+      const long long row = (long long)mt * kBM + row_in_tile;
+      const bool row_ok = row < C;
+      int carry_b = -1;           // query whose columns continue into the next N tile
+      float c1 = -INFINITY, c2 = -INFINITY;
+      int ci = 0;
+      for (int nt = 0; nt < n_tiles; ++nt) {
+        if (!mbar_wait(smem_u32(&accf[buf]), acc_phase, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+#pragma unroll 1
+        for (int c32 = 0; c32 < BN / 32; ++c32) {
+          const int col0 = nt * BN + c32 * 32;
+          if (col0 >= ql.row0[ql.n_queries]) break;  // trailing padding columns
+          uint32_t r[32];
+          tmem_ld32(tbase + (uint32_t)(c32 * 32), r);
+          tmem_wait_ld();
+          int lo = 0, hi = ql.n_queries;  // owner: largest b with row0[b] <= col0
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (ql.row0[mid] <= col0) lo = mid; else hi = mid;
+          }
+          const int b = lo;
+          const int t0 = col0 - ql.row0[b];            // token index of column col0 in query b
+          const int valid = min(32, ql.len[b] - t0);
+          float m1 = -INFINITY, m2 = -INFINITY;
+          int i1 = 0;
+          if (b == carry_b) {
+            m1 = c1;
+            m2 = c2;
+            i1 = ci;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(r[i]);
+            if (i < valid) {
+              if (x > m1) {
+                m2 = m1;
+                m1 = x;
+                i1 = t0 + i;
+              } else {
+                m2 = fmaxf(m2, x);
+              }
+            }
+          }
+          if (t0 + 32 >= ql.len[b]) {
+            if (row_ok) {
+              const long long o = ((long long)b * L + l) * C + row;
+              m_out[o] = m1;
+              aux_out[o] = make_int2(__float_as_int(m2), i1);
+            }
+            carry_b = -1;
+          } else {
+            carry_b = b;
+            c1 = m1;
+            c2 = m2;
+            ci = i1;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&acce[buf]));
+        if (++buf == 2) {
+          buf = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, K::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 row-major [rows][1024] map with a box of [box_rows][64] and the 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kKDim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kKDim * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
+  using K = Cfg<BN>;
+  CUtensorMap ma, mb;
+  const uint64_t rows_a = (uint64_t)a.L * (uint64_t)a.C;
+  if (!make_map(&ma, a.kr_hat, rows_a, kBM) || !make_map(&mb, a.qt, (uint64_t)a.L * a.n_rows, BN)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return 1;
+  }
+  const int m_tiles = (int)((a.C + kBM - 1) / kBM);
+  const long long units = (long long)a.L * m_tiles;
+  int grid = msa::sm_count();
+  if (units < grid) grid = (int)units;
+  if (cudaFuncSetAttribute(route_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) !=
+      cudaSuccess) {
+    *why = "cudaFuncSetAttribute (shared memory)";
+    return 1;
+  }
+  route_tc_kernel<BN><<<grid, kThreads, K::kSmem, s>>>(ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
+                                                       a.aux, a.dev_err);
+  if (cudaGetLastError() != cudaSuccess) {
+    *why = "kernel launch";
+    return 1;
+  }
+  return 0;
+}
+
+}  // namespace
+
+bool supported(int n_kv_heads) { return n_kv_heads == 8; }
 
 int launch(const LaunchArgs& a, cudaStream_t s, int* launches, const char** why) {
-  (void)a; (void)s;
   *launches = 0;
-  *why = "tensor-core routing path not available in this build";
-  return 1;
+  if ((long long)a.L * a.C >= (1ll << 31) || (long long)a.L * a.n_rows >= (1ll << 31)) {
+    *why = "bank too large for 32-bit TMA row coordinates";
+    return 1;
+  }
+  const int bn = tile_n(a.n_rows);
+  if (a.n_rows % bn != 0) {
+    *why = "operand rows not a multiple of the N tile";
+    return 1;
+  }
+  int r;
+  if (bn == 64) r = launch_bn<64>(a, s, why);
+  else if (bn == 128) r = launch_bn<128>(a, s, why);
+  else r = launch_bn<256>(a, s, why);
+  if (r == 0) *launches = 1;
+  return r;
 }
 
 }  // namespace route_tc

@@ -8,24 +8,55 @@ namespace route_tc {
 constexpr int kMaxQueries = 256;
 // Query lengths up to this many tokens (all queries of a call together) use the scan.
 constexpr int kScanMaxTokens = 8;
+// Every query's tokens start on a multiple of this many operand rows, so that each
+// 32-column slice of the accumulator belongs to a single query.
+constexpr int kQueryAlign = 32;
+// N tile of the MMA (columns = query tokens); the padded token count is a multiple.
+constexpr int kMaxTileN = 256;
 
-// Rows of the bf16 query operand: padded to the tensor-core N tile.
-inline int padded_tokens(int t) { return (t + 63) / 64 * 64; }
+// Padded operand row of every query: row0[b] = sum over b' < b of round_up(T_b', 32).
+inline int padded_rows(const int* q_off, int n_queries, int* row0) {
+  int r = 0;
+  for (int b = 0; b < n_queries; ++b) {
+    if (row0) row0[b] = r;
+    const int t = q_off[b + 1] - q_off[b];
+    r += (t + kQueryAlign - 1) / kQueryAlign * kQueryAlign;
+  }
+  if (row0) row0[n_queries] = r;
+  return r;
+}
+
+// N tile for a padded token count: the smallest of 64/128/256 covering it, else 256.
+inline int tile_n(int rows) { return rows <= 64 ? 64 : (rows <= 128 ? 128 : 256); }
+
+// Rows of the bf16 query operand per layer: padded rows rounded up to the N tile.
+inline int operand_rows(const int* q_off, int n_queries) {
+  const int r = padded_rows(q_off, n_queries, nullptr);
+  const int bn = tile_n(r);
+  return (r + bn - 1) / bn * bn;
+}
 
 bool supported(int n_kv_heads);
 
-struct LaunchArgs {
-  const void* kr_hat;  // bf16 [L][C][8][128]
-  const void* qt;      // bf16 [L][n_pad][8][128], rows >= total tokens are zero
-  int L;
-  int64_t C;
-  int n_pad;
+struct QueryLayout {
   int n_queries;
-  int q_off[kMaxQueries + 1];
-  float* m;            // [B][L][C]
+  int row0[kMaxQueries + 1];   // first operand row of each query (aligned to 32)
+  int len[kMaxQueries];        // tokens of each query
 };
 
-// Enqueues the score kernel(s); returns 0 on success (launches += kernels enqueued).
+struct LaunchArgs {
+  const void* kr_hat;  // bf16 [L][C][8][128]
+  const void* qt;      // bf16 [L][n_rows][8][128], padding rows are zero
+  int L;
+  int64_t C;
+  int n_rows;          // operand rows per layer (multiple of the N tile)
+  QueryLayout ql;
+  float* m;            // [B][L][C]  approximate max over the query's tokens
+  int2* aux;           // [B][L][C]  (bits of the second-largest score, argmax token in the query)
+  int32_t* dev_err;
+};
+
+// Enqueues the score kernel; returns 0 on success (launches += kernels enqueued).
 int launch(const LaunchArgs& a, cudaStream_t s, int* launches, const char** why);
 
 }  // namespace route_tc
