@@ -1,0 +1,477 @@
+"""Benchmark of the MSA hot path on the 100M-token bank.
+
+One step = one query through the whole online path: route + top-16 over all 18 routing
+layers of a 100M-token bank (1.5625M blocks, routing keys resident in HBM), gather of the
+selected documents' compressed K/V from page-locked host memory on a side stream, and 128
+decode tokens of 32/8-head GQA attention over [gathered memory ; local KV].  The offline
+block pooling of the bank runs once before the timed region (it is also timed on its own
+and reported under "pool").
+
+Prints one JSON line.  --impl reference times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "bank tokens routed/s + K̄ᵣ scan GB/s vs HBM peak at 100M; p50 route+decode ms"
+WORKLOAD = ("100M-token bank (100,000 docs, lognormal lengths rounded to 64, 1,562,500 blocks), "
+            "18 routing layers x 8 heads x 128 bf16 unit routing keys in HBM (57.6 GB); "
+            "query T=256 tokens with 16 planted target documents, top-16 per layer; gather of the "
+            "selected blocks' K/V from a page-locked host store; 128-token GQA 32/8 decode, local KV 256")
+N_DOCS, N_TOKENS, L, H, HQ, D, TOPK, T, DEC, SEED = 100_000, 100_000_000, 18, 8, 32, 128, 16, 256, 128, 3
+THETA = 1e6
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", 0)), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.rows = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            if len(r) < 9:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() in ("active", "0x1", "1"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+def smi_id(dev) -> str:
+    """nvidia-smi --id for a torch device: its PCI bus id when torch exposes it."""
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    bus, devno, dom = getattr(p, "pci_bus_id", None), getattr(p, "pci_device_id", None), getattr(p, "pci_domain_id", 0)
+    if bus is None or devno is None:
+        return str(dev.index or 0)
+    return f"{dom:08X}:{bus:02X}:{devno:02X}.0"
+
+
+# ----------------------------------------------------------------------------- workload
+
+def make_workload(dev, host_store_chunks: int):
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+
+    t0 = time.time()
+    lens = syn.doc_lengths_exact_total(SEED, N_DOCS, N_TOKENS)
+    bank = syn.make_bank(SEED, N_DOCS, lens, L)
+    C = bank.n_chunks
+    coffs = bank.doc_chunk_offsets
+    topic = torch.from_numpy(bank.topic).to(dev)
+    # routing keys: pooled-level draws (topic + noise/8), made unit per head by the pool
+    # kernel with 1-token blocks (no rotation)
+    kr_hat = torch.empty((L, C, H, D), dtype=torch.bfloat16, device=dev)
+    scratch = torch.empty((C, H, D), dtype=torch.bfloat16, device=dev)
+    row_topic = torch.from_numpy(syn.chunk_docs(coffs)).to(dev)
+    ones = torch.arange(C + 1, dtype=torch.int64, device=dev)
+    for l in range(L):
+        syn.device_fill(scratch, SEED, syn.STREAM_KRBAR, l, 0, 0, C, H * D, syn.POOLED_NOISE, topic, row_topic)
+        msa.msa_pool_blocks(None, None, scratch, ones, ones, C, C, H, D, 1, 0.0, None, None, kr_hat[l], None, None,
+                            in_dtype=msa.MSA_BF16)
+    del scratch, row_topic, ones
+    torch.cuda.synchronize(dev)
+    log(f"routing keys ready: {C} blocks x {L} layers ({kr_hat.numel() * 2 / 1e9:.1f} GB) in {time.time() - t0:.1f}s")
+    # content store: host_store_chunks physical blocks per layer; document d reads the
+    # contiguous physical range starting at a hashed offset (same bytes per selection)
+    P = min(host_store_chunks, C)
+    per_doc = np.diff(coffs)
+    h = syn.hashes(syn.tensor_key(SEED, syn.STREAM_TARGETS, 0, 99), np.arange(N_DOCS, dtype=np.uint64))
+    store_off = (h % np.uint64(max(1, P - int(per_doc.max())))).astype(np.int64) if P < C else coffs[:-1].copy()
+    host_kv = torch.empty((L, P, 2, H, D), dtype=torch.bfloat16, pin_memory=True)
+    stage = torch.empty((2, P, H * D), dtype=torch.bfloat16, device=dev)
+    for l in range(L):
+        syn.device_fill(stage[0], SEED, syn.STREAM_KBAR, l, 0, 0, P, H * D, syn.POOLED_NOISE)
+        syn.device_fill(stage[1], SEED, syn.STREAM_VBAR, l, 0, 0, P, H * D, syn.POOLED_NOISE)
+        host_kv[l].copy_(stage.permute(1, 0, 2).reshape(P, 2, H, D))
+    del stage
+    log(f"host content store: {P} blocks x {L} layers ({host_kv.numel() * 2 / 1e9:.1f} GB pinned)")
+    return bank, kr_hat, host_kv, store_off, topic
+
+
+def make_queries(dev, bank, topic, n_queries: int):
+    import torch
+
+    import msa_synth as syn
+    qs, targets = [], []
+    for b in range(n_queries):
+        tg = syn.pick_targets(SEED, N_DOCS, TOPK, sub=b)
+        targets.append(tg)
+        q = torch.empty((L, T, HQ, D), dtype=torch.bfloat16, device=dev)
+        rt = torch.from_numpy(np.repeat(tg[np.arange(T) % TOPK], HQ).astype(np.int32)).to(dev)
+        for l in range(L):
+            syn.device_fill(q[l], SEED, syn.STREAM_QR, l, b, 0, T * HQ, D, 0.5, topic, rt)
+        qs.append(q)
+    return qs, targets
+
+
+def make_decode_inputs(dev):
+    import torch
+
+    import msa_synth as syn
+    dq = torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16, device=dev)
+    dk = torch.empty((DEC, 1, L, H, D), dtype=torch.bfloat16, device=dev)
+    dv = torch.empty_like(dk)
+    for s in range(DEC):
+        syn.device_fill(dq[s], SEED, syn.STREAM_DEC_Q, s, 0, 0, L * HQ, D)
+        syn.device_fill(dk[s], SEED, syn.STREAM_DEC_K, s, 0, 0, L * H, D)
+        syn.device_fill(dv[s], SEED, syn.STREAM_DEC_V, s, 0, 0, L * H, D)
+    pk = torch.empty((L, H, T, D), dtype=torch.bfloat16, device=dev)
+    pv = torch.empty_like(pk)
+    syn.device_fill(pk, SEED, syn.STREAM_LOCAL_K, 0, 0, 0, L * H * T, D)
+    syn.device_fill(pv, SEED, syn.STREAM_LOCAL_V, 0, 0, 0, L * H * T, D)
+    return dq, dk, dv, pk, pv
+
+
+def time_pool(dev):
+    """Offline pooling throughput on raw bf16 tokens of a 1M-token bank, one layer."""
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+    lens = syn.doc_lengths_lognormal(1, 1000)
+    bank = syn.make_bank(1, 1000, lens, 1)
+    n, C = bank.n_tokens, bank.n_chunks
+    x = [torch.empty((n, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    for i, st in enumerate((syn.STREAM_K, syn.STREAM_V, syn.STREAM_KR)):
+        syn.device_fill(x[i], 1, st, 0, 0, 0, n, H * D, 1.0, torch.from_numpy(bank.topic).to(dev) if i == 2 else None,
+                        torch.from_numpy(syn.token_docs(bank.doc_tok_offsets)).to(dev) if i == 2 else None)
+    toff = torch.from_numpy(bank.doc_tok_offsets).to(dev)
+    coff = torch.from_numpy(bank.doc_chunk_offsets).to(dev)
+    out = [torch.empty((C, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    nr = torch.empty((C, H), device=dev)
+
+    def run():
+        msa.msa_pool_blocks(x[0], x[1], x[2], toff, coff, 1000, C, H, D, 64, THETA, out[0], out[1], out[2], nr, None)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    s.record()
+    for _ in range(reps):
+        run()
+    e.record()
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / reps
+    by = n * 3 * H * D * 2 + C * (3 * H * D * 2 + H * 4)
+    return {"tokens": n, "blocks": C, "ms": round(ms, 4), "gbs": round(by / ms / 1e6, 1),
+            "bytes_per_token": round(by / n, 1)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import top_kv_routing_b200 as msa
+    from top_kv_routing_b200.engine import SparseMemory
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm_peak, bf16_peak, bf16_sus, peak_src = measured_peaks()
+
+    bank, kr_hat, host_kv, store_off, topic = make_workload(dev, args.host_store_blocks)
+    qs, targets = make_queries(dev, bank, topic, args.queries)
+    dq, dk, dv, pk, pv = make_decode_inputs(dev)
+    out = torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16, device=dev)
+    eng = SparseMemory(kr_hat, bank.doc_chunk_offsets, host_kv, store_off, n_q_heads=HQ, top_k=TOPK,
+                       query_tokens=T, local_cap=T + DEC, rope_theta=THETA)
+    eng.set_local_prefix(pk, pv)
+    ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_a.record()
+    ev_b.record()
+    torch.cuda.synchronize(dev)
+    msa.msa_route_set_profile_events(ev_a, ev_b)
+    eng.qr.copy_(qs[0])
+    graph = eng.capture(dq, dk, dv, out)
+    msa.msa_route_set_profile_events(None, None)
+    launches = eng.launches_per_query
+
+    def score_kernel_ms(reps=5):
+        # the score kernel's own device time: the events recorded around it inside the
+        # graph, else the same call outside a graph with the events set
+        vals = []
+        try:
+            for i in range(reps):
+                eng.qr.copy_(qs[i % len(qs)])
+                graph.replay()
+                torch.cuda.synchronize(dev)
+                vals.append(ev_a.elapsed_time(ev_b))
+        except RuntimeError:
+            vals = []
+            msa.msa_route_set_profile_events(ev_a, ev_b)
+            for i in range(reps):
+                eng.qr.copy_(qs[i % len(qs)])
+                msa.msa_route_topk(eng.qr, [0, T], eng.kr_hat, eng.doc_chunk_offsets, eng.n_docs, eng.C, L, HQ, H,
+                                   D, TOPK, eng.ids, eng.scores, eng.ws)
+                torch.cuda.synchronize(dev)
+                vals.append(ev_a.elapsed_time(ev_b))
+            msa.msa_route_set_profile_events(None, None)
+        return float(np.mean(vals))
+
+    def step(i, host=None):
+        if host is None:
+            eng.qr.copy_(qs[i % len(qs)])
+        else:
+            eng.qr.copy_(host["qr"][i % len(qs)], non_blocking=True)
+            dq.copy_(host["dq"], non_blocking=True)
+            dk.copy_(host["dk"], non_blocking=True)
+            dv.copy_(host["dv"], non_blocking=True)
+        graph.replay()
+        if host is not None:
+            host["ids"].copy_(eng.ids, non_blocking=True)
+            host["scores"].copy_(eng.scores, non_blocking=True)
+            host["out"].copy_(out, non_blocking=True)
+
+    # correctness guard on the benchmark's own output: planted documents are selected
+    eng.dev_err.zero_()
+    step(0)
+    torch.cuda.synchronize(dev)
+    got = eng.ids.cpu().numpy()[0]
+    hits = np.mean([len(set(got[l].tolist()) & set(targets[0].tolist())) / TOPK for l in range(L)])
+    dev_err = int(eng.dev_err.item())
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(smi_id(dev)) as clk:
+        starts[0].record()
+        for i in range(args.steps):
+            step(i)
+            starts[i + 1].record()
+        torch.cuda.synchronize(dev)
+    per_step = [starts[i].elapsed_time(starts[i + 1]) for i in range(args.steps)]
+    total_ms = starts[0].elapsed_time(starts[-1])
+    gemm_avg = score_kernel_ms()
+
+    # end to end: pinned host inputs in, results out, every step
+    host = {"qr": [q.cpu().pin_memory() for q in qs], "dq": dq.cpu().pin_memory(), "dk": dk.cpu().pin_memory(),
+            "dv": dv.cpu().pin_memory(), "ids": torch.empty((1, L, TOPK), dtype=torch.int32).pin_memory(),
+            "scores": torch.empty((1, L, TOPK), dtype=torch.float32).pin_memory(),
+            "out": torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16).pin_memory()}
+    for i in range(2):
+        step(i, host)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        step(i, host)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = host["qr"][0].numel() * 2 + (dq.numel() + dk.numel() + dv.numel()) * 2
+    d2h = host["ids"].numel() * 4 + host["scores"].numel() * 4 + host["out"].numel() * 2
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+    pool = time_pool(dev) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms = total_ms / args.steps
+    units = N_TOKENS * args.steps * world
+    value = units / (total_ms / 1e3)
+    algo_bytes = L * bank.n_chunks * H * D * 2
+    achieved = algo_bytes / (gemm_avg / 1e3) / 1e9
+    flops = 2.0 * T * H * D * L * bank.n_chunks
+    p = sorted(per_step)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "bank tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n_docs": N_DOCS, "n_tokens": N_TOKENS, "n_blocks": bank.n_chunks,
+                   "layers": L, "kv_heads": H, "q_heads": HQ, "head_dim": D, "query_tokens": T, "top_k": TOPK,
+                   "decode_tokens": DEC, "distinct_queries": len(qs), "host_store_blocks": int(host_kv.shape[1]),
+                   "l2": "inputs larger than L2 (57.6 GB of routing keys stream through every step)",
+                   "graph": "one CUDA graph per query (route, gather on a side stream, 128 decode steps)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "scan_gbs": round(achieved, 1),
+        "p50_route_decode_ms": round(p[len(p) // 2], 4),
+        "p99_route_decode_ms": round(p[min(len(p) - 1, int(0.99 * len(p)))], 4),
+        "roofline": {"bound": "hbm", "kernel": "route score GEMM (tcgen05)", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes": algo_bytes, "kernel_ms": round(gemm_avg, 4),
+                     "tflops": round(flops / (gemm_avg / 1e3) / 1e12, 1),
+                     "tensor_frac": round(flops / (gemm_avg / 1e3) / 1e12 / bf16_peak, 4),
+                     "frac_of_8tbs": round(achieved / 8000.0, 4)},
+        "e2e": {"value": round(units / (e2e_ms / 1e3), 1), "unit": "bank tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+        "pool": pool,
+        "planted_recall": round(float(hits), 4),
+        "dev_err": dev_err,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def _oracle_sample(n_blocks: int):
+    """Layer-0 routing keys of the first n_blocks blocks of the 100M bank and the T=256 query."""
+    import msa_synth as syn
+    lens = syn.doc_lengths_exact_total(SEED, N_DOCS, N_TOKENS)
+    bank = syn.make_bank(SEED, N_DOCS, lens, L)
+    coffs = bank.doc_chunk_offsets
+    n_docs = int(np.searchsorted(coffs, n_blocks, side="right")) - 1
+    n_docs = max(1, n_docs)
+    nb = int(coffs[n_docs])
+    keys = syn.bf16_bits_to_f32(syn.pooled_router_keys(bank, 0, 0, nb))
+    tg = syn.pick_targets(SEED, N_DOCS, TOPK, sub=0)
+    q = syn.query_router(SEED, 0, 0, T, HQ, D, bank.topic, tg, dtype="bf16")
+    return syn.bf16_bits_to_f32(q), keys, coffs[:n_docs + 1].copy(), nb
+
+
+def cpu_baseline(seconds: float):
+    """The CPU oracle's routing (explicit cosine form, one core) on a bounded sample."""
+    import oracle
+    t_probe = time.time()
+    q, keys, offs, nb = _oracle_sample(64)
+    t0 = time.time()
+    oracle.route(q, keys, offs, TOPK)
+    per_block = (time.time() - t0) / nb
+    n = max(64, int(seconds / max(per_block, 1e-9)))
+    q, keys, offs, nb = _oracle_sample(n)
+    t0 = time.time()
+    oracle.route(q, keys, offs, TOPK)
+    dt = time.time() - t0
+    # bank tokens routed per second over all 18 layers: 64 tokens per block, 1 of 18 layers
+    value = nb * 64 / L / dt
+    return {"value": round(value, 3), "unit": "bank tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"layer 0 of 18, first {nb} of 1,562,500 blocks, T=256 query, explicit cosine form "
+                      f"({dt:.1f} s); rate scaled to all 18 layers", "setup_s": round(t0 - t_probe, 1)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline(min(2.0, args.cpu_seconds))
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(args.cpu_seconds / max(1, args.steps)))
+    v = float(np.mean([x["value"] for x in vals]))
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "bank tokens/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": round(v, 3), "unit": "bank tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": round(v, 3), "unit": "bank tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--queries", type=int, default=4, help="distinct synthetic queries cycled over the steps")
+    ap.add_argument("--host-store-blocks", type=int, default=163_840,
+                    help="physical blocks per layer in the page-locked content store")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

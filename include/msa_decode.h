@@ -17,6 +17,10 @@
 extern "C" {
 #endif
 
+/* Workspace bytes of one msa_sparse_decode call (partial softmax sums of the key splits). */
+msa_status msa_sparse_decode_workspace_size(int32_t n_queries, int32_t n_layers, int32_t n_q_heads,
+                                            int32_t n_kv_heads, size_t* bytes);
+
 /* One decode step for every query b and layer l.  With i = local_len[b] (read on the
  * device) and p = rope_pos_offset + i:
  *   q' = RoPE(q, p), k' = RoPE(k_new, p)  (rotate-half, angle p * theta^(-2j/d), fp64-reduced)
@@ -35,16 +39,23 @@ extern "C" {
  *           (msa_gather_kv output); mem_len DEVICE int32 [n_queries][n_layers]
  *   out     DEVICE bf16 [n_queries][n_layers][n_q_heads][head_dim]
  *   head_dim = 128; n_q_heads / n_kv_heads in {1, 2, 4, 8}; n_kv_heads <= 16.
+ *   workspace  DEVICE, >= msa_sparse_decode_workspace_size bytes, 16-byte aligned, zeroed
+ *              (e.g. cudaMemset) once before its first use; every call leaves it ready for
+ *              the next (its arrival counters return to zero).  Calls that share a
+ *              workspace must not overlap on the device.
+ * The keys of each (query, layer, key head) are split over several CTAs (flash-decoding);
+ * the last CTA of each to finish merges the partial softmax sums, and the last merge of
+ * a query advances its local_len.
  * A query whose cache is full (local_len >= local_cap) is skipped (out untouched, length
  * not advanced) and sets MSA_DEVERR_LOCAL_FULL; mem_len > max_mem_chunks is clamped with
- * MSA_DEVERR_CAPACITY.  Two kernel launches, asynchronous on stream, graph-capturable
+ * MSA_DEVERR_CAPACITY.  One kernel launch, asynchronous on stream, graph-capturable
  * (every per-step quantity is read on the device). */
 msa_status msa_sparse_decode(const void* q, const void* k_new, const void* v_new, int32_t n_queries,
                              int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                              void* local_k, void* local_v, int32_t* local_len, int32_t local_cap,
                              const void* mem_kv, const int32_t* mem_len, int32_t max_mem_chunks,
                              int32_t rope_pos_offset, float rope_theta, float softmax_scale, void* out,
-                             int32_t* dev_err, msa_stream_t stream);
+                             void* workspace, size_t workspace_bytes, int32_t* dev_err, msa_stream_t stream);
 
 const char* msa_decode_last_error(void);
 

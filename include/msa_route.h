@@ -66,6 +66,13 @@ msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_of
  * (for launch accounting). */
 int32_t msa_route_last_launch_count(void);
 
+/* Measurement hook: when both are non-NULL (cudaEvent_t handles created by the caller),
+ * every later msa_route_topk call on this thread records start_event right before and
+ * stop_event right after its score kernel (scan or tensor-core GEMM) on the call's
+ * stream, so cudaEventElapsedTime gives that kernel's device time (also inside a CUDA
+ * graph capture).  NULL, NULL turns it off.  Returns MSA_OK. */
+msa_status msa_route_set_profile_events(void* start_event, void* stop_event);
+
 const char* msa_route_last_error(void);
 
 #ifdef __cplusplus

@@ -71,7 +71,7 @@ def test_invalid_arguments_rejected_without_gpu(msa):
     with pytest.raises(msa.MsaError) as e:   # 32 query heads over 5 key heads
         z = np.zeros(16, np.uint16)
         msa.msa_sparse_decode(z, z, z, 1, 1, 32, 5, 128, z, z, np.zeros(1, np.int32), 4, z, np.zeros(1, np.int32),
-                              4, 16, 1e6, 0.1, z, stream=0)
+                              4, 16, 1e6, 0.1, z, z, stream=0)
     assert e.value.status == msa.MSA_ERR_INVALID_ARG
 
 

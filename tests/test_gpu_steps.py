@@ -312,8 +312,9 @@ def _decode_case(msa, B, L, M_max, mem_len, len0, cap, steps, offset, seed=0, hq
         kb = syn.fill(seed, syn.STREAM_DEC_K, s, 0, 0, B * L * h, D, dtype="bf16").reshape(B, L, h, D)
         vb = syn.fill(seed, syn.STREAM_DEC_V, s, 0, 0, B * L * h, D, dtype="bf16").reshape(B, L, h, D)
         out = torch.full((B, L, hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(msa.msa_sparse_decode_workspace_size(B, L, hq, h), dtype=torch.uint8, device="cuda")
         msa.msa_sparse_decode(bf16_tensor(qb), bf16_tensor(kb), bf16_tensor(vb), B, L, hq, h, D, d_lk, d_lv, d_len, cap,
-                              d_mem, d_mlen, M_max, offset, 1e6, scale, out, err)
+                              d_mem, d_mlen, M_max, offset, 1e6, scale, out, ws, err)
         torch.cuda.synchronize()
         got = bf16_to_np(out)
         for b in range(B):
@@ -357,9 +358,10 @@ def test_decode_full_cache_sets_flag_and_skips(msa):
     d_len = torch.tensor([cap], dtype=torch.int32, device="cuda")
     err = _err()
     z = lambda *s: torch.zeros(s, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(msa.msa_sparse_decode_workspace_size(B, L, HQ, H), dtype=torch.uint8, device="cuda")
     msa.msa_sparse_decode(z(B, L, HQ, D), z(B, L, H, D), z(B, L, H, D), B, L, HQ, H, D, z(B, L, H, cap, D),
                           z(B, L, H, cap, D), d_len, cap, z(B, L, 2, H, M, D),
-                          torch.tensor([[M]], dtype=torch.int32, device="cuda"), M, 4, 1e6, 0.1, out, err)
+                          torch.tensor([[M]], dtype=torch.int32, device="cuda"), M, 4, 1e6, 0.1, out, ws, err)
     torch.cuda.synchronize()
     assert int(err.item()) & msa.MSA_DEVERR_LOCAL_FULL
     assert int(d_len.item()) == cap and float(out.float().abs().sum()) == 0.0

@@ -1,179 +1,18 @@
 """B200-native Memory Sparse Attention (MSA) hot path.
 
-Thin ctypes binding over the four C-ABI libraries in ``lib/`` (see ``include/*.h``):
-argument marshalling only; every step runs in the libraries' CUDA kernels.  PyTorch is
-used by callers for device memory and streams.  There is no CPU fallback: importing this
-package fails if the libraries have not been built (``python -m top_kv_routing_b200.build``).
+The C-ABI libraries (``lib/libmsa_{pool,route,gather,decode}.so``, declared in
+``include/*.h``) are bound in ``abi``; their entry points are re-exported here under the
+same names and loaded on first use.  There is no CPU fallback: the first access raises
+ImportError if the libraries have not been built (``python top_kv_routing_b200/build.py``).
 """
 from __future__ import annotations
 
-import ctypes
-import os
+import importlib
 
-import numpy as np
-
-_HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_DIR = os.path.join(_HERE, "lib")
-
-MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY, MSA_ERR_TIMEOUT = range(6)
-MSA_F32, MSA_BF16 = 0, 1
-MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR = 0, 1, 2
-(MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS, MSA_DEVERR_TIMEOUT,
- MSA_DEVERR_UNCERTIFIED) = 1, 2, 4, 8, 16, 32
-
-_STATUS = {1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA", 4: "MSA_ERR_CAPACITY",
-           5: "MSA_ERR_TIMEOUT"}
+_SUBMODULES = {"abi", "build", "engine"}
 
 
-class MsaError(RuntimeError):
-    def __init__(self, status: int, where: str, msg: str):
-        super().__init__(f"{where}: {_STATUS.get(status, status)}: {msg}")
-        self.status = status
-
-
-def _load(name: str) -> ctypes.CDLL:
-    path = os.path.join(LIB_DIR, f"libmsa_{name}.so")
-    if not os.path.exists(path):
-        raise ImportError(f"{path} is missing: build the CUDA libraries first "
-                          "(python -m top_kv_routing_b200.build)")
-    return ctypes.CDLL(path)
-
-
-_p, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
-
-pool_lib = _load("pool")
-route_lib = _load("route")
-gather_lib = _load("gather")
-decode_lib = _load("decode")
-
-pool_lib.msa_count_chunks.argtypes = [_p, _i32, _i32, _p]
-pool_lib.msa_count_chunks.restype = _i64
-pool_lib.msa_pool_blocks.argtypes = [_p, _p, _p, _i32, _p, _p, _i32, _i64, _i32, _i32, _i32, _f32,
-                                     _p, _p, _p, _p, _p, _p]
-pool_lib.msa_pool_blocks.restype = _i32
-pool_lib.msa_pool_last_error.restype = ctypes.c_char_p
-
-route_lib.msa_route_topk_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i32, _i32,
-                                                    ctypes.POINTER(_sz)]
-route_lib.msa_route_topk_workspace_size.restype = _i32
-route_lib.msa_route_topk.argtypes = [_p, _i32, _p, _i32, _p, _p, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
-                                     _p, _p, _p, _sz, _i32, _p, _p]
-route_lib.msa_route_topk.restype = _i32
-route_lib.msa_route_last_launch_count.restype = _i32
-route_lib.msa_route_last_error.restype = ctypes.c_char_p
-
-gather_lib.msa_gather_kv.argtypes = [_p, _i64, _p, _p, _i32, _p, _i32, _i32, _i32, _i32, _i32, _i32, _p, _p,
-                                     _p, _p]
-gather_lib.msa_gather_kv.restype = _i32
-gather_lib.msa_gather_last_error.restype = ctypes.c_char_p
-
-decode_lib.msa_sparse_decode.argtypes = [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _i32, _p, _p,
-                                         _i32, _i32, _f32, _f32, _p, _p, _p]
-decode_lib.msa_sparse_decode.restype = _i32
-decode_lib.msa_decode_last_error.restype = ctypes.c_char_p
-
-# Kernel launches enqueued by each entry point (the route count is read back per call).
-LAUNCHES_POOL = 1
-LAUNCHES_GATHER = 1
-LAUNCHES_DECODE = 2
-
-
-def loaded_libraries() -> list[str]:
-    return [os.path.join(LIB_DIR, f"libmsa_{n}.so") for n in ("pool", "route", "gather", "decode")]
-
-
-def _ptr(t) -> int | None:
-    """Raw address of a torch tensor / numpy array (None stays NULL)."""
-    if t is None:
-        return None
-    if isinstance(t, np.ndarray):
-        return t.ctypes.data
-    return t.data_ptr()
-
-
-def _stream(stream) -> int | None:
-    if stream is None:
-        import torch
-        return torch.cuda.current_stream().cuda_stream
-    return getattr(stream, "cuda_stream", stream)
-
-
-def _check(status: int, where: str, lib, err_fn: str):
-    if status != MSA_OK:
-        raise MsaError(status, where, (getattr(lib, err_fn)() or b"").decode())
-
-
-# ----------------------------------------------------------------------------- step 1
-
-def msa_count_chunks(doc_tok_offsets, chunk: int = 64):
-    """Host: (block count, per-document block offsets int64 [n_docs+1])."""
-    o = np.ascontiguousarray(doc_tok_offsets, dtype=np.int64)
-    out = np.empty_like(o)
-    n = pool_lib.msa_count_chunks(o.ctypes.data, len(o) - 1, chunk, out.ctypes.data)
-    if n < 0:
-        raise MsaError(MSA_ERR_INVALID_ARG, "msa_count_chunks", "bad offsets")
-    return int(n), out
-
-
-def msa_pool_blocks(k, v, kr, doc_tok_offsets, doc_chunk_offsets, n_docs: int, n_chunks: int, n_heads: int,
-                    head_dim: int, chunk: int, rope_theta: float, k_bar=None, v_bar=None, kr_hat=None,
-                    kr_norm=None, dev_err=None, in_dtype: int | None = None, stream=None):
-    if in_dtype is None:
-        x = next(t for t in (k, v, kr) if t is not None)
-        in_dtype = MSA_BF16 if str(x.dtype) == "torch.bfloat16" else MSA_F32
-    st = pool_lib.msa_pool_blocks(_ptr(k), _ptr(v), _ptr(kr), in_dtype, _ptr(doc_tok_offsets),
-                                  _ptr(doc_chunk_offsets), n_docs, n_chunks, n_heads, head_dim, chunk,
-                                  rope_theta, _ptr(k_bar), _ptr(v_bar), _ptr(kr_hat), _ptr(kr_norm),
-                                  _ptr(dev_err), _stream(stream))
-    _check(st, "msa_pool_blocks", pool_lib, "msa_pool_last_error")
-
-
-# ----------------------------------------------------------------------------- step 2
-
-def msa_route_topk_workspace_size(n_layers: int, n_queries: int, total_q_tokens: int, n_kv_heads: int,
-                                  n_chunks: int, n_docs: int, top_k: int) -> int:
-    out = _sz(0)
-    st = route_lib.msa_route_topk_workspace_size(n_layers, n_queries, total_q_tokens, n_kv_heads, n_chunks,
-                                                 n_docs, top_k, ctypes.byref(out))
-    _check(st, "msa_route_topk_workspace_size", route_lib, "msa_route_last_error")
-    return int(out.value)
-
-
-def msa_route_topk(qr, q_offsets, kr_hat, doc_chunk_offsets, n_docs: int, n_chunks: int, n_layers: int,
-                   n_q_heads: int, n_kv_heads: int, head_dim: int, top_k: int, out_ids, out_scores, workspace,
-                   flags: int = MSA_ROUTE_AUTO, dev_err=None, q_dtype: int | None = None, stream=None) -> int:
-    """Returns the number of kernels the call enqueued."""
-    qo = np.ascontiguousarray(q_offsets, dtype=np.int32)
-    if q_dtype is None:
-        q_dtype = MSA_BF16 if str(qr.dtype) == "torch.bfloat16" else MSA_F32
-    ws_bytes = workspace.numel() * workspace.element_size()
-    st = route_lib.msa_route_topk(_ptr(qr), q_dtype, qo.ctypes.data, len(qo) - 1, _ptr(kr_hat),
-                                  _ptr(doc_chunk_offsets), n_docs, n_chunks, n_layers, n_q_heads, n_kv_heads,
-                                  head_dim, top_k, _ptr(out_ids), _ptr(out_scores), _ptr(workspace), ws_bytes,
-                                  flags, _ptr(dev_err), _stream(stream))
-    _check(st, "msa_route_topk", route_lib, "msa_route_last_error")
-    return int(route_lib.msa_route_last_launch_count())
-
-
-# ----------------------------------------------------------------------------- step 3
-
-def msa_gather_kv(host_kv, n_store_chunks: int, doc_chunk_offsets, doc_store_offsets, n_docs: int, ids,
-                  n_queries: int, n_layers: int, top_k: int, n_heads: int, head_dim: int, max_mem_chunks: int,
-                  dev_kv, mem_len, dev_err=None, stream=None):
-    st = gather_lib.msa_gather_kv(_ptr(host_kv), n_store_chunks, _ptr(doc_chunk_offsets), _ptr(doc_store_offsets),
-                                  n_docs, _ptr(ids), n_queries, n_layers, top_k, n_heads, head_dim,
-                                  max_mem_chunks, _ptr(dev_kv), _ptr(mem_len), _ptr(dev_err), _stream(stream))
-    _check(st, "msa_gather_kv", gather_lib, "msa_gather_last_error")
-
-
-# ----------------------------------------------------------------------------- step 4
-
-def msa_sparse_decode(q, k_new, v_new, n_queries: int, n_layers: int, n_q_heads: int, n_kv_heads: int,
-                      head_dim: int, local_k, local_v, local_len, local_cap: int, mem_kv, mem_len,
-                      max_mem_chunks: int, rope_pos_offset: int, rope_theta: float, softmax_scale: float, out,
-                      dev_err=None, stream=None):
-    st = decode_lib.msa_sparse_decode(_ptr(q), _ptr(k_new), _ptr(v_new), n_queries, n_layers, n_q_heads,
-                                      n_kv_heads, head_dim, _ptr(local_k), _ptr(local_v), _ptr(local_len),
-                                      local_cap, _ptr(mem_kv), _ptr(mem_len), max_mem_chunks, rope_pos_offset,
-                                      rope_theta, softmax_scale, _ptr(out), _ptr(dev_err), _stream(stream))
-    _check(st, "msa_sparse_decode", decode_lib, "msa_decode_last_error")
+def __getattr__(name: str):
+    if name.startswith("__") or name in _SUBMODULES:
+        raise AttributeError(name)
+    return getattr(importlib.import_module(__name__ + ".abi"), name)

@@ -1,6 +1,6 @@
 """Builds the four C-ABI libraries (and the synthetic-input device library) for sm_100a.
 
-Run ``python -m top_kv_routing_b200.build``; the shared objects land in-tree under
+Run ``python top_kv_routing_b200/build.py``; the shared objects land in-tree under
 ``top_kv_routing_b200/lib`` and ``msa_synth/`` so they travel with the source tree.
 """
 from __future__ import annotations

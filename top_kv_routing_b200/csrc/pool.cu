@@ -221,6 +221,79 @@ __global__ void __launch_bounds__(256) pool_kernel(
   }
 }
 
+// 1-token blocks without rotation: block c is token c, so each output row is its input
+// row (K, V copied to bf16; K_r made unit per head).  One warp per row; lane owns the
+// 8-element vectors lane + 32 i of the H*128-element row (head = (lane + 32 i) / 16).
+template <typename TIn, int NV>
+__global__ void __launch_bounds__(256) pool_rows_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
+                                                        const TIn* __restrict__ kr, int64_t n_rows,
+                                                        __nv_bfloat16* __restrict__ k_bar,
+                                                        __nv_bfloat16* __restrict__ v_bar,
+                                                        __nv_bfloat16* __restrict__ kr_hat,
+                                                        float* __restrict__ kr_norm) {
+  constexpr int R = NV * 256;
+  const int lane = threadIdx.x % 32;
+  const int64_t w0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
+  const int64_t nw = (int64_t)gridDim.x * blockDim.x / 32;
+  for (int64_t row = w0; row < n_rows; row += nw) {
+    const int64_t base = row * R;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int64_t e = base + 8 * (lane + 32 * i);
+      float x[8];
+      if (k != nullptr && k_bar != nullptr) {
+        Loader<TIn>::load8(k + e, x);
+        store8_bf16(k_bar + e, x);
+      }
+      if (v != nullptr && v_bar != nullptr) {
+        Loader<TIn>::load8(v + e, x);
+        store8_bf16(v_bar + e, x);
+      }
+    }
+    if (kr != nullptr) {
+      float x[NV][8];
+#pragma unroll
+      for (int i = 0; i < NV; ++i) Loader<TIn>::load8(kr + base + 8 * (lane + 32 * i), x[i]);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        float ss = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ss += x[i][u] * x[i][u];
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);   // 16 lanes share a head
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+        const float nrm = sqrtf(ss);
+        const float inv = 1.0f / fmaxf(nrm, 1e-8f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[i][u] *= inv;
+        if (kr_hat != nullptr) store8_bf16(kr_hat + base + 8 * (lane + 32 * i), x[i]);
+        if (kr_norm != nullptr && (lane & 15) == 0) kr_norm[row * (2 * NV) + ((lane + 32 * i) >> 4)] = nrm;
+      }
+    }
+  }
+}
+
+template <typename TIn>
+bool launch_rows(int H, const void* k, const void* v, const void* kr, int64_t n, void* kb, void* vb, void* krh,
+                 float* krn, cudaStream_t s) {
+  int64_t blocks = (n + 7) / 8;
+  const int64_t cap = (int64_t)msa::sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+#define MSA_ROWS(NV)                                                                                         \
+  pool_rows_kernel<TIn, NV><<<(unsigned)blocks, 256, 0, s>>>((const TIn*)k, (const TIn*)v, (const TIn*)kr, n, \
+                                                            (__nv_bfloat16*)kb, (__nv_bfloat16*)vb,           \
+                                                            (__nv_bfloat16*)krh, krn)
+  switch (H) {
+    case 2: MSA_ROWS(1); return true;
+    case 4: MSA_ROWS(2); return true;
+    case 8: MSA_ROWS(4); return true;
+    case 16: MSA_ROWS(8); return true;
+    default: return false;
+  }
+#undef MSA_ROWS
+}
+
 }  // namespace
 
 extern "C" int64_t msa_count_chunks(const int64_t* doc_tok_offsets_host, int32_t n_docs, int32_t chunk,
@@ -263,6 +336,17 @@ extern "C" msa_status msa_pool_blocks(const void* k, const void* v, const void* 
   if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
   if (n_chunks == 0 || n_docs == 0 || (!k && !v && !kr)) return msa_ok();
 
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (chunk == 1 && (k == nullptr || rope_theta == 0.0f)) {
+    // every block is one token: row-wise fast path (no positions, so no offsets needed)
+    const bool ok = in_dtype == MSA_F32 ? launch_rows<float>(n_heads, k, v, kr, n_chunks, k_bar, v_bar, kr_hat, kr_norm, s)
+                                        : launch_rows<__nv_bfloat16>(n_heads, k, v, kr, n_chunks, k_bar, v_bar, kr_hat,
+                                                                     kr_norm, s);
+    if (ok) {
+      MSA_CUDA_TRY(cudaGetLastError());
+      return msa_ok();
+    }
+  }
   const size_t smem = sizeof(PoolSmem);
   const int threads = 16 * n_heads;
   const int use_rope = (rope_theta != 0.0f && k != nullptr) ? 1 : 0;
@@ -270,7 +354,6 @@ extern "C" msa_status msa_pool_blocks(const void* k, const void* v, const void* 
   const int per_sm = 2;
   int64_t grid = (int64_t)msa::sm_count() * per_sm;
   if (grid > n_chunks) grid = n_chunks;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (in_dtype == MSA_F32) {
     MSA_CUDA_TRY(cudaFuncSetAttribute(pool_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     pool_kernel<float><<<(unsigned)grid, threads, smem, s>>>(

@@ -47,6 +47,7 @@ int rescore_count(int32_t n_docs, int32_t k) {
 }
 
 static thread_local int32_t g_launches = 0;
+static thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
 
 struct QueryOffsets {
   int32_t n;
@@ -57,7 +58,7 @@ struct QueryOffsets {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int topk_blocks(int32_t n_docs) {
-  int nb = (n_docs + 2047) / 2048;
+  int nb = (n_docs + 511) / 512;
   if (nb < 1) nb = 1;
   if (nb > kMaxBlocks) nb = kMaxBlocks;
   return nb;
@@ -317,9 +318,16 @@ __global__ void __launch_bounds__(kTopkThreads) docmax_topk_kernel(const float* 
     if (i < n) {
       const int doc = d0 + i;
       const int64_t c0 = __ldg(doc_chunk_off + doc), c1 = __ldg(doc_chunk_off + doc + 1);
-      float s = -INFINITY;
-      for (int64_t c = c0; c < c1; ++c) s = fmaxf(s, __ldg(mb + c));
-      key = make_key(s, doc);
+      float s0 = -INFINITY, s1 = -INFINITY, s2 = -INFINITY, s3 = -INFINITY;
+      int64_t c = c0;
+      for (; c + 4 <= c1; c += 4) {
+        s0 = fmaxf(s0, __ldg(mb + c));
+        s1 = fmaxf(s1, __ldg(mb + c + 1));
+        s2 = fmaxf(s2, __ldg(mb + c + 2));
+        s3 = fmaxf(s3, __ldg(mb + c + 3));
+      }
+      for (; c < c1; ++c) s0 = fmaxf(s0, __ldg(mb + c));
+      key = make_key(fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)), doc);
     }
     tk_smem[i] = key;
   }
@@ -360,10 +368,14 @@ __global__ void __launch_bounds__(kTopkThreads) merge_topk_kernel(const unsigned
 
 // ---------------------------------------------------------------------------- 2c. exact rescoring
 // grid (K2, L, B), 128 threads: exact fp32 score of filter candidate r of (b, l).  The
-// document's exact best (block, token) pair has a filter score within 2 E of the
-// document's filter maximum, and within 2 E of its block's filter maximum; so only
-// blocks with m >= max - 2E are visited, and in those only the argmax token unless the
-// runner-up is also within 2E (then every token of the query).
+// document's exact best (block, token) pair has a filter score within 2E of the
+// document's filter maximum and within 2E of its block's filter maximum, so only blocks
+// with m >= max - 2E are visited: in those, the argmax token alone when the runner-up is
+// more than 2E below, else every token of the query.  Blocks of the second kind are
+// staged (unit rows, fp32) in shared memory kRescoreRows at a time so that each query
+// token row is read once per group.
+constexpr int kRescoreRows = 16;
+
 template <int NV>
 __global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __restrict__ kr_hat,
                                                       const float* __restrict__ qt, int L, int64_t C, int T_total,
@@ -372,7 +384,10 @@ __global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __res
                                                       const unsigned long long* __restrict__ apx, int K2, float err,
                                                       float* __restrict__ exact) {
   constexpr int R = NV * 256;
+  extern __shared__ float4 rows[];  // [kRescoreRows][R / 4] in lane-vector order
   __shared__ float red[4];
+  __shared__ int full_list[kRescoreRows];
+  __shared__ int n_full;
   const int r = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t o = ((int64_t)b * L + l) * K2 + r;
@@ -388,20 +403,67 @@ __global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __res
   const float* qbase = qt + (int64_t)l * T_total * R;
   const float window = 2.0f * err;
   float best = -INFINITY;
-  for (int64_t c = c0 + warp; c < c1; c += 4) {
-    const float m1 = m[mrow + c];
-    if (!(m1 >= doc_apx - window)) continue;
-    const int2 ax = aux[mrow + c];
-    const float m2 = __int_as_float(ax.x);
-    float kx[NV][8];
-    load_unit_row<NV>(kr_hat + ((int64_t)l * C + c) * R, lane, kx);
-    if (m2 < m1 - window) {
-      const int t = qo.off[b] + ax.y;
-      best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
-    } else {
-      for (int t = qo.off[b]; t < qo.off[b + 1]; ++t)
+  // blocks are scanned in windows of 4 * kRescoreRows; each window's full-scan blocks
+  // (at most kRescoreRows per pass) are collected, staged and scanned together
+  for (int64_t w0 = c0; w0 < c1; w0 += kRescoreRows) {
+    if (threadIdx.x == 0) n_full = 0;
+    __syncthreads();
+    for (int64_t c = w0 + warp; c < min(c1, w0 + kRescoreRows); c += 4) {
+      const float m1 = m[mrow + c];
+      if (!(m1 >= doc_apx - window)) continue;
+      const int2 ax = aux[mrow + c];
+      const float m2 = __int_as_float(ax.x);
+      if (m2 < m1 - window) {
+        float kx[NV][8];
+        load_unit_row<NV>(kr_hat + ((int64_t)l * C + c) * R, lane, kx);
+        const int t = qo.off[b] + ax.y;
         best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
+      } else if (lane == 0) {
+        full_list[atomicAdd(&n_full, 1)] = (int)(c - w0);
+      }
     }
+    __syncthreads();
+    const int nf = n_full;
+    if (nf == 0) continue;
+    for (int rr = warp; rr < nf; rr += 4) {
+      float kx[NV][8];
+      load_unit_row<NV>(kr_hat + ((int64_t)l * C + w0 + full_list[rr]) * R, lane, kx);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        rows[rr * (R / 4) + 2 * (lane + 32 * i)] = make_float4(kx[i][0], kx[i][1], kx[i][2], kx[i][3]);
+        rows[rr * (R / 4) + 2 * (lane + 32 * i) + 1] = make_float4(kx[i][4], kx[i][5], kx[i][6], kx[i][7]);
+      }
+    }
+    __syncthreads();
+    for (int t = qo.off[b] + warp; t < qo.off[b + 1]; t += 4) {
+      const float4* qv = reinterpret_cast<const float4*>(qbase + (int64_t)t * R);
+      float q[NV][8];
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const float4 x = __ldg(qv + 2 * (lane + 32 * i));
+        const float4 y = __ldg(qv + 2 * (lane + 32 * i) + 1);
+        q[i][0] = x.x; q[i][1] = x.y; q[i][2] = x.z; q[i][3] = x.w;
+        q[i][4] = y.x; q[i][5] = y.y; q[i][6] = y.z; q[i][7] = y.w;
+      }
+      for (int rr = 0; rr < nf; ++rr) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const float4 x = rows[rr * (R / 4) + 2 * (lane + 32 * i)];
+          const float4 y = rows[rr * (R / 4) + 2 * (lane + 32 * i) + 1];
+          acc = fmaf(q[i][0], x.x, acc);
+          acc = fmaf(q[i][1], x.y, acc);
+          acc = fmaf(q[i][2], x.z, acc);
+          acc = fmaf(q[i][3], x.w, acc);
+          acc = fmaf(q[i][4], y.x, acc);
+          acc = fmaf(q[i][5], y.y, acc);
+          acc = fmaf(q[i][6], y.z, acc);
+          acc = fmaf(q[i][7], y.w, acc);
+        }
+        best = fmaxf(best, warp_sum(acc));
+      }
+    }
+    __syncthreads();
   }
   if (lane == 0) red[warp] = best;
   __syncthreads();
@@ -461,6 +523,12 @@ extern "C" msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_
 }
 
 extern "C" int32_t msa_route_last_launch_count(void) { return g_launches; }
+
+extern "C" msa_status msa_route_set_profile_events(void* start_event, void* stop_event) {
+  g_prof_start = (start_event && stop_event) ? reinterpret_cast<cudaEvent_t>(start_event) : nullptr;
+  g_prof_stop = (start_event && stop_event) ? reinterpret_cast<cudaEvent_t>(stop_event) : nullptr;
+  return msa_ok();
+}
 
 extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
                                      int32_t n_queries, const void* kr_hat, const int64_t* doc_chunk_offsets,
@@ -530,6 +598,7 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
   if (n_chunks > 0) {
+    if (g_prof_start) MSA_CUDA_TRY(cudaEventRecord(g_prof_start, s));
     if (!tensor) {
       int64_t warps = (int64_t)n_layers * n_chunks;
       int64_t blocks = (warps + 7) / 8;
@@ -562,6 +631,7 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
         return msa_fail(MSA_ERR_CUDA, "tensor-core route: %s", why ? why : "launch failed");
       g_launches += launches;
     }
+    if (g_prof_stop) MSA_CUDA_TRY(cudaEventRecord(g_prof_stop, s));
   }
   const int per = (n_docs + w.nblk - 1) / w.nblk;
   const int doc_pow2 = pow2_at_least(per > 0 ? per : 1);
@@ -601,7 +671,9 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
                                                                           nullptr, nullptr);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
-  rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, 0, s>>>(
+  const size_t rs_smem = (size_t)kRescoreRows * H * kD * sizeof(float);
+  MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs_smem));
+  rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, rs_smem, s>>>(
       (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks, T_total, qo, doc_chunk_offsets, m,
       reinterpret_cast<const int2*>(ws + w.aux), apx, K2, kFilterErr, exact);
   ++g_launches;

@@ -339,53 +339,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+        // two 32-column slices per TMEM round trip
 #pragma unroll 1
-        for (int c32 = 0; c32 < BN / 32; ++c32) {
-          const int col0 = nt * BN + c32 * 32;
-          if (col0 >= ql.row0[ql.n_queries]) break;  // trailing padding columns
-          uint32_t r[32];
-          tmem_ld32(tbase + (uint32_t)(c32 * 32), r);
+        for (int c64 = 0; c64 < BN / 64; ++c64) {
+          const int colA = nt * BN + c64 * 64;
+          if (colA >= ql.row0[ql.n_queries]) break;  // trailing padding columns
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tbase + (uint32_t)(c64 * 64), ra);
+          tmem_ld32(tbase + (uint32_t)(c64 * 64 + 32), rb);
           tmem_wait_ld();
-          int lo = 0, hi = ql.n_queries;  // owner: largest b with row0[b] <= col0
-          while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (ql.row0[mid] <= col0) lo = mid; else hi = mid;
-          }
-          const int b = lo;
-          const int t0 = col0 - ql.row0[b];            // token index of column col0 in query b
-          const int valid = min(32, ql.len[b] - t0);
-          float m1 = -INFINITY, m2 = -INFINITY;
-          int i1 = 0;
-          if (b == carry_b) {
-            m1 = c1;
-            m2 = c2;
-            i1 = ci;
-          }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(r[i]);
-            if (i < valid) {
-              if (x > m1) {
-                m2 = m1;
-                m1 = x;
-                i1 = t0 + i;
-              } else {
-                m2 = fmaxf(m2, x);
+          for (int half = 0; half < 2; ++half) {
+            const int col0 = colA + 32 * half;
+            if (col0 >= ql.row0[ql.n_queries]) break;
+            int lo = 0, hi = ql.n_queries;  // owner: largest b with row0[b] <= col0
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (ql.row0[mid] <= col0) lo = mid; else hi = mid;
+            }
+            const int b = lo;
+            const int t0 = col0 - ql.row0[b];  // token index of column col0 in query b
+            const int valid = min(32, ql.len[b] - t0);
+            float m1 = -INFINITY, m2 = -INFINITY;
+            int i1 = 0;
+            if (b == carry_b) {
+              m1 = c1;
+              m2 = c2;
+              i1 = ci;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = i < valid ? __uint_as_float(half ? rb[i] : ra[i]) : -INFINITY;
+              m2 = fmaxf(m2, fminf(m1, x));
+              i1 = x > m1 ? t0 + i : i1;
+              m1 = fmaxf(m1, x);
+            }
+            if (t0 + 32 >= ql.len[b]) {
+              if (row_ok) {
+                const long long o = ((long long)b * L + l) * C + row;
+                m_out[o] = m1;
+                aux_out[o] = make_int2(__float_as_int(m2), i1);
               }
+              carry_b = -1;
+            } else {
+              carry_b = b;
+              c1 = m1;
+              c2 = m2;
+              ci = i1;
             }
-          }
-          if (t0 + 32 >= ql.len[b]) {
-            if (row_ok) {
-              const long long o = ((long long)b * L + l) * C + row;
-              m_out[o] = m1;
-              aux_out[o] = make_int2(__float_as_int(m2), i1);
-            }
-            carry_b = -1;
-          } else {
-            carry_b = b;
-            c1 = m1;
-            c2 = m2;
-            ci = i1;
           }
         }
         tc_fence_before();
