@@ -73,6 +73,11 @@ int32_t msa_route_last_launch_count(void);
  * graph capture).  NULL, NULL turns it off.  Returns MSA_OK. */
 msa_status msa_route_set_profile_events(void* start_event, void* stop_event);
 
+/* Tensor-core path tiling on this thread: 1 (default) runs N tiles of 128 / 256 query
+ * tokens as M=256 tiles on pairs of SMs (tcgen05 cta_group::2, each SM streaming half of
+ * the query tile); 0 keeps one CTA per M=128 tile.  Results are identical.  Returns MSA_OK. */
+msa_status msa_route_set_pair_mode(int32_t enabled);
+
 const char* msa_route_last_error(void);
 
 #ifdef __cplusplus

@@ -208,6 +208,18 @@ def test_route_tensor_long_queries_span_tiles(msa, Ts):
     _route_case(msa, 7, lens, 2, Ts, 64, 2, n_targets=4)
 
 
+@pytest.mark.parametrize("pair", [True, False])
+@pytest.mark.parametrize("Ts", [[256], [100, 156], [129]])
+def test_route_tensor_pair_and_single_cta_tiles(msa, pair, Ts):
+    # N tiles of 128 / 256 run on SM pairs (M = 256) by default; both tilings must match the oracle
+    lens = syn.doc_lengths_lognormal(11, 180)
+    msa.msa_route_set_pair_mode(pair)
+    try:
+        _route_case(msa, 11, lens, 2, Ts, 32, 2, n_targets=4)
+    finally:
+        msa.msa_route_set_pair_mode(True)
+
+
 def test_route_tensor_selection_is_certified_for_planted_needles(msa):
     # k = number of planted documents: the k-th exact score sits far above the filter's
     # margin over the best document left out, so the certification bit stays clear

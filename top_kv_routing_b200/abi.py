@@ -60,6 +60,8 @@ route_lib.msa_route_topk.argtypes = [_p, _i32, _p, _i32, _p, _p, _i32, _i64, _i3
 route_lib.msa_route_topk.restype = _i32
 route_lib.msa_route_last_launch_count.restype = _i32
 route_lib.msa_route_last_error.restype = ctypes.c_char_p
+route_lib.msa_route_set_pair_mode.argtypes = [_i32]
+route_lib.msa_route_set_pair_mode.restype = _i32
 route_lib.msa_route_set_profile_events.argtypes = [_p, _p]
 route_lib.msa_route_set_profile_events.restype = _i32
 
@@ -164,6 +166,11 @@ def msa_route_topk(qr, q_offsets, kr_hat, doc_chunk_offsets, n_docs: int, n_chun
                                   flags, _ptr(dev_err), _stream(stream))
     _check(st, "msa_route_topk", route_lib, "msa_route_last_error")
     return int(route_lib.msa_route_last_launch_count())
+
+
+def msa_route_set_pair_mode(enabled: bool) -> None:
+    """Tensor-core routing on SM pairs (M=256 tiles, the default) or one CTA per tile."""
+    route_lib.msa_route_set_pair_mode(1 if enabled else 0)
 
 
 def msa_route_set_profile_events(start_event=None, stop_event=None):

@@ -48,6 +48,7 @@ int rescore_count(int32_t n_docs, int32_t k) {
 
 static thread_local int32_t g_launches = 0;
 static thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+static thread_local bool g_pair_mode = true;
 
 struct QueryOffsets {
   int32_t n;
@@ -524,6 +525,11 @@ extern "C" msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_
 
 extern "C" int32_t msa_route_last_launch_count(void) { return g_launches; }
 
+extern "C" msa_status msa_route_set_pair_mode(int32_t enabled) {
+  g_pair_mode = enabled != 0;
+  return msa_ok();
+}
+
 extern "C" msa_status msa_route_set_profile_events(void* start_event, void* stop_event) {
   g_prof_start = (start_event && stop_event) ? reinterpret_cast<cudaEvent_t>(start_event) : nullptr;
   g_prof_stop = (start_event && stop_event) ? reinterpret_cast<cudaEvent_t>(stop_event) : nullptr;
@@ -625,6 +631,7 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
       a.m = m;
       a.aux = reinterpret_cast<int2*>(ws + w.aux);
       a.dev_err = dev_err;
+      a.pair = g_pair_mode;
       int launches = 0;
       const char* why = nullptr;
       if (route_tc::launch(a, s, &launches, &why) != 0)

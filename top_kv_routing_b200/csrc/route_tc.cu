@@ -9,12 +9,18 @@
 // pairs that can hold the maximum exactly.
 //
 // Warp roles of the persistent kernel (192 threads, one CTA per SM):
-//   warp 0      TMA producer: A tile [128 blocks x 64] + B tile [BN tokens x 64] per
+//   warp 0      TMA producer: A tile [128 blocks x 64] + B tile [tokens x 64] per
 //               K-block into a ring of shared-memory stages (128-byte swizzle)
-//   warp 1      one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
-//               accumulators and commits stage / accumulator completion to mbarriers
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max over each query's
-//               columns, store; then release the accumulator
+//   warp 1      one thread issues tcgen05.mma (bf16 in, fp32 accumulate, K=16) into one of
+//               two TMEM accumulators and commits stage / accumulator completion to mbarriers
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max / runner-up / argmax over
+//               each query's columns, store; then release the accumulator
+// Paired mode (PAIR, for N tiles of 128 and 256): a cluster of two CTAs on two SMs runs
+// M=256 tiles with tcgen05.mma.cta_group::2.  Each CTA loads its 128 key rows and half of
+// the query tile, so each SM streams half the query bytes per key byte of the single-CTA
+// form.  The leader (rank 0) issues the MMAs; both CTAs' loads complete on the leader's
+// stage barrier; commits are multicast to both CTAs; the peer's epilogue releases the
+// accumulator on the leader's barrier.  No load uses cluster multicast.
 // Every wait is bounded (2 s on the global timer); on a timeout the kernel sets
 // MSA_DEVERR_TIMEOUT, drains its own copies and MMAs (bounded) and frees TMEM.
 #include <cuda.h>
@@ -33,12 +39,14 @@ constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kThreads = 192;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
-template <int BN>
+template <int BN, bool PAIR>
 struct Cfg {
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;  // query rows of the B tile held per CTA
+  static constexpr int kBBytes = kBRows * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kStages = (196 * 1024) / kStage > 8 ? 8 : (196 * 1024) / kStage;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators: 128, 256 or 512 columns
+  static constexpr int kRows = PAIR ? 2 * kBM : kBM;  // key rows per unit (M of the MMA)
   static constexpr int kBarBytes = 256;
   static constexpr int kSmem = kStages * kStage + 1024 + kBarBytes;
 };
@@ -99,6 +107,28 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -121,32 +151,70 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Paired variant: the cta_group::2 form, completing on a barrier that may be in the peer CTA.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+template <bool PAIR>
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_slot), "r"(ncols)
-               : "memory");
+  if (PAIR)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_slot), "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_slot), "r"(ncols)
+                 : "memory");
 }
+template <bool PAIR>
 __device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  if (PAIR) asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  else asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
+template <bool PAIR>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  if (PAIR) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+template <bool PAIR>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if (PAIR)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
+// Arrives (once all earlier MMAs of this thread finish) on the barrier at this shared
+// offset: in this CTA, or in both CTAs of the pair.
+template <bool PAIR>
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+  if (PAIR)
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"((uint16_t)3)
+        : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -181,12 +249,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN>
+template <int BN, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int L,
                     long long C, int n_rows, int m_tiles, const __grid_constant__ QueryLayout ql,
                     float* __restrict__ m_out, int2* __restrict__ aux_out, int32_t* dev_err) {
-  using K = Cfg<BN>;
+  using K = Cfg<BN, PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::kStages * K::kStage);
@@ -201,6 +269,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_tiles = n_rows / BN;
   const int units = L * m_tiles;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int first_unit = PAIR ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
+  const int unit_stride = PAIR ? (int)(gridDim.x / 2) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < K::kStages; ++s) {
@@ -209,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&accf[b]), 1);
-      mbar_init(smem_u32(&acce[b]), 4);
+      mbar_init(smem_u32(&acce[b]), PAIR ? 8 : 4);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -217,17 +289,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), K::kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<PAIR>(smem_u32(tmem_slot), K::kTmemCols);
+    tmem_relinquish<PAIR>();
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync_all();  // barriers of both CTAs initialised before any remote use
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- TMA producer (both CTAs of a pair)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_a)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b)) : "memory");
       const uint64_t pol_a = policy_evict_first(), pol_b = policy_evict_last();
@@ -237,11 +310,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = first_unit; u < units && ok; u += unit_stride) {
         const int l = u / m_tiles, mt = u % m_tiles;
-        const int row_a = (int)((long long)l * C) + mt * kBM;
+        const int row_a = (int)((long long)l * C) + mt * K::kRows + (int)rank * kBM;
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
-          const int row_b = l * n_rows + nt * BN;
+          const int row_b = l * n_rows + nt * BN + (int)rank * K::kBRows;
           for (int kb = 0; kb < kKBlocks; ++kb) {
             if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
               ok = false;
@@ -249,9 +322,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const uint32_t fb = smem_u32(&full[stage]);
             const uint32_t sa = smem_u32(smem + stage * K::kStage);
-            mbar_arrive_expect_tx(fb, K::kStage);
-            tma_load_2d(sa, &tm_a, fb, kb * kBK, row_a, pol_a);
-            tma_load_2d(sa + kABytes, &tm_b, fb, kb * kBK, row_b, pol_b);
+            if (PAIR) {
+              const uint32_t fb_lead = map_to_rank(fb, 0);  // both CTAs' bytes land on the leader's barrier
+              if (leader) mbar_arrive_expect_tx(fb, 2 * K::kStage);
+              tma_load_2d_pair(sa, &tm_a, fb_lead, kb * kBK, row_a, pol_a);
+              tma_load_2d_pair(sa + kABytes, &tm_b, fb_lead, kb * kBK, row_b, pol_b);
+            } else {
+              mbar_arrive_expect_tx(fb, K::kStage);
+              tma_load_2d(sa, &tm_a, fb, kb * kBK, row_a, pol_a);
+              tma_load_2d(sa + kABytes, &tm_b, fb, kb * kBK, row_b, pol_b);
+            }
             armed[stage] = (int)phase;
             if (++stage == K::kStages) {
               stage = 0;
@@ -263,19 +343,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
-        // let every copy this thread issued land before the CTA can exit
-        for (int s = 0; s < K::kStages; ++s)
-          if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
+        // let the copies this CTA issued land (the leader's barriers see both CTAs' bytes)
+        if (leader)
+          for (int s = 0; s < K::kStages; ++s)
+            if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      constexpr uint32_t idesc = idesc_bf16(kBM, BN);
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the leader of a pair issues for both CTAs)
+      constexpr uint32_t idesc = idesc_bf16(K::kRows, BN);
       int stage = 0, buf = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = first_unit; u < units && ok; u += unit_stride) {
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
           if (!mbar_wait(smem_u32(&acce[buf]), acc_phase ^ 1u, abort_flag)) {
             ok = false;
@@ -293,16 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t da = sw128_desc(sa), db = sw128_desc(sa + kABytes);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k)
-              umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc, (kb | k) != 0 ? 1u : 0u);
+              umma_bf16<PAIR>(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
+                              (kb | k) != 0 ? 1u : 0u);
             issued = true;
-            umma_commit(smem_u32(&empty[stage]));
+            umma_commit<PAIR>(smem_u32(&empty[stage]));
             if (++stage == K::kStages) {
               stage = 0;
               phase ^= 1u;
             }
           }
           if (!ok) break;
-          umma_commit(smem_u32(&accf[buf]));
+          umma_commit<PAIR>(smem_u32(&accf[buf]));
           if (++buf == 2) {
             buf = 0;
             acc_phase ^= 1u;
@@ -313,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
         if (issued) {
-          umma_commit(smem_u32(drain));  // arrives once every MMA issued so far has finished
+          umma_commit<PAIR>(smem_u32(drain));  // arrives once every MMA issued so far has finished
           mbar_drain(smem_u32(drain), 0u);
         }
       }
@@ -322,12 +404,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue (warps 2..5 -> TMEM lane quarters 2, 3, 0, 1)
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
+    const uint32_t acce_lead0 = PAIR ? map_to_rank(smem_u32(&acce[0]), 0) : smem_u32(&acce[0]);
     int buf = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = first_unit; u < units && ok; u += unit_stride) {
       const int l = u / m_tiles, mt = u % m_tiles;
-      const long long row = (long long)mt * kBM + row_in_tile;
+      const long long row = (long long)mt * K::kRows + (long long)rank * kBM + row_in_tile;
       const bool row_ok = row < C;
       int carry_b = -1;           // query whose columns continue into the next N tile
       float c1 = -INFINITY, c2 = -INFINITY;
@@ -391,7 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&acce[buf]));
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_cluster(acce_lead0 + (uint32_t)(buf * 8));
+          else mbar_arrive(smem_u32(&acce[buf]));
+        }
         if (++buf == 2) {
           buf = 0;
           acc_phase ^= 1u;
@@ -404,10 +490,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  __syncthreads();
+  tc_fence_before();
+  if (PAIR) cluster_sync_all();  // no CTA exits while its peer may still signal its barriers
+  else __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, K::kTmemCols);
+    tmem_dealloc<PAIR>(tmem_base, K::kTmemCols);
   }
 }
 
@@ -441,27 +529,39 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
-  using K = Cfg<BN>;
+  using K = Cfg<BN, PAIR>;
   CUtensorMap ma, mb;
   const uint64_t rows_a = (uint64_t)a.L * (uint64_t)a.C;
-  if (!make_map(&ma, a.kr_hat, rows_a, kBM) || !make_map(&mb, a.qt, (uint64_t)a.L * a.n_rows, BN)) {
+  if (!make_map(&ma, a.kr_hat, rows_a, kBM) || !make_map(&mb, a.qt, (uint64_t)a.L * a.n_rows, K::kBRows)) {
     *why = "cuTensorMapEncodeTiled failed";
     return 1;
   }
-  const int m_tiles = (int)((a.C + kBM - 1) / kBM);
+  const int m_tiles = (int)((a.C + K::kRows - 1) / K::kRows);
   const long long units = (long long)a.L * m_tiles;
-  int grid = msa::sm_count();
-  if (units < grid) grid = (int)units;
-  if (cudaFuncSetAttribute(route_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) !=
+  const int per_unit = PAIR ? 2 : 1;
+  int grid = msa::sm_count() / per_unit * per_unit;
+  if (units * per_unit < grid) grid = (int)(units * per_unit);
+  if (cudaFuncSetAttribute(route_tc_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) !=
       cudaSuccess) {
     *why = "cudaFuncSetAttribute (shared memory)";
     return 1;
   }
-  route_tc_kernel<BN><<<grid, kThreads, K::kSmem, s>>>(ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
-                                                       a.aux, a.dev_err);
-  if (cudaGetLastError() != cudaSuccess) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = K::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = per_unit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
+                         a.aux, a.dev_err) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
   }
@@ -484,9 +584,11 @@ int launch(const LaunchArgs& a, cudaStream_t s, int* launches, const char** why)
     return 1;
   }
   int r;
-  if (bn == 64) r = launch_bn<64>(a, s, why);
-  else if (bn == 128) r = launch_bn<128>(a, s, why);
-  else r = launch_bn<256>(a, s, why);
+  if (bn == 64) r = launch_bn<64, false>(a, s, why);
+  else if (a.pair && bn == 128) r = launch_bn<128, true>(a, s, why);
+  else if (bn == 128) r = launch_bn<128, false>(a, s, why);
+  else if (a.pair) r = launch_bn<256, true>(a, s, why);
+  else r = launch_bn<256, false>(a, s, why);
   if (r == 0) *launches = 1;
   return r;
 }

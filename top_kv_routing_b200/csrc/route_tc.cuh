@@ -54,6 +54,7 @@ struct LaunchArgs {
   float* m;            // [B][L][C]  approximate max over the query's tokens
   int2* aux;           // [B][L][C]  (bits of the second-largest score, argmax token in the query)
   int32_t* dev_err;
+  bool pair;           // M=256 tiles on CTA pairs (cta_group::2) for N tiles of 128 / 256
 };
 
 // Enqueues the score kernel; returns 0 on success (launches += kernels enqueued).
