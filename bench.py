@@ -31,6 +31,7 @@ WORKLOAD = ("100M-token bank (100,000 docs, lognormal lengths rounded to 64, 1,5
             "query T=256 tokens with 16 planted target documents, top-16 per layer; gather of the "
             "selected blocks' K/V from a page-locked host store; 128-token GQA 32/8 decode, local KV 256")
 N_DOCS, N_TOKENS, L, H, HQ, D, TOPK, T, DEC, SEED = 100_000, 100_000_000, 18, 8, 32, 128, 16, 256, 128, 3
+TOKENS_PER_DOC = 1000
 THETA = 1e6
 
 
@@ -110,6 +111,12 @@ def smi_id(dev) -> str:
 
 
 # ----------------------------------------------------------------------------- workload
+
+def set_bank_size(n_docs: int) -> None:
+    """Scales the bank (documents x 1000 tokens); the default is the 100M-token bank."""
+    global N_DOCS, N_TOKENS
+    N_DOCS, N_TOKENS = n_docs, n_docs * TOKENS_PER_DOC
+
 
 def make_workload(dev, host_store_chunks: int):
     import torch
@@ -244,103 +251,115 @@ def run_gpu(args):
     bank, kr_hat, host_kv, store_off, topic = make_workload(dev, args.host_store_blocks)
     qs, targets = make_queries(dev, bank, topic, args.queries)
     dq, dk, dv, pk, pv = make_decode_inputs(dev)
-    out = torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16, device=dev)
+    n_slots = args.pipeline
+    dec_inputs = [(dq.clone(), dk.clone(), dv.clone(), torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16,
+                                                                   device=dev)) for _ in range(n_slots)]
     eng = SparseMemory(kr_hat, bank.doc_chunk_offsets, host_kv, store_off, n_q_heads=HQ, top_k=TOPK,
-                       query_tokens=T, local_cap=T + DEC, rope_theta=THETA)
+                       query_tokens=T, local_cap=T + DEC, rope_theta=THETA, slots=n_slots)
     eng.set_local_prefix(pk, pv)
-    ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev_a.record()
-    ev_b.record()
-    torch.cuda.synchronize(dev)
-    msa.msa_route_set_profile_events(ev_a, ev_b)
-    eng.qr.copy_(qs[0])
-    graph = eng.capture(dq, dk, dv, out)
-    msa.msa_route_set_profile_events(None, None)
+    for s_ in eng.slots:
+        s_.qr.copy_(qs[0])
+    eng.capture(dec_inputs)
     launches = eng.launches_per_query
+    slot0 = eng.slots[0]
 
     def score_kernel_ms(reps=5):
-        # the score kernel's own device time: the events recorded around it inside the
-        # graph, else the same call outside a graph with the events set
+        # the score kernel's own device time: CUDA events the route library records right
+        # before and after it, on the route stream, for direct (non-graph) calls of the same
+        # route on the same buffers
+        ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_a.record()
+        ev_b.record()
+        torch.cuda.synchronize(dev)
+        msa.msa_route_set_profile_events(ev_a, ev_b)
         vals = []
         try:
             for i in range(reps):
-                eng.qr.copy_(qs[i % len(qs)])
-                graph.replay()
+                slot0.qr.copy_(qs[i % len(qs)])
+                torch.cuda.synchronize(dev)
+                with torch.cuda.stream(eng.route_stream):
+                    eng.enqueue_route(slot0, eng.route_stream)
                 torch.cuda.synchronize(dev)
                 vals.append(ev_a.elapsed_time(ev_b))
-        except RuntimeError:
-            vals = []
-            msa.msa_route_set_profile_events(ev_a, ev_b)
-            for i in range(reps):
-                eng.qr.copy_(qs[i % len(qs)])
-                msa.msa_route_topk(eng.qr, [0, T], eng.kr_hat, eng.doc_chunk_offsets, eng.n_docs, eng.C, L, HQ, H,
-                                   D, TOPK, eng.ids, eng.scores, eng.ws)
-                torch.cuda.synchronize(dev)
-                vals.append(ev_a.elapsed_time(ev_b))
+        finally:
             msa.msa_route_set_profile_events(None, None)
         return float(np.mean(vals))
 
-    def step(i, host=None):
-        if host is None:
-            eng.qr.copy_(qs[i % len(qs)])
-        else:
-            eng.qr.copy_(host["qr"][i % len(qs)], non_blocking=True)
-            dq.copy_(host["dq"], non_blocking=True)
-            dk.copy_(host["dk"], non_blocking=True)
-            dv.copy_(host["dv"], non_blocking=True)
-        graph.replay()
-        if host is not None:
-            host["ids"].copy_(eng.ids, non_blocking=True)
-            host["scores"].copy_(eng.scores, non_blocking=True)
-            host["out"].copy_(out, non_blocking=True)
+    def run(n, host=None, times=None):
+        """n queries through the two-slot pipeline; times: per-query (start, end) events."""
+        for i in range(n):
+            def load(slot, st, i=i):
+                if host is None:
+                    slot.qr.copy_(qs[i % len(qs)])
+                else:
+                    slot.qr.copy_(host["qr"][i % len(qs)], non_blocking=True)
+                    k = eng.slots.index(slot)
+                    for src, dst in zip((host["dq"], host["dk"], host["dv"]), dec_inputs[k][:3]):
+                        dst.copy_(src, non_blocking=True)
+                if times is not None:
+                    times[i][0].record(st)
+
+            def unload(slot, st, i=i):
+                if host is not None:
+                    k = eng.slots.index(slot)
+                    host["ids"][k].copy_(slot.ids, non_blocking=True)
+                    host["scores"][k].copy_(slot.scores, non_blocking=True)
+                    host["out"][k].copy_(dec_inputs[k][3], non_blocking=True)
+                if times is not None:
+                    times[i][1].record(st)
+            eng.launch(i, load, unload)
+        eng.drain()
 
     # correctness guard on the benchmark's own output: planted documents are selected
-    eng.dev_err.zero_()
-    step(0)
+    slot0.dev_err.zero_()
+    run(1)
     torch.cuda.synchronize(dev)
-    got = eng.ids.cpu().numpy()[0]
+    got = slot0.ids.cpu().numpy()[0]
     hits = np.mean([len(set(got[l].tolist()) & set(targets[0].tolist())) / TOPK for l in range(L)])
-    dev_err = int(eng.dev_err.item())
+    dev_err = int(slot0.dev_err.item())
 
-    for i in range(args.warmup):
-        step(i)
+    # isolated latency of one query (route + gather + decode, nothing overlapping)
+    iso = []
+    for i in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        tm = [(e0, e1)]
+        run(1, times=tm)
+        torch.cuda.synchronize(dev)
+        iso.append(e0.elapsed_time(e1))
+
+    run(args.warmup)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    times = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     with ClockSampler(smi_id(dev)) as clk:
-        starts[0].record()
-        for i in range(args.steps):
-            step(i)
-            starts[i + 1].record()
+        run(args.steps, times=times)
         torch.cuda.synchronize(dev)
-    per_step = [starts[i].elapsed_time(starts[i + 1]) for i in range(args.steps)]
-    total_ms = starts[0].elapsed_time(starts[-1])
+    per_query = [a.elapsed_time(b) for a, b in times]
+    total_ms = times[0][0].elapsed_time(times[-1][1])
     gemm_avg = score_kernel_ms()
 
-    # end to end: pinned host inputs in, results out, every step
+    # end to end: pinned host inputs in, results out, every query
     host = {"qr": [q.cpu().pin_memory() for q in qs], "dq": dq.cpu().pin_memory(), "dk": dk.cpu().pin_memory(),
-            "dv": dv.cpu().pin_memory(), "ids": torch.empty((1, L, TOPK), dtype=torch.int32).pin_memory(),
-            "scores": torch.empty((1, L, TOPK), dtype=torch.float32).pin_memory(),
-            "out": torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16).pin_memory()}
-    for i in range(2):
-        step(i, host)
+            "dv": dv.cpu().pin_memory(),
+            "ids": [torch.empty((1, L, TOPK), dtype=torch.int32).pin_memory() for _ in range(n_slots)],
+            "scores": [torch.empty((1, L, TOPK), dtype=torch.float32).pin_memory() for _ in range(n_slots)],
+            "out": [torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16).pin_memory() for _ in range(n_slots)]}
+    run(2, host)
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        step(i, host)
-    e1.record()
+    etimes = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    run(args.steps, host, times=etimes)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = etimes[0][0].elapsed_time(etimes[-1][1])
     h2d = host["qr"][0].numel() * 2 + (dq.numel() + dk.numel() + dv.numel()) * 2
-    d2h = host["ids"].numel() * 4 + host["scores"].numel() * 4 + host["out"].numel() * 2
+    d2h = host["ids"][0].numel() * 4 + host["scores"][0].numel() * 4 + host["out"][0].numel() * 2
 
     if world > 1:
         t = torch.tensor([total_ms, e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms, e2e_ms = float(t[0]), float(t[1])
-    pool = time_pool(dev) if rank == 0 else None
+    pool = time_pool(dev) if (rank == 0 and not args.no_pool) else None
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -353,7 +372,8 @@ def run_gpu(args):
     algo_bytes = L * bank.n_chunks * H * D * 2
     achieved = algo_bytes / (gemm_avg / 1e3) / 1e9
     flops = 2.0 * T * H * D * L * bank.n_chunks
-    p = sorted(per_step)
+    p = sorted(per_query)
+    iso_s = sorted(iso)
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -367,15 +387,19 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_docs": N_DOCS, "n_tokens": N_TOKENS, "n_blocks": bank.n_chunks,
+        "config": {"workload": WORKLOAD if N_DOCS == 100_000 else f"{N_TOKENS:,}-token bank (profiling size)",
+                   "n_docs": N_DOCS, "n_tokens": N_TOKENS, "n_blocks": bank.n_chunks,
                    "layers": L, "kv_heads": H, "q_heads": HQ, "head_dim": D, "query_tokens": T, "top_k": TOPK,
                    "decode_tokens": DEC, "distinct_queries": len(qs), "host_store_blocks": int(host_kv.shape[1]),
                    "l2": "inputs larger than L2 (57.6 GB of routing keys stream through every step)",
-                   "graph": "one CUDA graph per query (route, gather on a side stream, 128 decode steps)",
+                   "graph": "per query two CUDA graphs: route; gather + 128 decode steps",
+                   "pipeline": (f"{n_slots} query slots: the gather+decode of query i overlaps the route of "
+                                "query i+1" if n_slots > 1 else "one query at a time"),
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "scan_gbs": round(achieved, 1),
         "p50_route_decode_ms": round(p[len(p) // 2], 4),
         "p99_route_decode_ms": round(p[min(len(p) - 1, int(0.99 * len(p)))], 4),
+        "p50_isolated_ms": round(iso_s[len(iso_s) // 2], 4),
         "roofline": {"bound": "hbm", "kernel": "route score GEMM (tcgen05)", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "peak_source": peak_src, "traffic": None,
@@ -466,7 +490,13 @@ def main():
                     help="physical blocks per layer in the page-locked content store")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-pool", action="store_true", help="skip the separate pooling measurement")
+    ap.add_argument("--pipeline", type=int, default=1, choices=[1, 2],
+                    help="queries in flight (2 overlaps a query's gather+decode with the next route)")
+    ap.add_argument("--docs", type=int, default=N_DOCS,
+                    help="documents in the bank (x1000 tokens); smaller banks serve profiling captures")
     args = ap.parse_args()
+    set_bank_size(args.docs)
     if args.impl == "reference":
         run_reference(args)
     else:
