@@ -57,6 +57,25 @@ msa_status msa_sparse_decode(const void* q, const void* k_new, const void* v_new
                              int32_t rope_pos_offset, float rope_theta, float softmax_scale, void* out,
                              void* workspace, size_t workspace_bytes, int32_t* dev_err, msa_stream_t stream);
 
+/* msa_sparse_decode without a caller workspace.  There is no counterpart in the MSA
+ * pages: this exists for callers that cannot allocate device memory at all (for example
+ * a host that hands the library only the buffers it already owns, or code running where
+ * allocation is forbidden mid-stream).  The scratch is a fixed array inside this library,
+ * MSA_DECODE_STATIC_SCRATCH_BYTES in size, which every GPU that loads the library keeps
+ * until the process exits; sizes that need more fail with MSA_ERR_CAPACITY.  The first
+ * call on a device looks the array's device address up (issue that first call before any
+ * stream capture).  Each call clears the part that must start at zero with one
+ * cudaMemsetAsync on `stream` and allocates nothing.  All calls share the one array:
+ * calls that overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.  Same arguments, results and errors as msa_sparse_decode. */
+#define MSA_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+msa_status msa_sparse_decode_static(const void* q, const void* k_new, const void* v_new, int32_t n_queries,
+                                    int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                    void* local_k, void* local_v, int32_t* local_len, int32_t local_cap,
+                                    const void* mem_kv, const int32_t* mem_len, int32_t max_mem_chunks,
+                                    int32_t rope_pos_offset, float rope_theta, float softmax_scale, void* out,
+                                    int32_t* dev_err, msa_stream_t stream);
+
 const char* msa_decode_last_error(void);
 
 #ifdef __cplusplus

@@ -76,6 +76,10 @@ decode_lib.msa_sparse_decode_workspace_size.argtypes = [_i32, _i32, _i32, _i32, 
 decode_lib.msa_sparse_decode_workspace_size.restype = _i32
 decode_lib.msa_sparse_decode.restype = _i32
 decode_lib.msa_decode_last_error.restype = ctypes.c_char_p
+decode_lib.msa_sparse_decode_static.argtypes = [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _i32, _p, _p,
+                                                _i32, _i32, _f32, _f32, _p, _p, _p]
+decode_lib.msa_sparse_decode_static.restype = _i32
+MSA_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
 # Kernel launches enqueued by each entry point (the route count is read back per call).
 LAUNCHES_POOL = 1
@@ -212,3 +216,17 @@ def msa_sparse_decode(q, k_new, v_new, n_queries: int, n_layers: int, n_q_heads:
                                       rope_theta, softmax_scale, _ptr(out), _ptr(workspace), ws_bytes, _ptr(dev_err),
                                       _stream(stream))
     _check(st, "msa_sparse_decode", decode_lib, "msa_decode_last_error")
+
+
+def msa_sparse_decode_static(q, k_new, v_new, n_queries: int, n_layers: int, n_q_heads: int, n_kv_heads: int,
+                             head_dim: int, local_k, local_v, local_len, local_cap: int, mem_kv, mem_len,
+                             max_mem_chunks: int, rope_pos_offset: int, rope_theta: float, softmax_scale: float,
+                             out, dev_err=None, stream=None):
+    """msa_sparse_decode with the library's built-in scratch instead of a caller workspace,
+    for callers that cannot allocate device memory (see include/msa_decode.h)."""
+    st = decode_lib.msa_sparse_decode_static(_ptr(q), _ptr(k_new), _ptr(v_new), n_queries, n_layers, n_q_heads,
+                                             n_kv_heads, head_dim, _ptr(local_k), _ptr(local_v), _ptr(local_len),
+                                             local_cap, _ptr(mem_kv), _ptr(mem_len), max_mem_chunks,
+                                             rope_pos_offset, rope_theta, softmax_scale, _ptr(out), _ptr(dev_err),
+                                             _stream(stream))
+    _check(st, "msa_sparse_decode_static", decode_lib, "msa_decode_last_error")

@@ -17,6 +17,8 @@
 #include "common.cuh"
 #include "msa_decode.h"
 
+#include <mutex>
+
 MSA_DEFINE_LAST_ERROR(msa_decode_last_error)
 
 namespace {
@@ -370,4 +372,53 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
 #undef MSA_DECODE_LAUNCH
   MSA_CUDA_TRY(cudaGetLastError());
   return msa_ok();
+}
+
+// ---------------------------------------------------------------------------- no-allocation entry
+// Decode scratch that lives in the library itself, for callers that cannot allocate
+// device memory.  Every GPU that loads this library holds these bytes until the process
+// exits.  The host-side symbol is only a stand-in for the device address, so the address
+// is looked up once per device (cudaGetSymbolAddress, that device current) and passed to
+// the kernel.
+static __device__ __align__(256) unsigned char g_decode_scratch[MSA_DECODE_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[64];  // per device ordinal; nullptr until looked up
+}  // namespace
+
+extern "C" msa_status msa_sparse_decode_static(const void* q, const void* k_new, const void* v_new,
+                                               int32_t n_queries, int32_t n_layers, int32_t n_q_heads,
+                                               int32_t n_kv_heads, int32_t head_dim, void* local_k, void* local_v,
+                                               int32_t* local_len, int32_t local_cap, const void* mem_kv,
+                                               const int32_t* mem_len, int32_t max_mem_chunks,
+                                               int32_t rope_pos_offset, float rope_theta, float softmax_scale,
+                                               void* out, int32_t* dev_err, msa_stream_t stream) {
+  if (n_queries < 1 || n_layers < 1 || n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads != 0)
+    return msa_fail(MSA_ERR_INVALID_ARG, "bad sizes");
+  const size_t need = ws_bytes(n_queries, n_layers, n_q_heads, n_kv_heads);
+  if (need > MSA_DECODE_STATIC_SCRATCH_BYTES)
+    return msa_fail(MSA_ERR_CAPACITY, "static decode scratch holds %u bytes, these sizes need %zu",
+                    MSA_DECODE_STATIC_SCRATCH_BYTES, need);
+  int dev = 0;
+  MSA_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return msa_fail(MSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+      void* p = nullptr;
+      MSA_CUDA_TRY(cudaGetSymbolAddress(&p, g_decode_scratch));
+      g_scratch_addr[dev] = p;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  // the arrival counters must start at zero: their place depends on the sizes, and the
+  // array keeps whatever the previous call left there
+  const size_t counters_at = ws_floats(n_queries, n_layers, n_q_heads, n_kv_heads) * sizeof(float);
+  MSA_CUDA_TRY(cudaMemsetAsync(static_cast<unsigned char*>(scratch) + counters_at, 0, need - counters_at,
+                               reinterpret_cast<cudaStream_t>(stream)));
+  return msa_sparse_decode(q, k_new, v_new, n_queries, n_layers, n_q_heads, n_kv_heads, head_dim, local_k, local_v,
+                           local_len, local_cap, mem_kv, mem_len, max_mem_chunks, rope_pos_offset, rope_theta,
+                           softmax_scale, out, scratch, MSA_DECODE_STATIC_SCRATCH_BYTES, dev_err, stream);
 }
