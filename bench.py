@@ -33,6 +33,9 @@ WORKLOAD = ("100M-token bank (100,000 docs, lognormal lengths rounded to 64, 1,5
 N_DOCS, N_TOKENS, L, H, HQ, D, TOPK, T, DEC, SEED = 100_000, 100_000_000, 18, 8, 32, 128, 16, 256, 128, 3
 TOKENS_PER_DOC = 1000
 THETA = 1e6
+# DRAM bytes per (block, layer) of the routing GEMM, read + write, from the ncu capture in
+# profiles/route_tc_kernel_2M_T256.md (2M-token bank, same kernel), scaled by blocks.
+GEMM_TRAFFIC_PER_BLOCK_LAYER = 2074.5
 
 
 def log(*a):
@@ -402,7 +405,9 @@ def run_gpu(args):
         "p50_isolated_ms": round(iso_s[len(iso_s) // 2], 4),
         "roofline": {"bound": "hbm", "kernel": "route score GEMM (tcgen05)", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "peak_source": peak_src, "traffic": None,
+                     "peak_source": peak_src,
+                     "traffic": round(GEMM_TRAFFIC_PER_BLOCK_LAYER * L * bank.n_chunks),
+                     "traffic_source": "ncu dram bytes of a 2M-token launch scaled by blocks",
                      "algorithmic_bytes": algo_bytes, "kernel_ms": round(gemm_avg, 4),
                      "tflops": round(flops / (gemm_avg / 1e3) / 1e12, 1),
                      "tensor_frac": round(flops / (gemm_avg / 1e3) / 1e12 / bf16_peak, 4),
