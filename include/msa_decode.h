@@ -17,7 +17,8 @@
 extern "C" {
 #endif
 
-/* Workspace bytes of one msa_sparse_decode call (partial softmax sums of the key splits). */
+/* Workspace bytes of one msa_sparse_decode call (partial softmax sums of up to 4 key
+ * splits per (query, layer, key head), and the arrival counters). */
 msa_status msa_sparse_decode_workspace_size(int32_t n_queries, int32_t n_layers, int32_t n_q_heads,
                                             int32_t n_kv_heads, size_t* bytes);
 
@@ -43,9 +44,11 @@ msa_status msa_sparse_decode_workspace_size(int32_t n_queries, int32_t n_layers,
  *              (e.g. cudaMemset) once before its first use; every call leaves it ready for
  *              the next (its arrival counters return to zero).  Calls that share a
  *              workspace must not overlap on the device.
- * The keys of each (query, layer, key head) are split over several CTAs (flash-decoding);
- * the last CTA of each to finish merges the partial softmax sums, and the last merge of
- * a query advances its local_len.
+ * One CTA per (query, layer, key head) streams its keys in tiles of 16 through the tensor
+ * cores; when there are fewer such units than SMs, the keys of each are split over up to
+ * 4 CTAs and the last of them to finish merges the partial softmax sums.  Every CTA of
+ * a query announces on an arrival counter that it has read local_len; the last one
+ * advances it.
  * A query whose cache is full (local_len >= local_cap) is skipped (out untouched, length
  * not advanced) and sets MSA_DEVERR_LOCAL_FULL; mem_len > max_mem_chunks is clamped with
  * MSA_DEVERR_CAPACITY.  One kernel launch, asynchronous on stream, graph-capturable

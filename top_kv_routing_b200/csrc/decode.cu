@@ -4,19 +4,29 @@
 // selected compressed K/V with the local K/V; 全局 RoPE offset by k) and the MSA paper
 // reading notes, section 推理全流程 (memory KV fixed, local KV grows per token).
 //
-// Flash-decoding in one launch: the keys of every (query b, layer l, key head h) are cut
-// into kSplits contiguous ranges, one 128-thread CTA each: one key per thread for the
-// scores of the CTA's G query heads, a local softmax, and P.V with each warp taking 32
-// keys and each lane 4 dims (coalesced 8-byte rows).  Each CTA publishes its
-// unnormalised partial output with its running max and sum; the last CTA of a (b, l, h)
-// to finish (a self-resetting arrival counter) merges the splits and writes the output,
-// and the last merging CTA of query b advances local_len[b].  Only the CTA whose range
-// holds the new key appends it (rotated) to the cache, and it uses its own copy of it.
-// RoPE angles: p * w_j with w_j / pi precomputed in fp64 on the host; the product is
-// reduced modulo 2 pi in fp64 and evaluated by fp32 sincospif.
+// One 256-thread CTA per (query b, layer l, key head h) and key split (several splits
+// only when there are fewer (b, l, h) units than SMs).  The keys are cut into tiles of
+// 16 (memory rows, then local rows); warp w of the CTA takes tiles w, w + 8, ... and
+// streams each through its own 3-stage cp.async ring in shared memory (16 K rows and
+// 16 V rows, 16-byte chunks XOR-swizzled by row so ldmatrix reads are conflict-free).
+// Per tile, on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//   S = Q K^T   with the G query heads of h as A rows: row g carries bf16(q'_g) and row
+//               g + 8 the bf16 residual q'_g - bf16(q'_g), so S_g = row g + row g + 8 keeps
+//               about 16 mantissa bits of the rotated query (K is exact bf16);
+//   O += P V    with P split the same way (row g = bf16(p), row g + 8 = residual), the S
+//               accumulators being reused as the A fragments and V read by ldmatrix.trans.
+// Online softmax per warp in the log2 domain (softmax_scale * log2 e folded into q'),
+// then the 8 warps' (max, sum, O) are merged in shared memory.  With one split the CTA
+// writes the output; with several, each publishes its partial and the last CTA of the
+// (b, l, h) to arrive (a self-resetting counter) merges them.  The last CTA of query b
+// advances local_len[b].  Split 0 appends the rotated new key (rounded to the cache's
+// bf16) and the new value to the cache and folds that key into the state of its last
+// warp directly, in fp32.  RoPE angles: p * w_j with w_j / pi precomputed in fp64 on the
+// host; the product is reduced modulo 2 pi in fp64 and evaluated by fp32 sincospif.
 #include "common.cuh"
 #include "msa_decode.h"
 
+#include <algorithm>
 #include <mutex>
 
 MSA_DEFINE_LAST_ERROR(msa_decode_last_error)
@@ -25,19 +35,26 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kHalf = 64;
-constexpr int kThreads = 128;
-constexpr int kTile = kThreads;
-constexpr int kWarps = kThreads / 32;
-constexpr int kSplits = 5;  // 5 x 8 heads x 18 layers fits one wave of 5 CTAs per SM
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTileKeys = 16;
+constexpr int kStages = 3;
+constexpr int kRowBytes = kD * 2;                        // one bf16 key or value row
+constexpr int kStageBytes = 2 * kTileKeys * kRowBytes;   // 16 K rows then 16 V rows
+constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+constexpr int kMaxSplits = 4;
+constexpr int kRedStride = kD + 4;                       // merge rows, padded against bank conflicts
+constexpr float kLog2e = 1.4426950408889634f;
+static_assert(kWarps * 8 * kRedStride * 4 <= kRingBytes, "merge buffer reuses the ring");
 
 struct RopeTable {
   double w_over_pi[kHalf];  // theta^(-2j/d) / pi
 };
 
-// Workspace: per (b, l, h, split) the partial output [G][128] and (max, sum) per head,
+// Workspace: per (b, l, h, split slot) the partial output [G][128] and (max, sum) per head,
 // then one arrival counter per (b, l, h) and one per query b.
 size_t ws_floats(int B, int L, int Hq, int H) {
-  const size_t units = (size_t)B * L * H * kSplits;
+  const size_t units = (size_t)B * L * H * kMaxSplits;
   const int G = Hq / H;
   return units * (size_t)G * (kD + 2);
 }
@@ -45,30 +62,82 @@ size_t ws_bytes(int B, int L, int Hq, int H) {
   return ws_floats(B, L, Hq, H) * sizeof(float) + ((size_t)B * L * H + (size_t)B) * sizeof(int);
 }
 
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global -> shared copy; bytes = 0 fills the destination with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D += A B, A 16x16 (row-major fragments a[4]), B 16x8 (b0, b1), fp32 accumulators d[4].
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Adds 1 with release semantics at GPU scope (orders this CTA's earlier reads, made
+// before the preceding barrier, before the arrival) and returns the previous count.
+__device__ __forceinline__ int arrive_release(int* counter) {
+  int old;
+  asm volatile("atom.release.gpu.global.add.s32 %0, [%1], 1;\n" : "=r"(old) : "l"(counter) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+
+// x0, x1 -> (bf16 pair of x, bf16 pair of the residuals)
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+  hi = pack_bf16(h0, h1);
+  lo = pack_bf16(__float2bfloat16_rn(x0 - __bfloat162float(h0)), __float2bfloat16_rn(x1 - __bfloat162float(h1)));
+}
+
 template <int G>
-__global__ void __launch_bounds__(kThreads, 5) decode_split_kernel(
+__global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
     const __nv_bfloat16* __restrict__ v_new, int L, int H,
-    // the CTA that appends the new row never reads it back from memory
+    // rows [0, len) are read; row len is written by split 0 only and read by nobody here
     __nv_bfloat16* local_k, __nv_bfloat16* local_v, int32_t* local_len, int cap,
     const __nv_bfloat16* __restrict__ mem_kv, const int32_t* __restrict__ mem_len, int M_max, int pos_off,
-    const __grid_constant__ RopeTable rope, float scale, float* part, float2* stat, int* unit_count,
+    const __grid_constant__ RopeTable rope, float qscale, int splits, float* part, float2* stat, int* unit_count,
     int* query_count, __nv_bfloat16* __restrict__ out, int32_t* dev_err) {
-  __shared__ __align__(16) float qs[G][kD];
+  extern __shared__ __align__(128) unsigned char ring[];
+  __shared__ __align__(16) float qs[8][kD];
   __shared__ __align__(16) float knew[kD];
   __shared__ __align__(16) float vnew[kD];
-  __shared__ float lg[G][kTile];
   __shared__ float2 cs[kHalf];
-  __shared__ float s_max[G], s_sum[G], s_fac[G];
-  __shared__ __align__(16) float red[kWarps][G][kD];
+  __shared__ float2 wml[kWarps][8];
+  __shared__ int s_last;
   const int split = blockIdx.x, h = blockIdx.y;
-  const int b = blockIdx.z / L, l = blockIdx.z % L;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int b = blockIdx.z / L;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int Hq = H * G;
-  const int64_t bl = (int64_t)b * L + l;
-  const int64_t unit = (bl * H + h) * kSplits + split;
-  float* my_part = part + unit * G * kD;
-  float2* my_stat = stat + unit * G;
+  const int64_t bl = blockIdx.z;
+  const int64_t uh = bl * H + h;
   const int len = local_len[b];
   const bool full = len >= cap;
   int M = mem_len[bl];
@@ -77,237 +146,290 @@ __global__ void __launch_bounds__(kThreads, 5) decode_split_kernel(
     M = M_max;
   }
   if (M < 0) M = 0;
-  const int n_keys = M + len + 1;
-  const int per = (n_keys + kSplits - 1) / kSplits;
-  const int k0 = split * per, k1 = min(n_keys, k0 + per);
-  const int new_key = M + len;
-  const bool has_new = new_key >= k0 && new_key < k1;
+  int arrived = 0;  // tid 0: arrivals on query_count[b] before this CTA's
+
   if (full) {
-    if (tid == 0 && split == 0 && h == 0 && l == 0) msa::set_err(dev_err, MSA_DEVERR_LOCAL_FULL);
-    if (tid < G) my_stat[tid] = make_float2(-INFINITY, -1.f);  // unit skipped
-  } else if (k0 >= k1) {
-    if (tid < G) my_stat[tid] = make_float2(-INFINITY, 0.f);   // empty split
+    if (tid == 0 && split == 0 && h == 0 && (bl % L) == 0) msa::set_err(dev_err, MSA_DEVERR_LOCAL_FULL);
+    if (splits > 1 && tid < G) stat[(uh * kMaxSplits + split) * G + tid] = make_float2(-INFINITY, -1.f);
+    __syncthreads();
+    if (tid == 0) arrived = arrive_release(&query_count[b]);
   } else {
-  const double pos = (double)pos_off + (double)len;
-  if (tid < kHalf) {
-    double u = pos * rope.w_over_pi[tid];  // angle / pi
-    u -= 2.0 * rint(0.5 * u);             // in [-1, 1]
-    float sn, c;
-    sincospif((float)u, &sn, &c);
-    cs[tid] = make_float2(c, sn);
-  }
-  if (tid < G) {
-    s_max[tid] = -INFINITY;
-    s_sum[tid] = 0.f;
-  }
-  __syncthreads();
-  for (int e = tid; e < G * kHalf; e += kThreads) {
-    const int g = e / kHalf, j = e % kHalf;
-    const __nv_bfloat16* qp = q + (bl * Hq + (int64_t)h * G + g) * kD;
-    const float a = __bfloat162float(qp[j]), bb = __bfloat162float(qp[j + kHalf]);
-    const float2 c = cs[j];
-    qs[g][j] = (a * c.x - bb * c.y) * scale;
-    qs[g][j + kHalf] = (bb * c.x + a * c.y) * scale;
-  }
-  if (has_new) {
-    // rotate k_new, round to the cache's bf16 (the value every later step reads) and append
-    const int64_t cache_row = ((bl * H + h) * (int64_t)cap + len) * kD;
+    // loads that depend on nothing else start first
+    float qx[2][2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int e = tid + r * kThreads, gg = e / kHalf, j = e % kHalf;
+      qx[r][0] = qx[r][1] = 0.f;
+      if (gg < G) {
+        const __nv_bfloat16* qp = q + (bl * Hq + (int64_t)h * G + gg) * kD;
+        qx[r][0] = __bfloat162float(qp[j]);
+        qx[r][1] = __bfloat162float(qp[j + kHalf]);
+      }
+    }
+    float kx0 = 0.f, kx1 = 0.f;
+    __nv_bfloat16 vx = __float2bfloat16_rn(0.f);
+    if (split == 0) {
+      if (tid < kHalf) {
+        kx0 = __bfloat162float(k_new[uh * kD + tid]);
+        kx1 = __bfloat162float(k_new[uh * kD + tid + kHalf]);
+      } else if (tid < kHalf + kD) {
+        vx = v_new[uh * kD + tid - kHalf];
+      }
+    }
+
+    // ---- this warp's tiles: the first ones are requested before anything else
+    const int nt_mem = (M + kTileKeys - 1) / kTileKeys;
+    const int nt = nt_mem + (len + kTileKeys - 1) / kTileKeys;
+    const int per = (nt + splits - 1) / splits;
+    const int t0 = min(nt, split * per), t1 = min(nt, t0 + per);
+    const int first = t0 + warp;
+    const int my_n = first < t1 ? (t1 - first + kWarps - 1) / kWarps : 0;
+    const __nv_bfloat16* memk = mem_kv + ((bl * 2 + 0) * H + h) * (int64_t)M_max * kD;
+    const __nv_bfloat16* memv = mem_kv + ((bl * 2 + 1) * H + h) * (int64_t)M_max * kD;
+    const __nv_bfloat16* lock = local_k + uh * (int64_t)cap * kD;
+    const __nv_bfloat16* locv = local_v + uh * (int64_t)cap * kD;
+    const uint32_t my_ring = smem_u32(ring) + warp * (kStages * kStageBytes);
+
+    auto tile_rows = [&](int i, const __nv_bfloat16*& kp, const __nv_bfloat16*& vp) -> int {
+      const int ti = first + i * kWarps;
+      if (ti < nt_mem) {
+        kp = memk + (int64_t)ti * kTileKeys * kD;
+        vp = memv + (int64_t)ti * kTileKeys * kD;
+        return min(kTileKeys, M - ti * kTileKeys);
+      }
+      const int j = ti - nt_mem;
+      kp = lock + (int64_t)j * kTileKeys * kD;
+      vp = locv + (int64_t)j * kTileKeys * kD;
+      return min(kTileKeys, len - j * kTileKeys);
+    };
+    auto issue = [&](int i) {
+      const __nv_bfloat16 *kp, *vp;
+      const int nvalid = tile_rows(i, kp, vp);
+      const uint32_t st = my_ring + (i % kStages) * kStageBytes;
+      const int chunk = lane & 15;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int row = 2 * j + (lane >> 4);  // 0..15 K rows, 16..31 V rows
+        const int key = row & 15;
+        const bool ok = key < nvalid;
+        const __nv_bfloat16* src = (j < 8 ? kp : vp) + (ok ? key * kD + chunk * 8 : 0);
+        cp_async16(st + row * kRowBytes + ((chunk ^ (row & 7)) << 4), src, ok ? 16u : 0u);
+      }
+    };
+#pragma unroll
+    for (int p = 0; p < kStages - 1; ++p) {
+      if (p < my_n) issue(p);
+      cp_async_commit();
+    }
+
+    // ---- rotated, scaled query (rows >= G are zero) and, in split 0, the new key
+    const double pos = (double)pos_off + (double)len;
     if (tid < kHalf) {
-      const __nv_bfloat16* kp = k_new + (bl * H + h) * kD;
-      const float a = __bfloat162float(kp[tid]), bb = __bfloat162float(kp[tid + kHalf]);
-      const float2 c = cs[tid];
-      const __nv_bfloat16 lo = __float2bfloat16_rn(a * c.x - bb * c.y);
-      const __nv_bfloat16 hi = __float2bfloat16_rn(bb * c.x + a * c.y);
-      local_k[cache_row + tid] = lo;
-      local_k[cache_row + tid + kHalf] = hi;
-      knew[tid] = __bfloat162float(lo);
-      knew[tid + kHalf] = __bfloat162float(hi);
-    }
-    const __nv_bfloat16 vv = v_new[(bl * H + h) * kD + tid];
-    local_v[cache_row + tid] = vv;
-    vnew[tid] = __bfloat162float(vv);
-  }
-  __syncthreads();
-
-  const __nv_bfloat16* memk = mem_kv + ((bl * 2 + 0) * H + h) * (int64_t)M_max * kD;
-  const __nv_bfloat16* memv = mem_kv + ((bl * 2 + 1) * H + h) * (int64_t)M_max * kD;
-  const __nv_bfloat16* lock = local_k + (bl * H + h) * (int64_t)cap * kD;
-  const __nv_bfloat16* locv = local_v + (bl * H + h) * (int64_t)cap * kD;
-  float acc[G][4];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc[g][u] = 0.f;
-  }
-
-  for (int t0 = k0; t0 < k1; t0 += kTile) {
-    const int i = t0 + tid;
-    if (i < k1) {
-      float dotv[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) dotv[g] = 0.f;
-      if (i == new_key) {
-        for (int j = 0; j < kD; j += 4) {
-          const float4 kk = *reinterpret_cast<const float4*>(&knew[j]);
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float4 qa = *reinterpret_cast<const float4*>(&qs[g][j]);
-            float d = dotv[g];
-            d = fmaf(kk.x, qa.x, d); d = fmaf(kk.y, qa.y, d); d = fmaf(kk.z, qa.z, d); d = fmaf(kk.w, qa.w, d);
-            dotv[g] = d;
-          }
-        }
-      } else {
-        const __nv_bfloat16* kr = i < M ? memk + (int64_t)i * kD : lock + (int64_t)(i - M) * kD;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-        uint4 w[kD / 16];
-#pragma unroll
-        for (int v8 = 0; v8 < kD / 16; ++v8) w[v8] = *reinterpret_cast<const uint4*>(kr + 64 * half + 8 * v8);
-#pragma unroll
-        for (int v8 = 0; v8 < kD / 16; ++v8) {
-          const int e8 = 64 * half + 8 * v8;
-          const float2 f0 = msa::bf16x2_to_float2(w[v8].x), f1 = msa::bf16x2_to_float2(w[v8].y);
-          const float2 f2 = msa::bf16x2_to_float2(w[v8].z), f3 = msa::bf16x2_to_float2(w[v8].w);
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float4 qa = *reinterpret_cast<const float4*>(&qs[g][e8]);
-            const float4 qb = *reinterpret_cast<const float4*>(&qs[g][e8 + 4]);
-            float d = dotv[g];
-            d = fmaf(f0.x, qa.x, d); d = fmaf(f0.y, qa.y, d); d = fmaf(f1.x, qa.z, d); d = fmaf(f1.y, qa.w, d);
-            d = fmaf(f2.x, qb.x, d); d = fmaf(f2.y, qb.y, d); d = fmaf(f3.x, qb.z, d); d = fmaf(f3.y, qb.w, d);
-            dotv[g] = d;
-          }
-        }
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) lg[g][tid] = dotv[g];
-    } else {
-#pragma unroll
-      for (int g = 0; g < G; ++g) lg[g][tid] = -INFINITY;
+      double u = pos * rope.w_over_pi[tid];  // angle / pi
+      u -= 2.0 * rint(0.5 * u);             // in [-1, 1]
+      float sn, c;
+      sincospif((float)u, &sn, &c);
+      cs[tid] = make_float2(c, sn);
     }
     __syncthreads();
-    for (int g = warp; g < G; g += kWarps) {
-      float mx = -INFINITY;
-      for (int u = lane; u < kTile; u += 32) mx = fmaxf(mx, lg[g][u]);
+    // every thread has read local_len[b]: announce it (the last CTA of the query to
+    // arrive advances the length at its end)
+    if (tid == 0) arrived = arrive_release(&query_count[b]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float old = s_max[g];
-      const float nm = fmaxf(old, mx);
-      float sum = 0.f;
-      for (int u = lane; u < kTile; u += 32) {
-        const float p = expf(lg[g][u] - nm);
-        lg[g][u] = p;
-        sum += p;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) {
-        const float fac = expf(old - nm);  // 0 on the first tile (old = -inf)
-        s_fac[g] = fac;
-        s_sum[g] = s_sum[g] * fac + sum;
-        s_max[g] = nm;
+    for (int r = 0; r < 2; ++r) {
+      const int e = tid + r * kThreads, gg = e / kHalf, j = e % kHalf;
+      const float2 c = cs[j];
+      qs[gg][j] = (qx[r][0] * c.x - qx[r][1] * c.y) * qscale;
+      qs[gg][j + kHalf] = (qx[r][1] * c.x + qx[r][0] * c.y) * qscale;
+    }
+    if (split == 0) {
+      const int64_t cache_row = (uh * (int64_t)cap + len) * kD;
+      if (tid < kHalf) {
+        const float2 c = cs[tid];
+        const __nv_bfloat16 lo = __float2bfloat16_rn(kx0 * c.x - kx1 * c.y);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(kx1 * c.x + kx0 * c.y);
+        local_k[cache_row + tid] = lo;
+        local_k[cache_row + tid + kHalf] = hi;
+        knew[tid] = __bfloat162float(lo);
+        knew[tid + kHalf] = __bfloat162float(hi);
+      } else if (tid < kHalf + kD) {
+        const int j = tid - kHalf;
+        local_v[cache_row + j] = vx;
+        vnew[j] = __bfloat162float(vx);
       }
     }
     __syncthreads();
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float f = s_fac[g];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[g][u] *= f;
-    }
-    const int kbeg = warp * 32;
-    const int kend = min(kbeg + 32, k1 - t0);
-    for (int kk0 = kbeg; kk0 < kend; kk0 += 8) {
-      uint2 vw[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int ii = t0 + kk0 + u;
-        vw[u] = make_uint2(0u, 0u);
-        if (kk0 + u < kend && ii != new_key) {
-          const __nv_bfloat16* vr = ii < M ? memv + (int64_t)ii * kD : locv + (int64_t)(ii - M) * kD;
-          vw[u] = *reinterpret_cast<const uint2*>(vr + 4 * lane);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int kk = kk0 + u;
-        if (kk < kend) {
-          float v0, v1, v2, v3;
-          if (t0 + kk == new_key) {
-            const float4 x = *reinterpret_cast<const float4*>(&vnew[4 * lane]);
-            v0 = x.x; v1 = x.y; v2 = x.z; v3 = x.w;
-          } else {
-            const float2 a = msa::bf16x2_to_float2(vw[u].x), c = msa::bf16x2_to_float2(vw[u].y);
-            v0 = a.x; v1 = a.y; v2 = c.x; v3 = c.y;
-          }
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float p = lg[g][kk];
-            acc[g][0] = fmaf(p, v0, acc[g][0]);
-            acc[g][1] = fmaf(p, v1, acc[g][1]);
-            acc[g][2] = fmaf(p, v2, acc[g][2]);
-            acc[g][3] = fmaf(p, v3, acc[g][3]);
-          }
-        }
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-    *reinterpret_cast<float4*>(&red[warp][g][4 * lane]) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-  __syncthreads();
-  for (int o = tid; o < G * kD; o += kThreads) {
-    const int g = o / kD, j = o % kD;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += red[w][g][j];
-    my_part[o] = v;
-  }
-  if (tid < G) my_stat[tid] = make_float2(s_max[tid], s_sum[tid]);
-  }  // work of a non-empty split
 
-  // ---- arrival: the last split CTA of (b, l, h) merges the splits
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  const int64_t uh = bl * H + h;
-  if (tid == 0) s_last = atomicAdd(&unit_count[uh], 1) == kSplits - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int64_t unit0 = uh * kSplits;
-  const bool skipped = __ldcg(&stat[unit0 * G]).y < 0.f;
-  if (!skipped) {
-    for (int o = tid; o < G * kD; o += kThreads) {
-      const int g = o / kD;
+    // query fragments: rows g = bf16(q'), rows g + 8 = bf16 residual
+    uint32_t qa[8][4];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const float2 x = *reinterpret_cast<const float2*>(&qs[g][16 * ks + 2 * t]);
+      const float2 y = *reinterpret_cast<const float2*>(&qs[g][16 * ks + 8 + 2 * t]);
+      split_pair(x.x, x.y, qa[ks][0], qa[ks][1]);
+      split_pair(y.x, y.y, qa[ks][2], qa[ks][3]);
+    }
+
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m = -INFINITY, lsum = 0.f;
+    if (split == 0 && warp == kWarps - 1) {
+      // the new key, in fp32: every lane owns dims 8n + 2t + {0, 1} of its head g
+      float d = 0.f;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const int c = 8 * n + 2 * t;
+        d = fmaf(qs[g][c], knew[c], d);
+        d = fmaf(qs[g][c + 1], knew[c + 1], d);
+        o[n][0] = vnew[c];
+        o[n][1] = vnew[c + 1];
+      }
+      d += __shfl_xor_sync(0xffffffffu, d, 1);
+      d += __shfl_xor_sync(0xffffffffu, d, 2);
+      m = d;
+      lsum = t == 0 ? 1.f : 0.f;
+    }
+
+    for (int i = 0; i < my_n; ++i) {
+      __syncwarp();  // every lane is done with the stage about to be refilled
+      if (i + kStages - 1 < my_n) issue(i + kStages - 1);
+      cp_async_commit();
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
+      const __nv_bfloat16 *kp, *vp;
+      const int nvalid = tile_rows(i, kp, vp);
+      const uint32_t st = my_ring + (i % kStages) * kStageBytes;
+
+      // two accumulators per 8-key half (even / odd k-steps) keep the MMA chains short
+      float s[2][2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) s[j][u][0] = s[j][u][1] = s[j][u][2] = s[j][u][3] = 0.f;
+      }
+#pragma unroll
+      for (int ks2 = 0; ks2 < 4; ++ks2) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int row = 8 * j + (lane & 7);
+          const int chunk = 4 * ks2 + (lane >> 3);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(st + row * kRowBytes + ((chunk ^ (row & 7)) << 4), b0, b1, b2, b3);
+          mma_bf16(s[j][0], qa[2 * ks2], b0, b1);
+          mma_bf16(s[j][1], qa[2 * ks2 + 1], b2, b3);
+        }
+      }
+      float sc[4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = 8 * j + 2 * t + e;
+          sc[2 * j + e] = key < nvalid ? (s[j][0][e] + s[j][0][2 + e]) + (s[j][1][e] + s[j][1][2 + e]) : -INFINITY;
+        }
+      }
+      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m, mx);
+      const float alpha = exp2f(m - m_new);  // 0 while m is still -inf
+      float pr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) pr[u] = exp2f(sc[u] - m_new);
+      lsum = fmaf(lsum, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
+      m = m_new;
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          o[n][0] *= alpha; o[n][1] *= alpha; o[n][2] *= alpha; o[n][3] *= alpha;
+        }
+      }
+      uint32_t pa[4];
+      split_pair(pr[0], pr[1], pa[0], pa[1]);
+      split_pair(pr[2], pr[3], pa[2], pa[3]);
+      const int vkey = (lane & 7) + 8 * ((lane >> 3) & 1);
+      const int vrow = kTileKeys + vkey;
+#pragma unroll
+      for (int i2 = 0; i2 < 8; ++i2) {
+        const int chunk = 2 * i2 + (lane >> 4);
+        uint32_t v0, v1, v2, v3;
+        ldsm_x4_t(st + vrow * kRowBytes + ((chunk ^ (vrow & 7)) << 4), v0, v1, v2, v3);
+        mma_bf16(o[2 * i2], pa, v0, v1);
+        mma_bf16(o[2 * i2 + 1], pa, v2, v3);
+      }
+    }
+    cp_async_wait<0>();
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+
+    // ---- merge the warps (the ring is free once every warp is here)
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(ring);
+    if (t == 0) wml[warp][g] = make_float2(m, lsum);
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<float2*>(&red[(warp * 8 + g) * kRedStride + 8 * n + 2 * t]) =
+          make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
+    __syncthreads();
+    const int64_t unit = uh * kMaxSplits + split;
+    for (int oi = tid; oi < G * kD; oi += kThreads) {
+      const int gg = oi / kD, d = oi % kD;
       float mx = -INFINITY;
 #pragma unroll
-      for (int sp = 0; sp < kSplits; ++sp) mx = fmaxf(mx, __ldcg(&stat[(unit0 + sp) * G + g]).x);
+      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, wml[w][gg].x);
       float num = 0.f, den = 0.f;
 #pragma unroll
-      for (int sp = 0; sp < kSplits; ++sp) {
-        const float2 st = __ldcg(&stat[(unit0 + sp) * G + g]);
+      for (int w = 0; w < kWarps; ++w) {
+        const float2 st = wml[w][gg];
         if (st.y > 0.f) {
-          const float w = expf(st.x - mx);
-          num = fmaf(w, __ldcg(&part[(unit0 + sp) * G * kD + o]), num);
-          den = fmaf(w, st.y, den);
+          const float f = exp2f(st.x - mx);
+          num = fmaf(f, red[(w * 8 + gg) * kRedStride + d], num);
+          den = fmaf(f, st.y, den);
         }
       }
-      out[(bl * Hq + (int64_t)h * G + g) * kD + (o % kD)] = __float2bfloat16_rn(num / den);
+      if (splits == 1) {
+        out[(bl * Hq + (int64_t)h * G + gg) * kD + d] = __float2bfloat16_rn(num / den);
+      } else {
+        part[unit * G * kD + oi] = num;
+        if (d == 0) stat[unit * G + gg] = make_float2(mx, den);
+      }
     }
   }
-  if (tid == 0) {
-    unit_count[uh] = 0;  // ready for the next call
-    // the last merged (l, h) of query b advances its local length (every CTA of this
-    // call that reads local_len[b] has arrived by then)
+
+  if (splits > 1) {
+    // ---- the last split CTA of (b, l, h) to finish merges the splits
     __threadfence();
-    if (atomicAdd(&query_count[b], 1) == L * H - 1) {
-      if (!skipped) local_len[b] = len + 1;
-      query_count[b] = 0;
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&unit_count[uh], 1) == splits - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const int64_t unit0 = uh * kMaxSplits;
+      if (!full) {
+        for (int oi = tid; oi < G * kD; oi += kThreads) {
+          const int gg = oi / kD;
+          float mx = -INFINITY;
+          for (int sp = 0; sp < splits; ++sp) mx = fmaxf(mx, __ldcg(&stat[(unit0 + sp) * G + gg]).x);
+          float num = 0.f, den = 0.f;
+          for (int sp = 0; sp < splits; ++sp) {
+            const float2 st = __ldcg(&stat[(unit0 + sp) * G + gg]);
+            if (st.y > 0.f) {
+              const float w = exp2f(st.x - mx);
+              num = fmaf(w, __ldcg(&part[(unit0 + sp) * G * kD + oi]), num);
+              den = fmaf(w, st.y, den);
+            }
+          }
+          out[(bl * Hq + (int64_t)h * G + gg) * kD + (oi % kD)] = __float2bfloat16_rn(num / den);
+        }
+      }
+      if (tid == 0) unit_count[uh] = 0;  // ready for the next call
     }
+  }
+  // every CTA of query b arrived after reading local_len[b]; the last one advances it
+  if (tid == 0 && arrived == L * H * splits - 1) {
+    if (!full) local_len[b] = len + 1;
+    query_count[b] = 0;  // ready for the next call
   }
 }
 
@@ -339,7 +461,7 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   if (n_queries < 1 || n_layers < 1 || (int64_t)n_queries * n_layers > 65535 || local_cap < 1 || max_mem_chunks < 1)
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_queries * n_layers <= 65535)");
   if (!(rope_theta > 1.0f)) return msa_fail(MSA_ERR_INVALID_ARG, "rope_theta must be > 1");
-  if (!msa::aligned16(mem_kv) || !msa::aligned16(local_k) || !msa::aligned16(workspace))
+  if (!msa::aligned16(mem_kv) || !msa::aligned16(local_k) || !msa::aligned16(local_v) || !msa::aligned16(workspace))
     return msa_fail(MSA_ERR_INVALID_ARG, "16-byte alignment");
   const size_t need = ws_bytes(n_queries, n_layers, n_q_heads, n_kv_heads);
   if (workspace_bytes < need)
@@ -348,20 +470,24 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
   if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t units = (size_t)n_queries * n_layers * n_kv_heads * kSplits;
+  const int64_t units = (int64_t)n_queries * n_layers * n_kv_heads;
+  const int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, msa::sm_count() / units));
   float* part = reinterpret_cast<float*>(workspace);
-  float2* stat = reinterpret_cast<float2*>(part + units * G * kD);
+  float2* stat = reinterpret_cast<float2*>(part + (size_t)units * kMaxSplits * G * kD);
   int* unit_count = reinterpret_cast<int*>(part + ws_floats(n_queries, n_layers, n_q_heads, n_kv_heads));
-  int* query_count = unit_count + (size_t)n_queries * n_layers * n_kv_heads;
-  const dim3 grid(kSplits, n_kv_heads, n_queries * n_layers);
+  int* query_count = unit_count + units;
+  const dim3 grid(splits, n_kv_heads, n_queries * n_layers);
   RopeTable rope;
   for (int j = 0; j < kHalf; ++j)
     rope.w_over_pi[j] = pow((double)rope_theta, -2.0 * (double)j / (double)kD) / 3.14159265358979323846;
+  const float qscale = softmax_scale * kLog2e;
 #define MSA_DECODE_LAUNCH(GG)                                                                                    \
-  decode_split_kernel<GG><<<grid, kThreads, 0, s>>>(                                                             \
+  MSA_CUDA_TRY(cudaFuncSetAttribute(decode_mma_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                    kRingBytes));                                                                 \
+  decode_mma_kernel<GG><<<grid, kThreads, kRingBytes, s>>>(                                                       \
       (const __nv_bfloat16*)q, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_layers, n_kv_heads,     \
       (__nv_bfloat16*)local_k, (__nv_bfloat16*)local_v, local_len, local_cap, (const __nv_bfloat16*)mem_kv,        \
-      mem_len, max_mem_chunks, rope_pos_offset, rope, softmax_scale, part, stat, unit_count, query_count,         \
+      mem_len, max_mem_chunks, rope_pos_offset, rope, qscale, splits, part, stat, unit_count, query_count,        \
       (__nv_bfloat16*)out, dev_err)
   switch (G) {
     case 1: MSA_DECODE_LAUNCH(1); break;
