@@ -33,9 +33,9 @@ WORKLOAD = ("100M-token bank (100,000 docs, lognormal lengths rounded to 64, 1,5
 N_DOCS, N_TOKENS, L, H, HQ, D, TOPK, T, DEC, SEED = 100_000, 100_000_000, 18, 8, 32, 128, 16, 256, 128, 3
 TOKENS_PER_DOC = 1000
 THETA = 1e6
-# DRAM bytes per (block, layer) of the routing GEMM, read + write, from the ncu capture in
-# profiles/route_tc_kernel_2M_T256.md (2M-token bank, same kernel), scaled by blocks.
-GEMM_TRAFFIC_PER_BLOCK_LAYER = 2074.5
+# DRAM bytes per (block, layer) of the routing GEMM, read + write, from the ncu captures in
+# profiles/ (2M-token bank, same kernels), scaled by blocks; None where not captured yet.
+GEMM_TRAFFIC_PER_BLOCK_LAYER = {"bf16": 2074.5, "e4m3": None}
 
 
 def log(*a):
@@ -121,7 +121,7 @@ def set_bank_size(n_docs: int) -> None:
     N_DOCS, N_TOKENS = n_docs, n_docs * TOKENS_PER_DOC
 
 
-def make_workload(dev, host_store_chunks: int):
+def make_workload(dev, host_store_chunks: int, f8: bool):
     import torch
 
     import msa_synth as syn
@@ -146,6 +146,17 @@ def make_workload(dev, host_store_chunks: int):
     del scratch, row_topic, ones
     torch.cuda.synchronize(dev)
     log(f"routing keys ready: {C} blocks x {L} layers ({kr_hat.numel() * 2 / 1e9:.1f} GB) in {time.time() - t0:.1f}s")
+    kr_f8, f8_ms = None, None
+    if f8:
+        # the E4M3 filter copy of the keys (built once per bank, like the keys themselves)
+        kr_f8 = torch.empty((L, C, H, D), dtype=torch.uint8, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        msa.msa_route_filter_keys(kr_hat, L, C, H, D, kr_f8)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        f8_ms = e0.elapsed_time(e1)
+        log(f"E4M3 filter keys: {kr_f8.numel() / 1e9:.1f} GB in {f8_ms:.1f} ms")
     # content store: host_store_chunks physical blocks per layer; document d reads the
     # contiguous physical range starting at a hashed offset (same bytes per selection)
     P = min(host_store_chunks, C)
@@ -160,7 +171,7 @@ def make_workload(dev, host_store_chunks: int):
         host_kv[l].copy_(stage.permute(1, 0, 2).reshape(P, 2, H, D))
     del stage
     log(f"host content store: {P} blocks x {L} layers ({host_kv.numel() * 2 / 1e9:.1f} GB pinned)")
-    return bank, kr_hat, host_kv, store_off, topic
+    return bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic
 
 
 def make_queries(dev, bank, topic, n_queries: int):
@@ -251,14 +262,15 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     hbm_peak, bf16_peak, bf16_sus, peak_src = measured_peaks()
 
-    bank, kr_hat, host_kv, store_off, topic = make_workload(dev, args.host_store_blocks)
+    f8 = args.filter == "e4m3"
+    bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic = make_workload(dev, args.host_store_blocks, f8)
     qs, targets = make_queries(dev, bank, topic, args.queries)
     dq, dk, dv, pk, pv = make_decode_inputs(dev)
     n_slots = args.pipeline
     dec_inputs = [(dq.clone(), dk.clone(), dv.clone(), torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16,
                                                                    device=dev)) for _ in range(n_slots)]
     eng = SparseMemory(kr_hat, bank.doc_chunk_offsets, host_kv, store_off, n_q_heads=HQ, top_k=TOPK,
-                       query_tokens=T, local_cap=T + DEC, rope_theta=THETA, slots=n_slots)
+                       query_tokens=T, local_cap=T + DEC, rope_theta=THETA, slots=n_slots, kr_f8=kr_f8)
     eng.set_local_prefix(pk, pv)
     for s_ in eng.slots:
         s_.qr.copy_(qs[0])
@@ -320,6 +332,17 @@ def run_gpu(args):
     got = slot0.ids.cpu().numpy()[0]
     hits = np.mean([len(set(got[l].tolist()) & set(targets[0].tolist())) / TOPK for l in range(L)])
     dev_err = int(slot0.dev_err.item())
+    same_as_bf16 = None
+    if f8:
+        # the same query through the bf16 filter: both end in exact rescoring, so the
+        # selections must agree
+        ids2 = torch.empty_like(slot0.ids)
+        sc2 = torch.empty_like(slot0.scores)
+        msa.msa_route_topk(slot0.qr, [0, T], kr_hat, eng.doc_chunk_offsets, eng.n_docs, eng.C, L, HQ, H, D, TOPK,
+                           ids2, sc2, slot0.ws, flags=msa.MSA_ROUTE_TENSOR, dev_err=slot0.dev_err)
+        torch.cuda.synchronize(dev)
+        same_as_bf16 = bool(torch.equal(ids2, slot0.ids) and torch.equal(sc2, slot0.scores))
+        dev_err |= int(slot0.dev_err.item())
 
     # isolated latency of one query (route + gather + decode, nothing overlapping)
     iso = []
@@ -372,9 +395,18 @@ def run_gpu(args):
     ms = total_ms / args.steps
     units = N_TOKENS * args.steps * world
     value = units / (total_ms / 1e3)
-    algo_bytes = L * bank.n_chunks * H * D * 2
+    elem = 1 if f8 else 2
+    algo_bytes = L * bank.n_chunks * H * D * elem
     achieved = algo_bytes / (gemm_avg / 1e3) / 1e9
     flops = 2.0 * T * H * D * L * bank.n_chunks
+    tflops = flops / (gemm_avg / 1e3) / 1e12
+    # tensor peak of the operand type: E4M3 = 2 x the measured bf16 figure (the nominal
+    # dense ratio); sustained, as the GEMM runs for milliseconds back to back
+    tc_peak = (bf16_sus or bf16_peak) * (2.0 if f8 else 1.0)
+    t_hbm = algo_bytes / (hbm_peak * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    bound = "tensor" if t_tc > t_hbm else "hbm"
+    traffic_pbl = GEMM_TRAFFIC_PER_BLOCK_LAYER["e4m3" if f8 else "bf16"]
     p = sorted(per_query)
     iso_s = sorted(iso)
     line = {
@@ -388,13 +420,16 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3 filter + fp32 rescoring" if f8 else "bf16 filter + fp32 rescoring",
         "data": "synthetic",
         "config": {"workload": WORKLOAD if N_DOCS == 100_000 else f"{N_TOKENS:,}-token bank (profiling size)",
+                   "filter": ("E4M3 copy of the unit keys (x256), tcgen05 kind::f8f6f4; top candidates rescored "
+                              "exactly in fp32 from the bf16 keys" if f8 else
+                              "bf16 keys, tcgen05 kind::f16; top candidates rescored exactly in fp32"),
                    "n_docs": N_DOCS, "n_tokens": N_TOKENS, "n_blocks": bank.n_chunks,
                    "layers": L, "kv_heads": H, "q_heads": HQ, "head_dim": D, "query_tokens": T, "top_k": TOPK,
                    "decode_tokens": DEC, "distinct_queries": len(qs), "host_store_blocks": int(host_kv.shape[1]),
-                   "l2": "inputs larger than L2 (57.6 GB of routing keys stream through every step)",
+                   "l2": f"inputs larger than L2 ({algo_bytes / 1e9:.1f} GB of routing keys stream through every step)",
                    "graph": "per query two CUDA graphs: route; gather + 128 decode steps",
                    "pipeline": (f"{n_slots} query slots: the gather+decode of query i overlaps the route of "
                                 "query i+1" if n_slots > 1 else "one query at a time"),
@@ -403,15 +438,21 @@ def run_gpu(args):
         "p50_route_decode_ms": round(p[len(p) // 2], 4),
         "p99_route_decode_ms": round(p[min(len(p) - 1, int(0.99 * len(p)))], 4),
         "p50_isolated_ms": round(iso_s[len(iso_s) // 2], 4),
-        "roofline": {"bound": "hbm", "kernel": "route score GEMM (tcgen05)", "achieved": round(achieved, 1),
-                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "peak_source": peak_src,
-                     "traffic": round(GEMM_TRAFFIC_PER_BLOCK_LAYER * L * bank.n_chunks),
-                     "traffic_source": "ncu dram bytes of a 2M-token launch scaled by blocks",
+        "roofline": {"bound": bound, "kernel": "route score GEMM (tcgen05, %s)" % ("E4M3" if f8 else "bf16"),
+                     "achieved": round(tflops if bound == "tensor" else achieved, 1),
+                     "peak": round(tc_peak if bound == "tensor" else hbm_peak, 1),
+                     "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                     "frac": round(tflops / tc_peak if bound == "tensor" else achieved / hbm_peak, 4),
+                     "peak_source": (f"{peak_src}: " + ("sustained bf16 x 2 (E4M3/bf16 nominal ratio)" if f8 else
+                                                        "sustained bf16") if bound == "tensor" else
+                                     f"{peak_src}: HBM copy"),
+                     "traffic": None if traffic_pbl is None else round(traffic_pbl * L * bank.n_chunks),
+                     "traffic_source": ("ncu dram bytes of a 2M-token launch scaled by blocks" if traffic_pbl
+                                        else "not captured for this kernel yet"),
                      "algorithmic_bytes": algo_bytes, "kernel_ms": round(gemm_avg, 4),
-                     "tflops": round(flops / (gemm_avg / 1e3) / 1e12, 1),
-                     "tensor_frac": round(flops / (gemm_avg / 1e3) / 1e12 / bf16_peak, 4),
-                     "frac_of_8tbs": round(achieved / 8000.0, 4)},
+                     "gbs": round(achieved, 1), "hbm_frac": round(achieved / hbm_peak, 4),
+                     "tflops": round(tflops, 1), "tensor_frac": round(tflops / tc_peak, 4),
+                     "roofline_ms": round(max(t_hbm, t_tc) * 1e3, 4)},
         "e2e": {"value": round(units / (e2e_ms / 1e3), 1), "unit": "bank tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
@@ -419,6 +460,8 @@ def run_gpu(args):
         "pool": pool,
         "planted_recall": round(float(hits), 4),
         "dev_err": dev_err,
+        "filter_keys_ms": None if f8_ms is None else round(f8_ms, 2),
+        "ids_match_bf16_filter": same_as_bf16,
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -498,6 +541,8 @@ def main():
     ap.add_argument("--no-pool", action="store_true", help="skip the separate pooling measurement")
     ap.add_argument("--pipeline", type=int, default=1, choices=[1, 2],
                     help="queries in flight (2 overlaps a query's gather+decode with the next route)")
+    ap.add_argument("--filter", default="e4m3", choices=["e4m3", "bf16"],
+                    help="operands of the routing filter GEMM (both end in exact fp32 rescoring)")
     ap.add_argument("--docs", type=int, default=N_DOCS,
                     help="documents in the bank (x1000 tokens); smaller banks serve profiling captures")
     args = ap.parse_args()

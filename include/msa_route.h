@@ -33,11 +33,24 @@ extern "C" {
 #define MSA_ROUTE_AUTO 0    /* pick by query length                                  */
 #define MSA_ROUTE_SCAN 1    /* CUDA-core streaming scan (few query tokens)           */
 #define MSA_ROUTE_TENSOR 2  /* tcgen05 tensor-core GEMM with fused token-max epilogue */
+#define MSA_ROUTE_TENSOR_F8 3 /* the same GEMM on the E4M3 copy of the keys            */
 
 /* Workspace bytes for one msa_route_topk call with these sizes. */
 msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, int32_t total_q_tokens,
                                          int32_t n_kv_heads, int64_t n_chunks, int32_t n_docs, int32_t top_k,
                                          size_t* bytes);
+
+/* E4M3 filter copy of the unit routing keys, for MSA_ROUTE_TENSOR_F8.  The MSA pages have
+ * no counterpart: this is an index the tensor-core filter streams instead of kr_hat
+ * (half the bytes, twice the tensor-core rate); the selection is still decided on exact
+ * fp32 scores of kr_hat.  Every head of kr_hat is renormalised in fp32 (scale
+ * 1 / max(||k||, 1e-8)), multiplied by 256 and rounded to E4M3 (OCP FP8, nearest even,
+ * saturating at 448).
+ *   kr_hat  DEVICE bf16 [n_layers][n_chunks][n_kv_heads][head_dim], 16-byte aligned
+ *   kr_f8   DEVICE bytes, same shape, 16-byte aligned (caller-owned, written)
+ *   head_dim = 128.  One kernel, asynchronous on stream. */
+msa_status msa_route_filter_keys(const void* kr_hat, int32_t n_layers, int64_t n_chunks, int32_t n_kv_heads,
+                                 int32_t head_dim, void* kr_f8, msa_stream_t stream);
 
 /* Routes n_queries queries over n_layers routing layers (each layer selects its own
  * top_k documents).
@@ -48,15 +61,24 @@ msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, in
  *                    (every query has at least one token); read during the call only.
  *   kr_hat           DEVICE bf16 [n_layers][n_chunks][n_kv_heads][head_dim], unit-norm
  *                    routing keys (msa_pool_blocks), 16-byte aligned.
+ *   kr_f8            DEVICE, msa_route_filter_keys(kr_hat), or NULL.  Required by
+ *                    MSA_ROUTE_TENSOR_F8; with MSA_ROUTE_AUTO its presence selects that path
+ *                    for queries beyond the scan length.
  *   doc_chunk_offsets DEVICE int64 [n_docs + 1], doc_chunk_offsets[n_docs] = n_chunks.
  *   head_dim = 128; n_kv_heads = 8 on the tensor-core path; n_q_heads % n_kv_heads = 0;
  *   1 <= top_k <= 64; 1 <= n_queries <= 256; n_kv_heads in {2, 4, 8, 16}; n_q_heads <= 64.
  *   out_ids, out_scores DEVICE [n_queries][n_layers][top_k] int32 / fp32.
  *   workspace        DEVICE, >= msa_route_topk_workspace_size bytes, 256-byte aligned.
- *   flags            MSA_ROUTE_AUTO / _SCAN / _TENSOR.
+ *   flags            MSA_ROUTE_AUTO / _SCAN / _TENSOR / _TENSOR_F8.
+ * The tensor paths score with low-precision operands as a filter, rescore the best
+ * candidates exactly in fp32 and take the top_k from the exact scores.  A layer whose
+ * selection cannot be certified against the filter's error bound (1e-3 for bf16
+ * operands, 2^-6 for E4M3) sets MSA_DEVERR_UNCERTIFIED in dev_err; the ids are then the
+ * best of the rescored candidates, and re-routing with a tighter filter (_TENSOR or
+ * _SCAN) is the caller's choice.
  * Asynchronous on stream; no host synchronisation. */
 msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
-                          int32_t n_queries, const void* kr_hat, const int64_t* doc_chunk_offsets,
+                          int32_t n_queries, const void* kr_hat, const void* kr_f8, const int64_t* doc_chunk_offsets,
                           int32_t n_docs, int64_t n_chunks, int32_t n_layers, int32_t n_q_heads,
                           int32_t n_kv_heads, int32_t head_dim, int32_t top_k, int32_t* out_ids,
                           float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,

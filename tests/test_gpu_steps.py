@@ -143,6 +143,13 @@ def _route_bank(bank, layers):
     return bits, bf16_tensor(bits), _dev_i64(bank.doc_chunk_offsets)
 
 
+def _filter_keys(msa, kr_hat):
+    L, C = kr_hat.shape[0], kr_hat.shape[1]
+    kr_f8 = torch.empty(kr_hat.shape, dtype=torch.uint8, device="cuda")
+    msa.msa_route_filter_keys(kr_hat, L, C, H, D, kr_f8)
+    return kr_f8
+
+
 def _route_gpu(msa, qr, q_offsets, kr_hat, coffs, n_docs, C, L, k, flags):
     B = len(q_offsets) - 1
     T = int(q_offsets[-1])
@@ -150,8 +157,9 @@ def _route_gpu(msa, qr, q_offsets, kr_hat, coffs, n_docs, C, L, k, flags):
     ids = torch.full((B, L, k), -7, dtype=torch.int32, device="cuda")
     sc = torch.full((B, L, k), float("nan"), device="cuda")
     err = _err()
+    kr_f8 = _filter_keys(msa, kr_hat) if flags == msa.MSA_ROUTE_TENSOR_F8 else None
     msa.msa_route_topk(torch.from_numpy(np.ascontiguousarray(qr, dtype=np.float32)).cuda(), q_offsets, kr_hat,
-                       coffs, n_docs, C, L, HQ, H, D, k, ids, sc, ws, flags=flags, dev_err=err)
+                       coffs, n_docs, C, L, HQ, H, D, k, ids, sc, ws, flags=flags, dev_err=err, kr_f8=kr_f8)
     torch.cuda.synchronize()
     return ids.cpu().numpy(), sc.cpu().numpy(), int(err.item())
 
@@ -182,50 +190,86 @@ def _route_case(msa, seed, lens, L, Ts, k, flags, n_targets=2):
     return ids, sc, err
 
 
-@pytest.mark.parametrize("flags", [1, 2])
+@pytest.mark.parametrize("flags", [1, 2, 3])
 def test_route_multi_query_multi_layer(msa, flags):
     lens = syn.doc_lengths_lognormal(1, 200)
     _route_case(msa, 1, lens, 2, [1, 5, 2], 16, flags)
 
 
-@pytest.mark.parametrize("flags", [1, 2])
+@pytest.mark.parametrize("flags", [1, 2, 3])
 def test_route_fewer_docs_than_k_and_empty_docs(msa, flags):
     lens = np.array([100, 0, 64, 0, 1, 300])
     ids, sc, _ = _route_case(msa, 2, lens, 1, [3], 8, flags)
     assert list(ids[0, 0, 6:]) == [-1, -1] and np.all(np.isneginf(sc[0, 0, 4:]))
 
 
-@pytest.mark.parametrize("flags", [1, 2])
+@pytest.mark.parametrize("flags", [1, 2, 3])
 def test_route_single_document(msa, flags):
     _route_case(msa, 3, np.array([65]), 1, [2], 4, flags, n_targets=1)
 
 
+@pytest.mark.parametrize("flags", [2, 3])
 @pytest.mark.parametrize("Ts", [[300, 40, 257], [64], [129], [33, 31, 1, 64]])
-def test_route_tensor_long_queries_span_tiles(msa, Ts):
+def test_route_tensor_long_queries_span_tiles(msa, Ts, flags):
     # several N tiles per block tile (queries crossing tile edges), ragged last M tile,
     # two layers (tiles at the layer boundary)
     lens = syn.doc_lengths_lognormal(7, 150)
-    _route_case(msa, 7, lens, 2, Ts, 64, 2, n_targets=4)
+    _route_case(msa, 7, lens, 2, Ts, 64, flags, n_targets=4)
 
 
+@pytest.mark.parametrize("flags", [2, 3])
 @pytest.mark.parametrize("pair", [True, False])
 @pytest.mark.parametrize("Ts", [[256], [100, 156], [129]])
-def test_route_tensor_pair_and_single_cta_tiles(msa, pair, Ts):
+def test_route_tensor_pair_and_single_cta_tiles(msa, pair, Ts, flags):
     # N tiles of 128 / 256 run on SM pairs (M = 256) by default; both tilings must match the oracle
     lens = syn.doc_lengths_lognormal(11, 180)
     msa.msa_route_set_pair_mode(pair)
     try:
-        _route_case(msa, 11, lens, 2, Ts, 32, 2, n_targets=4)
+        _route_case(msa, 11, lens, 2, Ts, 32, flags, n_targets=4)
     finally:
         msa.msa_route_set_pair_mode(True)
 
 
-def test_route_tensor_selection_is_certified_for_planted_needles(msa):
+@pytest.mark.parametrize("flags", [2, 3])
+def test_route_tensor_selection_is_certified_for_planted_needles(msa, flags):
     # k = number of planted documents: the k-th exact score sits far above the filter's
     # margin over the best document left out, so the certification bit stays clear
     lens = syn.doc_lengths_lognormal(9, 400)
-    _, _, err = _route_case(msa, 9, lens, 1, [64], 4, 2, n_targets=4)
+    _, _, err = _route_case(msa, 9, lens, 1, [64], 4, flags, n_targets=4)
     assert err == 0
+
+
+def _e4m3_decode(b):
+    b = b.astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e, m = (b >> 3) & 15, b & 7
+    return sign * np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7.0))
+
+
+def test_route_filter_keys_round_unit_heads_to_e4m3(msa):
+    # every element is the E4M3 value nearest to 256 x the element of the unit head
+    # (within half a unit in the last place of E4M3), a zero head stays zero
+    L, C = 2, 77
+    x = syn.fill(12, syn.STREAM_KRBAR, 0, 0, 0, L * C * H, D, sigma=0.3, dtype="bf16").reshape(L, C, H, D)
+    x[1, 5, 2] = 0
+    x[0, 0, 0, :4] = syn.f32_to_bf16_bits(np.array([3.0, -2.0, 1e-3, 0.0], dtype=np.float32))
+    got = _e4m3_decode(_filter_keys(msa, bf16_tensor(x)).cpu().numpy())
+    f = syn.bf16_bits_to_f32(x).astype(np.float64)
+    ref = 256.0 * f / np.maximum(np.linalg.norm(f, axis=3, keepdims=True), 1e-8)
+    a = np.abs(ref)
+    ulp = np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -6))) - 3))
+    assert np.all(np.abs(got - ref) <= 0.5 * ulp * (1 + 1e-5) + 1e-9)
+    assert np.all(got[1, 5, 2] == 0)
+    assert np.abs(got).max() <= 256.0
+
+
+def test_route_f8_and_bf16_filters_select_the_same_documents(msa):
+    # both filters end in exact fp32 rescoring: on a planted bank the selections agree
+    lens = syn.doc_lengths_lognormal(13, 500)
+    a = _route_case(msa, 13, lens, 2, [256], 16, 2, n_targets=16)
+    b = _route_case(msa, 13, lens, 2, [256], 16, 3, n_targets=16)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    assert a[2] == 0 and b[2] == 0
 
 
 def test_route_auto_picks_tensor_for_long_query_and_scan_for_short(msa):
@@ -233,13 +277,14 @@ def test_route_auto_picks_tensor_for_long_query_and_scan_for_short(msa):
     bank = syn.make_bank(8, 60, lens, 1)
     _, kr_hat, coffs = _route_bank(bank, 1)
     C = bank.n_chunks
+    kr_f8 = _filter_keys(msa, kr_hat)
     # scan: qprep + scan + 2 top-k; tensor: zero-pad + qprep + GEMM + 2 top-k + rescore + final
-    for T, expect in ((4, 4), (40, 7)):
+    for T, f8, expect in ((4, None, 4), (40, None, 7), (4, kr_f8, 4), (40, kr_f8, 7)):
         ws = torch.empty(msa.msa_route_topk_workspace_size(1, 1, T, H, C, 60, 16), dtype=torch.uint8, device="cuda")
         ids = torch.empty((1, 1, 16), dtype=torch.int32, device="cuda")
         sc = torch.empty((1, 1, 16), device="cuda")
         n = msa.msa_route_topk(torch.randn((1, T, HQ, D), device="cuda"), [0, T], kr_hat, coffs, 60, C, 1, HQ, H, D,
-                               16, ids, sc, ws)
+                               16, ids, sc, ws, kr_f8=f8)
         assert n == expect
 
 

@@ -16,7 +16,7 @@ LIB_DIR = os.path.join(_HERE, "lib")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY, MSA_ERR_TIMEOUT = range(6)
 MSA_F32, MSA_BF16 = 0, 1
-MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR = 0, 1, 2
+MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR, MSA_ROUTE_TENSOR_F8 = 0, 1, 2, 3
 (MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS, MSA_DEVERR_TIMEOUT,
  MSA_DEVERR_UNCERTIFIED) = 1, 2, 4, 8, 16, 32
 
@@ -55,8 +55,10 @@ pool_lib.msa_pool_last_error.restype = ctypes.c_char_p
 route_lib.msa_route_topk_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i32, _i32,
                                                     ctypes.POINTER(_sz)]
 route_lib.msa_route_topk_workspace_size.restype = _i32
-route_lib.msa_route_topk.argtypes = [_p, _i32, _p, _i32, _p, _p, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
+route_lib.msa_route_topk.argtypes = [_p, _i32, _p, _i32, _p, _p, _p, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
                                      _p, _p, _p, _sz, _i32, _p, _p]
+route_lib.msa_route_filter_keys.argtypes = [_p, _i32, _i64, _i32, _i32, _p, _p]
+route_lib.msa_route_filter_keys.restype = _i32
 route_lib.msa_route_topk.restype = _i32
 route_lib.msa_route_last_launch_count.restype = _i32
 route_lib.msa_route_last_error.restype = ctypes.c_char_p
@@ -158,18 +160,29 @@ def msa_route_topk_workspace_size(n_layers: int, n_queries: int, total_q_tokens:
 
 def msa_route_topk(qr, q_offsets, kr_hat, doc_chunk_offsets, n_docs: int, n_chunks: int, n_layers: int,
                    n_q_heads: int, n_kv_heads: int, head_dim: int, top_k: int, out_ids, out_scores, workspace,
-                   flags: int = MSA_ROUTE_AUTO, dev_err=None, q_dtype: int | None = None, stream=None) -> int:
-    """Returns the number of kernels the call enqueued."""
+                   flags: int = MSA_ROUTE_AUTO, dev_err=None, q_dtype: int | None = None, stream=None,
+                   kr_f8=None) -> int:
+    """Returns the number of kernels the call enqueued.  kr_f8: the E4M3 keys written by
+    msa_route_filter_keys (needed by MSA_ROUTE_TENSOR_F8, picked by MSA_ROUTE_AUTO)."""
     qo = np.ascontiguousarray(q_offsets, dtype=np.int32)
     if q_dtype is None:
         q_dtype = MSA_BF16 if str(qr.dtype) == "torch.bfloat16" else MSA_F32
     ws_bytes = _nbytes(workspace)
-    st = route_lib.msa_route_topk(_ptr(qr), q_dtype, qo.ctypes.data, len(qo) - 1, _ptr(kr_hat),
+    st = route_lib.msa_route_topk(_ptr(qr), q_dtype, qo.ctypes.data, len(qo) - 1, _ptr(kr_hat), _ptr(kr_f8),
                                   _ptr(doc_chunk_offsets), n_docs, n_chunks, n_layers, n_q_heads, n_kv_heads,
                                   head_dim, top_k, _ptr(out_ids), _ptr(out_scores), _ptr(workspace), ws_bytes,
                                   flags, _ptr(dev_err), _stream(stream))
     _check(st, "msa_route_topk", route_lib, "msa_route_last_error")
     return int(route_lib.msa_route_last_launch_count())
+
+
+def msa_route_filter_keys(kr_hat, n_layers: int, n_chunks: int, n_kv_heads: int, head_dim: int, kr_f8,
+                          stream=None) -> None:
+    """E4M3 filter copy of the unit routing keys (x 256, per-head renormalised) into kr_f8
+    (uint8 tensor of kr_hat's shape)."""
+    st = route_lib.msa_route_filter_keys(_ptr(kr_hat), n_layers, n_chunks, n_kv_heads, head_dim, _ptr(kr_f8),
+                                         _stream(stream))
+    _check(st, "msa_route_filter_keys", route_lib, "msa_route_last_error")
 
 
 def msa_route_set_pair_mode(enabled: bool) -> None:

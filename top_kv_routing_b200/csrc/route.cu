@@ -9,8 +9,9 @@
 //               (fp32 for the exact kernels, bf16 rows padded per query for the GEMM)
 //   2. score    m[b][l][c] = max_{t in b} cos-score(t, c)
 //               scan path (few tokens): exact fp32 on CUDA cores, keys normalised per head
-//               tensor path: tcgen05 GEMM on bf16 operands (a filter; also the runner-up
-//               score and the argmax token of each block)
+//               tensor path: tcgen05 GEMM on bf16 operands, or on the E4M3 filter copy of
+//               the keys (a filter; also the runner-up score and the argmax token of each
+//               block)
 //   3. docmax   S[doc] = max of m over the document's blocks; per-CTA best candidates
 //   4. merge    the per-CTA candidates -> top_k (scan) or the K2 filter candidates (tensor)
 //   tensor path only:
@@ -18,6 +19,8 @@
 //               pairs whose filter score lies within the filter's error window of the max
 //   6. final    top_k of the exact scores; certification of the selection
 // The score matrix s[t][c] only ever lives in registers / TMEM.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "msa_route.h"
 #include "route_tc.cuh"
@@ -38,6 +41,9 @@ constexpr int kMaxBlocks = 64;       // docmax CTAs per (query, layer)
 // within 2x of it from a block's best are rescored; a selection is certified when the
 // k-th exact score beats the best filter score left out by more than it.
 constexpr float kFilterErr = 1e-3f;
+// The same for the E4M3 filter (3 mantissa bits on both operands): rms error ~8e-4,
+// largest seen ~5e-3 over 8M (block, token) pairs of bank-like data; 2^-6 is ~19 rms.
+constexpr float kFilterErrF8 = 0.015625f;
 
 // Candidates rescored exactly on the tensor-core path.
 int rescore_count(int32_t n_docs, int32_t k) {
@@ -114,7 +120,8 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
 // goes to operand row row0[b] + (t - off[b]) of layer l (n_rows rows per layer).
 __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr, int q_is_bf16, int T_total,
                                                     int Hq, int H, int n_rows, QueryOffsets qo,
-                                                    float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16) {
+                                                    float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16,
+                                                    uint8_t* __restrict__ qt_f8) {
   __shared__ float qhat[64][kD];
   const int t = blockIdx.x, l = blockIdx.y;
   int qb = 0;
@@ -158,6 +165,9 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
     acc *= inv_hq;
     qt_f32[((int64_t)l * T_total + t) * H * kD + e] = acc;
     if (qt_bf16 != nullptr) qt_bf16[((int64_t)l * n_rows + orow) * H * kD + e] = __float2bfloat16_rn(acc);
+    if (qt_f8 != nullptr)
+      qt_f8[((int64_t)l * n_rows + orow) * H * kD + e] =
+          __nv_cvt_float_to_fp8(acc * route_tc::kF8QueryScale, __NV_SATFINITE, __NV_E4M3);
   }
 }
 
@@ -174,6 +184,52 @@ __global__ void zero_pad_kernel(uint4* __restrict__ qt_bf16, int n_rows, int wor
     }
     const bool token_row = r < qo.row0[qo.n] && (r - qo.row0[lo]) < (qo.off[lo + 1] - qo.off[lo]);
     if (!token_row) qt_bf16[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// ---------------------------------------------------------------------------- E4M3 keys
+// 8 threads per (row, head): 16 bf16 each; the head is renormalised in fp32 (the same
+// 1 / max(||k||, 1e-8) as the exact kernels) and stored x kF8KeyScale as E4M3.  The loop
+// runs per warp (4 heads a pass) so every lane takes part in the shuffles.
+__global__ void __launch_bounds__(256) filter_keys_kernel(const __nv_bfloat16* __restrict__ kr, int64_t n_heads,
+                                                          uint8_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int64_t warp0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t base = warp0 * 4; base < n_heads; base += n_warps * 4) {
+    const int64_t hh = base + (lane >> 3);
+    const bool ok = hh < n_heads;
+    float x[16];
+    float ss = 0.f;
+    if (ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(kr + hh * kD) + 2 * sub;
+      const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
+      const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 f = msa::bf16x2_to_float2(w[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ss = fmaf(x[i], x[i], ss);
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+    if (ok) {
+      const float sc = route_tc::kF8KeyScale / fmaxf(sqrtf(ss), 1e-8f);
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i] * sc, x[4 * i + 1] * sc), __NV_SATFINITE,
+                                                     __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i + 2] * sc, x[4 * i + 3] * sc),
+                                                     __NV_SATFINITE, __NV_E4M3);
+        o[i] = lo | (hi << 16);
+      }
+      __stcs(reinterpret_cast<uint4*>(out + hh * kD) + sub, make_uint4(o[0], o[1], o[2], o[3]));
+    }
   }
 }
 
@@ -536,8 +592,30 @@ extern "C" msa_status msa_route_set_profile_events(void* start_event, void* stop
   return msa_ok();
 }
 
+extern "C" msa_status msa_route_filter_keys(const void* kr_hat, int32_t n_layers, int64_t n_chunks,
+                                            int32_t n_kv_heads, int32_t head_dim, void* kr_f8, msa_stream_t stream) {
+  if (!kr_hat || !kr_f8) return msa_fail(MSA_ERR_INVALID_ARG, "null pointer");
+  if (head_dim != kD) return msa_fail(MSA_ERR_INVALID_ARG, "head_dim must be 128");
+  if (n_layers < 1 || n_chunks < 0 || n_kv_heads < 1 || n_kv_heads > 16)
+    return msa_fail(MSA_ERR_INVALID_ARG, "bad sizes");
+  if (!msa::aligned16(kr_hat) || !msa::aligned16(kr_f8)) return msa_fail(MSA_ERR_INVALID_ARG, "16-byte alignment");
+  const int arch = msa::current_device_is_sm100(nullptr);
+  if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
+  if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
+  const int64_t n_heads = (int64_t)n_layers * n_chunks * n_kv_heads;
+  if (n_heads == 0) return msa_ok();
+  int64_t blocks = (n_heads + 31) / 32;  // 256 threads = 32 heads a pass
+  const int64_t cap = (int64_t)msa::sm_count() * 16;
+  if (blocks > cap) blocks = cap;
+  filter_keys_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(kr_hat), n_heads, reinterpret_cast<uint8_t*>(kr_f8));
+  MSA_CUDA_TRY(cudaGetLastError());
+  return msa_ok();
+}
+
 extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
-                                     int32_t n_queries, const void* kr_hat, const int64_t* doc_chunk_offsets,
+                                     int32_t n_queries, const void* kr_hat, const void* kr_f8,
+                                     const int64_t* doc_chunk_offsets,
                                      int32_t n_docs, int64_t n_chunks, int32_t n_layers, int32_t n_q_heads,
                                      int32_t n_kv_heads, int32_t head_dim, int32_t top_k, int32_t* out_ids,
                                      float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,
@@ -555,9 +633,12 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   if (n_layers < 1 || n_chunks < 0 || n_docs < 0 || n_docs > kMaxDocs)
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_docs <= 2^20)");
   if (q_dtype != MSA_F32 && q_dtype != MSA_BF16) return msa_fail(MSA_ERR_UNSUPPORTED, "q_dtype");
-  if (flags < MSA_ROUTE_AUTO || flags > MSA_ROUTE_TENSOR) return msa_fail(MSA_ERR_INVALID_ARG, "flags");
-  if (!msa::aligned16(qr) || !msa::aligned16(kr_hat) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return msa_fail(MSA_ERR_INVALID_ARG, "alignment: qr/kr_hat 16 B, workspace 256 B");
+  if (flags < MSA_ROUTE_AUTO || flags > MSA_ROUTE_TENSOR_F8) return msa_fail(MSA_ERR_INVALID_ARG, "flags");
+  if (flags == MSA_ROUTE_TENSOR_F8 && !kr_f8)
+    return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_TENSOR_F8 needs the E4M3 keys (msa_route_filter_keys)");
+  if (!msa::aligned16(qr) || !msa::aligned16(kr_hat) || !msa::aligned16(kr_f8) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return msa_fail(MSA_ERR_INVALID_ARG, "alignment: qr/kr_hat/kr_f8 16 B, workspace 256 B");
   QueryOffsets qo;
   qo.n = n_queries;
   if (q_offsets_host[0] != 0) return msa_fail(MSA_ERR_INVALID_ARG, "q_offsets[0] must be 0");
@@ -584,23 +665,29 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + w.cand);
   const int H = n_kv_heads;
 
-  // Path: the CUDA-core scan while the query is a handful of tokens, tensor cores beyond.
+  // Path: the CUDA-core scan while the query is a handful of tokens, tensor cores beyond
+  // (on the E4M3 keys when the caller has them).
   int path = flags;
-  if (path == MSA_ROUTE_AUTO) path = (T_total <= route_tc::kScanMaxTokens) ? MSA_ROUTE_SCAN : MSA_ROUTE_TENSOR;
-  if (path == MSA_ROUTE_TENSOR && !route_tc::supported(H)) {
-    if (flags == MSA_ROUTE_TENSOR) return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
+  if (path == MSA_ROUTE_AUTO)
+    path = (T_total <= route_tc::kScanMaxTokens) ? MSA_ROUTE_SCAN : (kr_f8 ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
+  if ((path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && !route_tc::supported(H)) {
+    if (flags != MSA_ROUTE_AUTO) return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
     path = MSA_ROUTE_SCAN;
   }
-  const bool tensor = path == MSA_ROUTE_TENSOR && n_chunks > 0;
+  const bool tensor = (path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && n_chunks > 0;
+  const bool f8 = tensor && path == MSA_ROUTE_TENSOR_F8;
+  const float filter_err = f8 ? kFilterErrF8 : kFilterErr;
 
   if (tensor) {
-    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(reinterpret_cast<uint4*>(qt_bf16), n_rows, H * kD / 8,
-                                                         n_layers, qo);
+    // (the E4M3 operand, one byte per element, reuses the bf16 operand's buffer)
+    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(reinterpret_cast<uint4*>(qt_bf16), n_rows,
+                                                         H * kD * (f8 ? 1 : 2) / 16, n_layers, qo);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
   qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
-                                                      qt_f32, tensor ? qt_bf16 : nullptr);
+                                                      qt_f32, tensor && !f8 ? qt_bf16 : nullptr,
+                                                      f8 ? reinterpret_cast<uint8_t*>(qt_bf16) : nullptr);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
   if (n_chunks > 0) {
@@ -620,8 +707,9 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
       MSA_CUDA_TRY(cudaGetLastError());
     } else {
       route_tc::LaunchArgs a;
-      a.kr_hat = kr_hat;
+      a.kr_hat = f8 ? kr_f8 : kr_hat;
       a.qt = qt_bf16;
+      a.f8 = f8;
       a.L = n_layers;
       a.C = n_chunks;
       a.n_rows = n_rows;
@@ -682,10 +770,10 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs_smem));
   rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, rs_smem, s>>>(
       (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks, T_total, qo, doc_chunk_offsets, m,
-      reinterpret_cast<const int2*>(ws + w.aux), apx, K2, kFilterErr, exact);
+      reinterpret_cast<const int2*>(ws + w.aux), apx, K2, filter_err, exact);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
-  select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, kFilterErr,
+  select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, filter_err,
                                                                out_ids, out_scores, dev_err);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());

@@ -2,16 +2,20 @@
 //
 // Per layer l the scores of every memory block c against every query token t are
 //   D[c][t] = < kr_hat[l][c][:], qt[l][t][:] >      (K = 8 heads x 128 = 1024)
-// a dense bf16 GEMM with fp32 accumulation (M = blocks, N = query tokens).  The
-// epilogue reduces each row over the columns of every query and writes, per (query,
+// a dense GEMM with fp32 accumulation (M = blocks, N = query tokens) on bf16 operands
+// (kind::f16) or on E4M3 operands (kind::f8f6f4; keys stored x 2^8, queries x 2^11, the
+// product rescaled by 2^-19 in the epilogue).  One 128-byte shared-memory row holds 64
+// bf16 or 128 E4M3 elements and one MMA consumes 32 bytes of K either way, so both
+// forms share the tiling, swizzle and descriptors; E4M3 halves the K-blocks per tile.
+// The epilogue reduces each row over the columns of every query and writes, per (query,
 // layer, block), the largest score m, the second largest and the argmax token; D itself
-// never leaves TMEM.  These bf16-operand scores are a filter: the caller rescores the
+// never leaves TMEM.  These low-precision scores are a filter: the caller rescores the
 // pairs that can hold the maximum exactly.
 //
 // Warp roles of the persistent kernel (192 threads, one CTA per SM):
-//   warp 0      TMA producer: A tile [128 blocks x 64] + B tile [tokens x 64] per
+//   warp 0      TMA producer: A tile [128 blocks x 128 B] + B tile [tokens x 128 B] per
 //               K-block into a ring of shared-memory stages (128-byte swizzle)
-//   warp 1      one thread issues tcgen05.mma (bf16 in, fp32 accumulate, K=16) into one of
+//   warp 1      one thread issues tcgen05.mma (fp32 accumulate, 32 bytes of K each) into one of
 //               two TMEM accumulators and commits stage / accumulator completion to mbarriers
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max / runner-up / argmax over
 //               each query's columns, store; then release the accumulator
@@ -32,17 +36,19 @@ namespace route_tc {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBK = 64;                  // bf16 elements per 128-byte row
+constexpr int kRowBytes = 128;           // one swizzled shared-memory row per K-block
 constexpr int kKDim = 1024;              // 8 key heads x 128
-constexpr int kKBlocks = kKDim / kBK;    // 16
-constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+constexpr int kABytes = kBM * kRowBytes; // 16 KB
 constexpr int kThreads = 192;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool F8>
 struct Cfg {
+  static constexpr int kElem = F8 ? 1 : 2;                 // operand bytes
+  static constexpr int kBK = kRowBytes / kElem;            // elements per K-block
+  static constexpr int kKBlocks = kKDim / kBK;             // 16 (bf16) or 8 (E4M3)
   static constexpr int kBRows = PAIR ? BN / 2 : BN;  // query rows of the B tile held per CTA
-  static constexpr int kBBytes = kBRows * kBK * 2;
+  static constexpr int kBBytes = kBRows * kRowBytes;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kStages = (196 * 1024) / kStage > 8 ? 8 : (196 * 1024) / kStage;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators: 128, 256 or 512 columns
@@ -183,14 +189,28 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-template <bool PAIR>
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  if (PAIR)
+template <bool PAIR, bool F8>
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                     uint32_t accumulate) {
+  if (PAIR && F8)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else if (PAIR)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else if (F8)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
   else
@@ -243,18 +263,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+// Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A and B both K-major, A / B
+// formats in bits 7-9 / 10-12 (kind::f16: bf16 = 1; kind::f8f6f4: E4M3 = 0), N / 8 in
+// bits 17-22, M / 16 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_make(int m, int n, bool f8) {
+  return (1u << 4) | (f8 ? 0u : (1u << 7) | (1u << 10)) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int L,
                     long long C, int n_rows, int m_tiles, const __grid_constant__ QueryLayout ql,
                     float* __restrict__ m_out, int2* __restrict__ aux_out, int32_t* dev_err) {
-  using K = Cfg<BN, PAIR>;
+  using K = Cfg<BN, PAIR, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::kStages * K::kStage);
@@ -315,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row_a = (int)((long long)l * C) + mt * K::kRows + (int)rank * kBM;
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
           const int row_b = l * n_rows + nt * BN + (int)rank * K::kBRows;
-          for (int kb = 0; kb < kKBlocks; ++kb) {
+          for (int kb = 0; kb < K::kKBlocks; ++kb) {
             if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
               ok = false;
               break;
@@ -325,12 +347,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (PAIR) {
               const uint32_t fb_lead = map_to_rank(fb, 0);  // both CTAs' bytes land on the leader's barrier
               if (leader) mbar_arrive_expect_tx(fb, 2 * K::kStage);
-              tma_load_2d_pair(sa, &tm_a, fb_lead, kb * kBK, row_a, pol_a);
-              tma_load_2d_pair(sa + kABytes, &tm_b, fb_lead, kb * kBK, row_b, pol_b);
+              tma_load_2d_pair(sa, &tm_a, fb_lead, kb * K::kBK, row_a, pol_a);
+              tma_load_2d_pair(sa + kABytes, &tm_b, fb_lead, kb * K::kBK, row_b, pol_b);
             } else {
               mbar_arrive_expect_tx(fb, K::kStage);
-              tma_load_2d(sa, &tm_a, fb, kb * kBK, row_a, pol_a);
-              tma_load_2d(sa + kABytes, &tm_b, fb, kb * kBK, row_b, pol_b);
+              tma_load_2d(sa, &tm_a, fb, kb * K::kBK, row_a, pol_a);
+              tma_load_2d(sa + kABytes, &tm_b, fb, kb * K::kBK, row_b, pol_b);
             }
             armed[stage] = (int)phase;
             if (++stage == K::kStages) {
@@ -352,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (the leader of a pair issues for both CTAs)
-      constexpr uint32_t idesc = idesc_bf16(K::kRows, BN);
+      constexpr uint32_t idesc = idesc_make(K::kRows, BN, F8);
       int stage = 0, buf = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
@@ -364,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
-          for (int kb = 0; kb < kKBlocks; ++kb) {
+          for (int kb = 0; kb < K::kKBlocks; ++kb) {
             if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag)) {
               ok = false;
               break;
@@ -373,9 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sa = smem_u32(smem + stage * K::kStage);
             const uint64_t da = sw128_desc(sa), db = sw128_desc(sa + kABytes);
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k)
-              umma_bf16<PAIR>(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
-                              (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < kRowBytes / 32; ++k)  // 32 bytes of K per MMA
+              umma<PAIR, F8>(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc, (kb | k) != 0 ? 1u : 0u);
             issued = true;
             umma_commit<PAIR>(smem_u32(&empty[stage]));
             if (++stage == K::kStages) {
@@ -460,8 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t0 + 32 >= ql.len[b]) {
               if (row_ok) {
                 const long long o = ((long long)b * L + l) * C + row;
-                m_out[o] = m1;
-                aux_out[o] = make_int2(__float_as_int(m2), i1);
+                m_out[o] = F8 ? m1 * kF8ScoreScale : m1;
+                aux_out[o] = make_int2(__float_as_int(F8 ? m2 * kF8ScoreScale : m2), i1);
               }
               carry_b = -1;
             } else {
@@ -516,25 +537,27 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D bf16 row-major [rows][1024] map with a box of [box_rows][64] and the 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+// 2D row-major [rows][1024] map (bf16 or bytes) with a box of [box_rows][128 bytes] and
+// the 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows, bool f8) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const int elem = f8 ? 1 : 2;
   const cuuint64_t dims[2] = {(cuuint64_t)kKDim, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kKDim * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kKDim * elem};
+  const cuuint32_t box[2] = {(cuuint32_t)(kRowBytes / elem), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool F8>
 int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
-  using K = Cfg<BN, PAIR>;
+  using K = Cfg<BN, PAIR, F8>;
   CUtensorMap ma, mb;
   const uint64_t rows_a = (uint64_t)a.L * (uint64_t)a.C;
-  if (!make_map(&ma, a.kr_hat, rows_a, kBM) || !make_map(&mb, a.qt, (uint64_t)a.L * a.n_rows, K::kBRows)) {
+  if (!make_map(&ma, a.kr_hat, rows_a, kBM, F8) || !make_map(&mb, a.qt, (uint64_t)a.L * a.n_rows, K::kBRows, F8)) {
     *why = "cuTensorMapEncodeTiled failed";
     return 1;
   }
@@ -543,7 +566,7 @@ int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
   const int per_unit = PAIR ? 2 : 1;
   int grid = msa::sm_count() / per_unit * per_unit;
   if (units * per_unit < grid) grid = (int)(units * per_unit);
-  if (cudaFuncSetAttribute(route_tc_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) !=
+  if (cudaFuncSetAttribute(route_tc_kernel<BN, PAIR, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) !=
       cudaSuccess) {
     *why = "cudaFuncSetAttribute (shared memory)";
     return 1;
@@ -560,7 +583,7 @@ int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
+  if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR, F8>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
                          a.aux, a.dev_err) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
@@ -584,11 +607,19 @@ int launch(const LaunchArgs& a, cudaStream_t s, int* launches, const char** why)
     return 1;
   }
   int r;
-  if (bn == 64) r = launch_bn<64, false>(a, s, why);
-  else if (a.pair && bn == 128) r = launch_bn<128, true>(a, s, why);
-  else if (bn == 128) r = launch_bn<128, false>(a, s, why);
-  else if (a.pair) r = launch_bn<256, true>(a, s, why);
-  else r = launch_bn<256, false>(a, s, why);
+  if (a.f8) {
+    if (bn == 64) r = launch_bn<64, false, true>(a, s, why);
+    else if (a.pair && bn == 128) r = launch_bn<128, true, true>(a, s, why);
+    else if (bn == 128) r = launch_bn<128, false, true>(a, s, why);
+    else if (a.pair) r = launch_bn<256, true, true>(a, s, why);
+    else r = launch_bn<256, false, true>(a, s, why);
+  } else {
+    if (bn == 64) r = launch_bn<64, false, false>(a, s, why);
+    else if (a.pair && bn == 128) r = launch_bn<128, true, false>(a, s, why);
+    else if (bn == 128) r = launch_bn<128, false, false>(a, s, why);
+    else if (a.pair) r = launch_bn<256, true, false>(a, s, why);
+    else r = launch_bn<256, false, false>(a, s, why);
+  }
   if (r == 0) *launches = 1;
   return r;
 }

@@ -38,6 +38,13 @@ inline int operand_rows(const int* q_off, int n_queries) {
 
 bool supported(int n_kv_heads);
 
+// E4M3 operand scales: unit keys are stored x 2^8 (|x| <= 256), the query operand rows
+// (each element at most 1 / n_kv_heads = 1/8 in magnitude) x 2^11 (|x| <= 256); both stay
+// inside the E4M3 range (448) and the GEMM result is rescaled by 2^-19.
+constexpr float kF8KeyScale = 256.0f;
+constexpr float kF8QueryScale = 2048.0f;
+constexpr float kF8ScoreScale = 1.0f / (256.0f * 2048.0f);
+
 struct QueryLayout {
   int n_queries;
   int row0[kMaxQueries + 1];   // first operand row of each query (aligned to 32)
@@ -45,8 +52,8 @@ struct QueryLayout {
 };
 
 struct LaunchArgs {
-  const void* kr_hat;  // bf16 [L][C][8][128]
-  const void* qt;      // bf16 [L][n_rows][8][128], padding rows are zero
+  const void* kr_hat;  // bf16 [L][C][8][128], or E4M3 x kF8KeyScale when f8
+  const void* qt;      // bf16 [L][n_rows][8][128] (E4M3 x kF8QueryScale when f8), padding rows zero
   int L;
   int64_t C;
   int n_rows;          // operand rows per layer (multiple of the N tile)
@@ -55,6 +62,7 @@ struct LaunchArgs {
   int2* aux;           // [B][L][C]  (bits of the second-largest score, argmax token in the query)
   int32_t* dev_err;
   bool pair;           // M=256 tiles on CTA pairs (cta_group::2) for N tiles of 128 / 256
+  bool f8;             // E4M3 operands (kind::f8f6f4)
 };
 
 // Enqueues the score kernel; returns 0 on success (launches += kernels enqueued).

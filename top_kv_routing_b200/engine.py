@@ -50,8 +50,12 @@ class SparseMemory:
     def __init__(self, kr_hat: torch.Tensor, doc_chunk_offsets: np.ndarray, host_kv: torch.Tensor,
                  doc_store_offsets: np.ndarray | None = None, *, n_q_heads: int = 32, top_k: int = 16,
                  query_tokens: int = 256, local_cap: int = 384, rope_theta: float = 1e6,
-                 max_mem_chunks: int | None = None, route_flags: int = MSA_ROUTE_AUTO, slots: int = 2):
+                 max_mem_chunks: int | None = None, route_flags: int = MSA_ROUTE_AUTO, slots: int = 2,
+                 kr_f8: torch.Tensor | None = None):
+        """kr_f8: optional E4M3 filter copy of kr_hat (msa_route_filter_keys); with the
+        default route flags, routes of long queries then filter on it."""
         assert kr_hat.is_cuda and kr_hat.dtype == torch.bfloat16 and kr_hat.dim() == 4
+        assert kr_f8 is None or (kr_f8.is_cuda and kr_f8.dtype == torch.uint8 and kr_f8.shape == kr_hat.shape)
         assert host_kv.is_pinned() and host_kv.dim() == 5 and host_kv.shape[2] == 2
         dev = kr_hat.device
         self.dev = dev
@@ -63,6 +67,7 @@ class SparseMemory:
         self.theta = rope_theta
         self.flags = route_flags
         self.kr_hat = kr_hat
+        self.kr_f8 = kr_f8
         offs = np.ascontiguousarray(doc_chunk_offsets, dtype=np.int64)
         self.n_docs = len(offs) - 1
         self.doc_chunk_offsets = torch.from_numpy(offs).to(dev)
@@ -89,7 +94,7 @@ class SparseMemory:
     def enqueue_route(self, slot: _Slot, stream) -> int:
         return msa_route_topk(slot.qr, [0, self.T], self.kr_hat, self.doc_chunk_offsets, self.n_docs, self.C,
                               self.L, self.Hq, self.H, self.D, self.k, slot.ids, slot.scores, slot.ws,
-                              flags=self.flags, dev_err=slot.dev_err, stream=stream)
+                              flags=self.flags, dev_err=slot.dev_err, stream=stream, kr_f8=self.kr_f8)
 
     def enqueue_tail(self, slot: _Slot, dec_q, dec_k, dec_v, out, stream) -> int:
         """Gather of slot's selection, then one decode step per row of dec_q [S][1][L][Hq][D]
