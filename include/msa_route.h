@@ -71,11 +71,13 @@ msa_status msa_route_filter_keys(const void* kr_hat, int32_t n_layers, int64_t n
  *   workspace        DEVICE, >= msa_route_topk_workspace_size bytes, 256-byte aligned.
  *   flags            MSA_ROUTE_AUTO / _SCAN / _TENSOR / _TENSOR_F8.
  * The tensor paths score with low-precision operands as a filter, rescore the best
- * candidates exactly in fp32 and take the top_k from the exact scores.  A layer whose
- * selection cannot be certified against the filter's error bound (1e-3 for bf16
- * operands, 2^-6 for E4M3) sets MSA_DEVERR_UNCERTIFIED in dev_err; the ids are then the
- * best of the rescored candidates, and re-routing with a tighter filter (_TENSOR or
- * _SCAN) is the caller's choice.
+ * candidates exactly in fp32 and take the top_k from the exact scores.  A selection is
+ * certified when its k-th exact score beats the best filter score left out by more than
+ * the filter's error bound (1e-3 for bf16 operands, 2^-6 for E4M3).  On the E4M3 path,
+ * layers that fail are filtered again with bf16 operands and rescored within the same
+ * call (its kernels return at once when every layer is certified); a layer that fails
+ * the bf16 bound sets MSA_DEVERR_UNCERTIFIED in dev_err, its ids being the best of the
+ * rescored candidates (MSA_ROUTE_SCAN is exact).
  * Asynchronous on stream; no host synchronisation. */
 msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
                           int32_t n_queries, const void* kr_hat, const void* kr_f8, const int64_t* doc_chunk_offsets,

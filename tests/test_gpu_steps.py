@@ -239,6 +239,23 @@ def test_route_tensor_selection_is_certified_for_planted_needles(msa, flags):
     assert err == 0
 
 
+def test_route_f8_layers_without_margin_fall_back_to_the_bf16_filter(msa):
+    # router queries of pure noise: the top-k boundary sits inside the E4M3 error window,
+    # so those layers cannot be certified from the E4M3 pass and are re-filtered in bf16;
+    # the result must still be the exact top-k (and certified)
+    lens = syn.doc_lengths_lognormal(14, 600)
+    bank = syn.make_bank(14, len(lens), lens, 2)
+    bits, kr_hat, coffs = _route_bank(bank, 2)
+    T, k = 96, 16
+    qr = syn.fill(14, syn.STREAM_QR, 0, 0, 0, 2 * T * HQ, D).reshape(2, T, HQ, D)
+    ids, sc, err = _route_gpu(msa, qr, [0, T], kr_hat, coffs, len(lens), bank.n_chunks, 2, k, msa.MSA_ROUTE_TENSOR_F8)
+    assert err == 0
+    for l in range(2):
+        _, _, doc_scores, _ = oracle.route(qr[l], syn.bf16_bits_to_f32(bits[l]), bank.doc_chunk_offsets, k,
+                                           grouped=True)
+        check_topk(ids[0, l], sc[0, l], doc_scores, k)
+
+
 def _e4m3_decode(b):
     b = b.astype(np.int64)
     sign = np.where(b >> 7, -1.0, 1.0)
@@ -278,8 +295,9 @@ def test_route_auto_picks_tensor_for_long_query_and_scan_for_short(msa):
     _, kr_hat, coffs = _route_bank(bank, 1)
     C = bank.n_chunks
     kr_f8 = _filter_keys(msa, kr_hat)
-    # scan: qprep + scan + 2 top-k; tensor: zero-pad + qprep + GEMM + 2 top-k + rescore + final
-    for T, f8, expect in ((4, None, 4), (40, None, 7), (4, kr_f8, 4), (40, kr_f8, 7)):
+    # scan: qprep + scan + 2 top-k; tensor: zero-pad + qprep + GEMM + 2 top-k + rescore + final;
+    # E4M3: the same plus the bf16 pass over uncertified layers (GEMM + 2 top-k + rescore + final)
+    for T, f8, expect in ((4, None, 4), (40, None, 7), (4, kr_f8, 4), (40, kr_f8, 12)):
         ws = torch.empty(msa.msa_route_topk_workspace_size(1, 1, T, H, C, 60, 16), dtype=torch.uint8, device="cuda")
         ids = torch.empty((1, 1, 16), dtype=torch.int32, device="cuda")
         sc = torch.empty((1, 1, 16), device="cuda")

@@ -78,7 +78,7 @@ int pow2_at_least(int n) {
 }
 
 struct WsLayout {
-  size_t qt_f32, qt_bf16, m, aux, cand, apx, exact, total;
+  size_t qt_f32, qt_bf16, qt_f8, m, aux, cand, apx, exact, redo, total;
   int n_pad;
   int nblk;
   int k2;
@@ -101,6 +101,8 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   o += align256((size_t)L * T_total * H * kD * sizeof(float));
   w.qt_bf16 = o;
   o += align256((size_t)L * w.n_pad * H * kD * 2);
+  w.qt_f8 = o;
+  o += align256((size_t)L * w.n_pad * H * kD);
   w.m = o;
   o += align256((size_t)B * L * (size_t)C * sizeof(float));
   w.aux = o;
@@ -111,6 +113,8 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(unsigned long long));
   w.exact = o;
   o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(float));
+  w.redo = o;
+  o += align256((size_t)L * sizeof(int32_t));
   w.total = o;
   return w;
 }
@@ -121,9 +125,12 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
 __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr, int q_is_bf16, int T_total,
                                                     int Hq, int H, int n_rows, QueryOffsets qo,
                                                     float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16,
-                                                    uint8_t* __restrict__ qt_f8) {
+                                                    uint8_t* __restrict__ qt_f8, int32_t* __restrict__ redo,
+                                                    int n_layers) {
   __shared__ float qhat[64][kD];
   const int t = blockIdx.x, l = blockIdx.y;
+  if (redo != nullptr && t == 0 && l == 0)
+    for (int i = threadIdx.x; i < n_layers; i += blockDim.x) redo[i] = 0;
   int qb = 0;
   {
     int lo = 0, hi = qo.n;  // largest b with off[b] <= t
@@ -173,17 +180,23 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
 
 // Zero every operand row that holds no query token (per-query alignment gaps and the
 // tail up to n_rows), in 16-byte words.
-__global__ void zero_pad_kernel(uint4* __restrict__ qt_bf16, int n_rows, int words_per_row, int L, QueryOffsets qo) {
+// (a second buffer with rows of words_per_row2 words is padded the same way when given)
+__global__ void zero_pad_kernel(uint4* __restrict__ qt, int n_rows, int words_per_row, int L, QueryOffsets qo,
+                                uint4* __restrict__ qt2, int words_per_row2) {
   const int64_t total = (int64_t)L * n_rows * words_per_row;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int r = (int)((i / words_per_row) % n_rows);
+  const int64_t total2 = qt2 != nullptr ? (int64_t)L * n_rows * words_per_row2 : 0;
+  const int64_t all = total + total2;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < all; i += (int64_t)gridDim.x * blockDim.x) {
+    const bool second = i >= total;
+    const int64_t j = second ? i - total : i;
+    const int r = (int)((j / (second ? words_per_row2 : words_per_row)) % n_rows);
     int lo = 0, hi = qo.n;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (qo.row0[mid] <= r) lo = mid; else hi = mid;
     }
     const bool token_row = r < qo.row0[qo.n] && (r - qo.row0[lo]) < (qo.off[lo + 1] - qo.off[lo]);
-    if (!token_row) qt_bf16[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (!token_row) (second ? qt2 : qt)[j] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -361,9 +374,11 @@ __device__ void block_sort_desc(unsigned long long* keys, int n) {
 __global__ void __launch_bounds__(kTopkThreads) docmax_topk_kernel(const float* __restrict__ m,
                                                                    const int64_t* __restrict__ doc_chunk_off,
                                                                    int n_docs, int64_t C, int L, int k_sel,
-                                                                   int n_pow2, unsigned long long* __restrict__ cand) {
+                                                                   int n_pow2, unsigned long long* __restrict__ cand,
+                                                                   const int32_t* __restrict__ only) {
   extern __shared__ unsigned long long tk_smem[];
   const int blk = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
+  if (only != nullptr && only[l] == 0) return;
   const int nblk = gridDim.x;
   const int per = (n_docs + nblk - 1) / nblk;
   const int d0 = blk * per;
@@ -400,9 +415,11 @@ __global__ void __launch_bounds__(kTopkThreads) merge_topk_kernel(const unsigned
                                                                   int nblk, int L, int k_sel, int n_pow2,
                                                                   unsigned long long* __restrict__ keys_out,
                                                                   int32_t* __restrict__ out_ids,
-                                                                  float* __restrict__ out_scores) {
+                                                                  float* __restrict__ out_scores,
+                                                                  const int32_t* __restrict__ only) {
   extern __shared__ unsigned long long tk_smem[];
   const int l = blockIdx.x, b = blockIdx.y;
+  if (only != nullptr && only[l] == 0) return;
   const int n = nblk * k_sel;
   const unsigned long long* src = cand + ((int64_t)b * L + l) * n;
   for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) tk_smem[i] = i < n ? src[i] : 0ull;
@@ -439,13 +456,14 @@ __global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __res
                                                       QueryOffsets qo, const int64_t* __restrict__ doc_chunk_off,
                                                       const float* __restrict__ m, const int2* __restrict__ aux,
                                                       const unsigned long long* __restrict__ apx, int K2, float err,
-                                                      float* __restrict__ exact) {
+                                                      float* __restrict__ exact, const int32_t* __restrict__ only) {
   constexpr int R = NV * 256;
   extern __shared__ float4 rows[];  // [kRescoreRows][R / 4] in lane-vector order
   __shared__ float red[4];
   __shared__ int full_list[kRescoreRows];
   __shared__ int n_full;
   const int r = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
+  if (only != nullptr && only[l] == 0) return;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t o = ((int64_t)b * L + l) * K2 + r;
   int doc;
@@ -529,14 +547,19 @@ __global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __res
 
 // grid (L, B), 128 threads: final top-k of the K2 exactly rescored candidates.  The
 // selection is certified when the k-th exact score beats the best filter score left out
-// (the K2-th) by more than the filter's error bound; otherwise MSA_DEVERR_UNCERTIFIED.
+// (the K2-th) by more than the filter's error bound.  Otherwise: with redo given (a first,
+// E4M3 pass) the layer is marked for the bf16 pass; without it MSA_DEVERR_UNCERTIFIED.
+// With only given, layers it does not mark are left as they are.
 __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long long* __restrict__ apx,
                                                            const float* __restrict__ exact, int K2, int k,
                                                            int n_docs, int L, float err,
                                                            int32_t* __restrict__ out_ids,
-                                                           float* __restrict__ out_scores, int32_t* dev_err) {
+                                                           float* __restrict__ out_scores, int32_t* dev_err,
+                                                           int32_t* __restrict__ redo,
+                                                           const int32_t* __restrict__ only) {
   __shared__ unsigned long long keys[kMaxCandidates];
   const int l = blockIdx.x, b = blockIdx.y;
+  if (only != nullptr && only[l] == 0) return;
   const int64_t base = ((int64_t)b * L + l) * K2;
   const int n_pow2 = K2 <= 1 ? 1 : (1 << (32 - __clz(K2 - 1)));
   for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
@@ -563,7 +586,10 @@ __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long l
     float s_left, s_kth;
     split_key(apx[base + K2 - 1], &d_left, &s_left);
     split_key(keys[k - 1], &d_kth, &s_kth);
-    if (!(s_kth > s_left + err)) msa::set_err(dev_err, MSA_DEVERR_UNCERTIFIED);
+    if (!(s_kth > s_left + err)) {
+      if (redo != nullptr) redo[l] = 1;
+      else msa::set_err(dev_err, MSA_DEVERR_UNCERTIFIED);
+    }
   }
 }
 
@@ -678,18 +704,47 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   const bool f8 = tensor && path == MSA_ROUTE_TENSOR_F8;
   const float filter_err = f8 ? kFilterErrF8 : kFilterErr;
 
+  uint8_t* qt_f8 = reinterpret_cast<uint8_t*>(ws + w.qt_f8);
+  int32_t* redo = reinterpret_cast<int32_t*>(ws + w.redo);
   if (tensor) {
-    // (the E4M3 operand, one byte per element, reuses the bf16 operand's buffer)
-    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(reinterpret_cast<uint4*>(qt_bf16), n_rows,
-                                                         H * kD * (f8 ? 1 : 2) / 16, n_layers, qo);
+    // the E4M3 pass also prepares the bf16 operand, for layers it cannot certify
+    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(reinterpret_cast<uint4*>(qt_bf16), n_rows, H * kD * 2 / 16,
+                                                         n_layers, qo, f8 ? reinterpret_cast<uint4*>(qt_f8) : nullptr,
+                                                         H * kD / 16);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
   qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
-                                                      qt_f32, tensor && !f8 ? qt_bf16 : nullptr,
-                                                      f8 ? reinterpret_cast<uint8_t*>(qt_bf16) : nullptr);
+                                                      qt_f32, tensor ? qt_bf16 : nullptr, f8 ? qt_f8 : nullptr,
+                                                      f8 ? redo : nullptr, n_layers);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
+
+  // tcgen05 filter GEMM over all blocks of the layers `only` marks (all when null)
+  auto gemm = [&](bool e4m3, const int32_t* only) -> msa_status {
+    route_tc::LaunchArgs a;
+    a.kr_hat = e4m3 ? kr_f8 : kr_hat;
+    a.qt = e4m3 ? static_cast<const void*>(qt_f8) : static_cast<const void*>(qt_bf16);
+    a.f8 = e4m3;
+    a.layer_only = only;
+    a.L = n_layers;
+    a.C = n_chunks;
+    a.n_rows = n_rows;
+    a.ql.n_queries = n_queries;
+    for (int b = 0; b <= n_queries; ++b) a.ql.row0[b] = qo.row0[b];
+    for (int b = 0; b < n_queries; ++b) a.ql.len[b] = qo.off[b + 1] - qo.off[b];
+    a.m = m;
+    a.aux = reinterpret_cast<int2*>(ws + w.aux);
+    a.dev_err = dev_err;
+    a.pair = g_pair_mode;
+    int launches = 0;
+    const char* why = nullptr;
+    if (route_tc::launch(a, s, &launches, &why) != 0)
+      return msa_fail(MSA_ERR_CUDA, "tensor-core route: %s", why ? why : "launch failed");
+    g_launches += launches;
+    return msa_ok();
+  };
+
   if (n_chunks > 0) {
     if (g_prof_start) MSA_CUDA_TRY(cudaEventRecord(g_prof_start, s));
     if (!tensor) {
@@ -706,25 +761,8 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
       ++g_launches;
       MSA_CUDA_TRY(cudaGetLastError());
     } else {
-      route_tc::LaunchArgs a;
-      a.kr_hat = f8 ? kr_f8 : kr_hat;
-      a.qt = qt_bf16;
-      a.f8 = f8;
-      a.L = n_layers;
-      a.C = n_chunks;
-      a.n_rows = n_rows;
-      a.ql.n_queries = n_queries;
-      for (int b = 0; b <= n_queries; ++b) a.ql.row0[b] = qo.row0[b];
-      for (int b = 0; b < n_queries; ++b) a.ql.len[b] = qo.off[b + 1] - qo.off[b];
-      a.m = m;
-      a.aux = reinterpret_cast<int2*>(ws + w.aux);
-      a.dev_err = dev_err;
-      a.pair = g_pair_mode;
-      int launches = 0;
-      const char* why = nullptr;
-      if (route_tc::launch(a, s, &launches, &why) != 0)
-        return msa_fail(MSA_ERR_CUDA, "tensor-core route: %s", why ? why : "launch failed");
-      g_launches += launches;
+      const msa_status st = gemm(f8, nullptr);
+      if (st != MSA_OK) return st;
     }
     if (g_prof_stop) MSA_CUDA_TRY(cudaEventRecord(g_prof_stop, s));
   }
@@ -740,11 +778,11 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     if (mg_smem > 48 * 1024)
       MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
     docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
-        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, top_k, doc_pow2, cand);
+        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, top_k, doc_pow2, cand, nullptr);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, top_k, mg_pow2,
-                                                                            nullptr, out_ids, out_scores);
+                                                                            nullptr, out_ids, out_scores, nullptr);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     return msa_ok();
@@ -758,24 +796,37 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
   if (mg_smem > 48 * 1024)
     MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
-  docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
-      m, doc_chunk_offsets, n_docs, n_chunks, n_layers, K2, doc_pow2, cand);
-  ++g_launches;
-  MSA_CUDA_TRY(cudaGetLastError());
-  merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, K2, mg_pow2, apx,
-                                                                          nullptr, nullptr);
-  ++g_launches;
-  MSA_CUDA_TRY(cudaGetLastError());
   const size_t rs_smem = (size_t)kRescoreRows * H * kD * sizeof(float);
   MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs_smem));
-  rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, rs_smem, s>>>(
-      (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks, T_total, qo, doc_chunk_offsets, m,
-      reinterpret_cast<const int2*>(ws + w.aux), apx, K2, filter_err, exact);
-  ++g_launches;
-  MSA_CUDA_TRY(cudaGetLastError());
-  select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, filter_err,
-                                                               out_ids, out_scores, dev_err);
-  ++g_launches;
-  MSA_CUDA_TRY(cudaGetLastError());
+  // candidates -> exact rescoring -> final top-k (+ certification), on the layers `only`
+  // marks; uncertified layers go to redo_out when given
+  auto select = [&](float err, int32_t* redo_out, const int32_t* only) -> msa_status {
+    docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
+        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, K2, doc_pow2, cand, only);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, K2, mg_pow2,
+                                                                            apx, nullptr, nullptr, only);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, rs_smem, s>>>(
+        (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks, T_total, qo, doc_chunk_offsets, m,
+        reinterpret_cast<const int2*>(ws + w.aux), apx, K2, err, exact, only);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, err,
+                                                                 out_ids, out_scores, dev_err, redo_out, only);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    return msa_ok();
+  };
+  msa_status st = select(filter_err, f8 ? redo : nullptr, nullptr);
+  if (st != MSA_OK || !f8) return st;
+  // E4M3 layers that could not be certified: bf16 filter over them, then the same steps
+  // with the bf16 error bound (every kernel returns at once on certified layers)
+  st = gemm(false, redo);
+  if (st != MSA_OK) return st;
+  st = select(kFilterErr, nullptr, redo);
+  if (st != MSA_OK) return st;
   return msa_ok();
 }

@@ -275,7 +275,8 @@ template <int BN, bool PAIR, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int L,
                     long long C, int n_rows, int m_tiles, const __grid_constant__ QueryLayout ql,
-                    float* __restrict__ m_out, int2* __restrict__ aux_out, int32_t* dev_err) {
+                    float* __restrict__ m_out, int2* __restrict__ aux_out, int32_t* dev_err,
+                    const int32_t* __restrict__ layer_only) {
   using K = Cfg<BN, PAIR, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -334,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int u = first_unit; u < units && ok; u += unit_stride) {
         const int l = u / m_tiles, mt = u % m_tiles;
+        if (layer_only != nullptr && layer_only[l] == 0) continue;
         const int row_a = (int)((long long)l * C) + mt * K::kRows + (int)rank * kBM;
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
           const int row_b = l * n_rows + nt * BN + (int)rank * K::kBRows;
@@ -379,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
       for (int u = first_unit; u < units && ok; u += unit_stride) {
+        if (layer_only != nullptr && layer_only[u / m_tiles] == 0) continue;
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
           if (!mbar_wait(smem_u32(&acce[buf]), acc_phase ^ 1u, abort_flag)) {
             ok = false;
@@ -431,6 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int u = first_unit; u < units && ok; u += unit_stride) {
       const int l = u / m_tiles, mt = u % m_tiles;
+      if (layer_only != nullptr && layer_only[l] == 0) continue;
       const long long row = (long long)mt * K::kRows + (long long)rank * kBM + row_in_tile;
       const bool row_ok = row < C;
       int carry_b = -1;           // query whose columns continue into the next N tile
@@ -584,7 +588,7 @@ int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR, F8>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
-                         a.aux, a.dev_err) != cudaSuccess) {
+                         a.aux, a.dev_err, a.layer_only) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
   }

@@ -63,6 +63,7 @@ struct LaunchArgs {
   int32_t* dev_err;
   bool pair;           // M=256 tiles on CTA pairs (cta_group::2) for N tiles of 128 / 256
   bool f8;             // E4M3 operands (kind::f8f6f4)
+  const int32_t* layer_only = nullptr;  // DEVICE [L]: when given, layers marked 0 are skipped
 };
 
 // Enqueues the score kernel; returns 0 on success (launches += kernels enqueued).
