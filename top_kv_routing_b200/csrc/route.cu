@@ -15,9 +15,10 @@
 //   3. docmax   S[doc] = max of m over the document's blocks; per-CTA best candidates
 //   4. merge    the per-CTA candidates -> top_k (scan) or the K2 filter candidates (tensor)
 //   tensor path only:
-//   5. rescore  exact fp32 scores of the K2 candidates, evaluating only the (block, token)
-//               pairs whose filter score lies within the filter's error window of the max
-//   6. final    top_k of the exact scores; certification of the selection
+//   5. rescore  exact scores of the K2 candidates: every block of the document against
+//               every token of the query, on the tensor cores with ~fp32 operands
+//   6. final    top_k of the exact scores; certification of the selection (E4M3: layers
+//               that fail go through steps 2-6 again with the bf16 filter)
 // The score matrix s[t][c] only ever lives in registers / TMEM.
 #include <cuda_fp8.h>
 
@@ -37,9 +38,9 @@ constexpr int kTopkThreads = 512;
 constexpr int kMaxDocs = 1 << 20;    // documents per bank
 constexpr int kMaxBlocks = 64;       // docmax CTAs per (query, layer)
 // Error bound assumed for the tensor-core filter scores (bf16 operands, fp32 accumulate):
-// the observed error is ~1e-4 (3e-4 worst seen), this is ~10 standard deviations.  Pairs
-// within 2x of it from a block's best are rescored; a selection is certified when the
-// k-th exact score beats the best filter score left out by more than it.
+// the observed error is ~1e-4 (3e-4 worst seen), this is ~10 standard deviations.  A
+// selection is certified when the k-th exact score beats the best filter score left out
+// by more than it.
 constexpr float kFilterErr = 1e-3f;
 // The same for the E4M3 filter (3 mantissa bits on both operands): rms error ~8e-4,
 // largest seen ~5e-3 over 8M (block, token) pairs of bank-like data; 2^-6 is ~19 rms.
@@ -78,7 +79,7 @@ int pow2_at_least(int n) {
 }
 
 struct WsLayout {
-  size_t qt_f32, qt_bf16, qt_f8, m, aux, cand, apx, exact, redo, total;
+  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, aux, cand, apx, exact, redo, total;
   int n_pad;
   int nblk;
   int k2;
@@ -100,6 +101,8 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   w.qt_f32 = o;
   o += align256((size_t)L * T_total * H * kD * sizeof(float));
   w.qt_bf16 = o;
+  o += align256((size_t)L * w.n_pad * H * kD * 2);
+  w.qt_lo = o;
   o += align256((size_t)L * w.n_pad * H * kD * 2);
   w.qt_f8 = o;
   o += align256((size_t)L * w.n_pad * H * kD);
@@ -125,8 +128,8 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
 __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr, int q_is_bf16, int T_total,
                                                     int Hq, int H, int n_rows, QueryOffsets qo,
                                                     float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16,
-                                                    uint8_t* __restrict__ qt_f8, int32_t* __restrict__ redo,
-                                                    int n_layers) {
+                                                    __nv_bfloat16* __restrict__ qt_lo, uint8_t* __restrict__ qt_f8,
+                                                    int32_t* __restrict__ redo, int n_layers) {
   __shared__ float qhat[64][kD];
   const int t = blockIdx.x, l = blockIdx.y;
   if (redo != nullptr && t == 0 && l == 0)
@@ -170,33 +173,40 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
     float acc = 0.f;
     for (int u = 0; u < G; ++u) acc += qhat[g * G + u][j];
     acc *= inv_hq;
-    qt_f32[((int64_t)l * T_total + t) * H * kD + e] = acc;
-    if (qt_bf16 != nullptr) qt_bf16[((int64_t)l * n_rows + orow) * H * kD + e] = __float2bfloat16_rn(acc);
-    if (qt_f8 != nullptr)
-      qt_f8[((int64_t)l * n_rows + orow) * H * kD + e] =
-          __nv_cvt_float_to_fp8(acc * route_tc::kF8QueryScale, __NV_SATFINITE, __NV_E4M3);
+    if (qt_f32 != nullptr) qt_f32[((int64_t)l * T_total + t) * H * kD + e] = acc;
+    const int64_t oi = ((int64_t)l * n_rows + orow) * H * kD + e;
+    if (qt_bf16 != nullptr) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+      qt_bf16[oi] = hi;
+      if (qt_lo != nullptr) qt_lo[oi] = __float2bfloat16_rn(acc - __bfloat162float(hi));
+    }
+    if (qt_f8 != nullptr) qt_f8[oi] = __nv_cvt_float_to_fp8(acc * route_tc::kF8QueryScale, __NV_SATFINITE, __NV_E4M3);
   }
 }
 
 // Zero every operand row that holds no query token (per-query alignment gaps and the
-// tail up to n_rows), in 16-byte words.
-// (a second buffer with rows of words_per_row2 words is padded the same way when given)
-__global__ void zero_pad_kernel(uint4* __restrict__ qt, int n_rows, int words_per_row, int L, QueryOffsets qo,
-                                uint4* __restrict__ qt2, int words_per_row2) {
-  const int64_t total = (int64_t)L * n_rows * words_per_row;
-  const int64_t total2 = qt2 != nullptr ? (int64_t)L * n_rows * words_per_row2 : 0;
-  const int64_t all = total + total2;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < all; i += (int64_t)gridDim.x * blockDim.x) {
-    const bool second = i >= total;
-    const int64_t j = second ? i - total : i;
-    const int r = (int)((j / (second ? words_per_row2 : words_per_row)) % n_rows);
-    int lo = 0, hi = qo.n;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (qo.row0[mid] <= r) lo = mid; else hi = mid;
+// tail up to n_rows), in 16-byte words, in up to three operand buffers.
+struct PadTargets {
+  uint4* buf[3];
+  int words_per_row[3];
+};
+
+__global__ void zero_pad_kernel(PadTargets pt, int n_rows, int L, QueryOffsets qo) {
+  for (int k = 0; k < 3; ++k) {
+    if (pt.buf[k] == nullptr) continue;
+    const int wpr = pt.words_per_row[k];
+    const int64_t total = (int64_t)L * n_rows * wpr;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+      const int r = (int)((i / wpr) % n_rows);
+      int lo = 0, hi = qo.n;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (qo.row0[mid] <= r) lo = mid; else hi = mid;
+      }
+      const bool token_row = r < qo.row0[qo.n] && (r - qo.row0[lo]) < (qo.off[lo + 1] - qo.off[lo]);
+      if (!token_row) pt.buf[k][i] = make_uint4(0u, 0u, 0u, 0u);
     }
-    const bool token_row = r < qo.row0[qo.n] && (r - qo.row0[lo]) < (qo.off[lo + 1] - qo.off[lo]);
-    if (!token_row) (second ? qt2 : qt)[j] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -441,108 +451,149 @@ __global__ void __launch_bounds__(kTopkThreads) merge_topk_kernel(const unsigned
 }
 
 // ---------------------------------------------------------------------------- 2c. exact rescoring
-// grid (K2, L, B), 128 threads: exact fp32 score of filter candidate r of (b, l).  The
-// document's exact best (block, token) pair has a filter score within 2E of the
-// document's filter maximum and within 2E of its block's filter maximum, so only blocks
-// with m >= max - 2E are visited: in those, the argmax token alone when the runner-up is
-// more than 2E below, else every token of the query.  Blocks of the second kind are
-// staged (unit rows, fp32) in shared memory kRescoreRows at a time so that each query
-// token row is read once per group.
-constexpr int kRescoreRows = 16;
+// grid (K2, L, B), 128 threads: the exact score of filter candidate r of (b, l), i.e. the
+// maximum over all of the document's blocks and all of the query's tokens of
+//   s[t][c] = sum_h rho[c][h] * < qt[t][h], k[c][h] >,  rho = 1 / max(||k[c][h]||, 1e-8)
+// with k the stored bf16 keys.  The dots run on the tensor cores (mma.sync m16n8k16,
+// fp32 accumulate): A = 16 blocks of keys (exact in bf16), B = 8 query tokens carried as
+// bf16(qt) plus its bf16 residual (two MMAs, ~16 mantissa bits of qt); each head's dot is
+// scaled by rho in fp32 and summed over the heads.
+//
+// K-dimension order: MMA k-step ks covers head h = ks / 8, and within it thread t's four
+// k-indices {2t, 2t+1, 2t+8, 2t+9} are the memory dims 128h + 32t + 4(ks % 8) + {0..3},
+// so every thread reads each query token with 16-byte loads; the key tile is written to
+// shared memory in the same order (rows of 64 k-steps x 32 bytes, 16-byte chunks XOR-
+// swizzled by row for conflict-free ldmatrix).
+constexpr int kRsRows = 16;  // key blocks per tile (MMA M)
 
-template <int NV>
-__global__ void __launch_bounds__(128) rescore_kernel(const __nv_bfloat16* __restrict__ kr_hat,
-                                                      const float* __restrict__ qt, int L, int64_t C, int T_total,
-                                                      QueryOffsets qo, const int64_t* __restrict__ doc_chunk_off,
-                                                      const float* __restrict__ m, const int2* __restrict__ aux,
-                                                      const unsigned long long* __restrict__ apx, int K2, float err,
-                                                      float* __restrict__ exact, const int32_t* __restrict__ only) {
-  constexpr int R = NV * 256;
-  extern __shared__ float4 rows[];  // [kRescoreRows][R / 4] in lane-vector order
+__device__ __forceinline__ void rs_ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void rs_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(128) rescore_mma_kernel(const __nv_bfloat16* __restrict__ kr_hat,
+                                                          const __nv_bfloat16* __restrict__ q_hi,
+                                                          const __nv_bfloat16* __restrict__ q_lo, int L, int64_t C,
+                                                          int n_rows, QueryOffsets qo,
+                                                          const int64_t* __restrict__ doc_chunk_off,
+                                                          const unsigned long long* __restrict__ apx, int K2,
+                                                          float* __restrict__ exact,
+                                                          const int32_t* __restrict__ only) {
+  constexpr int kRowBytes = 8 * kD * 2;  // 2048
+  __shared__ __align__(128) uint8_t ktile[kRsRows * kRowBytes];
+  __shared__ float rho[kRsRows][8];
   __shared__ float red[4];
-  __shared__ int full_list[kRescoreRows];
-  __shared__ int n_full;
   const int r = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
   if (only != nullptr && only[l] == 0) return;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t o = ((int64_t)b * L + l) * K2 + r;
   int doc;
   float doc_apx;
   split_key(apx[o], &doc, &doc_apx);
   if (doc < 0) {
-    if (threadIdx.x == 0) exact[o] = -INFINITY;
+    if (tid == 0) exact[o] = -INFINITY;
     return;
   }
   const int64_t c0 = doc_chunk_off[doc], c1 = doc_chunk_off[doc + 1];
-  const int64_t mrow = ((int64_t)b * L + l) * C;
-  const float* qbase = qt + (int64_t)l * T_total * R;
-  const float window = 2.0f * err;
+  const int T = qo.off[b + 1] - qo.off[b];
+  const int n_tiles = (T + 7) / 8;
+  const int64_t qrow0 = (int64_t)l * n_rows + qo.row0[b];
+  const uint32_t kt_base = static_cast<uint32_t>(__cvta_generic_to_shared(ktile));
   float best = -INFINITY;
-  // blocks are scanned in windows of 4 * kRescoreRows; each window's full-scan blocks
-  // (at most kRescoreRows per pass) are collected, staged and scanned together
-  for (int64_t w0 = c0; w0 < c1; w0 += kRescoreRows) {
-    if (threadIdx.x == 0) n_full = 0;
-    __syncthreads();
-    for (int64_t c = w0 + warp; c < min(c1, w0 + kRescoreRows); c += 4) {
-      const float m1 = m[mrow + c];
-      if (!(m1 >= doc_apx - window)) continue;
-      const int2 ax = aux[mrow + c];
-      const float m2 = __int_as_float(ax.x);
-      if (m2 < m1 - window) {
-        float kx[NV][8];
-        load_unit_row<NV>(kr_hat + ((int64_t)l * C + c) * R, lane, kx);
-        const int t = qo.off[b] + ax.y;
-        best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
-      } else if (lane == 0) {
-        full_list[atomicAdd(&n_full, 1)] = (int)(c - w0);
+  for (int64_t g0 = c0; g0 < c1; g0 += kRsRows) {
+    const int nb = (int)(c1 - g0 < kRsRows ? c1 - g0 : kRsRows);
+    // stage the key tile in MMA k order: 16-byte chunk m' of a row holds memory dims
+    // 8m' .. 8m'+7 = head h, thread t', k-steps 2m, 2m+1 (dims 4 apart per k-step)
+    for (int i = tid; i < kRsRows * 128; i += blockDim.x) {
+      const int row = i >> 7, mp = i & 127;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (row < nb) w = __ldg(reinterpret_cast<const uint4*>(kr_hat + ((int64_t)l * C + g0 + row) * 8 * kD) + mp);
+      const int h = mp >> 4, tp = (mp >> 2) & 3, m = mp & 3;
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int ks = 8 * h + 2 * m + (j >> 1), half = j & 1;  // word j: dims 2j, 2j+1 of the chunk
+        const int chunk = (2 * ks + half) ^ (row & 7);
+        *reinterpret_cast<uint32_t*>(ktile + row * kRowBytes + chunk * 16 + tp * 4) = wv[j];
       }
     }
     __syncthreads();
-    const int nf = n_full;
-    if (nf == 0) continue;
-    for (int rr = warp; rr < nf; rr += 4) {
-      float kx[NV][8];
-      load_unit_row<NV>(kr_hat + ((int64_t)l * C + w0 + full_list[rr]) * R, lane, kx);
+    {  // 1 / ||k|| per (row, head): a head is 16 whole chunks of the row, in any order
+      const int row = tid >> 3, h = tid & 7;
+      const uint4* src = reinterpret_cast<const uint4*>(ktile + row * kRowBytes + h * 256);
+      float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        rows[rr * (R / 4) + 2 * (lane + 32 * i)] = make_float4(kx[i][0], kx[i][1], kx[i][2], kx[i][3]);
-        rows[rr * (R / 4) + 2 * (lane + 32 * i) + 1] = make_float4(kx[i][4], kx[i][5], kx[i][6], kx[i][7]);
+      for (int i = 0; i < 16; ++i) {
+        const uint4 w = src[i];
+        const float2 f0 = msa::bf16x2_to_float2(w.x), f1 = msa::bf16x2_to_float2(w.y);
+        const float2 f2 = msa::bf16x2_to_float2(w.z), f3 = msa::bf16x2_to_float2(w.w);
+        ss = fmaf(f0.x, f0.x, ss); ss = fmaf(f0.y, f0.y, ss); ss = fmaf(f1.x, f1.x, ss); ss = fmaf(f1.y, f1.y, ss);
+        ss = fmaf(f2.x, f2.x, ss); ss = fmaf(f2.y, f2.y, ss); ss = fmaf(f3.x, f3.x, ss); ss = fmaf(f3.y, f3.y, ss);
       }
+      rho[row][h] = 1.0f / fmaxf(sqrtf(ss), 1e-8f);
     }
     __syncthreads();
-    for (int t = qo.off[b] + warp; t < qo.off[b + 1]; t += 4) {
-      const float4* qv = reinterpret_cast<const float4*>(qbase + (int64_t)t * R);
-      float q[NV][8];
+    // lane's ldmatrix row: matrix (lane >> 3): rows 0-7 / 8-15, k-indices 0-7 / 8-15
+    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lhalf = lane >> 4;
+    const uint32_t arow = kt_base + lrow * kRowBytes;
+    for (int nt = warp; nt < n_tiles; nt += 4) {
+      const int tok = 8 * nt + g;  // this lane's B column (token); padded rows are zero
+      const uint4* qh = reinterpret_cast<const uint4*>(q_hi + (qrow0 + tok) * 8 * kD) + 4 * t;
+      const uint4* ql = reinterpret_cast<const uint4*>(q_lo + (qrow0 + tok) * 8 * kD) + 4 * t;
+      float tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+      for (int h = 0; h < 8; ++h) {
+        uint4 xh[4], xl[4];  // dims 128h + 32t .. +32 of token tok
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const float4 x = __ldg(qv + 2 * (lane + 32 * i));
-        const float4 y = __ldg(qv + 2 * (lane + 32 * i) + 1);
-        q[i][0] = x.x; q[i][1] = x.y; q[i][2] = x.z; q[i][3] = x.w;
-        q[i][4] = y.x; q[i][5] = y.y; q[i][6] = y.z; q[i][7] = y.w;
-      }
-      for (int rr = 0; rr < nf; ++rr) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-          const float4 x = rows[rr * (R / 4) + 2 * (lane + 32 * i)];
-          const float4 y = rows[rr * (R / 4) + 2 * (lane + 32 * i) + 1];
-          acc = fmaf(q[i][0], x.x, acc);
-          acc = fmaf(q[i][1], x.y, acc);
-          acc = fmaf(q[i][2], x.z, acc);
-          acc = fmaf(q[i][3], x.w, acc);
-          acc = fmaf(q[i][4], y.x, acc);
-          acc = fmaf(q[i][5], y.y, acc);
-          acc = fmaf(q[i][6], y.z, acc);
-          acc = fmaf(q[i][7], y.w, acc);
+        for (int m = 0; m < 4; ++m) {
+          xh[m] = __ldg(qh + 16 * h + m);
+          xl[m] = __ldg(ql + 16 * h + m);
         }
-        best = fmaxf(best, warp_sum(acc));
+        float acc_h[4] = {0.f, 0.f, 0.f, 0.f}, acc_l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int ks = 8 * h + kk;
+          uint32_t a[4];
+          rs_ldsm_x4(arow + (((2 * ks + lhalf) ^ (lrow & 7)) << 4), a);
+          const uint4& vh = xh[kk >> 1];
+          const uint4& vl = xl[kk >> 1];
+          if (kk & 1) {
+            rs_mma(acc_h, a, vh.z, vh.w);
+            rs_mma(acc_l, a, vl.z, vl.w);
+          } else {
+            rs_mma(acc_h, a, vh.x, vh.y);
+            rs_mma(acc_l, a, vl.x, vl.y);
+          }
+        }
+        const float ra = rho[g][h], rb = rho[g + 8][h];
+        tot[0] = fmaf(ra, acc_h[0] + acc_l[0], tot[0]);
+        tot[1] = fmaf(ra, acc_h[1] + acc_l[1], tot[1]);
+        tot[2] = fmaf(rb, acc_h[2] + acc_l[2], tot[2]);
+        tot[3] = fmaf(rb, acc_h[3] + acc_l[3], tot[3]);
       }
+      // C: rows (blocks) g / g+8, columns (tokens) 8nt + 2t + {0, 1}
+      const int t0 = 8 * nt + 2 * t;
+      const bool r0 = g < nb, r1 = g + 8 < nb;
+      if (r0 && t0 < T) best = fmaxf(best, tot[0]);
+      if (r0 && t0 + 1 < T) best = fmaxf(best, tot[1]);
+      if (r1 && t0 < T) best = fmaxf(best, tot[2]);
+      if (r1 && t0 + 1 < T) best = fmaxf(best, tot[3]);
     }
-    __syncthreads();
+    __syncthreads();  // before the tile is restaged
   }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, s));
   if (lane == 0) red[warp] = best;
   __syncthreads();
-  if (threadIdx.x == 0) exact[o] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  if (tid == 0) exact[o] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
 }
 
 // grid (L, B), 128 threads: final top-k of the K2 exactly rescored candidates.  The
@@ -705,17 +756,25 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   const float filter_err = f8 ? kFilterErrF8 : kFilterErr;
 
   uint8_t* qt_f8 = reinterpret_cast<uint8_t*>(ws + w.qt_f8);
+  __nv_bfloat16* qt_lo = reinterpret_cast<__nv_bfloat16*>(ws + w.qt_lo);
   int32_t* redo = reinterpret_cast<int32_t*>(ws + w.redo);
   if (tensor) {
-    // the E4M3 pass also prepares the bf16 operand, for layers it cannot certify
-    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(reinterpret_cast<uint4*>(qt_bf16), n_rows, H * kD * 2 / 16,
-                                                         n_layers, qo, f8 ? reinterpret_cast<uint4*>(qt_f8) : nullptr,
-                                                         H * kD / 16);
+    // operand rows: bf16 (GEMM, and the high half of the exact rescoring), its residual
+    // (the low half) and, on the E4M3 path, E4M3
+    PadTargets pt;
+    pt.buf[0] = reinterpret_cast<uint4*>(qt_bf16);
+    pt.words_per_row[0] = H * kD * 2 / 16;
+    pt.buf[1] = reinterpret_cast<uint4*>(qt_lo);
+    pt.words_per_row[1] = H * kD * 2 / 16;
+    pt.buf[2] = f8 ? reinterpret_cast<uint4*>(qt_f8) : nullptr;
+    pt.words_per_row[2] = H * kD / 16;
+    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(pt, n_rows, n_layers, qo);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
   qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
-                                                      qt_f32, tensor ? qt_bf16 : nullptr, f8 ? qt_f8 : nullptr,
+                                                      tensor ? nullptr : qt_f32, tensor ? qt_bf16 : nullptr,
+                                                      tensor ? qt_lo : nullptr, f8 ? qt_f8 : nullptr,
                                                       f8 ? redo : nullptr, n_layers);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
@@ -796,8 +855,6 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
   if (mg_smem > 48 * 1024)
     MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
-  const size_t rs_smem = (size_t)kRescoreRows * H * kD * sizeof(float);
-  MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs_smem));
   // candidates -> exact rescoring -> final top-k (+ certification), on the layers `only`
   // marks; uncertified layers go to redo_out when given
   auto select = [&](float err, int32_t* redo_out, const int32_t* only) -> msa_status {
@@ -809,9 +866,9 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
                                                                             apx, nullptr, nullptr, only);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
-    rescore_kernel<4><<<dim3(K2, n_layers, n_queries), 128, rs_smem, s>>>(
-        (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks, T_total, qo, doc_chunk_offsets, m,
-        reinterpret_cast<const int2*>(ws + w.aux), apx, K2, err, exact, only);
+    rescore_mma_kernel<<<dim3(K2, n_layers, n_queries), 128, 0, s>>>(
+        (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx, K2,
+        exact, only);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, err,

@@ -40,6 +40,7 @@ constexpr int kRowBytes = 128;           // one swizzled shared-memory row per K
 constexpr int kKDim = 1024;              // 8 key heads x 128
 constexpr int kABytes = kBM * kRowBytes; // 16 KB
 constexpr int kThreads = 192;
+constexpr int kMaskLayers = 64;          // layer-mask entries kept in shared memory
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 template <int BN, bool PAIR, bool F8>
@@ -296,6 +297,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int first_unit = PAIR ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
   const int unit_stride = PAIR ? (int)(gridDim.x / 2) : (int)gridDim.x;
+  // with a layer mask: nothing to do returns before any set-up (every CTA of a pair reads
+  // the same mask); otherwise whole masked layers are stepped over, the same way by every role
+  __shared__ int s_active[kMaskLayers];
+  if (layer_only != nullptr) {
+    int any = 0;
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+      const int a = layer_only[i] != 0;
+      if (i < kMaskLayers) s_active[i] = a;
+      any |= a;
+    }
+    if (!__syncthreads_or(any)) return;
+  }
+  auto active = [&](int l) -> bool {
+    return layer_only == nullptr || (l < kMaskLayers ? s_active[l] != 0 : layer_only[l] != 0);
+  };
+  // the first unit >= u of this CTA's sequence (first_unit + i * unit_stride) in an active layer
+  auto next_active = [&](int u) -> int {
+    while (u < units && !active(u / m_tiles)) {
+      const int nxt = (u / m_tiles + 1) * m_tiles;
+      u = nxt + ((first_unit - nxt) % unit_stride + unit_stride) % unit_stride;
+    }
+    return u;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < K::kStages; ++s) {
@@ -333,9 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = first_unit; u < units && ok; u += unit_stride) {
+      for (int u = next_active(first_unit); u < units && ok; u = next_active(u + unit_stride)) {
         const int l = u / m_tiles, mt = u % m_tiles;
-        if (layer_only != nullptr && layer_only[l] == 0) continue;
         const int row_a = (int)((long long)l * C) + mt * K::kRows + (int)rank * kBM;
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
           const int row_b = l * n_rows + nt * BN + (int)rank * K::kBRows;
@@ -380,8 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, buf = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
-      for (int u = first_unit; u < units && ok; u += unit_stride) {
-        if (layer_only != nullptr && layer_only[u / m_tiles] == 0) continue;
+      for (int u = next_active(first_unit); u < units && ok; u = next_active(u + unit_stride)) {
         for (int nt = 0; nt < n_tiles && ok; ++nt) {
           if (!mbar_wait(smem_u32(&acce[buf]), acc_phase ^ 1u, abort_flag)) {
             ok = false;
@@ -432,9 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = first_unit; u < units && ok; u += unit_stride) {
+    for (int u = next_active(first_unit); u < units && ok; u = next_active(u + unit_stride)) {
       const int l = u / m_tiles, mt = u % m_tiles;
-      if (layer_only != nullptr && layer_only[l] == 0) continue;
       const long long row = (long long)mt * K::kRows + (long long)rank * kBM + row_in_tile;
       const bool row_ok = row < C;
       int carry_b = -1;           // query whose columns continue into the next N tile
