@@ -35,7 +35,7 @@ TOKENS_PER_DOC = 1000
 THETA = 1e6
 # DRAM bytes per (block, layer) of the routing GEMM, read + write, from the ncu captures in
 # profiles/ (2M-token bank, same kernels), scaled by blocks; None where not captured yet.
-GEMM_TRAFFIC_PER_BLOCK_LAYER = {"bf16": 2074.5, "e4m3": None}
+GEMM_TRAFFIC_PER_BLOCK_LAYER = {"bf16": None, "e4m3": 1039.8}
 
 
 def log(*a):

@@ -10,8 +10,7 @@
 //   2. score    m[b][l][c] = max_{t in b} cos-score(t, c)
 //               scan path (few tokens): exact fp32 on CUDA cores, keys normalised per head
 //               tensor path: tcgen05 GEMM on bf16 operands, or on the E4M3 filter copy of
-//               the keys (a filter; also the runner-up score and the argmax token of each
-//               block)
+//               the keys (a filter)
 //   3. docmax   S[doc] = max of m over the document's blocks; per-CTA best candidates
 //   4. merge    the per-CTA candidates -> top_k (scan) or the K2 filter candidates (tensor)
 //   tensor path only:
@@ -79,7 +78,7 @@ int pow2_at_least(int n) {
 }
 
 struct WsLayout {
-  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, aux, cand, apx, exact, redo, total;
+  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, cand, apx, exact, redo, total;
   int n_pad;
   int nblk;
   int k2;
@@ -108,8 +107,6 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   o += align256((size_t)L * w.n_pad * H * kD);
   w.m = o;
   o += align256((size_t)B * L * (size_t)C * sizeof(float));
-  w.aux = o;
-  o += align256((size_t)B * L * (size_t)C * sizeof(int2));
   w.cand = o;
   o += align256((size_t)B * L * w.nblk * ksel * sizeof(unsigned long long));
   w.apx = o;
@@ -793,7 +790,6 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     for (int b = 0; b <= n_queries; ++b) a.ql.row0[b] = qo.row0[b];
     for (int b = 0; b < n_queries; ++b) a.ql.len[b] = qo.off[b + 1] - qo.off[b];
     a.m = m;
-    a.aux = reinterpret_cast<int2*>(ws + w.aux);
     a.dev_err = dev_err;
     a.pair = g_pair_mode;
     int launches = 0;

@@ -8,8 +8,7 @@
 // bf16 or 128 E4M3 elements and one MMA consumes 32 bytes of K either way, so both
 // forms share the tiling, swizzle and descriptors; E4M3 halves the K-blocks per tile.
 // The epilogue reduces each row over the columns of every query and writes, per (query,
-// layer, block), the largest score m, the second largest and the argmax token; D itself
-// never leaves TMEM.  These low-precision scores are a filter: the caller rescores the
+// layer, block), the largest score m; D itself never leaves TMEM.  These low-precision scores are a filter: the caller rescores the
 // pairs that can hold the maximum exactly.
 //
 // Warp roles of the persistent kernel (192 threads, one CTA per SM):
@@ -17,8 +16,8 @@
 //               K-block into a ring of shared-memory stages (128-byte swizzle)
 //   warp 1      one thread issues tcgen05.mma (fp32 accumulate, 32 bytes of K each) into one of
 //               two TMEM accumulators and commits stage / accumulator completion to mbarriers
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max / runner-up / argmax over
-//               each query's columns, store; then release the accumulator
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max over each query's columns,
+//               store; then release the accumulator
 // Paired mode (PAIR, for N tiles of 128 and 256): a cluster of two CTAs on two SMs runs
 // M=256 tiles with tcgen05.mma.cta_group::2.  Each CTA loads its 128 key rows and half of
 // the query tile, so each SM streams half the query bytes per key byte of the single-CTA
@@ -276,7 +275,7 @@ template <int BN, bool PAIR, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int L,
                     long long C, int n_rows, int m_tiles, const __grid_constant__ QueryLayout ql,
-                    float* __restrict__ m_out, int2* __restrict__ aux_out, int32_t* dev_err,
+                    float* __restrict__ m_out, int32_t* dev_err,
                     const int32_t* __restrict__ layer_only) {
   using K = Cfg<BN, PAIR, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -459,8 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long row = (long long)mt * K::kRows + (long long)rank * kBM + row_in_tile;
       const bool row_ok = row < C;
       int carry_b = -1;           // query whose columns continue into the next N tile
-      float c1 = -INFINITY, c2 = -INFINITY;
-      int ci = 0;
+      float carry_m = -INFINITY;
       for (int nt = 0; nt < n_tiles; ++nt) {
         if (!mbar_wait(smem_u32(&accf[buf]), acc_phase, abort_flag)) {
           ok = false;
@@ -489,32 +487,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = lo;
             const int t0 = col0 - ql.row0[b];  // token index of column col0 in query b
             const int valid = min(32, ql.len[b] - t0);
-            float m1 = -INFINITY, m2 = -INFINITY;
-            int i1 = 0;
-            if (b == carry_b) {
-              m1 = c1;
-              m2 = c2;
-              i1 = ci;
-            }
+            const uint32_t* r = half ? rb : ra;
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (valid == 32) {  // (the same for every lane: a slice spans all the rows)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = i < valid ? __uint_as_float(half ? rb[i] : ra[i]) : -INFINITY;
-              m2 = fmaxf(m2, fminf(m1, x));
-              i1 = x > m1 ? t0 + i : i1;
-              m1 = fmaxf(m1, x);
+              for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (i < valid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
             }
+            float m1 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            if (b == carry_b) m1 = fmaxf(m1, carry_m);
             if (t0 + 32 >= ql.len[b]) {
-              if (row_ok) {
-                const long long o = ((long long)b * L + l) * C + row;
-                m_out[o] = F8 ? m1 * kF8ScoreScale : m1;
-                aux_out[o] = make_int2(__float_as_int(F8 ? m2 * kF8ScoreScale : m2), i1);
-              }
+              if (row_ok) m_out[((long long)b * L + l) * C + row] = F8 ? m1 * kF8ScoreScale : m1;
               carry_b = -1;
             } else {
               carry_b = b;
-              c1 = m1;
-              c2 = m2;
-              ci = i1;
+              carry_m = m1;
             }
           }
         }
@@ -609,7 +599,7 @@ int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR, F8>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
-                         a.aux, a.dev_err, a.layer_only) != cudaSuccess) {
+                         a.dev_err, a.layer_only) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
   }

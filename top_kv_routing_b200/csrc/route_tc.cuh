@@ -59,7 +59,6 @@ struct LaunchArgs {
   int n_rows;          // operand rows per layer (multiple of the N tile)
   QueryLayout ql;
   float* m;            // [B][L][C]  approximate max over the query's tokens
-  int2* aux;           // [B][L][C]  (bits of the second-largest score, argmax token in the query)
   int32_t* dev_err;
   bool pair;           // M=256 tiles on CTA pairs (cta_group::2) for N tiles of 128 / 256
   bool f8;             // E4M3 operands (kind::f8f6f4)
