@@ -295,9 +295,10 @@ def test_route_auto_picks_tensor_for_long_query_and_scan_for_short(msa):
     _, kr_hat, coffs = _route_bank(bank, 1)
     C = bank.n_chunks
     kr_f8 = _filter_keys(msa, kr_hat)
-    # scan: qprep + scan + 2 top-k; tensor: zero-pad + qprep + GEMM + 2 top-k + rescore + final;
-    # E4M3: the same plus the bf16 pass over uncertified layers (GEMM + 2 top-k + rescore + final)
-    for T, f8, expect in ((4, None, 4), (40, None, 7), (4, kr_f8, 4), (40, kr_f8, 12)):
+    # scan: qprep + scan + 2 top-k; tensor: prep + qprep + GEMM + top-k + rescore + final;
+    # E4M3: the same plus the bf16 pass over uncertified layers (reset + GEMM + top-k +
+    # rescore + final)
+    for T, f8, expect in ((4, None, 4), (40, None, 6), (4, kr_f8, 4), (40, kr_f8, 11)):
         ws = torch.empty(msa.msa_route_topk_workspace_size(1, 1, T, H, C, 60, 16), dtype=torch.uint8, device="cuda")
         ids = torch.empty((1, 1, 16), dtype=torch.int32, device="cuda")
         sc = torch.empty((1, 1, 16), device="cuda")

@@ -11,8 +11,11 @@
 //               scan path (few tokens): exact fp32 on CUDA cores, keys normalised per head
 //               tensor path: tcgen05 GEMM on bf16 operands, or on the E4M3 filter copy of
 //               the keys (a filter)
-//   3. docmax   S[doc] = max of m over the document's blocks; per-CTA best candidates
-//   4. merge    the per-CTA candidates -> top_k (scan) or the K2 filter candidates (tensor)
+//   3. docmax   scan path: S[doc] = max of m over the document's blocks; per-CTA best
+//               candidates.  Tensor path: the GEMM epilogue folds every block's maximum
+//               into its document's score directly (atomicMax), no block scores stored
+//   4. merge    scan path: the per-CTA candidates -> top_k.  Tensor path: radix selection
+//               of the K2 filter candidates from the document scores
 //   tensor path only:
 //   5. rescore  exact scores of the K2 candidates: every block of the document against
 //               every token of the query, on the tensor cores with ~fp32 operands
@@ -78,7 +81,7 @@ int pow2_at_least(int n) {
 }
 
 struct WsLayout {
-  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, cand, apx, exact, redo, total;
+  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, cand, apx, exact, redo, doc_score, block_doc, total;
   int n_pad;
   int nblk;
   int k2;
@@ -115,6 +118,10 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(float));
   w.redo = o;
   o += align256((size_t)L * sizeof(int32_t));
+  w.doc_score = o;
+  o += align256((size_t)B * L * (size_t)(n_docs > 0 ? n_docs : 1) * sizeof(uint32_t));
+  w.block_doc = o;
+  o += align256((size_t)(C > 0 ? C : 1) * sizeof(int32_t));
   w.total = o;
   return w;
 }
@@ -181,20 +188,30 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
   }
 }
 
+// Document scores are kept as the ordered bits of make_key's high word (monotonic as
+// unsigned ints, so atomicMax works on them); this is -inf, a document with no block.
+constexpr uint32_t kOrdNegInf = 0x007FFFFFu;
+
 // Zero every operand row that holds no query token (per-query alignment gaps and the
-// tail up to n_rows), in 16-byte words, in up to three operand buffers.
+// tail up to n_rows), in 16-byte words, in up to three operand buffers; on the tensor
+// path also write the block -> document map and set every (query, layer, document)
+// score to -inf.
 struct PadTargets {
   uint4* buf[3];
   int words_per_row[3];
 };
 
-__global__ void zero_pad_kernel(PadTargets pt, int n_rows, int L, QueryOffsets qo) {
+__global__ void route_prep_kernel(PadTargets pt, int n_rows, int L, QueryOffsets qo,
+                                  const int64_t* __restrict__ doc_chunk_off, int n_docs,
+                                  int32_t* __restrict__ block_doc, uint32_t* __restrict__ doc_score,
+                                  int64_t n_scores) {
+  const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int k = 0; k < 3; ++k) {
     if (pt.buf[k] == nullptr) continue;
     const int wpr = pt.words_per_row[k];
     const int64_t total = (int64_t)L * n_rows * wpr;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t i = i0; i < total; i += stride) {
       const int r = (int)((i / wpr) % n_rows);
       int lo = 0, hi = qo.n;
       while (hi - lo > 1) {
@@ -205,6 +222,20 @@ __global__ void zero_pad_kernel(PadTargets pt, int n_rows, int L, QueryOffsets q
       if (!token_row) pt.buf[k][i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  if (block_doc != nullptr)
+    for (int64_t d = i0; d < n_docs; d += stride)
+      for (int64_t c = doc_chunk_off[d]; c < doc_chunk_off[d + 1]; ++c) block_doc[c] = (int32_t)d;
+  if (doc_score != nullptr)
+    for (int64_t i = i0; i < n_scores; i += stride) doc_score[i] = kOrdNegInf;
+}
+
+// grid (L, B): the document scores of the layers `only` marks back to -inf
+__global__ void doc_reset_kernel(uint32_t* __restrict__ doc_score, int L, int n_docs,
+                                 const int32_t* __restrict__ only) {
+  const int l = blockIdx.x, b = blockIdx.y;
+  if (only[l] == 0) return;
+  uint32_t* sc = doc_score + ((int64_t)b * L + l) * n_docs;
+  for (int d = threadIdx.x; d < n_docs; d += blockDim.x) sc[d] = kOrdNegInf;
 }
 
 // ---------------------------------------------------------------------------- E4M3 keys
@@ -445,6 +476,115 @@ __global__ void __launch_bounds__(kTopkThreads) merge_topk_kernel(const unsigned
       out_scores[o] = s;
     }
   }
+}
+
+// grid (L, B), 1024 threads: the k_sel best documents of (b, l) by score (equal scores:
+// smaller id first), as keys in descending order (key 0: no document).  Radix selection
+// on the ordered score bits, 8 bits a pass (histograms with warp-aggregated shared
+// atomics), then the documents above the threshold value plus the lowest ids at it.
+constexpr int kSelThreads = 1024;
+
+__global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* __restrict__ doc_score, int L,
+                                                                int n_docs, int k_sel,
+                                                                unsigned long long* __restrict__ out,
+                                                                const int32_t* __restrict__ only) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_need, s_gt, s_taken;
+  __shared__ int wsum[kSelThreads / 32];
+  __shared__ unsigned long long keys[kMaxCandidates];
+  const int l = blockIdx.x, b = blockIdx.y;
+  if (only != nullptr && only[l] == 0) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t* sc = doc_score + ((int64_t)b * L + l) * n_docs;
+  unsigned long long* o = out + ((int64_t)b * L + l) * k_sel;
+  const int K = min(k_sel, n_docs);
+  if (tid == 0) {
+    s_prefix = 0u;
+    s_mask = 0u;
+    s_need = K;
+    s_gt = 0;
+    s_taken = 0;
+  }
+  if (K > 0) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
+      __syncthreads();
+      const uint32_t prefix = s_prefix, mask = s_mask;
+      for (int d0 = 0; d0 < n_docs; d0 += kSelThreads) {  // (uniform trip count for the match)
+        const int d = d0 + tid;
+        const uint32_t u = d < n_docs ? sc[d] : 0u;
+        const bool in = d < n_docs && (u & mask) == prefix;
+        const uint32_t bin = in ? (u >> shift) & 255u : 256u;
+        const uint32_t same = __match_any_sync(0xffffffffu, bin);
+        if (in && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane i owns bins 8i .. 8i+7; sfx = documents in bins >= 8i
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c += (int)hist[8 * lane + j];
+        int sfx = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int t = __shfl_down_sync(0xffffffffu, sfx, off);
+          if (lane + off < 32) sfx += t;
+        }
+        int nxt = __shfl_down_sync(0xffffffffu, sfx, 1);
+        if (lane == 31) nxt = 0;
+        const int need = s_need;
+        if (sfx >= need && nxt < need) {
+          int cum = nxt;
+          for (int j = 7; j >= 0; --j) {
+            const int bin = 8 * lane + j;
+            if (cum + (int)hist[bin] >= need) {
+              s_need = need - cum;
+              s_prefix = prefix | ((uint32_t)bin << shift);
+              s_mask = mask | (255u << shift);
+              break;
+            }
+            cum += (int)hist[bin];
+          }
+        }
+      }
+      __syncthreads();
+    }
+    // the documents above the threshold value, then the lowest ids at it
+    const uint32_t thr = s_prefix;
+    const int need = s_need;
+    for (int d = tid; d < n_docs; d += kSelThreads) {
+      const uint32_t u = sc[d];
+      if (u > thr) keys[atomicAdd(&s_gt, 1)] = ((unsigned long long)u << 32) | (0xFFFFFFFFull - (uint32_t)d);
+    }
+    __syncthreads();
+    const int n_gt = s_gt;  // = K - need
+    for (int d0 = 0; d0 < n_docs; d0 += kSelThreads) {
+      const int taken = s_taken;
+      if (taken >= need) break;  // (uniform: read after the barrier below)
+      const int d = d0 + tid;
+      const bool eq = d < n_docs && sc[d] == thr;
+      const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+      if (lane == 0) wsum[warp] = __popc(bal);
+      __syncthreads();
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += wsum[w];
+      const int rank = taken + before + __popc(bal & ((1u << lane) - 1u));
+      if (eq && rank < need) keys[n_gt + rank] = ((unsigned long long)thr << 32) | (0xFFFFFFFFull - (uint32_t)d);
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < kSelThreads / 32; ++w) tot += wsum[w];
+        s_taken = taken + tot;
+      }
+      __syncthreads();
+    }
+    const int n_pow2 = K <= 1 ? 1 : (1 << (32 - __clz(K - 1)));
+    for (int i = K + tid; i < n_pow2; i += kSelThreads) keys[i] = 0ull;
+    __syncthreads();
+    block_sort_desc(keys, n_pow2);
+  }
+  for (int r = tid; r < k_sel; r += kSelThreads) o[r] = r < K ? keys[r] : 0ull;
 }
 
 // ---------------------------------------------------------------------------- 2c. exact rescoring
@@ -753,6 +893,8 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   const float filter_err = f8 ? kFilterErrF8 : kFilterErr;
 
   uint8_t* qt_f8 = reinterpret_cast<uint8_t*>(ws + w.qt_f8);
+  uint32_t* doc_score = reinterpret_cast<uint32_t*>(ws + w.doc_score);
+  int32_t* block_doc = reinterpret_cast<int32_t*>(ws + w.block_doc);
   __nv_bfloat16* qt_lo = reinterpret_cast<__nv_bfloat16*>(ws + w.qt_lo);
   int32_t* redo = reinterpret_cast<int32_t*>(ws + w.redo);
   if (tensor) {
@@ -765,7 +907,9 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     pt.words_per_row[1] = H * kD * 2 / 16;
     pt.buf[2] = f8 ? reinterpret_cast<uint4*>(qt_f8) : nullptr;
     pt.words_per_row[2] = H * kD / 16;
-    zero_pad_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(pt, n_rows, n_layers, qo);
+    route_prep_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(pt, n_rows, n_layers, qo, doc_chunk_offsets, n_docs,
+                                                           block_doc, doc_score,
+                                                           (int64_t)n_queries * n_layers * n_docs);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
@@ -789,7 +933,9 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     a.ql.n_queries = n_queries;
     for (int b = 0; b <= n_queries; ++b) a.ql.row0[b] = qo.row0[b];
     for (int b = 0; b < n_queries; ++b) a.ql.len[b] = qo.off[b + 1] - qo.off[b];
-    a.m = m;
+    a.block_doc = block_doc;
+    a.doc_score = doc_score;
+    a.n_docs = n_docs;
     a.dev_err = dev_err;
     a.pair = g_pair_mode;
     int launches = 0;
@@ -847,19 +993,10 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   const int K2 = w.k2;
   unsigned long long* apx = reinterpret_cast<unsigned long long*>(ws + w.apx);
   float* exact = reinterpret_cast<float*>(ws + w.exact);
-  const int mg_pow2 = pow2_at_least(w.nblk * K2);
-  const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
-  if (mg_smem > 48 * 1024)
-    MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
   // candidates -> exact rescoring -> final top-k (+ certification), on the layers `only`
   // marks; uncertified layers go to redo_out when given
   auto select = [&](float err, int32_t* redo_out, const int32_t* only) -> msa_status {
-    docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
-        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, K2, doc_pow2, cand, only);
-    ++g_launches;
-    MSA_CUDA_TRY(cudaGetLastError());
-    merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, K2, mg_pow2,
-                                                                            apx, nullptr, nullptr, only);
+    topk_docs_kernel<<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs, K2, apx, only);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     rescore_mma_kernel<<<dim3(K2, n_layers, n_queries), 128, 0, s>>>(
@@ -877,6 +1014,9 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   if (st != MSA_OK || !f8) return st;
   // E4M3 layers that could not be certified: bf16 filter over them, then the same steps
   // with the bf16 error bound (every kernel returns at once on certified layers)
+  doc_reset_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(doc_score, n_layers, n_docs, redo);
+  ++g_launches;
+  MSA_CUDA_TRY(cudaGetLastError());
   st = gemm(false, redo);
   if (st != MSA_OK) return st;
   st = select(kFilterErr, nullptr, redo);

@@ -7,8 +7,9 @@
 // product rescaled by 2^-19 in the epilogue).  One 128-byte shared-memory row holds 64
 // bf16 or 128 E4M3 elements and one MMA consumes 32 bytes of K either way, so both
 // forms share the tiling, swizzle and descriptors; E4M3 halves the K-blocks per tile.
-// The epilogue reduces each row over the columns of every query and writes, per (query,
-// layer, block), the largest score m; D itself never leaves TMEM.  These low-precision scores are a filter: the caller rescores the
+// The epilogue reduces each row over the columns of every query, then over the rows of
+// the same document within the warp (runs of consecutive blocks), and folds the result
+// into the document's score with one atomicMax per run; D itself never leaves TMEM.  These low-precision scores are a filter: the caller rescores the
 // pairs that can hold the maximum exactly.
 //
 // Warp roles of the persistent kernel (192 threads, one CTA per SM):
@@ -16,8 +17,9 @@
 //               K-block into a ring of shared-memory stages (128-byte swizzle)
 //   warp 1      one thread issues tcgen05.mma (fp32 accumulate, 32 bytes of K each) into one of
 //               two TMEM accumulators and commits stage / accumulator completion to mbarriers
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max over each query's columns,
-//               store; then release the accumulator
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, max over each query's columns
+//               and over each document's rows, atomicMax per document; then release the
+//               accumulator
 // Paired mode (PAIR, for N tiles of 128 and 256): a cluster of two CTAs on two SMs runs
 // M=256 tiles with tcgen05.mma.cta_group::2.  Each CTA loads its 128 key rows and half of
 // the query tile, so each SM streams half the query bytes per key byte of the single-CTA
@@ -275,7 +277,8 @@ template <int BN, bool PAIR, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int L,
                     long long C, int n_rows, int m_tiles, const __grid_constant__ QueryLayout ql,
-                    float* __restrict__ m_out, int32_t* dev_err,
+                    const int32_t* __restrict__ block_doc, uint32_t* __restrict__ doc_score, int n_docs,
+                    int32_t* dev_err,
                     const int32_t* __restrict__ layer_only) {
   using K = Cfg<BN, PAIR, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -457,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int l = u / m_tiles, mt = u % m_tiles;
       const long long row = (long long)mt * K::kRows + (long long)rank * kBM + row_in_tile;
       const bool row_ok = row < C;
+      const int my_doc = row_ok ? __ldg(block_doc + row) : -1;
       int carry_b = -1;           // query whose columns continue into the next N tile
       float carry_m = -INFINITY;
       for (int nt = 0; nt < n_tiles; ++nt) {
@@ -499,8 +503,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             float m1 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             if (b == carry_b) m1 = fmaxf(m1, carry_m);
-            if (t0 + 32 >= ql.len[b]) {
-              if (row_ok) m_out[((long long)b * L + l) * C + row] = F8 ? m1 * kF8ScoreScale : m1;
+            if (t0 + 32 >= ql.len[b]) {  // (the same for every lane)
+              // the rows of one document are consecutive: max over each run of equal
+              // documents in the warp, one atomic per run
+              float v = F8 ? m1 * kF8ScoreScale : m1;
+#pragma unroll
+              for (int off = 1; off < 32; off <<= 1) {
+                const float vo = __shfl_down_sync(0xffffffffu, v, off);
+                const int dd = __shfl_down_sync(0xffffffffu, my_doc, off);
+                if (lane + off < 32 && dd == my_doc) v = fmaxf(v, vo);
+              }
+              const int dprev = __shfl_up_sync(0xffffffffu, my_doc, 1);
+              if (my_doc >= 0 && (lane == 0 || dprev != my_doc)) {
+                const uint32_t ub = __float_as_uint(v);
+                atomicMax(doc_score + ((long long)b * L + l) * n_docs + my_doc,
+                          (ub & 0x80000000u) ? ~ub : (ub | 0x80000000u));
+              }
               carry_b = -1;
             } else {
               carry_b = b;
@@ -598,8 +616,8 @@ int launch_bn(const LaunchArgs& a, cudaStream_t s, const char** why) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR, F8>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql, a.m,
-                         a.dev_err, a.layer_only) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, route_tc_kernel<BN, PAIR, F8>, ma, mb, a.L, (long long)a.C, a.n_rows, m_tiles, a.ql,
+                         a.block_doc, a.doc_score, a.n_docs, a.dev_err, a.layer_only) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
   }

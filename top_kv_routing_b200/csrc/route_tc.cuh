@@ -58,7 +58,9 @@ struct LaunchArgs {
   int64_t C;
   int n_rows;          // operand rows per layer (multiple of the N tile)
   QueryLayout ql;
-  float* m;            // [B][L][C]  approximate max over the query's tokens
+  const int32_t* block_doc;  // [C] document of each block
+  uint32_t* doc_score;       // [B][L][n_docs] ordered bits of the filter score, max-accumulated
+  int n_docs;
   int32_t* dev_err;
   bool pair;           // M=256 tiles on CTA pairs (cta_group::2) for N tiles of 128 / 256
   bool f8;             // E4M3 operands (kind::f8f6f4)
