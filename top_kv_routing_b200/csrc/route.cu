@@ -487,6 +487,7 @@ constexpr int kSelThreads = 1024;
 __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* __restrict__ doc_score, int L,
                                                                 int n_docs, int k_sel,
                                                                 unsigned long long* __restrict__ out,
+                                                                uint32_t* __restrict__ exact_bits,
                                                                 const int32_t* __restrict__ only) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix, s_mask;
@@ -584,12 +585,15 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
     __syncthreads();
     block_sort_desc(keys, n_pow2);
   }
-  for (int r = tid; r < k_sel; r += kSelThreads) o[r] = r < K ? keys[r] : 0ull;
+  for (int r = tid; r < k_sel; r += kSelThreads) {
+    o[r] = r < K ? keys[r] : 0ull;
+    exact_bits[((int64_t)b * L + l) * k_sel + r] = kOrdNegInf;  // the rescoring max-accumulates here
+  }
 }
 
 // ---------------------------------------------------------------------------- 2c. exact rescoring
-// grid (K2, L, B), 128 threads: the exact score of filter candidate r of (b, l), i.e. the
-// maximum over all of the document's blocks and all of the query's tokens of
+// The exact score of filter candidate r of (b, l) is the maximum over all of the
+// document's blocks and all of the query's tokens of
 //   s[t][c] = sum_h rho[c][h] * < qt[t][h], k[c][h] >,  rho = 1 / max(||k[c][h]||, 1e-8)
 // with k the stored bf16 keys.  The dots run on the tensor cores (mma.sync m16n8k16,
 // fp32 accumulate): A = 16 blocks of keys (exact in bf16), B = 8 query tokens carried as
@@ -601,7 +605,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
 // so every thread reads each query token with 16-byte loads; the key tile is written to
 // shared memory in the same order (rows of 64 k-steps x 32 bytes, 16-byte chunks XOR-
 // swizzled by row for conflict-free ldmatrix).
-constexpr int kRsRows = 16;  // key blocks per tile (MMA M)
 
 __device__ __forceinline__ void rs_ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
@@ -616,77 +619,132 @@ __device__ __forceinline__ void rs_mma(float (&d)[4], const uint32_t (&a)[4], ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(128) rescore_mma_kernel(const __nv_bfloat16* __restrict__ kr_hat,
-                                                          const __nv_bfloat16* __restrict__ q_hi,
-                                                          const __nv_bfloat16* __restrict__ q_lo, int L, int64_t C,
-                                                          int n_rows, QueryOffsets qo,
-                                                          const int64_t* __restrict__ doc_chunk_off,
-                                                          const unsigned long long* __restrict__ apx, int K2,
-                                                          float* __restrict__ exact,
-                                                          const int32_t* __restrict__ only) {
+// grid (x, L, B), 256 threads: the blocks of all K2 candidates of (b, l), laid end to
+// end, are cut into tiles of kRsTile blocks; CTA x takes tiles x, x + gridDim.x, ...
+// Each tile is staged once (64 KB of keys = 4 MMA row tiles), and every warp reads the
+// query rows of its tokens once per head for all four row tiles.  The maximum of every
+// (block, token) pair goes to its candidate through shared atomics on ordered bits, then
+// one global atomicMax per candidate into exact_bits (set to -inf by the selection).
+constexpr int kRsTile = 64;
+constexpr int kRsWarps = 8;
+constexpr size_t kRsSmem = (size_t)kRsTile * 8 * kD * 2;  // the staged keys
+
+__global__ void __launch_bounds__(kRsWarps * 32) rescore_mma_kernel(
+    const __nv_bfloat16* __restrict__ kr_hat, const __nv_bfloat16* __restrict__ q_hi,
+    const __nv_bfloat16* __restrict__ q_lo, int L, int64_t C, int n_rows, QueryOffsets qo,
+    const int64_t* __restrict__ doc_chunk_off, const unsigned long long* __restrict__ apx, int K2,
+    uint32_t* __restrict__ exact_bits, const int32_t* __restrict__ only) {
   constexpr int kRowBytes = 8 * kD * 2;  // 2048
-  __shared__ __align__(128) uint8_t ktile[kRsRows * kRowBytes];
-  __shared__ float rho[kRsRows][8];
-  __shared__ float red[4];
-  const int r = blockIdx.x, l = blockIdx.y, b = blockIdx.z;
+  extern __shared__ __align__(128) uint8_t ktile[];
+  __shared__ float rho[kRsTile][8];
+  __shared__ int64_t cand_c0[kMaxCandidates];
+  __shared__ int cand_start[kMaxCandidates + 1];
+  __shared__ int row_rank[kRsTile];
+  __shared__ uint32_t row_best[kRsTile];
+  __shared__ uint32_t best[kMaxCandidates];
+  const int l = blockIdx.y, b = blockIdx.z;
   if (only != nullptr && only[l] == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int64_t o = ((int64_t)b * L + l) * K2 + r;
-  int doc;
-  float doc_apx;
-  split_key(apx[o], &doc, &doc_apx);
-  if (doc < 0) {
-    if (tid == 0) exact[o] = -INFINITY;
-    return;
+  const int64_t o = ((int64_t)b * L + l) * K2;
+  // the candidates' block ranges, end to end
+  if (warp == 0) {
+    int cnt[kMaxCandidates / 32];
+    int run = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxCandidates / 32; ++i) {
+      const int r = 32 * i + lane;
+      int n = 0;
+      int64_t c0 = 0;
+      if (r < K2) {
+        int doc;
+        float sc;
+        split_key(apx[o + r], &doc, &sc);
+        if (doc >= 0) {
+          c0 = doc_chunk_off[doc];
+          n = (int)(doc_chunk_off[doc + 1] - c0);
+        }
+        cand_c0[r] = c0;
+      }
+      int incl = n;  // inclusive prefix over the 32 lanes
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (r < K2) cand_start[r] = run + incl - n;
+      cnt[i] = __shfl_sync(0xffffffffu, incl, 31);
+      run += cnt[i];
+    }
+    if (lane == 0) cand_start[K2] = run;
   }
-  const int64_t c0 = doc_chunk_off[doc], c1 = doc_chunk_off[doc + 1];
+  for (int r = tid; r < K2; r += blockDim.x) best[r] = 0x007FFFFFu;  // -inf
+  __syncthreads();
+  const int n_blocks = cand_start[K2];
   const int T = qo.off[b + 1] - qo.off[b];
   const int n_tiles = (T + 7) / 8;
   const int64_t qrow0 = (int64_t)l * n_rows + qo.row0[b];
   const uint32_t kt_base = static_cast<uint32_t>(__cvta_generic_to_shared(ktile));
-  float best = -INFINITY;
-  for (int64_t g0 = c0; g0 < c1; g0 += kRsRows) {
-    const int nb = (int)(c1 - g0 < kRsRows ? c1 - g0 : kRsRows);
-    // stage the key tile in MMA k order: 16-byte chunk m' of a row holds memory dims
-    // 8m' .. 8m'+7 = head h, thread t', k-steps 2m, 2m+1 (dims 4 apart per k-step)
-    for (int i = tid; i < kRsRows * 128; i += blockDim.x) {
+  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lhalf = lane >> 4;
+  for (int f0 = blockIdx.x * kRsTile; f0 < n_blocks; f0 += gridDim.x * kRsTile) {
+    if (tid < kRsTile) {
+      const int f = f0 + tid;
+      int rr = -1;
+      if (f < n_blocks) {  // candidate holding flat block f: the last start <= f
+        int lo = 0, hi = K2;
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (cand_start[mid] <= f) lo = mid; else hi = mid;
+        }
+        rr = lo;
+      }
+      row_rank[tid] = rr;
+      row_best[tid] = 0x007FFFFFu;
+    }
+    __syncthreads();
+    // stage the tile in MMA k order (see above); rows past the end are zero
+    for (int i = tid; i < kRsTile * 128; i += blockDim.x) {
       const int row = i >> 7, mp = i & 127;
+      const int rr = row_rank[row];
       uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (row < nb) w = __ldg(reinterpret_cast<const uint4*>(kr_hat + ((int64_t)l * C + g0 + row) * 8 * kD) + mp);
+      if (rr >= 0) {
+        const int64_t c = cand_c0[rr] + (f0 + row - cand_start[rr]);
+        w = __ldg(reinterpret_cast<const uint4*>(kr_hat + ((int64_t)l * C + c) * 8 * kD) + mp);
+      }
       const int h = mp >> 4, tp = (mp >> 2) & 3, m = mp & 3;
       const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int ks = 8 * h + 2 * m + (j >> 1), half = j & 1;  // word j: dims 2j, 2j+1 of the chunk
+        const int ks = 8 * h + 2 * m + (j >> 1), half = j & 1;
         const int chunk = (2 * ks + half) ^ (row & 7);
         *reinterpret_cast<uint32_t*>(ktile + row * kRowBytes + chunk * 16 + tp * 4) = wv[j];
       }
     }
     __syncthreads();
-    {  // 1 / ||k|| per (row, head): a head is 16 whole chunks of the row, in any order
-      const int row = tid >> 3, h = tid & 7;
-      const uint4* src = reinterpret_cast<const uint4*>(ktile + row * kRowBytes + h * 256);
+    for (int i = tid; i < kRsTile * 8; i += blockDim.x) {  // 1 / ||k|| per (row, head)
+      // (summed in the head's logical chunk order, so the value does not depend on the
+      // row's place in the tile)
+      const int row = i >> 3, h = i & 7;
+      const uint4* src = reinterpret_cast<const uint4*>(ktile + row * kRowBytes);
       float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint4 w = src[i];
-        const float2 f0 = msa::bf16x2_to_float2(w.x), f1 = msa::bf16x2_to_float2(w.y);
+      for (int j = 0; j < 16; ++j) {
+        const uint4 w = src[(16 * h + j) ^ (row & 7)];
+        const float2 f0v = msa::bf16x2_to_float2(w.x), f1 = msa::bf16x2_to_float2(w.y);
         const float2 f2 = msa::bf16x2_to_float2(w.z), f3 = msa::bf16x2_to_float2(w.w);
-        ss = fmaf(f0.x, f0.x, ss); ss = fmaf(f0.y, f0.y, ss); ss = fmaf(f1.x, f1.x, ss); ss = fmaf(f1.y, f1.y, ss);
+        ss = fmaf(f0v.x, f0v.x, ss); ss = fmaf(f0v.y, f0v.y, ss); ss = fmaf(f1.x, f1.x, ss); ss = fmaf(f1.y, f1.y, ss);
         ss = fmaf(f2.x, f2.x, ss); ss = fmaf(f2.y, f2.y, ss); ss = fmaf(f3.x, f3.x, ss); ss = fmaf(f3.y, f3.y, ss);
       }
       rho[row][h] = 1.0f / fmaxf(sqrtf(ss), 1e-8f);
     }
     __syncthreads();
-    // lane's ldmatrix row: matrix (lane >> 3): rows 0-7 / 8-15, k-indices 0-7 / 8-15
-    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lhalf = lane >> 4;
-    const uint32_t arow = kt_base + lrow * kRowBytes;
-    for (int nt = warp; nt < n_tiles; nt += 4) {
+    for (int nt = warp; nt < n_tiles; nt += kRsWarps) {
       const int tok = 8 * nt + g;  // this lane's B column (token); padded rows are zero
       const uint4* qh = reinterpret_cast<const uint4*>(q_hi + (qrow0 + tok) * 8 * kD) + 4 * t;
       const uint4* ql = reinterpret_cast<const uint4*>(q_lo + (qrow0 + tok) * 8 * kD) + 4 * t;
-      float tot[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
+      float tot[kRsTile / 16][4];
+#pragma unroll
+      for (int mt = 0; mt < kRsTile / 16; ++mt) tot[mt][0] = tot[mt][1] = tot[mt][2] = tot[mt][3] = 0.f;
+#pragma unroll 1
       for (int h = 0; h < 8; ++h) {
         uint4 xh[4], xl[4];  // dims 128h + 32t .. +32 of token tok
 #pragma unroll
@@ -694,43 +752,57 @@ __global__ void __launch_bounds__(128) rescore_mma_kernel(const __nv_bfloat16* _
           xh[m] = __ldg(qh + 16 * h + m);
           xl[m] = __ldg(ql + 16 * h + m);
         }
-        float acc_h[4] = {0.f, 0.f, 0.f, 0.f}, acc_l[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int ks = 8 * h + kk;
-          uint32_t a[4];
-          rs_ldsm_x4(arow + (((2 * ks + lhalf) ^ (lrow & 7)) << 4), a);
-          const uint4& vh = xh[kk >> 1];
-          const uint4& vl = xl[kk >> 1];
-          if (kk & 1) {
-            rs_mma(acc_h, a, vh.z, vh.w);
-            rs_mma(acc_l, a, vl.z, vl.w);
-          } else {
-            rs_mma(acc_h, a, vh.x, vh.y);
-            rs_mma(acc_l, a, vl.x, vl.y);
+        for (int mt = 0; mt < kRsTile / 16; ++mt) {
+          const uint32_t arow = kt_base + (16 * mt + lrow) * kRowBytes;
+          float acc_h[4] = {0.f, 0.f, 0.f, 0.f}, acc_l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int ks = 8 * h + kk;
+            uint32_t a4[4];
+            rs_ldsm_x4(arow + (((2 * ks + lhalf) ^ (lrow & 7)) << 4), a4);
+            const uint4& vh = xh[kk >> 1];
+            const uint4& vl = xl[kk >> 1];
+            if (kk & 1) {
+              rs_mma(acc_h, a4, vh.z, vh.w);
+              rs_mma(acc_l, a4, vl.z, vl.w);
+            } else {
+              rs_mma(acc_h, a4, vh.x, vh.y);
+              rs_mma(acc_l, a4, vl.x, vl.y);
+            }
           }
+          const float ra = rho[16 * mt + g][h], rb = rho[16 * mt + g + 8][h];
+          tot[mt][0] = fmaf(ra, acc_h[0] + acc_l[0], tot[mt][0]);
+          tot[mt][1] = fmaf(ra, acc_h[1] + acc_l[1], tot[mt][1]);
+          tot[mt][2] = fmaf(rb, acc_h[2] + acc_l[2], tot[mt][2]);
+          tot[mt][3] = fmaf(rb, acc_h[3] + acc_l[3], tot[mt][3]);
         }
-        const float ra = rho[g][h], rb = rho[g + 8][h];
-        tot[0] = fmaf(ra, acc_h[0] + acc_l[0], tot[0]);
-        tot[1] = fmaf(ra, acc_h[1] + acc_l[1], tot[1]);
-        tot[2] = fmaf(rb, acc_h[2] + acc_l[2], tot[2]);
-        tot[3] = fmaf(rb, acc_h[3] + acc_l[3], tot[3]);
       }
-      // C: rows (blocks) g / g+8, columns (tokens) 8nt + 2t + {0, 1}
+      // C: rows g / g+8 of each row tile, tokens 8nt + 2t + {0, 1}; the row's maximum
+      // over this warp's 8 tokens, then into the row's shared maximum
       const int t0 = 8 * nt + 2 * t;
-      const bool r0 = g < nb, r1 = g + 8 < nb;
-      if (r0 && t0 < T) best = fmaxf(best, tot[0]);
-      if (r0 && t0 + 1 < T) best = fmaxf(best, tot[1]);
-      if (r1 && t0 < T) best = fmaxf(best, tot[2]);
-      if (r1 && t0 + 1 < T) best = fmaxf(best, tot[3]);
+#pragma unroll
+      for (int mt = 0; mt < kRsTile / 16; ++mt) {
+        float va = -INFINITY, vb = -INFINITY;
+        if (t0 < T) { va = tot[mt][0]; vb = tot[mt][2]; }
+        if (t0 + 1 < T) { va = fmaxf(va, tot[mt][1]); vb = fmaxf(vb, tot[mt][3]); }
+        va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, 1));
+        va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, 2));
+        vb = fmaxf(vb, __shfl_xor_sync(0xffffffffu, vb, 1));
+        vb = fmaxf(vb, __shfl_xor_sync(0xffffffffu, vb, 2));
+        if (t == 0) {
+          const uint32_t ua = __float_as_uint(va), ub = __float_as_uint(vb);
+          atomicMax(&row_best[16 * mt + g], (ua & 0x80000000u) ? ~ua : (ua | 0x80000000u));
+          atomicMax(&row_best[16 * mt + g + 8], (ub & 0x80000000u) ? ~ub : (ub | 0x80000000u));
+        }
+      }
     }
+    __syncthreads();
+    if (tid < kRsTile && row_rank[tid] >= 0) atomicMax(&best[row_rank[tid]], row_best[tid]);
     __syncthreads();  // before the tile is restaged
   }
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, s));
-  if (lane == 0) red[warp] = best;
-  __syncthreads();
-  if (tid == 0) exact[o] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  for (int r = tid; r < K2; r += blockDim.x)
+    if (best[r] != 0x007FFFFFu) atomicMax(&exact_bits[o + r], best[r]);
 }
 
 // grid (L, B), 128 threads: final top-k of the K2 exactly rescored candidates.  The
@@ -739,7 +811,7 @@ __global__ void __launch_bounds__(128) rescore_mma_kernel(const __nv_bfloat16* _
 // E4M3 pass) the layer is marked for the bf16 pass; without it MSA_DEVERR_UNCERTIFIED.
 // With only given, layers it does not mark are left as they are.
 __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long long* __restrict__ apx,
-                                                           const float* __restrict__ exact, int K2, int k,
+                                                           const uint32_t* __restrict__ exact_bits, int K2, int k,
                                                            int n_docs, int L, float err,
                                                            int32_t* __restrict__ out_ids,
                                                            float* __restrict__ out_scores, int32_t* dev_err,
@@ -756,7 +828,7 @@ __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long l
       int doc;
       float s;
       split_key(apx[base + i], &doc, &s);
-      if (doc >= 0) key = make_key(exact[base + i], doc);
+      if (doc >= 0) key = ((unsigned long long)exact_bits[base + i] << 32) | (0xFFFFFFFFull - (uint32_t)doc);
     }
     keys[i] = key;
   }
@@ -992,14 +1064,19 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   // rescored exactly (fp32 cosines) and the final top-k is taken from the exact scores
   const int K2 = w.k2;
   unsigned long long* apx = reinterpret_cast<unsigned long long*>(ws + w.apx);
-  float* exact = reinterpret_cast<float*>(ws + w.exact);
+  uint32_t* exact = reinterpret_cast<uint32_t*>(ws + w.exact);
+  MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRsSmem));
+  // CTAs per (query, layer) of the rescoring: about two per SM in all, at most 8
+  int rs_x = (2 * msa::sm_count() + n_layers * n_queries - 1) / (n_layers * n_queries);
+  rs_x = rs_x < 1 ? 1 : (rs_x > 8 ? 8 : rs_x);
   // candidates -> exact rescoring -> final top-k (+ certification), on the layers `only`
   // marks; uncertified layers go to redo_out when given
   auto select = [&](float err, int32_t* redo_out, const int32_t* only) -> msa_status {
-    topk_docs_kernel<<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs, K2, apx, only);
+    topk_docs_kernel<<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs, K2, apx, exact,
+                                                                      only);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
-    rescore_mma_kernel<<<dim3(K2, n_layers, n_queries), 128, 0, s>>>(
+    rescore_mma_kernel<<<dim3(rs_x, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
         (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx, K2,
         exact, only);
     ++g_launches;
