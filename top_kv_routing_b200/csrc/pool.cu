@@ -4,12 +4,17 @@
 // pooling of K/V/K_r; 并行 RoPE: positions restart at 0 per document) and the MSA paper
 // reading notes, section 路由投影器 + Top-k 稀疏注意力 (64-token blocks).
 //
-// Design: persistent CTAs, one memory block (<= 64 tokens x H heads) per iteration.
-// Thread (parity p, head h, part q) owns dims [8q, 8q+8) and their rotate-half partners
-// [64+8q, 64+8q+8) of head h for tokens p, p+2, ... of the block, so a 16-byte load of
-// each half feeds the rotation with no exchange.  RoPE cos/sin for the block's 64
-// positions x 64 frequencies are built once per block in shared memory from a per-CTA
-// table cos/sin(i w_j) and the block's base angle (fp64 reduced), by angle addition.
+// Design: a streaming kernel, one CTA per SM, each owning a contiguous range of memory
+// blocks (so a block's document is found once by binary search and then advanced
+// incrementally).  A producer warp copies the blocks' token rows of K, V and K_r with
+// bulk asynchronous copies (cp.async.bulk, completion on mbarriers) into a ring of
+// shared-memory stages of S tokens; one consumer warp per head h accumulates them.
+// Lane (g, q) of that warp (g = lane / 8) owns dims [8q, 8q+8) and their rotate-half
+// partners [64+8q, 64+8q+8) of head h for the block's tokens g, g+4, g+8, ...; its 8
+// frequencies' cos/sin live in registers, exact at the lane's first token of the block
+// (angle / pi reduced in fp64, fp32 sincospif) and advanced by the fixed rotation of 4
+// positions per token.  At the block's end the four token groups meet through warp
+// shuffles.  Every wait is bounded (2 s); a timeout sets MSA_DEVERR_TIMEOUT.
 #include "common.cuh"
 #include "msa_pool.h"
 
@@ -21,39 +26,56 @@ constexpr int kD = 128;      // head_dim
 constexpr int kHalf = 64;    // rotate-half partner distance
 constexpr int kMaxChunk = 64;
 
-struct PoolSmem {
-  float2 inner[kMaxChunk][kHalf];   // (cos, sin)(i * w_j)
-  float2 table[kMaxChunk][kHalf];   // (cos, sin)((p0 + i) * w_j) for the current block
-  float2 base[kHalf];               // (cos, sin)(p0 * w_j)
-  double w[kHalf];                  // theta^(-2j/d)
-  float partial[3][8 * 16][16];     // odd-parity partial sums, [stream][thread][value]
-  int64_t tok0, n_tok, pos0;
-  int skip;
-};
-
 template <typename T>
 struct Loader;
 
+// 8 consecutive elements: raw() reads them (16 or 32 bytes), unpack() widens to fp32.
 template <>
 struct Loader<float> {
-  // 8 consecutive fp32 values
+  struct Raw {
+    float4 a, b;
+  };
+  static __device__ __forceinline__ void raw(const float* p, Raw& r) {
+    r.a = __ldg(reinterpret_cast<const float4*>(p));
+    r.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  static __device__ __forceinline__ void unpack(const Raw& r, float* x) {
+    x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+    x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+  }
   static __device__ __forceinline__ void load8(const float* p, float* x) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    Raw r;
+    raw(p, r);
+    unpack(r, x);
+  }
+  static __device__ __forceinline__ void load8_smem(const unsigned char* p, float* x) {
+    Raw r;
+    r.a = *reinterpret_cast<const float4*>(p);
+    r.b = *reinterpret_cast<const float4*>(p + 16);
+    unpack(r, x);
   }
 };
 
 template <>
 struct Loader<__nv_bfloat16> {
-  static __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* x) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  using Raw = uint4;
+  static __device__ __forceinline__ void raw(const __nv_bfloat16* p, Raw& r) {
+    r = __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  static __device__ __forceinline__ void unpack(const Raw& a, float* x) {
     float2 f;
     f = msa::bf16x2_to_float2(a.x); x[0] = f.x; x[1] = f.y;
     f = msa::bf16x2_to_float2(a.y); x[2] = f.x; x[3] = f.y;
     f = msa::bf16x2_to_float2(a.z); x[4] = f.x; x[5] = f.y;
     f = msa::bf16x2_to_float2(a.w); x[6] = f.x; x[7] = f.y;
+  }
+  static __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* x) {
+    Raw r;
+    raw(p, r);
+    unpack(r, x);
+  }
+  static __device__ __forceinline__ void load8_smem(const unsigned char* p, float* x) {
+    unpack(*reinterpret_cast<const uint4*>(p), x);
   }
 };
 
@@ -66,91 +88,233 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* x) {
   *reinterpret_cast<uint4*>(p) = o;
 }
 
-template <typename TIn>
-__global__ void __launch_bounds__(256) pool_kernel(
-    const TIn* __restrict__ k, const TIn* __restrict__ v, const TIn* __restrict__ kr,
-    const int64_t* __restrict__ doc_tok_off, const int64_t* __restrict__ doc_chunk_off, int n_docs,
-    int64_t n_chunks, int H, int chunk, double log2_theta, int use_rope,
-    __nv_bfloat16* __restrict__ k_bar, __nv_bfloat16* __restrict__ v_bar,
-    __nv_bfloat16* __restrict__ kr_hat, float* __restrict__ kr_norm, int32_t* dev_err) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  PoolSmem& sm = *reinterpret_cast<PoolSmem*>(smem_raw);
-  const int tid = threadIdx.x;
-  const int per_parity = 8 * H;
-  const int parity = tid / per_parity;
-  const int r = tid % per_parity;
-  const int h = r / 8;
-  const int q = r % 8;
-  const int64_t row = (int64_t)H * kD;
+constexpr int kStageBytesTarget = 48 * 1024;  // K, V and K_r rows of one stage
+constexpr int kRingBytes = 192 * 1024;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
-  if (blockIdx.x == 0 && tid == 0 && __ldg(doc_chunk_off + n_docs) != n_chunks)
-    msa::set_err(dev_err, MSA_DEVERR_BAD_OFFSETS);
+struct SliceMeta {
+  int64_t blk;    // memory block
+  int first;      // index in the block of the slice's first token
+  int rows;       // tokens in the slice
+  int n_block;    // tokens in the block
+  int pos0;       // position (in its document) of the block's first token
+  int last;       // last slice of the block
+  int state;      // 0 = tokens, 1 = skipped block (bad offsets), 2 = end of the sequence
+};
 
-  if (use_rope) {
-    for (int j = tid; j < kHalf; j += blockDim.x) sm.w[j] = exp2(-2.0 * (double)j / (double)kD * log2_theta);
-    __syncthreads();
-    for (int e = tid; e < chunk * kHalf; e += blockDim.x) {
-      const int i = e / kHalf, j = e % kHalf;
-      float c, s;
-      msa::angle_sincos((double)i, sm.w[j], &c, &s);
-      sm.inner[i][j] = make_float2(c, s);
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase with this parity; false after 2 s or once another warp has given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer() - t0 > kTimeoutNs) return false;
     }
   }
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// global -> shared bulk copy (no multicast), completing on an mbarrier of this CTA
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 
-  for (int64_t blk = blockIdx.x; blk < n_chunks; blk += gridDim.x) {
-    __syncthreads();  // previous block's smem readers are done
-    if (tid == 0) {
-      const int d = msa::upper_doc(doc_chunk_off, n_docs, blk);
+template <typename TIn, int kWarps>  // kWarps: heads + 1 at most
+__global__ void __launch_bounds__(kWarps * 32) pool_kernel(
+    const TIn* __restrict__ k, const TIn* __restrict__ v, const TIn* __restrict__ kr,
+    const int64_t* __restrict__ doc_tok_off, const int64_t* __restrict__ doc_chunk_off, int n_docs,
+    int64_t n_chunks, int64_t blocks_per_cta, int H, int chunk, int S, int n_stages, double log2_theta, int use_rope,
+    __nv_bfloat16* __restrict__ k_bar, __nv_bfloat16* __restrict__ v_bar,
+    __nv_bfloat16* __restrict__ kr_hat, float* __restrict__ kr_norm, int32_t* dev_err) {
+  extern __shared__ __align__(128) unsigned char ring[];
+  __shared__ SliceMeta meta[8];
+  __shared__ __align__(8) uint64_t full[8], empty[8];
+  __shared__ int abort_flag;
+  __shared__ double s_wpi[kHalf];  // theta^(-2j/d) / pi
+  __shared__ float2 s_r4[kHalf];   // (cos, sin) of 4 positions' angle, per frequency
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (use_rope)
+    for (int j = threadIdx.x; j < kHalf; j += blockDim.x) {
+      const double w = exp2(-2.0 * (double)j / (double)kD * log2_theta) * 0.31830988618379067154;
+      double x = 4.0 * w;
+      x -= 2.0 * rint(0.5 * x);
+      float sn, cs;
+      sincospif((float)x, &sn, &cs);
+      s_wpi[j] = w;
+      s_r4[j] = make_float2(cs, sn);
+    }
+  const int64_t row_elems = (int64_t)H * kD;
+  const uint32_t row_bytes = (uint32_t)(row_elems * sizeof(TIn));
+  const uint32_t region = (uint32_t)S * row_bytes;  // one stream's rows in a stage
+  const uint32_t stage_bytes = 3u * region;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < n_stages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), (uint32_t)H);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (blockIdx.x == 0 && __ldg(doc_chunk_off + n_docs) != n_chunks) msa::set_err(dev_err, MSA_DEVERR_BAD_OFFSETS);
+  }
+  __syncthreads();
+  const int64_t b_begin = blockIdx.x * blocks_per_cta;
+  const int64_t b_end = min(n_chunks, b_begin + blocks_per_cta);
+
+  if (warp == H) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0u, armed_phase = 0u;  // stages with a copy issued, and its phase bit
+    bool ok = true;
+    auto next_stage = [&]() -> bool {  // waits for a free stage
+      if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &abort_flag)) return false;
+      return true;
+    };
+    auto advance = [&]() {
+      armed |= 1u << stage;
+      armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+      if (++stage == n_stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    };
+    int d = b_begin < b_end ? msa::upper_doc(doc_chunk_off, n_docs, b_begin) : 0;
+    for (int64_t blk = b_begin; blk < b_end && ok; ++blk) {
+      while (d + 1 < n_docs && __ldg(doc_chunk_off + d + 1) <= blk) ++d;
       const int64_t j = blk - __ldg(doc_chunk_off + d);
       const int64_t t_begin = __ldg(doc_tok_off + d), t_end = __ldg(doc_tok_off + d + 1);
-      const int64_t start = t_begin + j * chunk;
-      sm.skip = 0;
-      if (start >= t_end || start < t_begin) {
-        msa::set_err(dev_err, MSA_DEVERR_BAD_OFFSETS);
-        sm.skip = 1;
+      const int64_t tok0 = t_begin + j * chunk;
+      const bool bad = tok0 >= t_end || tok0 < t_begin;
+      const int nb = bad ? 0 : (int)min((int64_t)chunk, t_end - tok0);
+      const int n_slices = bad ? 1 : (nb + S - 1) / S;
+      for (int sl = 0; sl < n_slices; ++sl) {
+        if (!next_stage()) {
+          ok = false;
+          break;
+        }
+        SliceMeta& m = meta[stage];
+        m.blk = blk;
+        m.first = sl * S;
+        m.rows = bad ? 0 : min(S, nb - sl * S);
+        m.n_block = nb;
+        m.pos0 = (int)(j * chunk);
+        m.last = sl == n_slices - 1;
+        m.state = bad ? 1 : 0;
+        if (bad) msa::set_err(dev_err, MSA_DEVERR_BAD_OFFSETS);
+        const uint32_t bytes = (uint32_t)m.rows * row_bytes;
+        const uint32_t fb = smem_u32(&full[stage]);
+        const uint32_t dst = smem_u32(ring) + stage * stage_bytes;
+        const int64_t src = (tok0 + sl * S) * row_elems;
+        mbar_arrive_expect_tx(fb, bytes * ((k != nullptr) + (v != nullptr) + (kr != nullptr)));
+        if (bytes > 0) {
+          if (k != nullptr) bulk_copy(dst, k + src, bytes, fb);
+          if (v != nullptr) bulk_copy(dst + region, v + src, bytes, fb);
+          if (kr != nullptr) bulk_copy(dst + 2 * region, kr + src, bytes, fb);
+        }
+        advance();
       }
-      sm.tok0 = start;
-      sm.n_tok = min((int64_t)chunk, t_end - start);
-      sm.pos0 = start - t_begin;
     }
-    __syncthreads();
-    if (sm.skip) continue;
-    const int64_t tok0 = sm.tok0;
-    const int n = (int)sm.n_tok;
-    if (use_rope && k != nullptr) {
-      for (int j = tid; j < kHalf; j += blockDim.x) {
-        float c, s;
-        msa::angle_sincos((double)sm.pos0, sm.w[j], &c, &s);
-        sm.base[j] = make_float2(c, s);
-      }
-      __syncthreads();
-      for (int e = tid; e < n * kHalf; e += blockDim.x) {
-        const int i = e / kHalf, j = e % kHalf;
-        const float2 b = sm.base[j], in = sm.inner[i][j];
-        sm.table[i][j] = make_float2(b.x * in.x - b.y * in.y, b.y * in.x + b.x * in.y);
-      }
-      __syncthreads();
+    if (ok && next_stage()) {  // the end marker
+      meta[stage].state = 2;
+      mbar_arrive_expect_tx(smem_u32(&full[stage]), 0u);
+      advance();
+    } else {
+      ok = false;
     }
+    if (!ok) {
+      abort_flag = 1;
+      msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+    }
+    // no copy may still be writing this CTA's shared memory when it exits
+    for (int i = 0; i < n_stages; ++i) {
+      if (!((armed >> i) & 1u)) continue;
+      const uint64_t t0 = global_timer();
+      while (!mbar_try_wait(smem_u32(&full[i]), (armed_phase >> i) & 1u))
+        if (global_timer() - t0 > kTimeoutNs) break;
+    }
+    return;
+  }
 
-    float ak[16], av[16], ar[16];
+  // -------------------------------------------------------------- consumers: warp h = head
+  const int h = warp, g = lane >> 3, q = lane & 7;
+  float ak[16], av[16], ar[16], c[8], sn[8];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) { ak[u] = 0.f; av[u] = 0.f; ar[u] = 0.f; }
-    if (parity < 2) {
-      const int64_t lo_off = (int64_t)h * kD + 8 * q;
-      const int64_t hi_off = lo_off + kHalf;
-#pragma unroll 2
-      for (int i = parity; i < n; i += 2) {
-        const int64_t base = (tok0 + i) * row;
+  for (int u = 0; u < 8; ++u) { c[u] = 1.f; sn[u] = 0.f; }
+  const uint32_t lo_byte = (uint32_t)((h * kD + 8 * q) * (int)sizeof(TIn));
+  const uint32_t hi_byte = lo_byte + (uint32_t)(kHalf * sizeof(TIn));
+  int stage = 0;
+  uint32_t phase = 0;
+  while (true) {
+    if (!mbar_wait(smem_u32(&full[stage]), phase, &abort_flag)) {
+      if (lane == 0) {
+        abort_flag = 1;
+        msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+      }
+      break;
+    }
+    const SliceMeta m = meta[stage];
+    if (m.state == 2) break;
+    if (m.state == 0) {
+      if (m.first == 0) {  // a new block
+#pragma unroll
+        for (int u = 0; u < 16; ++u) { ak[u] = 0.f; av[u] = 0.f; ar[u] = 0.f; }
+        if (use_rope && k != nullptr) {
+          const double pos = (double)(m.pos0 + g);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            double x = pos * s_wpi[8 * q + u];  // angle / pi
+            x -= 2.0 * rint(0.5 * x);
+            sincospif((float)x, &sn[u], &c[u]);
+          }
+        }
+      }
+      const unsigned char* st = ring + stage * stage_bytes;
+      for (int rr = g; rr < m.rows; rr += 4) {
+        const unsigned char* rowp = st + rr * row_bytes;
         float lo[8], hi[8];
         if (k != nullptr) {
-          Loader<TIn>::load8(k + base + lo_off, lo);
-          Loader<TIn>::load8(k + base + hi_off, hi);
+          Loader<TIn>::load8_smem(rowp + lo_byte, lo);
+          Loader<TIn>::load8_smem(rowp + hi_byte, hi);
           if (use_rope) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              const float2 cs = sm.table[i][8 * q + u];
-              ak[u] += lo[u] * cs.x - hi[u] * cs.y;
-              ak[8 + u] += hi[u] * cs.x + lo[u] * cs.y;
+              ak[u] += lo[u] * c[u] - hi[u] * sn[u];
+              ak[8 + u] += hi[u] * c[u] + lo[u] * sn[u];
+              const float2 r4 = s_r4[8 * q + u];  // advance 4 positions
+              const float cn = c[u] * r4.x - sn[u] * r4.y;
+              sn[u] = sn[u] * r4.x + c[u] * r4.y;
+              c[u] = cn;
             }
           } else {
 #pragma unroll
@@ -158,65 +322,71 @@ __global__ void __launch_bounds__(256) pool_kernel(
           }
         }
         if (v != nullptr) {
-          Loader<TIn>::load8(v + base + lo_off, lo);
-          Loader<TIn>::load8(v + base + hi_off, hi);
+          Loader<TIn>::load8_smem(rowp + region + lo_byte, lo);
+          Loader<TIn>::load8_smem(rowp + region + hi_byte, hi);
 #pragma unroll
           for (int u = 0; u < 8; ++u) { av[u] += lo[u]; av[8 + u] += hi[u]; }
         }
         if (kr != nullptr) {
-          Loader<TIn>::load8(kr + base + lo_off, lo);
-          Loader<TIn>::load8(kr + base + hi_off, hi);
+          Loader<TIn>::load8_smem(rowp + 2 * region + lo_byte, lo);
+          Loader<TIn>::load8_smem(rowp + 2 * region + hi_byte, hi);
 #pragma unroll
           for (int u = 0; u < 8; ++u) { ar[u] += lo[u]; ar[8 + u] += hi[u]; }
         }
       }
     }
-    if (parity == 1) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[stage]));  // the stage may be refilled
+    if (m.state == 0 && m.last) {
+      // the four token groups (lanes q, q+8, q+16, q+24) meet
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        sm.partial[0][r][u] = ak[u];
-        sm.partial[1][r][u] = av[u];
-        sm.partial[2][r][u] = ar[u];
+        ak[u] += __shfl_xor_sync(0xffffffffu, ak[u], 8);
+        ak[u] += __shfl_xor_sync(0xffffffffu, ak[u], 16);
+        av[u] += __shfl_xor_sync(0xffffffffu, av[u], 8);
+        av[u] += __shfl_xor_sync(0xffffffffu, av[u], 16);
+        ar[u] += __shfl_xor_sync(0xffffffffu, ar[u], 8);
+        ar[u] += __shfl_xor_sync(0xffffffffu, ar[u], 16);
+      }
+      const float inv_n = 1.0f / (float)m.n_block;
+      const int64_t o = m.blk * row_elems + (int64_t)h * kD + 8 * q;
+      float ss = 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        ak[u] *= inv_n;
+        av[u] *= inv_n;
+        ar[u] *= inv_n;
+        ss += ar[u] * ar[u];
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);  // the 8 q-lanes of the head
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      if (g == 0) {
+        if (k != nullptr && k_bar != nullptr) {
+          store8_bf16(k_bar + o, ak);
+          store8_bf16(k_bar + o + kHalf, ak + 8);
+        }
+        if (v != nullptr && v_bar != nullptr) {
+          store8_bf16(v_bar + o, av);
+          store8_bf16(v_bar + o + kHalf, av + 8);
+        }
+        if (kr != nullptr) {
+          const float nrm = sqrtf(ss);
+          const float inv = 1.0f / fmaxf(nrm, 1e-8f);
+          if (kr_hat != nullptr) {
+            float x[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) x[u] = ar[u] * inv;
+            store8_bf16(kr_hat + o, x);
+            store8_bf16(kr_hat + o + kHalf, x + 8);
+          }
+          if (kr_norm != nullptr && q == 0) kr_norm[m.blk * H + h] = nrm;
+        }
       }
     }
-    __syncthreads();
-    if (parity == 0) {
-      const float cnt = (float)n;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        ak[u] = (ak[u] + sm.partial[0][r][u]) / cnt;
-        av[u] = (av[u] + sm.partial[1][r][u]) / cnt;
-        ar[u] = (ar[u] + sm.partial[2][r][u]) / cnt;
-      }
-      const int64_t o = blk * row + (int64_t)h * kD + 8 * q;
-      if (k != nullptr && k_bar != nullptr) {
-        store8_bf16(k_bar + o, ak);
-        store8_bf16(k_bar + o + kHalf, ak + 8);
-      }
-      if (v != nullptr && v_bar != nullptr) {
-        store8_bf16(v_bar + o, av);
-        store8_bf16(v_bar + o + kHalf, av + 8);
-      }
-      if (kr != nullptr) {
-        float ss = 0.f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) ss += ar[u] * ar[u];
-        // the 8 threads of head h are 8 consecutive lanes (an aligned group) of one warp
-        const unsigned grp = 0xFFu << (threadIdx.x & 24);
-        ss += __shfl_xor_sync(grp, ss, 1);
-        ss += __shfl_xor_sync(grp, ss, 2);
-        ss += __shfl_xor_sync(grp, ss, 4);
-        const float nrm = sqrtf(ss);
-        const float inv = 1.0f / fmaxf(nrm, 1e-8f);
-        if (kr_hat != nullptr) {
-          float x[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) x[u] = ar[u] * inv;
-          store8_bf16(kr_hat + o, x);
-          store8_bf16(kr_hat + o + kHalf, x + 8);
-        }
-        if (kr_norm != nullptr && q == 0) kr_norm[blk * H + h] = nrm;
-      }
+    if (++stage == n_stages) {
+      stage = 0;
+      phase ^= 1u;
     }
   }
 }
@@ -347,27 +517,39 @@ extern "C" msa_status msa_pool_blocks(const void* k, const void* v, const void* 
       return msa_ok();
     }
   }
-  const size_t smem = sizeof(PoolSmem);
-  const int threads = 16 * n_heads;
   const int use_rope = (rope_theta != 0.0f && k != nullptr) ? 1 : 0;
   const double log2_theta = use_rope ? log2((double)rope_theta) : 0.0;
-  const int per_sm = 2;
-  int64_t grid = (int64_t)msa::sm_count() * per_sm;
+  // stages of S tokens of each stream (S a multiple of 4, the token groups of a warp)
+  const size_t esz = in_dtype == MSA_F32 ? 4 : 2;
+  const size_t row_bytes = (size_t)n_heads * kD * esz;
+  int S = (int)(kStageBytesTarget / (3 * row_bytes)) / 4 * 4;
+  if (S < 4) S = 4;
+  if (S > 64) S = 64;
+  int n_stages = (int)(kRingBytes / (3 * (size_t)S * row_bytes));
+  if (n_stages > 8) n_stages = 8;
+  if (n_stages < 2) return msa_fail(MSA_ERR_UNSUPPORTED, "token rows too large for the staging ring");
+  const size_t smem = (size_t)n_stages * 3 * S * row_bytes;
+  const int threads = 32 * (n_heads + 1);  // a warp per head + the producer warp
+  int64_t grid = msa::sm_count();           // one CTA per SM (the ring fills shared memory)
   if (grid > n_chunks) grid = n_chunks;
+  const int64_t per_cta = (n_chunks + grid - 1) / grid;
+  grid = (n_chunks + per_cta - 1) / per_cta;
+#define MSA_POOL_LAUNCH(T, W)                                                                                   \
+  do {                                                                                                         \
+    MSA_CUDA_TRY(cudaFuncSetAttribute(pool_kernel<T, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); \
+    pool_kernel<T, W><<<(unsigned)grid, threads, smem, s>>>(                                                    \
+        (const T*)k, (const T*)v, (const T*)kr, doc_tok_offsets, doc_chunk_offsets, n_docs, n_chunks, per_cta, \
+        n_heads, chunk, S, n_stages, log2_theta, use_rope, (__nv_bfloat16*)k_bar, (__nv_bfloat16*)v_bar,       \
+        (__nv_bfloat16*)kr_hat, kr_norm, dev_err);                                                              \
+  } while (0)
   if (in_dtype == MSA_F32) {
-    MSA_CUDA_TRY(cudaFuncSetAttribute(pool_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    pool_kernel<float><<<(unsigned)grid, threads, smem, s>>>(
-        (const float*)k, (const float*)v, (const float*)kr, doc_tok_offsets, doc_chunk_offsets, n_docs,
-        n_chunks, n_heads, chunk, log2_theta, use_rope, (__nv_bfloat16*)k_bar, (__nv_bfloat16*)v_bar,
-        (__nv_bfloat16*)kr_hat, kr_norm, dev_err);
+    if (n_heads <= 8) MSA_POOL_LAUNCH(float, 9);
+    else MSA_POOL_LAUNCH(float, 17);
   } else {
-    MSA_CUDA_TRY(cudaFuncSetAttribute(pool_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem));
-    pool_kernel<__nv_bfloat16><<<(unsigned)grid, threads, smem, s>>>(
-        (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (const __nv_bfloat16*)kr, doc_tok_offsets,
-        doc_chunk_offsets, n_docs, n_chunks, n_heads, chunk, log2_theta, use_rope, (__nv_bfloat16*)k_bar,
-        (__nv_bfloat16*)v_bar, (__nv_bfloat16*)kr_hat, kr_norm, dev_err);
+    if (n_heads <= 8) MSA_POOL_LAUNCH(__nv_bfloat16, 9);
+    else MSA_POOL_LAUNCH(__nv_bfloat16, 17);
   }
+#undef MSA_POOL_LAUNCH
   MSA_CUDA_TRY(cudaGetLastError());
   return msa_ok();
 }
