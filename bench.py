@@ -35,7 +35,7 @@ TOKENS_PER_DOC = 1000
 THETA = 1e6
 # DRAM bytes per (block, layer) of the routing GEMM, read + write, from the ncu captures in
 # profiles/ (2M-token bank, same kernels), scaled by blocks; None where not captured yet.
-GEMM_TRAFFIC_PER_BLOCK_LAYER = {"bf16": None, "e4m3": 1039.8}
+GEMM_TRAFFIC_PER_BLOCK_LAYER = {"bf16": None, "e4m3": 1039.5}
 
 
 def log(*a):
@@ -240,8 +240,9 @@ def time_pool(dev):
     torch.cuda.synchronize(dev)
     ms = s.elapsed_time(e) / reps
     by = n * 3 * H * D * 2 + C * (3 * H * D * 2 + H * 4)
+    hbm = measured_peaks()[0]
     return {"tokens": n, "blocks": C, "ms": round(ms, 4), "gbs": round(by / ms / 1e6, 1),
-            "bytes_per_token": round(by / n, 1)}
+            "hbm_frac": round(by / ms / 1e6 / hbm, 4), "bytes_per_token": round(by / n, 1)}
 
 
 # ----------------------------------------------------------------------------- GPU arm

@@ -256,6 +256,28 @@ def test_route_f8_layers_without_margin_fall_back_to_the_bf16_filter(msa):
         check_topk(ids[0, l], sc[0, l], doc_scores, k)
 
 
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_route_many_equal_documents_take_the_lowest_ids(msa, flags):
+    # 2,100 documents with identical blocks: every score ties, so the selection is the
+    # lowest ids (more documents share the threshold score than the selection collects at
+    # once, exercising the ordered fallback); ties cannot be certified, so the
+    # uncertified bit may be set
+    n_docs, per, k = 2100, 2, 16
+    lens = np.full(n_docs, 64 * per)
+    bank = syn.make_bank(15, n_docs, lens, 1)
+    row = syn.fill(15, syn.STREAM_KRBAR, 0, 0, 0, 1, H * D).reshape(H, D).astype(np.float64)
+    row /= np.linalg.norm(row, axis=1, keepdims=True)
+    bits = np.broadcast_to(syn.f32_to_bf16_bits(row.astype(np.float32)), (1, bank.n_chunks, H, D)).copy()
+    kr_hat = bf16_tensor(bits)
+    coffs = _dev_i64(bank.doc_chunk_offsets)
+    T = 1 if flags == 1 else 40
+    qr = syn.fill(15, syn.STREAM_QR, 0, 0, 0, T * HQ, D).reshape(1, T, HQ, D)
+    ids, sc, err = _route_gpu(msa, qr, [0, T], kr_hat, coffs, n_docs, bank.n_chunks, 1, k, flags)
+    assert err & ~msa.MSA_DEVERR_UNCERTIFIED == 0
+    assert ids[0, 0].tolist() == list(range(k))
+    assert np.all(sc[0, 0] == sc[0, 0, 0])
+
+
 def _e4m3_decode(b):
     b = b.astype(np.int64)
     sign = np.where(b >> 7, -1.0, 1.0)

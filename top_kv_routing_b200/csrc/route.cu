@@ -481,8 +481,12 @@ __global__ void __launch_bounds__(kTopkThreads) merge_topk_kernel(const unsigned
 // grid (L, B), 1024 threads: the k_sel best documents of (b, l) by score (equal scores:
 // smaller id first), as keys in descending order (key 0: no document).  Radix selection
 // on the ordered score bits, 8 bits a pass (histograms with warp-aggregated shared
-// atomics), then the documents above the threshold value plus the lowest ids at it.
+// atomics, kSelBatch independent loads per thread in flight), then one pass collecting
+// the documents above the threshold value and those at it; the lowest ids at it are
+// taken (an ordered scan only when more than kSelEqCap documents share that value).
 constexpr int kSelThreads = 1024;
+constexpr int kSelBatch = 16;
+constexpr int kSelEqCap = 1024;
 
 __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* __restrict__ doc_score, int L,
                                                                 int n_docs, int k_sel,
@@ -491,20 +495,23 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
                                                                 const int32_t* __restrict__ only) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_need, s_gt, s_taken;
+  __shared__ int s_need, s_gt, s_eq, s_taken;
   __shared__ int wsum[kSelThreads / 32];
   __shared__ unsigned long long keys[kMaxCandidates];
+  __shared__ int eq_docs[kSelEqCap];
   const int l = blockIdx.x, b = blockIdx.y;
   if (only != nullptr && only[l] == 0) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* sc = doc_score + ((int64_t)b * L + l) * n_docs;
   unsigned long long* o = out + ((int64_t)b * L + l) * k_sel;
   const int K = min(k_sel, n_docs);
+  constexpr int kSpan = kSelThreads * kSelBatch;
   if (tid == 0) {
     s_prefix = 0u;
     s_mask = 0u;
     s_need = K;
     s_gt = 0;
+    s_eq = 0;
     s_taken = 0;
   }
   if (K > 0) {
@@ -512,13 +519,21 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
       __syncthreads();
       const uint32_t prefix = s_prefix, mask = s_mask;
-      for (int d0 = 0; d0 < n_docs; d0 += kSelThreads) {  // (uniform trip count for the match)
-        const int d = d0 + tid;
-        const uint32_t u = d < n_docs ? sc[d] : 0u;
-        const bool in = d < n_docs && (u & mask) == prefix;
-        const uint32_t bin = in ? (u >> shift) & 255u : 256u;
-        const uint32_t same = __match_any_sync(0xffffffffu, bin);
-        if (in && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+      for (int d0 = 0; d0 < n_docs; d0 += kSpan) {  // (uniform trip count for the match)
+        uint32_t u[kSelBatch];
+#pragma unroll
+        for (int j = 0; j < kSelBatch; ++j) {
+          const int d = d0 + j * kSelThreads + tid;
+          u[j] = d < n_docs ? __ldcg(sc + d) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < kSelBatch; ++j) {
+          const int d = d0 + j * kSelThreads + tid;
+          const bool in = d < n_docs && (u[j] & mask) == prefix;
+          const uint32_t bin = in ? (u[j] >> shift) & 255u : 256u;
+          const uint32_t same = __match_any_sync(0xffffffffu, bin);
+          if (in && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+        }
       }
       __syncthreads();
       if (warp == 0) {
@@ -551,35 +566,79 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
       }
       __syncthreads();
     }
-    // the documents above the threshold value, then the lowest ids at it
+    // the documents above the threshold value, and those at it
     const uint32_t thr = s_prefix;
     const int need = s_need;
-    for (int d = tid; d < n_docs; d += kSelThreads) {
-      const uint32_t u = sc[d];
-      if (u > thr) keys[atomicAdd(&s_gt, 1)] = ((unsigned long long)u << 32) | (0xFFFFFFFFull - (uint32_t)d);
+    for (int d0 = 0; d0 < n_docs; d0 += kSpan) {
+      uint32_t u[kSelBatch];
+#pragma unroll
+      for (int j = 0; j < kSelBatch; ++j) {
+        const int d = d0 + j * kSelThreads + tid;
+        u[j] = d < n_docs ? __ldcg(sc + d) : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < kSelBatch; ++j) {
+        const int d = d0 + j * kSelThreads + tid;
+        if (d >= n_docs) continue;
+        if (u[j] > thr) {
+          keys[atomicAdd(&s_gt, 1)] = ((unsigned long long)u[j] << 32) | (0xFFFFFFFFull - (uint32_t)d);
+        } else if (u[j] == thr) {
+          const int slot = atomicAdd(&s_eq, 1);
+          if (slot < kSelEqCap) eq_docs[slot] = d;
+        }
+      }
     }
     __syncthreads();
     const int n_gt = s_gt;  // = K - need
-    for (int d0 = 0; d0 < n_docs; d0 += kSelThreads) {
-      const int taken = s_taken;
-      if (taken >= need) break;  // (uniform: read after the barrier below)
-      const int d = d0 + tid;
-      const bool eq = d < n_docs && sc[d] == thr;
-      const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) wsum[warp] = __popc(bal);
+    const int n_eq = s_eq;
+    if (n_eq <= kSelEqCap) {
+      // the need lowest ids among the documents at the threshold value
+      int n_pow = 1;
+      while (n_pow < n_eq) n_pow <<= 1;
+      for (int i = n_eq + tid; i < n_pow; i += kSelThreads) eq_docs[i] = 0x7FFFFFFF;
       __syncthreads();
-      int before = 0;
-      for (int w = 0; w < warp; ++w) before += wsum[w];
-      const int rank = taken + before + __popc(bal & ((1u << lane) - 1u));
-      if (eq && rank < need) keys[n_gt + rank] = ((unsigned long long)thr << 32) | (0xFFFFFFFFull - (uint32_t)d);
-      __syncthreads();
-      if (tid == 0) {
-        int tot = 0;
-        for (int w = 0; w < kSelThreads / 32; ++w) tot += wsum[w];
-        s_taken = taken + tot;
+      for (int kk = 2; kk <= n_pow; kk <<= 1) {  // ascending bitonic sort
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+          for (int i = tid; i < n_pow; i += kSelThreads) {
+            const int ixj = i ^ jj;
+            if (ixj > i) {
+              const int x = eq_docs[i], y = eq_docs[ixj];
+              const bool up = (i & kk) == 0;
+              if (up ? (x > y) : (x < y)) {
+                eq_docs[i] = y;
+                eq_docs[ixj] = x;
+              }
+            }
+          }
+          __syncthreads();
+        }
       }
-      __syncthreads();
+      for (int i = tid; i < need; i += kSelThreads)
+        keys[n_gt + i] = ((unsigned long long)thr << 32) | (0xFFFFFFFFull - (uint32_t)eq_docs[i]);
+    } else {
+      // very many documents share the threshold value: take the lowest ids in order
+      for (int d0 = 0; d0 < n_docs; d0 += kSelThreads) {
+        const int taken = s_taken;
+        if (taken >= need) break;  // (uniform: read after the barrier below)
+        const int d = d0 + tid;
+        const bool eq = d < n_docs && sc[d] == thr;
+        const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) wsum[warp] = __popc(bal);
+        __syncthreads();
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += wsum[w];
+        const int rank = taken + before + __popc(bal & ((1u << lane) - 1u));
+        if (eq && rank < need) keys[n_gt + rank] = ((unsigned long long)thr << 32) | (0xFFFFFFFFull - (uint32_t)d);
+        __syncthreads();
+        if (tid == 0) {
+          int tot = 0;
+          for (int w = 0; w < kSelThreads / 32; ++w) tot += wsum[w];
+          s_taken = taken + tot;
+        }
+        __syncthreads();
+      }
     }
+    __syncthreads();
     const int n_pow2 = K <= 1 ? 1 : (1 << (32 - __clz(K - 1)));
     for (int i = K + tid; i < n_pow2; i += kSelThreads) keys[i] = 0ull;
     __syncthreads();
