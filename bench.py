@@ -113,6 +113,41 @@ def smi_id(dev) -> str:
     return f"{dom:08X}:{bus:02X}:{devno:02X}.0"
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_env():
+    """(world, rank, local rank) from the launcher's environment (1, 0, 0 without one)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_ranks(backend: str, timeout_s: int = 600):
+    """One process per GPU: a process group when there is more than one rank."""
+    import datetime
+
+    import torch.distributed as dist
+    world, rank, local = rank_env()
+    if world > 1:
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return world, rank, local
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of a list of floats over all ranks (the list itself with one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def replica_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job units per second: every replica's units over the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- workload
 
 def set_bank_size(n_docs: int) -> None:
@@ -254,11 +289,7 @@ def run_gpu(args):
     import top_kv_routing_b200 as msa
     from top_kv_routing_b200.engine import SparseMemory
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    world, rank, local = init_ranks("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     hbm_peak, bf16_peak, bf16_sus, peak_src = measured_peaks()
@@ -382,10 +413,7 @@ def run_gpu(args):
     h2d = host["qr"][0].numel() * 2 + (dq.numel() + dk.numel() + dv.numel()) * 2
     d2h = host["ids"][0].numel() * 4 + host["scores"][0].numel() * 4 + host["out"][0].numel() * 2
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
     pool = time_pool(dev) if (rank == 0 and not args.no_pool) else None
     if world > 1:
         dist.barrier()
@@ -395,7 +423,7 @@ def run_gpu(args):
 
     ms = total_ms / args.steps
     units = N_TOKENS * args.steps * world
-    value = units / (total_ms / 1e3)
+    value = replica_throughput(N_TOKENS * args.steps, world, total_ms)
     elem = 1 if f8 else 2
     algo_bytes = L * bank.n_chunks * H * D * elem
     achieved = algo_bytes / (gemm_avg / 1e3) / 1e9
@@ -454,7 +482,8 @@ def run_gpu(args):
                      "gbs": round(achieved, 1), "hbm_frac": round(achieved / hbm_peak, 4),
                      "tflops": round(tflops, 1), "tensor_frac": round(tflops / tc_peak, 4),
                      "roofline_ms": round(max(t_hbm, t_tc) * 1e3, 4)},
-        "e2e": {"value": round(units / (e2e_ms / 1e3), 1), "unit": "bank tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(replica_throughput(N_TOKENS * args.steps, world, e2e_ms), 1), "unit": "bank tokens/s",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
@@ -513,12 +542,14 @@ def run_reference(args):
     vals = []
     for _ in range(args.warmup):
         cpu_baseline(min(2.0, args.cpu_seconds))
+    t0 = time.time()
     for _ in range(args.steps):
         vals.append(cpu_baseline(args.cpu_seconds / max(1, args.steps)))
+    step_ms = (time.time() - t0) * 1e3 / max(1, args.steps)
     v = float(np.mean([x["value"] for x in vals]))
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "bank tokens/s",
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": round(step_ms, 1), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD},
             "cpu_baseline": {"value": round(v, 3), "unit": "bank tokens/s", "cores": 1, "kind": "oracle",
