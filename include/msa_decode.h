@@ -40,6 +40,7 @@ msa_status msa_sparse_decode_workspace_size(int32_t n_queries, int32_t n_layers,
  *           (msa_gather_kv output); mem_len DEVICE int32 [n_queries][n_layers]
  *   out     DEVICE bf16 [n_queries][n_layers][n_q_heads][head_dim]
  *   head_dim = 128; n_q_heads / n_kv_heads in {1, 2, 4, 8}; n_kv_heads <= 16.
+ *   q, mem_kv, local_k, local_v  16-byte aligned.
  *   workspace  DEVICE, >= msa_sparse_decode_workspace_size bytes, 16-byte aligned, zeroed
  *              (e.g. cudaMemset) once before its first use; every call leaves it ready for
  *              the next (its arrival counters return to zero).  Calls that share a

@@ -19,10 +19,12 @@
 // then the 8 warps' (max, sum, O) are merged in shared memory.  With one split the CTA
 // writes the output; with several, each publishes its partial and the last CTA of the
 // (b, l, h) to arrive (a self-resetting counter) merges them.  The last CTA of query b
-// advances local_len[b].  Split 0 appends the rotated new key (rounded to the cache's
-// bf16) and the new value to the cache and folds that key into the state of its last
-// warp directly, in fp32.  RoPE angles: p * w_j with w_j / pi precomputed in fp64 on the
-// host; the product is reduced modulo 2 pi in fp64 and evaluated by fp32 sincospif.
+// advances local_len[b].  The rotated new key (rounded to the cache's bf16) and the new
+// value go to the cache (split 0) and into the zero-filled row of the last local tile
+// in shared memory, so they are scored like every other key.  RoPE angles: p * w_j with
+// w_j / pi in fp64, the product reduced modulo 2 pi in fp64, fp32 sincospif.  The query
+// fragments are built once per CTA in shared memory in MMA order (the kernel's per-launch
+// path is kept short: it runs with a cold instruction cache on every launch).
 #include "common.cuh"
 #include "msa_decode.h"
 
@@ -46,10 +48,6 @@ constexpr int kMaxSplits = 4;
 constexpr int kRedStride = kD + 4;                       // merge rows, padded against bank conflicts
 constexpr float kLog2e = 1.4426950408889634f;
 static_assert(kWarps * 8 * kRedStride * 4 <= kRingBytes, "merge buffer reuses the ring");
-
-struct RopeTable {
-  double w_over_pi[kHalf];  // theta^(-2j/d) / pi
-};
 
 // Workspace: per (b, l, h, split slot) the partial output [G][128] and (max, sum) per head,
 // then one arrival counter per (b, l, h) and one per query b.
@@ -119,17 +117,21 @@ template <int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
     const __nv_bfloat16* __restrict__ v_new, int L, int H,
-    // rows [0, len) are read; row len is written by split 0 only and read by nobody here
+    // rows [0, len) are read; row len is written by split 0 and read by nobody here
     __nv_bfloat16* local_k, __nv_bfloat16* local_v, int32_t* local_len, int cap,
     const __nv_bfloat16* __restrict__ mem_kv, const int32_t* __restrict__ mem_len, int M_max, int pos_off,
-    const __grid_constant__ RopeTable rope, float qscale, int splits, float* part, float2* stat, int* unit_count,
-    int* query_count, __nv_bfloat16* __restrict__ out, int32_t* dev_err) {
+    double log2_theta, float qscale, int splits, float* part, float2* stat, int* unit_count, int* query_count,
+    __nv_bfloat16* __restrict__ out, int32_t* dev_err) {
   extern __shared__ __align__(128) unsigned char ring[];
-  __shared__ __align__(16) float qs[8][kD];
-  __shared__ __align__(16) float knew[kD];
-  __shared__ __align__(16) float vnew[kD];
+  // query fragments in MMA order: row g*4 + t holds thread (g, t)'s 8 k-steps x 4 words,
+  // the 16-byte chunk of k-step ks at position ks ^ (row & 7)
+  __shared__ __align__(16) uint32_t qfrag[32][32];
+  __shared__ __align__(16) __nv_bfloat16 knew[kD];  // the rotated new key (as cached)
+  __shared__ __align__(16) __nv_bfloat16 vnew[kD];
   __shared__ float2 cs[kHalf];
   __shared__ float2 wml[kWarps][8];
+  __shared__ float fac[kWarps][8];
+  __shared__ float s_mx[8], s_den[8];
   __shared__ int s_last;
   const int split = blockIdx.x, h = blockIdx.y;
   const int b = blockIdx.z / L;
@@ -154,32 +156,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     __syncthreads();
     if (tid == 0) arrived = arrive_release(&query_count[b]);
   } else {
-    // loads that depend on nothing else start first
-    float qx[2][2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int e = tid + r * kThreads, gg = e / kHalf, j = e % kHalf;
-      qx[r][0] = qx[r][1] = 0.f;
-      if (gg < G) {
-        const __nv_bfloat16* qp = q + (bl * Hq + (int64_t)h * G + gg) * kD;
-        qx[r][0] = __bfloat162float(qp[j]);
-        qx[r][1] = __bfloat162float(qp[j + kHalf]);
-      }
+    // loads that depend on nothing else start first: thread (head gg, m) takes dims 2m,
+    // 2m+1 and their rotate-half partners 2m+64, 2m+65
+    const int gg = tid >> 5, mq = tid & 31;
+    uint32_t qlo = 0u, qhi = 0u;
+    if (gg < G) {
+      const __nv_bfloat16* qp = q + (bl * Hq + (int64_t)h * G + gg) * kD;
+      qlo = *reinterpret_cast<const uint32_t*>(qp + 2 * mq);
+      qhi = *reinterpret_cast<const uint32_t*>(qp + 2 * mq + kHalf);
     }
     float kx0 = 0.f, kx1 = 0.f;
     __nv_bfloat16 vx = __float2bfloat16_rn(0.f);
-    if (split == 0) {
-      if (tid < kHalf) {
-        kx0 = __bfloat162float(k_new[uh * kD + tid]);
-        kx1 = __bfloat162float(k_new[uh * kD + tid + kHalf]);
-      } else if (tid < kHalf + kD) {
-        vx = v_new[uh * kD + tid - kHalf];
-      }
+    if (tid < kHalf) {
+      kx0 = __bfloat162float(k_new[uh * kD + tid]);
+      kx1 = __bfloat162float(k_new[uh * kD + tid + kHalf]);
+    } else if (tid < kHalf + kD) {
+      vx = v_new[uh * kD + tid - kHalf];
     }
 
-    // ---- this warp's tiles: the first ones are requested before anything else
+    // ---- this warp's tiles (memory tiles, then local tiles; the new key, row len, rides
+    // in the last local tile): the first ones are requested before anything else
     const int nt_mem = (M + kTileKeys - 1) / kTileKeys;
-    const int nt = nt_mem + (len + kTileKeys - 1) / kTileKeys;
+    const int nt = nt_mem + len / kTileKeys + 1;
     const int per = (nt + splits - 1) / splits;
     const int t0 = min(nt, split * per), t1 = min(nt, t0 + per);
     const int first = t0 + warp;
@@ -190,29 +188,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     const __nv_bfloat16* locv = local_v + uh * (int64_t)cap * kD;
     const uint32_t my_ring = smem_u32(ring) + warp * (kStages * kStageBytes);
 
-    auto tile_rows = [&](int i, const __nv_bfloat16*& kp, const __nv_bfloat16*& vp) -> int {
+    struct Tile {
+      const __nv_bfloat16 *kp, *vp;
+      int n_copy;   // rows read from memory
+      int nvalid;   // rows that are keys
+      int new_row;  // row of the new key, or -1
+    };
+    auto tile = [&](int i) -> Tile {
       const int ti = first + i * kWarps;
+      Tile tl;
       if (ti < nt_mem) {
-        kp = memk + (int64_t)ti * kTileKeys * kD;
-        vp = memv + (int64_t)ti * kTileKeys * kD;
-        return min(kTileKeys, M - ti * kTileKeys);
+        tl.kp = memk + (int64_t)ti * kTileKeys * kD;
+        tl.vp = memv + (int64_t)ti * kTileKeys * kD;
+        tl.n_copy = tl.nvalid = min(kTileKeys, M - ti * kTileKeys);
+        tl.new_row = -1;
+      } else {
+        const int r0 = (ti - nt_mem) * kTileKeys;
+        tl.kp = lock + (int64_t)r0 * kD;
+        tl.vp = locv + (int64_t)r0 * kD;
+        tl.n_copy = max(0, min(kTileKeys, len - r0));
+        tl.nvalid = min(kTileKeys, len + 1 - r0);
+        tl.new_row = len - r0 < kTileKeys ? len - r0 : -1;
       }
-      const int j = ti - nt_mem;
-      kp = lock + (int64_t)j * kTileKeys * kD;
-      vp = locv + (int64_t)j * kTileKeys * kD;
-      return min(kTileKeys, len - j * kTileKeys);
+      return tl;
     };
     auto issue = [&](int i) {
-      const __nv_bfloat16 *kp, *vp;
-      const int nvalid = tile_rows(i, kp, vp);
+      const Tile tl = tile(i);
       const uint32_t st = my_ring + (i % kStages) * kStageBytes;
       const int chunk = lane & 15;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int row = 2 * j + (lane >> 4);  // 0..15 K rows, 16..31 V rows
         const int key = row & 15;
-        const bool ok = key < nvalid;
-        const __nv_bfloat16* src = (j < 8 ? kp : vp) + (ok ? key * kD + chunk * 8 : 0);
+        const bool ok = key < tl.n_copy;
+        const __nv_bfloat16* src = (j < 8 ? tl.kp : tl.vp) + (ok ? key * kD + chunk * 8 : 0);
         cp_async16(st + row * kRowBytes + ((chunk ^ (row & 7)) << 4), src, ok ? 16u : 0u);
       }
     };
@@ -222,11 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
       cp_async_commit();
     }
 
-    // ---- rotated, scaled query (rows >= G are zero) and, in split 0, the new key
+    // ---- RoPE angles of this step's position: w_j / pi in fp64, the product reduced
+    // modulo 2 pi in fp64, fp32 sincospif
     const double pos = (double)pos_off + (double)len;
     if (tid < kHalf) {
-      double u = pos * rope.w_over_pi[tid];  // angle / pi
-      u -= 2.0 * rint(0.5 * u);             // in [-1, 1]
+      double u = pos * (exp2(-2.0 * (double)tid / (double)kD * log2_theta) * 0.31830988618379067154);
+      u -= 2.0 * rint(0.5 * u);  // in [-1, 1]
       float sn, c;
       sincospif((float)u, &sn, &c);
       cs[tid] = make_float2(c, sn);
@@ -235,71 +245,81 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     // every thread has read local_len[b]: announce it (the last CTA of the query to
     // arrive advances the length at its end)
     if (tid == 0) arrived = arrive_release(&query_count[b]);
+    {  // rotated, scaled query pairs -> MMA fragments (bf16 value and bf16 residual)
+      float r[4] = {0.f, 0.f, 0.f, 0.f};  // dims 2m, 2m+1, 2m+64, 2m+65
+      if (gg < G) {
+        const float2 a = msa::bf16x2_to_float2(qlo), bb = msa::bf16x2_to_float2(qhi);
+        const float2 c0 = cs[2 * mq], c1 = cs[2 * mq + 1];
+        r[0] = (a.x * c0.x - bb.x * c0.y) * qscale;
+        r[1] = (a.y * c1.x - bb.y * c1.y) * qscale;
+        r[2] = (bb.x * c0.x + a.x * c0.y) * qscale;
+        r[3] = (bb.y * c1.x + a.y * c1.y) * qscale;
+      }
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int e = tid + r * kThreads, gg = e / kHalf, j = e % kHalf;
-      const float2 c = cs[j];
-      qs[gg][j] = (qx[r][0] * c.x - qx[r][1] * c.y) * qscale;
-      qs[gg][j + kHalf] = (qx[r][1] * c.x + qx[r][0] * c.y) * qscale;
+      for (int p2 = 0; p2 < 2; ++p2) {
+        const int d = 2 * mq + p2 * kHalf;  // first dim of the pair
+        const int ks = d >> 4, c = d & 15, tq = (c & 7) >> 1, half = c >> 3;
+        const int row = gg * 4 + tq;
+        uint32_t hi, lo;
+        split_pair(r[2 * p2], r[2 * p2 + 1], hi, lo);
+        uint32_t* w = &qfrag[row][((ks ^ (row & 7)) << 2)];
+        w[half ? 2 : 0] = hi;
+        w[half ? 3 : 1] = lo;
+      }
     }
-    if (split == 0) {
-      const int64_t cache_row = (uh * (int64_t)cap + len) * kD;
-      if (tid < kHalf) {
-        const float2 c = cs[tid];
-        const __nv_bfloat16 lo = __float2bfloat16_rn(kx0 * c.x - kx1 * c.y);
-        const __nv_bfloat16 hi = __float2bfloat16_rn(kx1 * c.x + kx0 * c.y);
+    if (tid < kHalf) {  // the new key, rotated and rounded to the cache's bf16
+      const float2 c = cs[tid];
+      const __nv_bfloat16 lo = __float2bfloat16_rn(kx0 * c.x - kx1 * c.y);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(kx1 * c.x + kx0 * c.y);
+      knew[tid] = lo;
+      knew[tid + kHalf] = hi;
+      if (split == 0) {
+        const int64_t cache_row = (uh * (int64_t)cap + len) * kD;
         local_k[cache_row + tid] = lo;
         local_k[cache_row + tid + kHalf] = hi;
-        knew[tid] = __bfloat162float(lo);
-        knew[tid + kHalf] = __bfloat162float(hi);
-      } else if (tid < kHalf + kD) {
-        const int j = tid - kHalf;
-        local_v[cache_row + j] = vx;
-        vnew[j] = __bfloat162float(vx);
       }
+    } else if (tid < kHalf + kD) {
+      const int j = tid - kHalf;
+      vnew[j] = vx;
+      if (split == 0) local_v[(uh * (int64_t)cap + len) * kD + j] = vx;
     }
     __syncthreads();
 
-    // query fragments: rows g = bf16(q'), rows g + 8 = bf16 residual
     uint32_t qa[8][4];
+    {
+      const int row = g * 4 + t;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const float2 x = *reinterpret_cast<const float2*>(&qs[g][16 * ks + 2 * t]);
-      const float2 y = *reinterpret_cast<const float2*>(&qs[g][16 * ks + 8 + 2 * t]);
-      split_pair(x.x, x.y, qa[ks][0], qa[ks][1]);
-      split_pair(y.x, y.y, qa[ks][2], qa[ks][3]);
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint4 w = *reinterpret_cast<const uint4*>(&qfrag[row][(ks ^ (row & 7)) << 2]);
+        qa[ks][0] = w.x;
+        qa[ks][1] = w.y;
+        qa[ks][2] = w.z;
+        qa[ks][3] = w.w;
+      }
     }
 
     float o[16][4];
 #pragma unroll
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     float m = -INFINITY, lsum = 0.f;
-    if (split == 0 && warp == kWarps - 1) {
-      // the new key, in fp32: every lane owns dims 8n + 2t + {0, 1} of its head g
-      float d = 0.f;
-#pragma unroll
-      for (int n = 0; n < 16; ++n) {
-        const int c = 8 * n + 2 * t;
-        d = fmaf(qs[g][c], knew[c], d);
-        d = fmaf(qs[g][c + 1], knew[c + 1], d);
-        o[n][0] = vnew[c];
-        o[n][1] = vnew[c + 1];
-      }
-      d += __shfl_xor_sync(0xffffffffu, d, 1);
-      d += __shfl_xor_sync(0xffffffffu, d, 2);
-      m = d;
-      lsum = t == 0 ? 1.f : 0.f;
-    }
-
     for (int i = 0; i < my_n; ++i) {
       __syncwarp();  // every lane is done with the stage about to be refilled
       if (i + kStages - 1 < my_n) issue(i + kStages - 1);
       cp_async_commit();
       cp_async_wait<kStages - 1>();
       __syncwarp();
-      const __nv_bfloat16 *kp, *vp;
-      const int nvalid = tile_rows(i, kp, vp);
+      const Tile tl = tile(i);
       const uint32_t st = my_ring + (i % kStages) * kStageBytes;
+      if (tl.new_row >= 0) {  // the new key and value into their (zero-filled) rows
+        const int row = (lane < 16 ? 0 : kTileKeys) + tl.new_row, chunk = lane & 15;
+        const uint4 w = *reinterpret_cast<const uint4*>((lane < 16 ? knew : vnew) + 8 * chunk);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(st + row * kRowBytes +
+                                                                          ((chunk ^ (row & 7)) << 4)),
+                     "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w)
+                     : "memory");
+        __syncwarp();
+      }
+      const int nvalid = tl.nvalid;
 
       // two accumulators per 8-key half (even / odd k-steps) keep the MMA chains short
       float s[2][2][4];
@@ -372,27 +392,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
       *reinterpret_cast<float2*>(&red[(warp * 8 + g) * kRedStride + 8 * n + 2 * t]) =
           make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
     __syncthreads();
+    if (tid < 64) {  // per head (8 lanes each): every warp's weight, and the sum
+      const int hg = tid >> 3, w = tid & 7;
+      const float2 st = wml[w][hg];
+      float mx = st.x;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      const float f = st.y > 0.f ? exp2f(st.x - mx) : 0.f;
+      float den = f * st.y;
+      den += __shfl_xor_sync(0xffffffffu, den, 1);
+      den += __shfl_xor_sync(0xffffffffu, den, 2);
+      den += __shfl_xor_sync(0xffffffffu, den, 4);
+      fac[w][hg] = splits == 1 ? f / den : f;
+      if (w == 0) {
+        s_mx[hg] = mx;
+        s_den[hg] = den;
+      }
+    }
+    __syncthreads();
     const int64_t unit = uh * kMaxSplits + split;
     for (int oi = tid; oi < G * kD; oi += kThreads) {
-      const int gg = oi / kD, d = oi % kD;
-      float mx = -INFINITY;
+      const int hg = oi / kD, d = oi % kD;
+      float num = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, wml[w][gg].x);
-      float num = 0.f, den = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float2 st = wml[w][gg];
-        if (st.y > 0.f) {
-          const float f = exp2f(st.x - mx);
-          num = fmaf(f, red[(w * 8 + gg) * kRedStride + d], num);
-          den = fmaf(f, st.y, den);
-        }
-      }
+      for (int w = 0; w < kWarps; ++w) num = fmaf(fac[w][hg], red[(w * 8 + hg) * kRedStride + d], num);
       if (splits == 1) {
-        out[(bl * Hq + (int64_t)h * G + gg) * kD + d] = __float2bfloat16_rn(num / den);
+        out[(bl * Hq + (int64_t)h * G + hg) * kD + d] = __float2bfloat16_rn(num);
       } else {
         part[unit * G * kD + oi] = num;
-        if (d == 0) stat[unit * G + gg] = make_float2(mx, den);
+        if (d == 0) stat[unit * G + hg] = make_float2(s_mx[hg], s_den[hg]);
       }
     }
   }
@@ -408,19 +437,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
       const int64_t unit0 = uh * kMaxSplits;
       if (!full) {
         for (int oi = tid; oi < G * kD; oi += kThreads) {
-          const int gg = oi / kD;
+          const int hg = oi / kD;
           float mx = -INFINITY;
-          for (int sp = 0; sp < splits; ++sp) mx = fmaxf(mx, __ldcg(&stat[(unit0 + sp) * G + gg]).x);
+          for (int sp = 0; sp < splits; ++sp) mx = fmaxf(mx, __ldcg(&stat[(unit0 + sp) * G + hg]).x);
           float num = 0.f, den = 0.f;
           for (int sp = 0; sp < splits; ++sp) {
-            const float2 st = __ldcg(&stat[(unit0 + sp) * G + gg]);
+            const float2 st = __ldcg(&stat[(unit0 + sp) * G + hg]);
             if (st.y > 0.f) {
               const float w = exp2f(st.x - mx);
               num = fmaf(w, __ldcg(&part[(unit0 + sp) * G * kD + oi]), num);
               den = fmaf(w, st.y, den);
             }
           }
-          out[(bl * Hq + (int64_t)h * G + gg) * kD + (oi % kD)] = __float2bfloat16_rn(num / den);
+          out[(bl * Hq + (int64_t)h * G + hg) * kD + (oi % kD)] = __float2bfloat16_rn(num / den);
         }
       }
       if (tid == 0) unit_count[uh] = 0;  // ready for the next call
@@ -461,8 +490,9 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   if (n_queries < 1 || n_layers < 1 || (int64_t)n_queries * n_layers > 65535 || local_cap < 1 || max_mem_chunks < 1)
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_queries * n_layers <= 65535)");
   if (!(rope_theta > 1.0f)) return msa_fail(MSA_ERR_INVALID_ARG, "rope_theta must be > 1");
-  if (!msa::aligned16(mem_kv) || !msa::aligned16(local_k) || !msa::aligned16(local_v) || !msa::aligned16(workspace))
-    return msa_fail(MSA_ERR_INVALID_ARG, "16-byte alignment");
+  if (!msa::aligned16(q) || !msa::aligned16(mem_kv) || !msa::aligned16(local_k) || !msa::aligned16(local_v) ||
+      !msa::aligned16(workspace))
+    return msa_fail(MSA_ERR_INVALID_ARG, "16-byte alignment (q, mem_kv, local_k, local_v, workspace)");
   const size_t need = ws_bytes(n_queries, n_layers, n_q_heads, n_kv_heads);
   if (workspace_bytes < need)
     return msa_fail(MSA_ERR_CAPACITY, "workspace too small (%zu < %zu)", workspace_bytes, need);
@@ -477,9 +507,7 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   int* unit_count = reinterpret_cast<int*>(part + ws_floats(n_queries, n_layers, n_q_heads, n_kv_heads));
   int* query_count = unit_count + units;
   const dim3 grid(splits, n_kv_heads, n_queries * n_layers);
-  RopeTable rope;
-  for (int j = 0; j < kHalf; ++j)
-    rope.w_over_pi[j] = pow((double)rope_theta, -2.0 * (double)j / (double)kD) / 3.14159265358979323846;
+  const double log2_theta = log2((double)rope_theta);
   const float qscale = softmax_scale * kLog2e;
 #define MSA_DECODE_LAUNCH(GG)                                                                                    \
   MSA_CUDA_TRY(cudaFuncSetAttribute(decode_mma_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
@@ -487,7 +515,7 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   decode_mma_kernel<GG><<<grid, kThreads, kRingBytes, s>>>(                                                       \
       (const __nv_bfloat16*)q, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_layers, n_kv_heads,     \
       (__nv_bfloat16*)local_k, (__nv_bfloat16*)local_v, local_len, local_cap, (const __nv_bfloat16*)mem_kv,        \
-      mem_len, max_mem_chunks, rope_pos_offset, rope, qscale, splits, part, stat, unit_count, query_count,        \
+      mem_len, max_mem_chunks, rope_pos_offset, log2_theta, qscale, splits, part, stat, unit_count, query_count,  \
       (__nv_bfloat16*)out, dev_err)
   switch (G) {
     case 1: MSA_DECODE_LAUNCH(1); break;
