@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_decode.argtypes = [_p, _p, _p, _p, _i32, _i32, _p, _p, _i32, _i32, _i64, _dbl,
                                        _dbl, _i32, _i32, _i32, _p]
         _lib.oracle_decode.restype = _i32
+        _lib.oracle_prefill.argtypes = [_p, _p, _p, _i32, _p, _i32, _i32, _p, _p, _i32, _i32, _i64, _dbl, _dbl,
+                                        _i32, _i32, _i32, _p]
+        _lib.oracle_prefill.restype = _i32
     return _lib
 
 
@@ -172,4 +175,25 @@ def decode(q, k_new, v_new, mem_kv, mem_len: int, local_k, local_v, local_len: i
                             _ptr(out))
     if r != 0:
         raise OverflowError("oracle decode: local cache full")
+    return out
+
+
+def prefill(q, k_new, v_new, mem_kv, mem_len: int, local_k, local_v, local_len: int, pos: int, theta: float,
+            scale: float):
+    """n new tokens for one (sequence, layer): token i is the decode step at local index
+    local_len + i, position pos + i.  q [n][Hq][d], k_new/v_new [n][H][d], mem_kv
+    [2][H][M_stride][d], local_k/local_v [H][Lcap][d] float64 (updated in place).
+    Returns out [n][Hq][d] (double)."""
+    q, k_new, v_new, mem_kv = _f32(q), _f32(k_new), _f32(v_new), _f32(mem_kv)
+    n, Hq, d = q.shape
+    H = k_new.shape[1]
+    M_stride = mem_kv.shape[2]
+    assert local_k.dtype == np.float64 and local_k.flags.c_contiguous
+    assert local_v.dtype == np.float64 and local_v.flags.c_contiguous
+    Lcap = local_k.shape[1]
+    out = np.empty((n, Hq, d), dtype=np.float64)
+    r = lib().oracle_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), n, _ptr(mem_kv), mem_len, M_stride, _ptr(local_k),
+                             _ptr(local_v), local_len, Lcap, pos, theta, scale, Hq, H, d, _ptr(out))
+    if r != 0:
+        raise OverflowError("oracle prefill: local cache full")
     return out

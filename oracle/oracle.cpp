@@ -357,4 +357,21 @@ int32_t oracle_decode(const float* q, const float* k_new, const float* v_new, co
   return 0;
 }
 
+// Prefill of n_new tokens (a query's own tokens): token i is the decode step at local
+// index local_len + i and position pos + i, so it sees the memory and every local key up
+// to and including its own.  [README] 推理流水线 step 3 / [NOTES] 推理全流程: the query is
+// processed over [selected memory ; local context] before generation continues.
+int32_t oracle_prefill(const float* q, const float* k_new, const float* v_new, int32_t n_new, const float* mem_kv,
+                       int32_t M, int32_t M_stride, double* local_k, double* local_v, int32_t local_len,
+                       int32_t Lcap, int64_t pos, double theta, double scale, int32_t Hq, int32_t H, int32_t d,
+                       double* out) {
+  for (int32_t i = 0; i < n_new; ++i) {
+    const int32_t r = oracle_decode(q + (size_t)i * Hq * d, k_new + (size_t)i * H * d, v_new + (size_t)i * H * d,
+                                    mem_kv, M, M_stride, local_k, local_v, local_len + i, Lcap, pos + i, theta,
+                                    scale, Hq, H, d, out + (size_t)i * Hq * d);
+    if (r != 0) return r;
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -371,3 +371,66 @@ def test_decode_local_cache_full_is_an_error():
     with pytest.raises(OverflowError):
         oracle.decode(np.zeros((1, 4)), np.zeros((1, 4)), np.zeros((1, 4)), np.zeros((2, 1, 1, 4)), 0,
                       lk, lv, 2, 0, 1e6, 1.0)
+
+
+def test_prefill_is_masked_gqa_attention_over_memory_prefix_and_causal_block():
+    # Prefill of T new tokens with memory and an existing local prefix: token i attends
+    # the memory, the prefix and the new tokens up to itself.  Compare with torch's
+    # scaled_dot_product_attention (fp64) given the rotated queries and keys and that mask.
+    rng = np.random.default_rng(21)
+    Hq, H, d, T, M, pre, off = 8, 2, 32, 7, 5, 3, 4
+    mem = rng.standard_normal((2, H, M + 2, d)).astype(np.float32)
+    lk, lv = _empty_local(H, pre + T, d)
+    pk = rng.standard_normal((H, pre, d))
+    pv = rng.standard_normal((H, pre, d))
+    lk[:, :pre], lv[:, :pre] = pk, pv
+    q = rng.standard_normal((T, Hq, d)).astype(np.float32)
+    kn = rng.standard_normal((T, H, d)).astype(np.float32)
+    vn = rng.standard_normal((T, H, d)).astype(np.float32)
+    out = oracle.prefill(q, kn, vn, mem, M, lk, lv, pre, off + pre, 1e6, d ** -0.5)
+    qr = np.stack([[oracle.rope(q[i, h].astype(np.float64), off + pre + i, 1e6) for h in range(Hq)]
+                   for i in range(T)])                                        # [T][Hq][d]
+    kr = np.stack([[oracle.rope(kn[i, h].astype(np.float64), off + pre + i, 1e6) for h in range(H)]
+                   for i in range(T)])                                        # [T][H][d]
+    keys = np.concatenate([mem[0, :, :M].astype(np.float64), pk, np.transpose(kr, (1, 0, 2))], axis=1)
+    vals = np.concatenate([mem[1, :, :M].astype(np.float64), pv, np.transpose(vn.astype(np.float64), (1, 0, 2))],
+                          axis=1)                                             # [H][M+pre+T][d]
+    n = M + pre + T
+    mask = np.ones((T, n), dtype=bool)
+    for i in range(T):
+        mask[i, M + pre + i + 1:] = False
+    kk = torch.from_numpy(np.repeat(keys, Hq // H, axis=0))[None]
+    vv = torch.from_numpy(np.repeat(vals, Hq // H, axis=0))[None]
+    qq = torch.from_numpy(np.transpose(qr, (1, 0, 2)))[None]                  # [1][Hq][T][d]
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=torch.from_numpy(mask))
+    np.testing.assert_allclose(out, np.transpose(ref[0].numpy(), (1, 0, 2)), atol=1e-12)
+    np.testing.assert_allclose(lk[:, pre:pre + T], np.transpose(kr, (1, 0, 2)), atol=0)
+
+
+def test_prefill_zero_queries_average_the_visible_values():
+    rng = np.random.default_rng(22)
+    Hq, H, d, T, M = 4, 2, 16, 5, 3
+    mem = rng.standard_normal((2, H, M, d)).astype(np.float32)
+    lk, lv = _empty_local(H, T, d)
+    vn = rng.standard_normal((T, H, d)).astype(np.float32)
+    out = oracle.prefill(np.zeros((T, Hq, d), np.float32), rng.standard_normal((T, H, d)).astype(np.float32), vn,
+                         mem, M, lk, lv, 0, 0, 1e6, 0.1)
+    for i in range(T):
+        for hq in range(Hq):
+            h = hq // (Hq // H)
+            vis = np.concatenate([mem[1, h].astype(np.float64), vn[:i + 1, h].astype(np.float64)])
+            np.testing.assert_allclose(out[i, hq], vis.mean(axis=0), atol=1e-12)
+
+
+def test_prefill_of_one_token_is_a_decode_step():
+    rng = np.random.default_rng(23)
+    Hq, H, d, M = 8, 2, 16, 4
+    mem = rng.standard_normal((2, H, M, d)).astype(np.float32)
+    q = rng.standard_normal((1, Hq, d)).astype(np.float32)
+    kn = rng.standard_normal((1, H, d)).astype(np.float32)
+    vn = rng.standard_normal((1, H, d)).astype(np.float32)
+    a_k, a_v = _empty_local(H, 3, d)
+    b_k, b_v = _empty_local(H, 3, d)
+    a = oracle.prefill(q, kn, vn, mem, M, a_k, a_v, 2, 9, 1e6, 0.2)
+    b = oracle.decode(q[0], kn[0], vn[0], mem, M, b_k, b_v, 2, 9, 1e6, 0.2)
+    np.testing.assert_array_equal(a[0], b)
