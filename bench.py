@@ -280,6 +280,63 @@ def time_pool(dev):
             "hbm_frac": round(by / ms / 1e6 / hbm, 4), "bytes_per_token": round(by / n, 1)}
 
 
+PREFILL_MEM = 256  # gathered memory rows per (query, layer): 16 documents of about 16 blocks
+
+
+def prefill_flops(n_layers: int, n_q_heads: int, T: int, M: int, prefix: int = 0) -> float:
+    """Algorithmic FLOPs of one prefill block: token i of each (layer, query head) scores
+    and weighs M + prefix + i + 1 keys, 2 d FLOPs each for QK^T and for PV."""
+    keys = T * (M + prefix) + T * (T + 1) / 2
+    return 4.0 * D * n_layers * n_q_heads * keys
+
+
+def time_prefill(dev):
+    """The query's own T tokens through sparse attention over 16 gathered documents: one
+    query, every layer, no earlier local rows.  L2 is flushed before every timed launch."""
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+    M = PREFILL_MEM
+    q = torch.empty((1, L, T, HQ, D), dtype=torch.bfloat16, device=dev)
+    kn = torch.empty((1, L, T, H, D), dtype=torch.bfloat16, device=dev)
+    vn = torch.empty_like(kn)
+    syn.device_fill(q, SEED, syn.STREAM_DEC_Q, 0, 1, 0, L * T * HQ, D)
+    syn.device_fill(kn, SEED, syn.STREAM_DEC_K, 0, 1, 0, L * T * H, D)
+    syn.device_fill(vn, SEED, syn.STREAM_DEC_V, 0, 1, 0, L * T * H, D)
+    mem = torch.empty((1, L, 2, H, M, D), dtype=torch.bfloat16, device=dev)
+    syn.device_fill(mem, SEED, syn.STREAM_KBAR, 0, 0, 0, L * 2 * H * M, D, syn.POOLED_NOISE)
+    mlen = torch.full((1, L), M, dtype=torch.int32, device=dev)
+    lk = torch.zeros((1, L, H, T, D), dtype=torch.bfloat16, device=dev)
+    lv = torch.zeros_like(lk)
+    llen = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def run():
+        msa.msa_sparse_prefill(q, kn, vn, T, 1, L, HQ, H, D, lk, lv, llen, T, mem, mlen, M, TOPK, THETA, D ** -0.5, out,
+                               err)
+    ev = []
+    for r in range(13):
+        llen.zero_()
+        flush.fill_(r & 0xFF)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        run()
+        e.record()
+        if r >= 3:
+            ev.append((s, e))
+    torch.cuda.synchronize(dev)
+    ms = sorted(a.elapsed_time(b) for a, b in ev)[len(ev) // 2]
+    fl = prefill_flops(L, HQ, T, M)
+    tf = fl / ms / 1e9
+    peak = measured_peaks()[1]
+    return {"tokens": T, "layers": L, "mem_rows": M, "ms_p50": round(ms, 4), "gflop": round(fl / 1e9, 2),
+            "tflops": round(tf, 1), "tensor_frac_of_bf16_burst": round(tf / peak, 4),
+            "launches": msa.LAUNCHES_PREFILL, "dev_err": int(err.item()), "l2": "flushed (256 MB write) before each"}
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args):
@@ -296,6 +353,7 @@ def run_gpu(args):
 
     # pooling is an offline pass of its own: timed first, on the idle GPU
     pool = time_pool(dev) if (rank == 0 and not args.no_pool) else None
+    prefill = time_prefill(dev) if (rank == 0 and not args.no_prefill) else None
     torch.cuda.empty_cache()
     f8 = args.filter == "e4m3"
     bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic = make_workload(dev, args.host_store_blocks, f8)
@@ -545,6 +603,7 @@ def run_gpu(args):
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
         "pool": pool,
+        "prefill": prefill,
         "planted_recall": round(float(hits), 4),
         "dev_err": dev_err,
         "filter_keys_ms": None if f8_ms is None else round(f8_ms, 2),
@@ -628,6 +687,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool", action="store_true", help="skip the separate pooling measurement")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the separate prefill measurement")
     ap.add_argument("--pipeline", type=int, default=1, choices=[1, 2],
                     help="queries in flight (2 overlaps a query's gather+decode with the next route)")
     ap.add_argument("--filter", default="e4m3", choices=["e4m3", "bf16"],

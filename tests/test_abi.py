@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADERS = {"pool": "msa_pool.h", "route": "msa_route.h", "gather": "msa_gather.h", "decode": "msa_decode.h"}
+HEADERS = {"pool": "msa_pool.h", "route": "msa_route.h", "gather": "msa_gather.h", "decode": "msa_decode.h",
+           "prefill": "msa_prefill.h"}
 
 
 def _declared(header):
@@ -81,6 +82,12 @@ def test_invalid_arguments_rejected_without_gpu(msa):
         msa.msa_sparse_decode(z, z, z, 1, 1, 32, 5, 128, z, z, np.zeros(1, np.int32), 4, z, np.zeros(1, np.int32),
                               4, 16, 1e6, 0.1, z, z, stream=0)
     assert e.value.status == msa.MSA_ERR_INVALID_ARG
+    z = np.zeros(16, np.uint16)
+    for n_new, hq, h in ((4, 32, 5), (0, 32, 8), (4, 32, 2)):   # ratio 6.4; no tokens; ratio 16
+        with pytest.raises(msa.MsaError) as e:
+            msa.msa_sparse_prefill(z, z, z, n_new, 1, 1, hq, h, 128, z, z, np.zeros(1, np.int32), 8, z,
+                                   np.zeros(1, np.int32), 4, 16, 1e6, 0.1, z, stream=0)
+        assert e.value.status == msa.MSA_ERR_INVALID_ARG
 
 
 def test_workspace_size_grows_with_bank(msa):

@@ -44,6 +44,7 @@ pool_lib = _load("pool")
 route_lib = _load("route")
 gather_lib = _load("gather")
 decode_lib = _load("decode")
+prefill_lib = _load("prefill")
 
 pool_lib.msa_count_chunks.argtypes = [_p, _i32, _i32, _p]
 pool_lib.msa_count_chunks.restype = _i64
@@ -83,14 +84,20 @@ decode_lib.msa_sparse_decode_static.argtypes = [_p, _p, _p, _i32, _i32, _i32, _i
 decode_lib.msa_sparse_decode_static.restype = _i32
 MSA_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
+prefill_lib.msa_sparse_prefill.argtypes = [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _i32, _p,
+                                           _p, _i32, _i32, _f32, _f32, _p, _p, _p]
+prefill_lib.msa_sparse_prefill.restype = _i32
+prefill_lib.msa_prefill_last_error.restype = ctypes.c_char_p
+
 # Kernel launches enqueued by each entry point (the route count is read back per call).
 LAUNCHES_POOL = 1
 LAUNCHES_GATHER = 1
 LAUNCHES_DECODE = 1
+LAUNCHES_PREFILL = 3
 
 
 def loaded_libraries() -> list[str]:
-    return [os.path.join(LIB_DIR, f"libmsa_{n}.so") for n in ("pool", "route", "gather", "decode")]
+    return [os.path.join(LIB_DIR, f"libmsa_{n}.so") for n in ("pool", "route", "gather", "decode", "prefill")]
 
 
 def _ptr(t) -> int | None:
@@ -243,3 +250,17 @@ def msa_sparse_decode_static(q, k_new, v_new, n_queries: int, n_layers: int, n_q
                                              rope_pos_offset, rope_theta, softmax_scale, _ptr(out), _ptr(dev_err),
                                              _stream(stream))
     _check(st, "msa_sparse_decode_static", decode_lib, "msa_decode_last_error")
+
+
+# ----------------------------------------------------------------------------- prefill
+
+def msa_sparse_prefill(q, k_new, v_new, n_new: int, n_queries: int, n_layers: int, n_q_heads: int, n_kv_heads: int,
+                       head_dim: int, local_k, local_v, local_len, local_cap: int, mem_kv, mem_len,
+                       max_mem_chunks: int, rope_pos_offset: int, rope_theta: float, softmax_scale: float, out,
+                       dev_err=None, stream=None):
+    """n_new tokens per query through sparse attention (include/msa_prefill.h)."""
+    st = prefill_lib.msa_sparse_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), n_new, n_queries, n_layers, n_q_heads,
+                                        n_kv_heads, head_dim, _ptr(local_k), _ptr(local_v), _ptr(local_len),
+                                        local_cap, _ptr(mem_kv), _ptr(mem_len), max_mem_chunks, rope_pos_offset,
+                                        rope_theta, softmax_scale, _ptr(out), _ptr(dev_err), _stream(stream))
+    _check(st, "msa_sparse_prefill", prefill_lib, "msa_prefill_last_error")

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
   const int64_t bl = blockIdx.z;
   const int64_t uh = bl * H + h;
   const int len = local_len[b];
-  const bool full = len >= cap;
+  const bool full = len < 0 || len >= cap;  // (a negative length is treated as unusable too)
   int M = mem_len[bl];
   if (M > M_max) {
     if (tid == 0 && split == 0 && h == 0 && !full) msa::set_err(dev_err, MSA_DEVERR_CAPACITY);
