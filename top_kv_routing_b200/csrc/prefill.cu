@@ -77,7 +77,7 @@ __global__ void prefill_advance_kernel(int32_t* local_len, int B, int T, int cap
 
 // (2) attention
 template <int G>
-__global__ void __launch_bounds__(kThreads) prefill_attn_kernel(
+__global__ void __launch_bounds__(kThreads, 3) prefill_attn_kernel(
     const __nv_bfloat16* __restrict__ q, int T, int L, int H, const __nv_bfloat16* __restrict__ local_k,
     const __nv_bfloat16* __restrict__ local_v, const int32_t* __restrict__ local_len, int cap,
     const __nv_bfloat16* __restrict__ mem_kv, const int32_t* __restrict__ mem_len, int M_max, int pos_off,
@@ -198,18 +198,23 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(
 #pragma unroll
       for (int u = 0; u < 2; ++u) s[j][u][0] = s[j][u][1] = s[j][u][2] = s[j][u][3] = 0.f;
     }
+    // s[j][0] accumulates the bf16(q') products of key group j, s[j][1] the residual's;
+    // dependent MMAs are issued four apart
 #pragma unroll
     for (int ks2 = 0; ks2 < 4; ++ks2) {
+      uint32_t b[2][4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int row = 8 * j + (lane & 7);
         const int chunk = 4 * ks2 + (lane >> 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(st + row * kRowBytes + ((chunk ^ (row & 7)) << 4), b0, b1, b2, b3);
-        mma_bf16(s[j][0], qh[2 * ks2], b0, b1);
-        mma_bf16(s[j][0], ql[2 * ks2], b0, b1);
-        mma_bf16(s[j][1], qh[2 * ks2 + 1], b2, b3);
-        mma_bf16(s[j][1], ql[2 * ks2 + 1], b2, b3);
+        ldsm_x4(st + row * kRowBytes + ((chunk ^ (row & 7)) << 4), b[j][0], b[j][1], b[j][2], b[j][3]);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma_bf16(s[j][0], qh[2 * ks2 + e], b[j][2 * e], b[j][2 * e + 1]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma_bf16(s[j][1], ql[2 * ks2 + e], b[j][2 * e], b[j][2 * e + 1]);
       }
     }
     // scores of rows ra (c0, c1) and rb (c2, c3) for keys 8j + 2t + e
@@ -259,14 +264,17 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(
     const int vkey = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int vrow = kTileKeys + vkey;
 #pragma unroll
-    for (int i2 = 0; i2 < 8; ++i2) {
-      const int chunk = 2 * i2 + (lane >> 4);
-      uint32_t v0, v1, v2, v3;
-      ldsm_x4_t(st + vrow * kRowBytes + ((chunk ^ (vrow & 7)) << 4), v0, v1, v2, v3);
-      mma_bf16(o[2 * i2], ph, v0, v1);
-      mma_bf16(o[2 * i2], pl, v0, v1);
-      mma_bf16(o[2 * i2 + 1], ph, v2, v3);
-      mma_bf16(o[2 * i2 + 1], pl, v2, v3);
+    for (int i4 = 0; i4 < 4; ++i4) {  // 32 output dims per round, dependent MMAs four apart
+      uint32_t v[2][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int chunk = 4 * i4 + 2 * u + (lane >> 4);
+        ldsm_x4_t(st + vrow * kRowBytes + ((chunk ^ (vrow & 7)) << 4), v[u][0], v[u][1], v[u][2], v[u][3]);
+      }
+#pragma unroll
+      for (int n = 0; n < 4; ++n) mma_bf16(o[4 * i4 + n], ph, v[n >> 1][2 * (n & 1)], v[n >> 1][2 * (n & 1) + 1]);
+#pragma unroll
+      for (int n = 0; n < 4; ++n) mma_bf16(o[4 * i4 + n], pl, v[n >> 1][2 * (n & 1)], v[n >> 1][2 * (n & 1) + 1]);
     }
   }
   cp_async_wait<0>();
