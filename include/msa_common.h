@@ -1,20 +1,23 @@
 /* Common types of the MSA (Memory Sparse Attention) hot-path libraries.
  *
- * Four shared libraries, one per step of the online/offline path described on the
- * MSA pages ("MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", sections 架构 and
- * 推理流水线):
+ * One shared library per step of the online/offline path described on the MSA pages
+ * ("MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", sections 架构 and 推理流水线), plus
+ * the query's prefill and bank persistence:
  *   libmsa_pool.so    offline block compression        (msa_pool.h)
  *   libmsa_route.so   routing scores + top-k documents (msa_route.h)
  *   libmsa_gather.so  host -> device load of selection (msa_gather.h)
  *   libmsa_decode.so  sparse decode attention          (msa_decode.h)
+ *   libmsa_prefill.so the query's own tokens through sparse attention (msa_prefill.h)
+ *   libmsa_bank.so    bank file save / load, append re-layout (msa_bank.h)
  *
  * Conventions shared by every entry point:
  *  - Every call returns an msa_status; nothing else crosses the ABI on failure.  The
  *    library's msa_<lib>_last_error() returns a thread-local message for the last
  *    failing call of that library on this thread.
  *  - Every buffer is owned by the caller.  The libraries never allocate device or
- *    host memory; calls that need scratch space take a caller buffer whose size comes
- *    from a *_workspace_size query.
+ *    host memory (the one exception, msa_sparse_decode_static, holds a fixed array of
+ *    its own); calls that need scratch space take a caller buffer whose size comes
+ *    from a *_workspace_size query or is stated in the header.
  *  - Calls are asynchronous on the stream they are given (NULL = legacy default
  *    stream).  Host-side argument checks happen before anything is enqueued.
  *  - Conditions only the GPU can see (capacity overflow, a bad document id, a full
@@ -38,7 +41,8 @@ typedef enum msa_status {
   MSA_ERR_UNSUPPORTED = 2, /* device is not sm_100, or a dtype the call does not take */
   MSA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   MSA_ERR_CAPACITY = 4,    /* a caller buffer is too small (workspace, cache) */
-  MSA_ERR_TIMEOUT = 5      /* reserved for host waits with a time limit */
+  MSA_ERR_TIMEOUT = 5,     /* reserved for host waits with a time limit */
+  MSA_ERR_IO = 6           /* a bank file cannot be opened, read or written, or fails its checks */
 } msa_status;
 
 typedef enum msa_dtype { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;

@@ -10,7 +10,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADERS = {"pool": "msa_pool.h", "route": "msa_route.h", "gather": "msa_gather.h", "decode": "msa_decode.h",
-           "prefill": "msa_prefill.h"}
+           "prefill": "msa_prefill.h", "bank": "msa_bank.h"}
 
 
 def _declared(header):

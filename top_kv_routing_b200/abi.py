@@ -14,14 +14,14 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_DIR = os.path.join(_HERE, "lib")
 
-MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY, MSA_ERR_TIMEOUT = range(6)
+MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY, MSA_ERR_TIMEOUT, MSA_ERR_IO = range(7)
 MSA_F32, MSA_BF16 = 0, 1
 MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR, MSA_ROUTE_TENSOR_F8 = 0, 1, 2, 3
 (MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS, MSA_DEVERR_TIMEOUT,
  MSA_DEVERR_UNCERTIFIED) = 1, 2, 4, 8, 16, 32
 
 _STATUS = {1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA", 4: "MSA_ERR_CAPACITY",
-           5: "MSA_ERR_TIMEOUT"}
+           5: "MSA_ERR_TIMEOUT", 6: "MSA_ERR_IO"}
 
 
 class MsaError(RuntimeError):
@@ -45,6 +45,7 @@ route_lib = _load("route")
 gather_lib = _load("gather")
 decode_lib = _load("decode")
 prefill_lib = _load("prefill")
+bank_lib = _load("bank")
 
 pool_lib.msa_count_chunks.argtypes = [_p, _i32, _i32, _p]
 pool_lib.msa_count_chunks.restype = _i64
@@ -89,6 +90,25 @@ prefill_lib.msa_sparse_prefill.argtypes = [_p, _p, _p, _i32, _i32, _i32, _i32, _
 prefill_lib.msa_sparse_prefill.restype = _i32
 prefill_lib.msa_prefill_last_error.restype = ctypes.c_char_p
 
+
+class MsaBankInfo(ctypes.Structure):
+    _fields_ = [("n_layers", _i32), ("n_heads", _i32), ("head_dim", _i32), ("block_tokens", _i32),
+                ("n_docs", _i64), ("n_blocks", _i64), ("fields", ctypes.c_uint32)]
+
+
+MSA_BANK_KR, MSA_BANK_KR_F8, MSA_BANK_KV, MSA_BANK_NORM = 1, 2, 4, 8
+bank_lib.msa_bank_save.argtypes = [ctypes.c_char_p, ctypes.POINTER(MsaBankInfo), _p, _p, _p, _p, _p, _p, _sz, _p]
+bank_lib.msa_bank_save.restype = _i32
+bank_lib.msa_bank_read_info.argtypes = [ctypes.c_char_p, ctypes.POINTER(MsaBankInfo)]
+bank_lib.msa_bank_read_info.restype = _i32
+bank_lib.msa_bank_load.argtypes = [ctypes.c_char_p, _p, _p, _p, _p, _p, _p, _sz, _p]
+bank_lib.msa_bank_load.restype = _i32
+bank_lib.msa_bank_relayout.argtypes = [_p, _p, _i32, _i64, _i64, _i64, _p]
+bank_lib.msa_bank_relayout.restype = _i32
+bank_lib.msa_bank_append_offsets.argtypes = [_p, _i64, _p, _i64, _p]
+bank_lib.msa_bank_append_offsets.restype = _i32
+bank_lib.msa_bank_last_error.restype = ctypes.c_char_p
+
 # Kernel launches enqueued by each entry point (the route count is read back per call).
 LAUNCHES_POOL = 1
 LAUNCHES_GATHER = 1
@@ -97,7 +117,7 @@ LAUNCHES_PREFILL = 3
 
 
 def loaded_libraries() -> list[str]:
-    return [os.path.join(LIB_DIR, f"libmsa_{n}.so") for n in ("pool", "route", "gather", "decode", "prefill")]
+    return [os.path.join(LIB_DIR, f"libmsa_{n}.so") for n in ("pool", "route", "gather", "decode", "prefill", "bank")]
 
 
 def _ptr(t) -> int | None:
@@ -264,3 +284,57 @@ def msa_sparse_prefill(q, k_new, v_new, n_new: int, n_queries: int, n_layers: in
                                         local_cap, _ptr(mem_kv), _ptr(mem_len), max_mem_chunks, rope_pos_offset,
                                         rope_theta, softmax_scale, _ptr(out), _ptr(dev_err), _stream(stream))
     _check(st, "msa_sparse_prefill", prefill_lib, "msa_prefill_last_error")
+
+
+# ----------------------------------------------------------------------------- bank files
+
+def _path(p) -> bytes:
+    return os.fsencode(p)
+
+
+def _bank_stream(stream):
+    """The bank calls also serve host arrays on machines without a GPU (stream 0 there)."""
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else 0
+    return _stream(stream)
+
+
+def msa_bank_save(path, info: MsaBankInfo, doc_chunk_offsets, kr_hat=None, kr_f8=None, content_kv=None,
+                  kr_norm=None, staging=None, stream=None):
+    """Writes a bank file (include/msa_bank.h); doc_chunk_offsets is a host int64 array."""
+    off = np.ascontiguousarray(doc_chunk_offsets, dtype=np.int64)
+    st = bank_lib.msa_bank_save(_path(path), ctypes.byref(info), _ptr(off), _ptr(kr_hat), _ptr(kr_f8),
+                                _ptr(content_kv), _ptr(kr_norm), _ptr(staging), _nbytes(staging) if staging is not None
+                                else 0, _bank_stream(stream))
+    _check(st, "msa_bank_save", bank_lib, "msa_bank_last_error")
+
+
+def msa_bank_read_info(path) -> MsaBankInfo:
+    info = MsaBankInfo()
+    st = bank_lib.msa_bank_read_info(_path(path), ctypes.byref(info))
+    _check(st, "msa_bank_read_info", bank_lib, "msa_bank_last_error")
+    return info
+
+
+def msa_bank_load(path, doc_chunk_offsets, kr_hat=None, kr_f8=None, content_kv=None, kr_norm=None, staging=None,
+                  stream=None):
+    """Reads a bank file into caller arrays; doc_chunk_offsets is a host int64 array [n_docs + 1]."""
+    st = bank_lib.msa_bank_load(_path(path), _ptr(doc_chunk_offsets), _ptr(kr_hat), _ptr(kr_f8), _ptr(content_kv),
+                                _ptr(kr_norm), _ptr(staging), _nbytes(staging) if staging is not None else 0,
+                                _bank_stream(stream))
+    _check(st, "msa_bank_load", bank_lib, "msa_bank_last_error")
+
+
+def msa_bank_relayout(src, dst, n_layers: int, rows_old: int, rows_new: int, row_bytes: int, stream=None):
+    st = bank_lib.msa_bank_relayout(_ptr(src), _ptr(dst), n_layers, rows_old, rows_new, row_bytes, _bank_stream(stream))
+    _check(st, "msa_bank_relayout", bank_lib, "msa_bank_last_error")
+
+
+def msa_bank_append_offsets(old_offsets, new_offsets) -> np.ndarray:
+    a = np.ascontiguousarray(old_offsets, dtype=np.int64)
+    b = np.ascontiguousarray(new_offsets, dtype=np.int64)
+    out = np.empty(len(a) + len(b) - 1, dtype=np.int64)
+    st = bank_lib.msa_bank_append_offsets(_ptr(a), len(a) - 1, _ptr(b), len(b) - 1, _ptr(out))
+    _check(st, "msa_bank_append_offsets", bank_lib, "msa_bank_last_error")
+    return out

@@ -28,11 +28,13 @@ TARGETS = {
     os.path.join(LIB, "libmsa_gather.so"): ["gather.cu"],
     os.path.join(LIB, "libmsa_decode.so"): ["decode.cu"],
     os.path.join(LIB, "libmsa_prefill.so"): ["prefill.cu"],
+    os.path.join(LIB, "libmsa_bank.so"): ["bank.cu"],
 }
 SYNTH_TARGET = os.path.join(SYNTH, "libmsa_synth.so")
 
 LIBRARIES = {"pool": "libmsa_pool.so", "route": "libmsa_route.so", "gather": "libmsa_gather.so",
-             "decode": "libmsa_decode.so", "prefill": "libmsa_prefill.so"}
+             "decode": "libmsa_decode.so", "prefill": "libmsa_prefill.so",
+             "bank": "libmsa_bank.so"}
 
 
 def nvcc() -> str:
