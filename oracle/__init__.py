@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_prefill.argtypes = [_p, _p, _p, _i32, _p, _i32, _i32, _p, _p, _i32, _i32, _i64, _dbl, _dbl,
                                         _i32, _i32, _i32, _p]
         _lib.oracle_prefill.restype = _i32
+        _lib.oracle_router_project.argtypes = [_p, _i32, _i32, _p, _i32, _p]
+        _lib.oracle_router_project.restype = None
     return _lib
 
 
@@ -197,3 +199,15 @@ def prefill(q, k_new, v_new, mem_kv, mem_len: int, local_k, local_v, local_len: 
     if r != 0:
         raise OverflowError("oracle prefill: local cache full")
     return out
+
+
+def router_project(h, w, n_q_heads: int):
+    """Router query projection of one layer: h [T][hidden] times w [n_q_heads * d][hidden]
+    transposed.  Returns Q_r [T][n_q_heads][d] (double)."""
+    h, w = _f32(h), _f32(w)
+    T, hidden = h.shape
+    F, hidden2 = w.shape
+    assert hidden == hidden2 and F % n_q_heads == 0
+    out = np.empty((T, F), dtype=np.float64)
+    lib().oracle_router_project(_ptr(h), T, hidden, _ptr(w), F, _ptr(out))
+    return out.reshape(T, n_q_heads, F // n_q_heads)

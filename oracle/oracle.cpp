@@ -374,4 +374,16 @@ int32_t oracle_prefill(const float* q, const float* k_new, const float* v_new, i
   return 0;
 }
 
+// Router query projection of one routing layer ([DEEP] 5.1: the decoupled router_q_proj
+// is a bias-free linear map hidden -> n_q_heads * head_dim; 5.2: it is applied to the
+// layer's input hidden states).  out[t][j] = sum_k h[t][k] * w[j][k], in double.
+void oracle_router_project(const float* h, int32_t T, int32_t hidden, const float* w, int32_t F, double* out) {
+  for (int32_t t = 0; t < T; ++t)
+    for (int32_t j = 0; j < F; ++j) {
+      double acc = 0.0;
+      for (int32_t k = 0; k < hidden; ++k) acc += (double)h[(size_t)t * hidden + k] * (double)w[(size_t)j * hidden + k];
+      out[(size_t)t * F + j] = acc;
+    }
+}
+
 }  // extern "C"

@@ -434,3 +434,41 @@ def test_prefill_of_one_token_is_a_decode_step():
     a = oracle.prefill(q, kn, vn, mem, M, a_k, a_v, 2, 9, 1e6, 0.2)
     b = oracle.decode(q[0], kn[0], vn[0], mem, M, b_k, b_v, 2, 9, 1e6, 0.2)
     np.testing.assert_array_equal(a[0], b)
+
+
+# ----------------------------------------------------------------------------- router projection
+
+def test_router_projection_hand_example():
+    # Q_r[t][j] = sum_k h[t][k] w[j][k] with w stored [features][hidden] (nn.Linear's
+    # weight layout), features grouped into heads of d = 2: worked by hand.
+    h = np.array([[1, 2], [3, -1]], np.float32)
+    w = np.array([[3, 4], [0, 1], [1, 0], [2, 2], [-1, 5], [0, 0]], np.float32)
+    q = oracle.router_project(h, w, 3)
+    assert q.shape == (2, 3, 2)
+    assert q.tolist() == [[[11, 2], [1, 6], [9, 0]], [[5, -1], [3, 4], [-8, 0]]]
+
+
+def test_router_projection_one_hot_rows_select_hidden_features():
+    rng = np.random.default_rng(31)
+    T, hidden, Hq, d = 5, 24, 3, 8
+    h = rng.standard_normal((T, hidden)).astype(np.float32)
+    pick = rng.integers(0, hidden, size=Hq * d)
+    w = np.zeros((Hq * d, hidden), np.float32)
+    w[np.arange(Hq * d), pick] = 1.0
+    q = oracle.router_project(h, w, Hq)
+    np.testing.assert_array_equal(q.reshape(T, Hq * d), h[:, pick].astype(np.float64))
+
+
+def test_routing_of_projected_queries_is_invariant_to_weight_scale():
+    # the routing score is a cosine per head: scaling the projection weights by a
+    # positive constant changes no score and no selection
+    rng = np.random.default_rng(32)
+    T, hidden, Hq, H, d, C = 4, 32, 4, 2, 8, 6
+    h = rng.standard_normal((T, hidden)).astype(np.float32)
+    w = rng.standard_normal((Hq * d, hidden)).astype(np.float32)
+    kr = rng.standard_normal((C, H, d)).astype(np.float32)
+    offs = np.array([0, 2, 3, 6])
+    a = oracle.route(oracle.router_project(h, w, Hq), kr, offs, 2)
+    b = oracle.route(oracle.router_project(h, 8 * w, Hq), kr, offs, 2)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_allclose(a[2], b[2], atol=1e-12)
