@@ -86,6 +86,29 @@ msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_of
                           float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,
                           int32_t* dev_err, msa_stream_t stream);
 
+/* msa_route_topk with the router's query projection fused in.  Defined by "【MSA】突破100M
+ * Token 上下文：记忆稀疏注意力架构深度解析", section 5.1 (each routing layer's decoupled
+ * router_q_proj: hidden -> n_q_heads x head_dim, no bias) and section 5.2 (the router
+ * query is that projection of the layer's input hidden states).  Per layer l and token t:
+ *   Q_r[l][t] = hidden[t] . w_router_q[l]^T          (head q = features q*128 .. q*128+127)
+ * computed on the tensor cores (bf16 operands, fp32 accumulation) and normalised per head
+ * and summed per key-head group inside the same kernel, straight into the routing
+ * operand; Q_r is never written to memory.  Everything after that, and every other
+ * argument, result and error, is as msa_route_topk with q_dtype bf16.
+ *   hidden      DEVICE bf16 [total tokens][hidden_size], 16-byte aligned (the tokens of
+ *               all queries back to back, as qr)
+ *   w_router_q  DEVICE bf16 [n_layers][n_q_heads * head_dim][hidden_size], 16-byte aligned
+ *   hidden_size a multiple of 64; n_q_heads / n_kv_heads in {1, 2, 4}.
+ * The workspace is msa_route_topk_workspace_size's.  One launch replaces the query
+ * preparation kernel (the launch count is unchanged). */
+msa_status msa_route_topk_hidden(const void* hidden, const void* w_router_q, int32_t hidden_size,
+                                 const int32_t* q_offsets_host, int32_t n_queries, const void* kr_hat,
+                                 const void* kr_f8, const int64_t* doc_chunk_offsets, int32_t n_docs,
+                                 int64_t n_chunks, int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads,
+                                 int32_t head_dim, int32_t top_k, int32_t* out_ids, float* out_scores,
+                                 void* workspace, size_t workspace_bytes, int32_t flags, int32_t* dev_err,
+                                 msa_stream_t stream);
+
 /* Number of kernel launches the last successful msa_route_topk on this thread enqueued
  * (for launch accounting). */
 int32_t msa_route_last_launch_count(void);

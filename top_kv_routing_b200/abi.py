@@ -59,6 +59,9 @@ route_lib.msa_route_topk_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64
 route_lib.msa_route_topk_workspace_size.restype = _i32
 route_lib.msa_route_topk.argtypes = [_p, _i32, _p, _i32, _p, _p, _p, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
                                      _p, _p, _p, _sz, _i32, _p, _p]
+route_lib.msa_route_topk_hidden.argtypes = [_p, _p, _i32, _p, _i32, _p, _p, _p, _i32, _i64, _i32, _i32, _i32, _i32,
+                                            _i32, _p, _p, _p, _sz, _i32, _p, _p]
+route_lib.msa_route_topk_hidden.restype = _i32
 route_lib.msa_route_filter_keys.argtypes = [_p, _i32, _i64, _i32, _i32, _p, _p]
 route_lib.msa_route_filter_keys.restype = _i32
 route_lib.msa_route_topk.restype = _i32
@@ -200,6 +203,22 @@ def msa_route_topk(qr, q_offsets, kr_hat, doc_chunk_offsets, n_docs: int, n_chun
                                   head_dim, top_k, _ptr(out_ids), _ptr(out_scores), _ptr(workspace), ws_bytes,
                                   flags, _ptr(dev_err), _stream(stream))
     _check(st, "msa_route_topk", route_lib, "msa_route_last_error")
+    return int(route_lib.msa_route_last_launch_count())
+
+
+def msa_route_topk_hidden(hidden, w_router_q, hidden_size: int, q_offsets, kr_hat, doc_chunk_offsets, n_docs: int,
+                          n_chunks: int, n_layers: int, n_q_heads: int, n_kv_heads: int, head_dim: int, top_k: int,
+                          out_ids, out_scores, workspace, flags: int = MSA_ROUTE_AUTO, dev_err=None, stream=None,
+                          kr_f8=None) -> int:
+    """msa_route_topk with the router query projection (hidden [T][hidden_size] bf16 times
+    w_router_q [L][Hq*128][hidden_size] bf16) fused in; returns the launches enqueued."""
+    qo = np.ascontiguousarray(q_offsets, dtype=np.int32)
+    st = route_lib.msa_route_topk_hidden(_ptr(hidden), _ptr(w_router_q), hidden_size, qo.ctypes.data, len(qo) - 1,
+                                         _ptr(kr_hat), _ptr(kr_f8), _ptr(doc_chunk_offsets), n_docs, n_chunks,
+                                         n_layers, n_q_heads, n_kv_heads, head_dim, top_k, _ptr(out_ids),
+                                         _ptr(out_scores), _ptr(workspace), _nbytes(workspace), flags, _ptr(dev_err),
+                                         _stream(stream))
+    _check(st, "msa_route_topk_hidden", route_lib, "msa_route_last_error")
     return int(route_lib.msa_route_last_launch_count())
 
 

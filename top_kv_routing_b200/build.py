@@ -24,7 +24,7 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "-X
 
 TARGETS = {
     os.path.join(LIB, "libmsa_pool.so"): ["pool.cu"],
-    os.path.join(LIB, "libmsa_route.so"): ["route.cu", "route_tc.cu"],
+    os.path.join(LIB, "libmsa_route.so"): ["route.cu", "route_tc.cu", "route_proj.cu"],
     os.path.join(LIB, "libmsa_gather.so"): ["gather.cu"],
     os.path.join(LIB, "libmsa_decode.so"): ["decode.cu"],
     os.path.join(LIB, "libmsa_prefill.so"): ["prefill.cu"],

@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "msa_route.h"
+#include "route_proj.cuh"
 #include "route_tc.cuh"
 
 MSA_DEFINE_LAST_ERROR(msa_route_last_error)
@@ -958,16 +959,31 @@ extern "C" msa_status msa_route_filter_keys(const void* kr_hat, int32_t n_layers
   return msa_ok();
 }
 
-extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
-                                     int32_t n_queries, const void* kr_hat, const void* kr_f8,
-                                     const int64_t* doc_chunk_offsets,
-                                     int32_t n_docs, int64_t n_chunks, int32_t n_layers, int32_t n_q_heads,
-                                     int32_t n_kv_heads, int32_t head_dim, int32_t top_k, int32_t* out_ids,
-                                     float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,
-                                     int32_t* dev_err, msa_stream_t stream) {
+namespace {
+// Where the routing query comes from: a given Q_r (qr), or hidden states projected by the
+// router's query weights inside the call (hidden, w).
+struct QuerySrc {
+  const void* qr;
+  msa_dtype q_dtype;
+  const void* hidden;
+  const void* w;
+  int32_t hidden_size;
+};
+
+msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_t n_queries, const void* kr_hat,
+                      const void* kr_f8, const int64_t* doc_chunk_offsets, int32_t n_docs, int64_t n_chunks,
+                      int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t top_k,
+                      int32_t* out_ids, float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,
+                      int32_t* dev_err, msa_stream_t stream) {
   g_launches = 0;
-  if (!qr || !q_offsets_host || !kr_hat || !doc_chunk_offsets || !out_ids || !out_scores || !workspace)
+  const void* qr = src.qr;
+  const msa_dtype q_dtype = src.q_dtype;
+  const bool project = src.hidden != nullptr;
+  if (!(qr || (project && src.w)) || !q_offsets_host || !kr_hat || !doc_chunk_offsets || !out_ids || !out_scores ||
+      !workspace)
     return msa_fail(MSA_ERR_INVALID_ARG, "null pointer");
+  if (project && !route_proj::supported(n_q_heads, n_kv_heads, src.hidden_size))
+    return msa_fail(MSA_ERR_INVALID_ARG, "projection: hidden_size a multiple of 64, n_q_heads / n_kv_heads in {1,2,4}");
   if (head_dim != kD) return msa_fail(MSA_ERR_INVALID_ARG, "head_dim must be 128");
   if (n_kv_heads != 2 && n_kv_heads != 4 && n_kv_heads != 8 && n_kv_heads != 16)
     return msa_fail(MSA_ERR_INVALID_ARG, "n_kv_heads must be 2, 4, 8 or 16");
@@ -977,13 +993,13 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   if (top_k < 1 || top_k > kMaxTopK) return msa_fail(MSA_ERR_INVALID_ARG, "top_k in [1,64]");
   if (n_layers < 1 || n_chunks < 0 || n_docs < 0 || n_docs > kMaxDocs)
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_docs <= 2^20)");
-  if (q_dtype != MSA_F32 && q_dtype != MSA_BF16) return msa_fail(MSA_ERR_UNSUPPORTED, "q_dtype");
+  if (!project && q_dtype != MSA_F32 && q_dtype != MSA_BF16) return msa_fail(MSA_ERR_UNSUPPORTED, "q_dtype");
   if (flags < MSA_ROUTE_AUTO || flags > MSA_ROUTE_TENSOR_F8) return msa_fail(MSA_ERR_INVALID_ARG, "flags");
   if (flags == MSA_ROUTE_TENSOR_F8 && !kr_f8)
     return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_TENSOR_F8 needs the E4M3 keys (msa_route_filter_keys)");
   if (!msa::aligned16(qr) || !msa::aligned16(kr_hat) || !msa::aligned16(kr_f8) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return msa_fail(MSA_ERR_INVALID_ARG, "alignment: qr/kr_hat/kr_f8 16 B, workspace 256 B");
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) || !msa::aligned16(src.hidden) || !msa::aligned16(src.w))
+    return msa_fail(MSA_ERR_INVALID_ARG, "alignment: qr/hidden/w/kr_hat/kr_f8 16 B, workspace 256 B");
   QueryOffsets qo;
   qo.n = n_queries;
   if (q_offsets_host[0] != 0) return msa_fail(MSA_ERR_INVALID_ARG, "q_offsets[0] must be 0");
@@ -1044,10 +1060,37 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
-  qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
-                                                      tensor ? nullptr : qt_f32, tensor ? qt_bf16 : nullptr,
-                                                      tensor ? qt_lo : nullptr, f8 ? qt_f8 : nullptr,
-                                                      f8 ? redo : nullptr, n_layers);
+  if (project) {
+    // Q_r = hidden W^T on the tensor cores, normalised and group-summed in the epilogue
+    route_proj::Args pa;
+    pa.hidden = src.hidden;
+    pa.w = src.w;
+    pa.T = T_total;
+    pa.hidden_size = src.hidden_size;
+    pa.L = n_layers;
+    pa.Hq = n_q_heads;
+    pa.H = H;
+    pa.n_rows = n_rows;
+    pa.lay.n_queries = n_queries;
+    for (int b = 0; b <= n_queries; ++b) {
+      pa.lay.off[b] = qo.off[b];
+      pa.lay.row0[b] = qo.row0[b];
+    }
+    pa.qt_f32 = tensor ? nullptr : qt_f32;
+    pa.qt_bf16 = tensor ? qt_bf16 : nullptr;
+    pa.qt_lo = tensor ? qt_lo : nullptr;
+    pa.qt_f8 = f8 ? qt_f8 : nullptr;
+    pa.redo = f8 ? redo : nullptr;
+    pa.dev_err = dev_err;
+    const char* why = nullptr;
+    if (route_proj::launch(pa, s, &why) != 0)
+      return msa_fail(MSA_ERR_CUDA, "router projection: %s", why ? why : "launch failed");
+  } else {
+    qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
+                                                        tensor ? nullptr : qt_f32, tensor ? qt_bf16 : nullptr,
+                                                        tensor ? qt_lo : nullptr, f8 ? qt_f8 : nullptr,
+                                                        f8 ? redo : nullptr, n_layers);
+  }
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
 
@@ -1158,4 +1201,33 @@ extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const in
   st = select(kFilterErr, nullptr, redo);
   if (st != MSA_OK) return st;
   return msa_ok();
+}
+
+}  // namespace
+
+extern "C" msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
+                                     int32_t n_queries, const void* kr_hat, const void* kr_f8,
+                                     const int64_t* doc_chunk_offsets,
+                                     int32_t n_docs, int64_t n_chunks, int32_t n_layers, int32_t n_q_heads,
+                                     int32_t n_kv_heads, int32_t head_dim, int32_t top_k, int32_t* out_ids,
+                                     float* out_scores, void* workspace, size_t workspace_bytes, int32_t flags,
+                                     int32_t* dev_err, msa_stream_t stream) {
+  const QuerySrc src{qr, q_dtype, nullptr, nullptr, 0};
+  return route_impl(src, q_offsets_host, n_queries, kr_hat, kr_f8, doc_chunk_offsets, n_docs, n_chunks, n_layers,
+                    n_q_heads, n_kv_heads, head_dim, top_k, out_ids, out_scores, workspace, workspace_bytes, flags,
+                    dev_err, stream);
+}
+
+extern "C" msa_status msa_route_topk_hidden(const void* hidden, const void* w_router_q, int32_t hidden_size,
+                                            const int32_t* q_offsets_host, int32_t n_queries, const void* kr_hat,
+                                            const void* kr_f8, const int64_t* doc_chunk_offsets, int32_t n_docs,
+                                            int64_t n_chunks, int32_t n_layers, int32_t n_q_heads,
+                                            int32_t n_kv_heads, int32_t head_dim, int32_t top_k, int32_t* out_ids,
+                                            float* out_scores, void* workspace, size_t workspace_bytes,
+                                            int32_t flags, int32_t* dev_err, msa_stream_t stream) {
+  if (!hidden || !w_router_q) return msa_fail(MSA_ERR_INVALID_ARG, "null pointer");
+  const QuerySrc src{nullptr, MSA_BF16, hidden, w_router_q, hidden_size};
+  return route_impl(src, q_offsets_host, n_queries, kr_hat, kr_f8, doc_chunk_offsets, n_docs, n_chunks, n_layers,
+                    n_q_heads, n_kv_heads, head_dim, top_k, out_ids, out_scores, workspace, workspace_bytes, flags,
+                    dev_err, stream);
 }
