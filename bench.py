@@ -321,6 +321,7 @@ def time_prefill(dev):
     for r in range(13):
         llen.zero_()
         flush.fill_(r & 0xFF)
+        torch.cuda._sleep(2_000_000)  # the GPU is busy while the host prepares the call
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
         run()
@@ -335,6 +336,70 @@ def time_prefill(dev):
     return {"tokens": T, "layers": L, "mem_rows": M, "ms_p50": round(ms, 4), "gflop": round(fl / 1e9, 2),
             "tflops": round(tf, 1), "tensor_frac_of_bf16_burst": round(tf / peak, 4),
             "launches": msa.LAUNCHES_PREFILL, "dev_err": int(err.item()), "l2": "flushed (256 MB write) before each"}
+
+
+HIDDEN = 2560  # hidden size of the 4B backbone the pages' model is built on
+
+
+def time_projection(dev, bank, kr_hat, kr_f8):
+    """Routing from hidden states (msa_route_topk_hidden): the router query projection of
+    the query's T tokens for every routing layer, fused with the normalisation and group
+    sum, then the same routing as the step.  Synthetic bf16 weights.  Reports the
+    projection kernel's device time (events around the query stage) and the whole call's."""
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+    C, n_docs = bank.n_chunks, len(bank.lengths)
+    # planted inputs: the first 128 hidden features carry a target document's topic (16
+    # targets over the tokens) and every head's weights are near-identity on them, so the
+    # projected queries find their documents and the E4M3 selections certify as in the step
+    hid = torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=dev)
+    w = torch.empty((L, HQ * D, HIDDEN), dtype=torch.bfloat16, device=dev)
+    syn.device_fill(hid, SEED, syn.STREAM_QR, 90, 0, 0, T, HIDDEN)
+    targets = syn.pick_targets(SEED, n_docs, 16, sub=77)
+    rt = torch.from_numpy(np.asarray(targets)[np.arange(T) % 16].astype(np.int32)).to(dev)
+    head = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    syn.device_fill(head, SEED, syn.STREAM_QR, 91, 0, 0, T, D, 0.5, torch.from_numpy(bank.topic).to(dev), rt)
+    hid[:, :D].copy_(head)
+    syn.device_fill(w, SEED, syn.STREAM_KBAR, 92, 0, 0, L * HQ * D, HIDDEN, 0.02)
+    eye = torch.eye(D, dtype=torch.bfloat16, device=dev)
+    w.view(L, HQ, D, HIDDEN)[..., :D] += eye
+    coffs = torch.from_numpy(bank.doc_chunk_offsets).to(dev)
+    ws = torch.empty(msa.msa_route_topk_workspace_size(L, 1, T, H, C, n_docs, TOPK), dtype=torch.uint8, device=dev)
+    ids = torch.empty((1, L, TOPK), dtype=torch.int32, device=dev)
+    sc = torch.empty((1, L, TOPK), device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flags = msa.MSA_ROUTE_TENSOR_F8 if kr_f8 is not None else msa.MSA_ROUTE_TENSOR
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q0.record()  # (creates the events; the route library re-records them around the query stage)
+    q1.record()
+    torch.cuda.synchronize(dev)
+    proj, whole = [], []
+    msa.msa_route_set_query_profile_events(q0, q1)
+    try:
+        for r in range(8):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(2_000_000)  # the GPU is busy while the host prepares the call
+            a.record()
+            msa.msa_route_topk_hidden(hid, w, HIDDEN, [0, T], kr_hat, coffs, n_docs, C, L, HQ, H, D, TOPK, ids, sc, ws,
+                                      flags=flags, dev_err=err, kr_f8=kr_f8)
+            b.record()
+            torch.cuda.synchronize(dev)
+            if r >= 3:
+                proj.append(q0.elapsed_time(q1))
+                whole.append(a.elapsed_time(b))
+    finally:
+        msa.msa_route_set_query_profile_events(None, None)
+    ms = sorted(proj)[len(proj) // 2]
+    fl = 2.0 * T * HIDDEN * HQ * D * L
+    peak = measured_peaks()[1]
+    want = set(np.asarray(targets).tolist())
+    found = float(np.mean([len(want & set(x.tolist())) / 16 for x in ids[0].cpu().numpy()]))
+    return {"hidden": HIDDEN, "tokens": T, "layers": L, "proj_ms_p50": round(ms, 4), "gflop": round(fl / 1e9, 1),
+            "planted_recall": round(found, 4),
+            "tflops": round(fl / ms / 1e9, 1), "tensor_frac_of_bf16_burst": round(fl / ms / 1e9 / peak, 4),
+            "route_hidden_ms_p50": round(sorted(whole)[len(whole) // 2], 3), "dev_err": int(err.item())}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -527,6 +592,8 @@ def run_gpu(args):
                                eng.slots[(args.steps - 1) % n_slots].ids))
     h2d = host["qr"][0].numel() * 2 + (dq.numel() + dk.numel() + dv.numel()) * 2
     d2h = host["ids"][0].numel() * 4 + host["scores"][0].numel() * 4 + host["out"][0].numel() * 2
+    # routing from hidden states (fused router projection), after the timed regions
+    projection = time_projection(dev, bank, kr_hat, kr_f8) if (rank == 0 and not args.no_projection) else None
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
     if world > 1:
@@ -604,6 +671,7 @@ def run_gpu(args):
         "clocks": clk.summary(),
         "pool": pool,
         "prefill": prefill,
+        "router_projection": projection,
         "planted_recall": round(float(hits), 4),
         "dev_err": dev_err,
         "filter_keys_ms": None if f8_ms is None else round(f8_ms, 2),
@@ -688,6 +756,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool", action="store_true", help="skip the separate pooling measurement")
     ap.add_argument("--no-prefill", action="store_true", help="skip the separate prefill measurement")
+    ap.add_argument("--no-projection", action="store_true",
+                    help="skip the separate routing-from-hidden-states measurement")
     ap.add_argument("--pipeline", type=int, default=1, choices=[1, 2],
                     help="queries in flight (2 overlaps a query's gather+decode with the next route)")
     ap.add_argument("--filter", default="e4m3", choices=["e4m3", "bf16"],
