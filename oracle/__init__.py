@@ -211,3 +211,25 @@ def router_project(h, w, n_q_heads: int):
     out = np.empty((T, F), dtype=np.float64)
     lib().oracle_router_project(_ptr(h), T, hidden, _ptr(w), F, _ptr(out))
     return out.reshape(T, n_q_heads, F // n_q_heads)
+
+
+def layer_mean_topk(doc_scores, k: int):
+    """Layer-aggregated selection: one top-k shared by every routing layer, ranking the
+    documents by the mean over layers of their per-layer document scores (a document with
+    no block scores -inf in every layer and so in the mean).  doc_scores [L][n_docs].
+    Returns (ids [k], scores [k], mean [n_docs])."""
+    ds = np.asarray(doc_scores, dtype=np.float64)
+    L = ds.shape[0]
+    mean = np.empty(ds.shape[1], dtype=np.float64)
+    for d in range(ds.shape[1]):  # in layer order, as written
+        col = ds[:, d]
+        mean[d] = -np.inf if np.isneginf(col).any() else sum(float(x) for x in col) / L
+    ids, sc = topk(mean, k)
+    return ids, sc, mean
+
+
+def route_layer_mean(q_layers, kr_layers, doc_chunk_offsets, top_k: int):
+    """Routing of one query with the layer-aggregated selection: q_layers [L][T][Hq][d],
+    kr_layers [L][C][H][d].  Returns (ids [k], scores [k], mean doc scores [n_docs])."""
+    per_layer = [route(q, kr, doc_chunk_offsets, top_k, grouped=True)[2] for q, kr in zip(q_layers, kr_layers)]
+    return layer_mean_topk(np.stack(per_layer), top_k)

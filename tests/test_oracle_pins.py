@@ -472,3 +472,34 @@ def test_routing_of_projected_queries_is_invariant_to_weight_scale():
     b = oracle.route(oracle.router_project(h, 8 * w, Hq), kr, offs, 2)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_allclose(a[2], b[2], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- layer-aggregated routing
+
+def test_layer_mean_selection_hand_example():
+    # per-layer document scores, worked by hand: means 0.5, 0.45, 0.5, -inf (doc 3 has no
+    # block, so it ranks last at -inf); the tie between documents 0 and 2 goes to the
+    # lower id; a fifth slot has no document (-1)
+    ds = [[0.9, 0.1, 0.5, -np.inf], [0.1, 0.8, 0.5, -np.inf]]
+    ids, sc, mean = oracle.layer_mean_topk(ds, 5)
+    assert ids.tolist() == [0, 2, 1, 3, -1]
+    assert np.isneginf(sc[4])
+    assert sc[:3].tolist() == [0.5, 0.5, 0.45] and np.isneginf(sc[3])
+    assert mean[:3].tolist() == [0.5, 0.45, 0.5]
+    # each layer alone would pick differently: layer 0 -> 0, layer 1 -> 1
+    assert oracle.layer_mean_topk(ds[:1], 1)[0].tolist() == [0]
+    assert oracle.layer_mean_topk(ds[1:], 1)[0].tolist() == [1]
+
+
+def test_layer_mean_routing_of_one_layer_or_equal_layers_is_the_per_layer_routing():
+    rng = np.random.default_rng(41)
+    T, Hq, H, d, k = 3, 4, 2, 8, 3
+    offs = np.array([0, 2, 2, 5, 9, 10])
+    kr = rng.standard_normal((10, H, d)).astype(np.float32)
+    q = rng.standard_normal((T, Hq, d)).astype(np.float32)
+    ref_ids, ref_sc, ref_ds, _ = oracle.route(q, kr, offs, k)
+    for L in (1, 3):
+        ids, sc, mean = oracle.route_layer_mean([q] * L, [kr] * L, offs, k)
+        assert ids.tolist() == ref_ids.tolist()
+        np.testing.assert_allclose(sc, ref_sc, rtol=1e-12)
+        assert np.isneginf(mean[1])  # the empty document
