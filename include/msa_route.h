@@ -34,6 +34,20 @@ extern "C" {
 #define MSA_ROUTE_SCAN 1    /* CUDA-core streaming scan (few query tokens)           */
 #define MSA_ROUTE_TENSOR 2  /* tcgen05 tensor-core GEMM with fused token-max epilogue */
 #define MSA_ROUTE_TENSOR_F8 3 /* the same GEMM on the E4M3 copy of the keys            */
+/* OR-ed with a path: one selection shared by every routing layer (the layer-aggregated
+ * variant).  Documents are ranked by the mean over the layers of their document scores
+ * (each layer's score defined as above), and the same top_k ids and mean scores are
+ * written for every layer.  A reading of the pages' single-selection variant: the
+ * "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文" page, section 架构, and the MSA paper
+ * reading notes, section 路由投影器 + Top-k 稀疏注意力, state the selection per query; where
+ * the layers' selections are to be one, their scores are averaged.  Runs on the tensor
+ * path (AUTO picks it at any query length; with MSA_ROUTE_SCAN it is MSA_ERR_INVALID_ARG;
+ * needs n_kv_heads = 8): the mean filter scores choose the candidates, every layer rescores
+ * them exactly, and the final top-k is certified on the mean exact scores against the
+ * best mean filter score left out (the same bounds as per layer: a mean of errors is
+ * within the largest).  On the E4M3 path an uncertified query sends every layer to the
+ * bf16 second pass. */
+#define MSA_ROUTE_LAYER_MEAN 16
 
 /* Workspace bytes for one msa_route_topk call with these sizes. */
 msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, int32_t total_q_tokens,
@@ -119,6 +133,10 @@ int32_t msa_route_last_launch_count(void);
  * stream, so cudaEventElapsedTime gives that kernel's device time (also inside a CUDA
  * graph capture).  NULL, NULL turns it off.  Returns MSA_OK. */
 msa_status msa_route_set_profile_events(void* start_event, void* stop_event);
+
+/* The same hook around the query stage: the query preparation kernel of msa_route_topk,
+ * or the fused projection kernel of msa_route_topk_hidden. */
+msa_status msa_route_set_query_profile_events(void* start_event, void* stop_event);
 
 /* Tensor-core path tiling on this thread: 1 (default) runs N tiles of 128 / 256 query
  * tokens as M=256 tiles on pairs of SMs (tcgen05 cta_group::2, each SM streaming half of

@@ -74,7 +74,9 @@ class DeviceBank:
         err = torch.zeros(1, dtype=torch.int32, device="cuda")
         msa.msa_route_topk(qr, q_offsets, self.kr_hat, self.d_coffs, self.n_docs, self.C, self.L, HQ, H, D, k, ids,
                            sc, ws, flags=flags, dev_err=err,
-                           kr_f8=self.kr_f8 if flags in (msa.MSA_ROUTE_AUTO, msa.MSA_ROUTE_TENSOR_F8) else None)
+                           kr_f8=self.kr_f8 if (flags & ~msa.MSA_ROUTE_LAYER_MEAN) in (msa.MSA_ROUTE_AUTO,
+                                                                                       msa.MSA_ROUTE_TENSOR_F8)
+                           else None)
         torch.cuda.synchronize()
         return ids.cpu().numpy(), sc.cpu().numpy(), int(err.item())
 

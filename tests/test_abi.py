@@ -46,7 +46,7 @@ def test_common_header_constants_match_binding(msa):
         v = int(re.search(rf"#define {name} (\d+)u", text).group(1))
         assert getattr(msa, name) == v
     text = open(os.path.join(ROOT, "include", "msa_route.h")).read()
-    for name in ("MSA_ROUTE_AUTO", "MSA_ROUTE_SCAN", "MSA_ROUTE_TENSOR", "MSA_ROUTE_TENSOR_F8"):
+    for name in ("MSA_ROUTE_AUTO", "MSA_ROUTE_SCAN", "MSA_ROUTE_TENSOR", "MSA_ROUTE_TENSOR_F8", "MSA_ROUTE_LAYER_MEAN"):
         assert getattr(msa, name) == int(re.search(rf"#define {name} (\d+)", text).group(1))
 
 
@@ -69,6 +69,12 @@ def test_invalid_arguments_rejected_without_gpu(msa):
         z = np.zeros(16, np.uint16)
         msa.msa_route_topk(z, [0, 1], z, np.zeros(2, np.int64), 1, 1, 1, 32, 8, 128, 4, np.zeros(4, np.int32),
                            np.zeros(4, np.float32), np.zeros(256, np.uint8), flags=msa.MSA_ROUTE_TENSOR_F8, stream=0)
+    assert e.value.status == msa.MSA_ERR_INVALID_ARG
+    with pytest.raises(msa.MsaError) as e:   # the layer-aggregated selection on the scan path
+        z = np.zeros(16, np.uint16)
+        msa.msa_route_topk(z, [0, 1], z, np.zeros(2, np.int64), 1, 1, 1, 32, 8, 128, 4, np.zeros(4, np.int32),
+                           np.zeros(4, np.float32), np.zeros(256, np.uint8),
+                           flags=msa.MSA_ROUTE_SCAN | msa.MSA_ROUTE_LAYER_MEAN, stream=0)
     assert e.value.status == msa.MSA_ERR_INVALID_ARG
     with pytest.raises(msa.MsaError) as e:   # head_dim 64
         msa.msa_route_filter_keys(np.zeros(16, np.uint16), 1, 1, 8, 64, np.zeros(16, np.uint8), stream=0)

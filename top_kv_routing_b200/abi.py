@@ -17,6 +17,7 @@ LIB_DIR = os.path.join(_HERE, "lib")
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY, MSA_ERR_TIMEOUT, MSA_ERR_IO = range(7)
 MSA_F32, MSA_BF16 = 0, 1
 MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR, MSA_ROUTE_TENSOR_F8 = 0, 1, 2, 3
+MSA_ROUTE_LAYER_MEAN = 16  # OR-ed with a path: one selection for all layers
 (MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS, MSA_DEVERR_TIMEOUT,
  MSA_DEVERR_UNCERTIFIED) = 1, 2, 4, 8, 16, 32
 
@@ -71,6 +72,8 @@ route_lib.msa_route_set_pair_mode.argtypes = [_i32]
 route_lib.msa_route_set_pair_mode.restype = _i32
 route_lib.msa_route_set_profile_events.argtypes = [_p, _p]
 route_lib.msa_route_set_profile_events.restype = _i32
+route_lib.msa_route_set_query_profile_events.argtypes = [_p, _p]
+route_lib.msa_route_set_query_profile_events.restype = _i32
 
 gather_lib.msa_gather_kv.argtypes = [_p, _i64, _p, _p, _i32, _p, _i32, _i32, _i32, _i32, _i32, _i32, _p, _p,
                                      _p, _p]
@@ -242,6 +245,13 @@ def msa_route_set_profile_events(start_event=None, stop_event=None):
     a = None if start_event is None else start_event.cuda_event
     b = None if stop_event is None else stop_event.cuda_event
     route_lib.msa_route_set_profile_events(a, b)
+
+
+def msa_route_set_query_profile_events(start_event=None, stop_event=None):
+    """The same around the query stage (preparation, or the fused projection)."""
+    a = None if start_event is None else start_event.cuda_event
+    b = None if stop_event is None else stop_event.cuda_event
+    route_lib.msa_route_set_query_profile_events(a, b)
 
 
 # ----------------------------------------------------------------------------- step 3

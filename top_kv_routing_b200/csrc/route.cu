@@ -58,6 +58,7 @@ int rescore_count(int32_t n_docs, int32_t k) {
 
 static thread_local int32_t g_launches = 0;
 static thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+static thread_local cudaEvent_t g_qprof_start = nullptr, g_qprof_stop = nullptr;
 static thread_local bool g_pair_mode = true;
 
 struct QueryOffsets {
@@ -82,7 +83,8 @@ int pow2_at_least(int n) {
 }
 
 struct WsLayout {
-  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, cand, apx, exact, redo, doc_score, block_doc, total;
+  size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, cand, apx, exact, redo, doc_score, block_doc, agg, apx_agg, exact_agg,
+      total;
   int n_pad;
   int nblk;
   int k2;
@@ -123,6 +125,13 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   o += align256((size_t)B * L * (size_t)(n_docs > 0 ? n_docs : 1) * sizeof(uint32_t));
   w.block_doc = o;
   o += align256((size_t)(C > 0 ? C : 1) * sizeof(int32_t));
+  // layer-aggregated selection: mean document scores and their candidates per query
+  w.agg = o;
+  o += align256((size_t)B * (size_t)(n_docs > 0 ? n_docs : 1) * sizeof(uint32_t));
+  w.apx_agg = o;
+  o += align256((size_t)B * (w.k2 > 0 ? w.k2 : 1) * sizeof(unsigned long long));
+  w.exact_agg = o;
+  o += align256((size_t)B * (w.k2 > 0 ? w.k2 : 1) * sizeof(uint32_t));
   w.total = o;
   return w;
 }
@@ -913,6 +922,96 @@ __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long l
   }
 }
 
+// ---------------------------------------------------------------------------- layer-aggregated selection
+// One selection shared by every layer: documents ranked by the mean over layers of their
+// scores.  Scores travel as ordered bits (make_key's high word).
+__device__ __forceinline__ float ord_to_float(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+__device__ __forceinline__ uint32_t float_to_ord(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// agg[b][d] = mean over layers of doc_score[b][l][d] (in layer order; -inf stays -inf).
+// gate: run only when gate[0] != 0 (the second pass), or always when null.
+__global__ void layer_mean_kernel(const uint32_t* __restrict__ doc_score, int B, int L, int n_docs,
+                                  uint32_t* __restrict__ agg, const int32_t* __restrict__ gate) {
+  if (gate != nullptr && gate[0] == 0) return;
+  const float inv_l = 1.0f / (float)L;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < (int64_t)B * n_docs;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t b = i / n_docs, d = i % n_docs;
+    float acc = 0.f;
+    for (int l = 0; l < L; ++l) acc += ord_to_float(doc_score[(b * L + l) * n_docs + d]);
+    agg[i] = float_to_ord(acc * inv_l);
+  }
+}
+
+// Every layer of query b takes the shared candidates; their exact scores restart at -inf.
+__global__ void replicate_candidates_kernel(const unsigned long long* __restrict__ apx_agg, int B, int L, int K2,
+                                            unsigned long long* __restrict__ apx, uint32_t* __restrict__ exact_bits,
+                                            const int32_t* __restrict__ gate) {
+  if (gate != nullptr && gate[0] == 0) return;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < (int64_t)B * L * K2;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t b = i / ((int64_t)L * K2), r = i % K2;
+    apx[i] = apx_agg[b * K2 + r];
+    exact_bits[i] = kOrdNegInf;
+  }
+}
+
+// grid (B): the final top-k of the shared candidates by the mean over layers of their
+// exact scores, written to every layer; certified when the k-th exact mean beats the best
+// mean filter score left out by more than err (else the redo mark on all layers, or
+// MSA_DEVERR_UNCERTIFIED).
+__global__ void __launch_bounds__(128) select_final_mean_kernel(
+    const unsigned long long* __restrict__ apx_agg, const uint32_t* __restrict__ exact_bits, int K2, int k, int n_docs,
+    int L, float err, int32_t* __restrict__ out_ids, float* __restrict__ out_scores, int32_t* dev_err,
+    int32_t* __restrict__ redo, const int32_t* __restrict__ gate) {
+  __shared__ unsigned long long keys[kMaxCandidates];
+  if (gate != nullptr && gate[0] == 0) return;
+  const int b = blockIdx.x;
+  const int n_pow2 = K2 <= 1 ? 1 : (1 << (32 - __clz(K2 - 1)));
+  const float inv_l = 1.0f / (float)L;
+  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+    unsigned long long key = 0ull;
+    if (i < K2) {
+      int doc;
+      float s;
+      split_key(apx_agg[(int64_t)b * K2 + i], &doc, &s);
+      if (doc >= 0) {
+        float acc = 0.f;
+        for (int l = 0; l < L; ++l) acc += ord_to_float(exact_bits[((int64_t)b * L + l) * K2 + i]);
+        key = make_key(acc * inv_l, doc);
+      }
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  block_sort_desc(keys, n_pow2);
+  for (int e = threadIdx.x; e < L * k; e += blockDim.x) {
+    const int l = e / k, r = e % k;
+    int doc;
+    float s;
+    split_key(r < n_pow2 ? keys[r] : 0ull, &doc, &s);
+    out_ids[((int64_t)b * L + l) * k + r] = doc;
+    out_scores[((int64_t)b * L + l) * k + r] = s;
+  }
+  if (threadIdx.x == 0 && n_docs > K2 && K2 >= k) {
+    int d_left, d_kth;
+    float s_left, s_kth;
+    split_key(apx_agg[(int64_t)b * K2 + K2 - 1], &d_left, &s_left);
+    split_key(keys[k - 1], &d_kth, &s_kth);
+    if (!(s_kth > s_left + err)) {
+      if (redo != nullptr)
+        for (int l = 0; l < L; ++l) redo[l] = 1;
+      else
+        msa::set_err(dev_err, MSA_DEVERR_UNCERTIFIED);
+    }
+  }
+}
+
 }  // namespace
 
 extern "C" msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, int32_t total_q_tokens,
@@ -929,6 +1028,12 @@ extern "C" int32_t msa_route_last_launch_count(void) { return g_launches; }
 
 extern "C" msa_status msa_route_set_pair_mode(int32_t enabled) {
   g_pair_mode = enabled != 0;
+  return msa_ok();
+}
+
+extern "C" msa_status msa_route_set_query_profile_events(void* start_event, void* stop_event) {
+  g_qprof_start = (start_event && stop_event) ? reinterpret_cast<cudaEvent_t>(start_event) : nullptr;
+  g_qprof_stop = (start_event && stop_event) ? reinterpret_cast<cudaEvent_t>(stop_event) : nullptr;
   return msa_ok();
 }
 
@@ -994,7 +1099,11 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   if (n_layers < 1 || n_chunks < 0 || n_docs < 0 || n_docs > kMaxDocs)
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_docs <= 2^20)");
   if (!project && q_dtype != MSA_F32 && q_dtype != MSA_BF16) return msa_fail(MSA_ERR_UNSUPPORTED, "q_dtype");
+  const bool layer_mean = (flags & MSA_ROUTE_LAYER_MEAN) != 0;
+  flags &= ~MSA_ROUTE_LAYER_MEAN;
   if (flags < MSA_ROUTE_AUTO || flags > MSA_ROUTE_TENSOR_F8) return msa_fail(MSA_ERR_INVALID_ARG, "flags");
+  if (layer_mean && flags == MSA_ROUTE_SCAN)
+    return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_LAYER_MEAN runs on the tensor path, not MSA_ROUTE_SCAN");
   if (flags == MSA_ROUTE_TENSOR_F8 && !kr_f8)
     return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_TENSOR_F8 needs the E4M3 keys (msa_route_filter_keys)");
   if (!msa::aligned16(qr) || !msa::aligned16(kr_hat) || !msa::aligned16(kr_f8) ||
@@ -1030,9 +1139,11 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   // (on the E4M3 keys when the caller has them).
   int path = flags;
   if (path == MSA_ROUTE_AUTO)
-    path = (T_total <= route_tc::kScanMaxTokens) ? MSA_ROUTE_SCAN : (kr_f8 ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
+    path = (T_total <= route_tc::kScanMaxTokens && !layer_mean) ? MSA_ROUTE_SCAN
+                                                                 : (kr_f8 ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
   if ((path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && !route_tc::supported(H)) {
-    if (flags != MSA_ROUTE_AUTO) return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
+    if (flags != MSA_ROUTE_AUTO || layer_mean)
+      return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
     path = MSA_ROUTE_SCAN;
   }
   const bool tensor = (path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && n_chunks > 0;
@@ -1060,6 +1171,7 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
+  if (g_qprof_start) MSA_CUDA_TRY(cudaEventRecord(g_qprof_start, s));
   if (project) {
     // Q_r = hidden W^T on the tensor cores, normalised and group-summed in the epilogue
     route_proj::Args pa;
@@ -1093,6 +1205,7 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   }
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
+  if (g_qprof_stop) MSA_CUDA_TRY(cudaEventRecord(g_qprof_stop, s));
 
   // tcgen05 filter GEMM over all blocks of the layers `only` marks (all when null)
   auto gemm = [&](bool e4m3, const int32_t* only) -> msa_status {
@@ -1189,6 +1302,48 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
     MSA_CUDA_TRY(cudaGetLastError());
     return msa_ok();
   };
+  // the layer-aggregated variant: shared candidates from the mean filter scores, exact
+  // rescoring in every layer, final top-k on the mean exact scores (gate: the second
+  // pass runs these only when the first marked the layers)
+  unsigned long long* apx_agg = reinterpret_cast<unsigned long long*>(ws + w.apx_agg);
+  uint32_t* agg = reinterpret_cast<uint32_t*>(ws + w.agg);
+  uint32_t* exact_agg = reinterpret_cast<uint32_t*>(ws + w.exact_agg);
+  auto select_mean = [&](float err, int32_t* redo_out, const int32_t* gate) -> msa_status {
+    const int64_t n_agg = (int64_t)n_queries * n_docs;
+    const int mean_blocks = (int)((n_agg + 255) / 256 < msa::sm_count() * 4 ? (n_agg + 255) / 256 : msa::sm_count() * 4);
+    layer_mean_kernel<<<mean_blocks > 0 ? mean_blocks : 1, 256, 0, s>>>(doc_score, n_queries, n_layers, n_docs, agg,
+                                                                        gate);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    topk_docs_kernel<<<dim3(1, n_queries), kSelThreads, 0, s>>>(agg, 1, n_docs, K2, apx_agg, exact_agg, gate);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    const int64_t n_rep = (int64_t)n_queries * n_layers * K2;
+    replicate_candidates_kernel<<<(int)((n_rep + 255) / 256), 256, 0, s>>>(apx_agg, n_queries, n_layers, K2, apx,
+                                                                          exact, gate);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    rescore_mma_kernel<<<dim3(rs_x, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
+        (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx, K2,
+        exact, gate);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    select_final_mean_kernel<<<n_queries, 128, 0, s>>>(apx_agg, exact, K2, top_k, n_docs, n_layers, err, out_ids,
+                                                       out_scores, dev_err, redo_out, gate);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    return msa_ok();
+  };
+  if (layer_mean) {
+    msa_status st = select_mean(filter_err, f8 ? redo : nullptr, nullptr);
+    if (st != MSA_OK || !f8) return st;
+    doc_reset_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(doc_score, n_layers, n_docs, redo);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    st = gemm(false, redo);
+    if (st != MSA_OK) return st;
+    return select_mean(kFilterErr, nullptr, redo);
+  }
   msa_status st = select(filter_err, f8 ? redo : nullptr, nullptr);
   if (st != MSA_OK || !f8) return st;
   // E4M3 layers that could not be certified: bf16 filter over them, then the same steps
