@@ -27,7 +27,7 @@ TARGETS = {
     os.path.join(LIB, "libmsa_route.so"): ["route.cu", "route_tc.cu", "route_proj.cu"],
     os.path.join(LIB, "libmsa_gather.so"): ["gather.cu"],
     os.path.join(LIB, "libmsa_decode.so"): ["decode.cu"],
-    os.path.join(LIB, "libmsa_prefill.so"): ["prefill.cu"],
+    os.path.join(LIB, "libmsa_prefill.so"): ["prefill.cu", "prefill_tc.cu"],
     os.path.join(LIB, "libmsa_bank.so"): ["bank.cu"],
 }
 SYNTH_TARGET = os.path.join(SYNTH, "libmsa_synth.so")

@@ -1,0 +1,27 @@
+// tcgen05 prefill attention (host-side interface used by prefill.cu; not part of the ABI).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace prefill_tc {
+
+struct Args {
+  const __nv_bfloat16* q;       // [B][L][T][H*G][128]
+  __nv_bfloat16* out;           // [B][L][T][H*G][128]
+  const __nv_bfloat16* local_k; // [B][L][H][cap][128] (the block's rows already appended)
+  const __nv_bfloat16* local_v;
+  const int32_t* local_len;     // [B] (before the block)
+  const __nv_bfloat16* mem_kv;  // [B][L][2][H][M_max][128]
+  const int32_t* mem_len;       // [B][L]
+  int T, B, L, H, G, cap, M_max, pos_off;
+  double log2_theta;
+  float qscale;                 // softmax scale x log2(e)
+  int32_t* dev_err;
+};
+
+// Sizes within the kernel's 32-bit tensor-map row coordinates.
+bool supported(const Args& a);
+int launch(const Args& a, cudaStream_t s, const char** why);
+
+}  // namespace prefill_tc

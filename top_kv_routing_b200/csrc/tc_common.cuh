@@ -200,6 +200,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the 128-byte
 // swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte offset), leading
 // byte offset unused for swizzled K-major layouts, descriptor version 1, swizzle mode 2.
@@ -213,11 +226,27 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major tile in the 128-byte swizzle: each
+// 128-byte row holds 64 consecutive MN elements of one K index, 8 K rows form a 1024-byte
+// atom; lbo = byte distance between atoms along MN (the next 64 elements), sbo = byte
+// distance between atoms along K (the next 8 K indices).
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A and B both K-major, A / B
 // formats in bits 7-9 / 10-12 (kind::f16: bf16 = 1; kind::f8f6f4: E4M3 = 0), N / 8 in
 // bits 17-22, M / 16 in bits 24-28.
 __host__ __device__ constexpr uint32_t idesc_make(int m, int n, bool f8) {
   return (1u << 4) | (f8 ? 0u : (1u << 7) | (1u << 10)) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
+// bf16 with B MN-major (bit 16: B read as [K rows of N-contiguous elements])
+__host__ __device__ constexpr uint32_t idesc_make_bmn(int m, int n) { return idesc_make(m, n, false) | (1u << 16); }
 
 }  // namespace tc
