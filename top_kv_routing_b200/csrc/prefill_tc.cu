@@ -6,18 +6,20 @@
 // times the values.  Follows "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", section
 // 推理流水线, and the MSA paper reading notes, section 推理全流程.
 //
-// One CTA (192 threads) per 128 rows: 128 / G tokens x the G query heads of key head h.
-//   warp 5, one thread   TMA producer: tiles of 64 keys (K as two 64-column boxes, then V
+// One CTA (320 threads) per 128 rows: 128 / G tokens x the G query heads of key head h.
+//   warp 9, one thread   TMA producer: tiles of 64 keys (K as two 64-column boxes, then V
 //                        the same), 128-byte swizzle, a 3-stage ring; memory tiles first,
 //                        then local tiles up to the CTA's last token
-//   warp 4, one thread   MMA issuer: S_i = Q K_i^T (M = 128, N = 64, K = 128) into one of two
+//   warp 8, one thread   MMA issuer: S_i = Q K_i^T (M = 128, N = 64, K = 128) into one of two
 //                        TMEM score buffers, then O += P_{i-1} V_{i-1} (M = 128, N = 128,
 //                        K = 64) into the TMEM output.  The rotated queries and the softmax
 //                        weights are each a bf16 value plus a bf16 residual (two MMAs), the
 //                        keys and values exact bf16; V is read MN-major straight from its
 //                        [key][d] rows
-//   warps 0..3           thread = row (TMEM lane): builds its rotated, scaled query row in
-//                        shared memory; per tile reads its score row, masks it (memory keys
+//   warps 0..7           two threads per row (TMEM lane), each with half of the row's dims
+//                        and half of every tile's keys: build the rotated, scaled query row
+//                        in shared memory (cos / sin once per token); per tile read the score
+//                        row, mask it (memory keys
 //                        < M, local keys <= its own local index), keeps a running maximum
 //                        that is raised (and O rescaled in TMEM) only when a score exceeds it
 //                        by more than 2^8, writes its weights exp2(s - m) as the A operand of
@@ -40,7 +42,9 @@ constexpr int kHalf = 64;
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
 constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kRowWarps = 8;                  // two threads per row: 32 keys of a tile each
+constexpr int kMmaWarp = kRowWarps, kTmaWarp = kRowWarps + 1;
+constexpr int kThreads = (kRowWarps + 2) * 32;
 constexpr int kQHalf = kRows * 128;      // 16 KB: 64 bf16 of every row
 constexpr int kQBytes = 2 * kQHalf;      // 32 KB: one bf16 copy of the CTA's queries
 constexpr int kPBytes = kRows * 128;     // 16 KB: 64 bf16 weights of every row
@@ -52,7 +56,7 @@ constexpr int kOffPhi = 2 * kQBytes;
 constexpr int kOffPlo = 2 * kQBytes + kPBytes;
 constexpr int kOffRing = 2 * kQBytes + 2 * kPBytes;
 constexpr int kSmemData = kOffRing + kStages * kTileBytes;
-constexpr int kSmem = kSmemData + 1024 + 256;
+constexpr int kSmem = kSmemData + 1024 + 256 + 4 * 128 * 4;  // + the row pairs' exchange buffer
 constexpr uint32_t kTmemCols = 256;  // S0 [0, 64) | S1 [64, 128) | O [128, 256)
 constexpr uint32_t kColO = 128;
 constexpr float kHeadroom = 8.0f;    // log2 growth of a row's maximum tolerated before rescaling
@@ -113,17 +117,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(bar_q), 4);
+    mbar_init(smem_u32(bar_q), kRowWarps);
     mbar_init(smem_u32(&bar_s[0]), 1);
     mbar_init(smem_u32(&bar_s[1]), 1);
-    mbar_init(smem_u32(bar_p), 4);
+    mbar_init(smem_u32(bar_p), kRowWarps);
     mbar_init(smem_u32(bar_pv), 1);
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc<false>(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish<false>();
   }
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
 
-  if (warp == 5) {
+  if (warp == kTmaWarp) {
     if (lane == 0) {
       // ---------------- TMA producer
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
@@ -175,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       // ---------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
@@ -233,106 +237,151 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- rows (warps 0..3, thread = TMEM lane = row)
-    const int r = tid;
+    // ---------------- rows (warps 0..7): thread (row r = TMEM lane, half hf) takes the row's
+    // dims 32 hf .. 32 hf + 31 and 64 + 32 hf .. 95 + 32 hf of the query, and keys
+    // 32 hf .. 32 hf + 31 of every tile; the pair meets in shared memory (warps w, w + 4)
+    const int r = tid & (kRows - 1), hf = tid >> 7;
     const int tl = r / G, hd = r % G;
     const int tok = tok0 + tl;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    {  // rotated, scaled query row: bf16 value and residual, 128-byte swizzled rows
-      float x[kD];
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const int pair_bar = 1 + (warp & 3);  // named barrier of warps w and w + 4
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
+    {  // rotated, scaled query: bf16 value and residual, 128-byte swizzled rows
+      // cos / sin of the block's tokens (G > 1: once per token, shared by its G rows, in the
+      // weight buffer, which is free until the first tile)
+      float2* tab = reinterpret_cast<float2*>(smem + kOffPhi);
+      if (G > 1) {
+        for (int e = tid; e < kTok * kHalf; e += kRowWarps * 32) {
+          const int t2 = e / kHalf, j = e % kHalf;
+          double u = ((double)pos_off + (double)(len + tok0 + t2)) * s_w[j];
+          u -= 2.0 * rint(0.5 * u);
+          float sn, cs;
+          sincospif((float)u, &sn, &cs);
+          tab[e] = make_float2(cs, sn);
+        }
+        asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory");
+      }
+      float xa[32], xb[32];  // dims 32 hf + e and 64 + 32 hf + e
       if (tok < T) {
-        const uint4* src = reinterpret_cast<const uint4*>(q + ((bl * T + tok) * Hq + (int64_t)h * G + hd) * kD);
+        const __nv_bfloat16* src = q + ((bl * T + tok) * Hq + (int64_t)h * G + hd) * kD;
+        const uint4* pa = reinterpret_cast<const uint4*>(src + 32 * hf);
+        const uint4* pb = reinterpret_cast<const uint4*>(src + kHalf + 32 * hf);
 #pragma unroll
-        for (int c = 0; c < kD / 8; ++c) {
-          const uint4 w = __ldg(src + c);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int c = 0; c < 4; ++c) {
+          const uint4 wa = __ldg(pa + c), wb = __ldg(pb + c);
+          const uint32_t va[4] = {wa.x, wa.y, wa.z, wa.w}, vb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            x[8 * c + 2 * e] = __uint_as_float(ww[e] << 16);
-            x[8 * c + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+            xa[8 * c + 2 * e] = __uint_as_float(va[e] << 16);
+            xa[8 * c + 2 * e + 1] = __uint_as_float(va[e] & 0xFFFF0000u);
+            xb[8 * c + 2 * e] = __uint_as_float(vb[e] << 16);
+            xb[8 * c + 2 * e + 1] = __uint_as_float(vb[e] & 0xFFFF0000u);
           }
         }
         const double pos = (double)pos_off + (double)(len + tok);
 #pragma unroll
-        for (int j = 0; j < kHalf; ++j) {
-          double u = pos * s_w[j];
-          u -= 2.0 * rint(0.5 * u);
+        for (int e = 0; e < 32; ++e) {
+          const int j = 32 * hf + e;
           float sn, cs;
-          sincospif((float)u, &sn, &cs);
-          const float a = x[j], bb = x[j + kHalf];
-          x[j] = (a * cs - bb * sn) * qscale;
-          x[j + kHalf] = (bb * cs + a * sn) * qscale;
+          if (G > 1) {
+            const float2 t2 = tab[tl * kHalf + j];
+            cs = t2.x;
+            sn = t2.y;
+          } else {
+            double u = pos * s_w[j];
+            u -= 2.0 * rint(0.5 * u);
+            sincospif((float)u, &sn, &cs);
+          }
+          const float a = xa[e], bb = xb[e];
+          xa[e] = (a * cs - bb * sn) * qscale;
+          xb[e] = (bb * cs + a * sn) * qscale;
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < kD; ++j) x[j] = 0.f;
+        for (int e = 0; e < 32; ++e) xa[e] = xb[e] = 0.f;
       }
 #pragma unroll
-      for (int c = 0; c < kD / 8; ++c) {  // chunk c: elements 8c .. 8c+7
+      for (int c = 0; c < 8; ++c) {  // chunks of 8 dims: 4 hf .. 4 hf + 3 (xa) and 8 + 4 hf .. (xb)
+        const float* x = c < 4 ? &xa[8 * c] : &xb[8 * (c - 4)];
+        const int chunk = c < 4 ? 4 * hf + c : 8 + 4 * hf + (c - 4);
         uint32_t hw[4], lw[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split2(x[8 * c + 2 * e], x[8 * c + 2 * e + 1], hw[e], lw[e]);
-        const uint32_t off = (uint32_t)((c >> 3) * kQHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+        for (int e = 0; e < 4; ++e) split2(x[2 * e], x[2 * e + 1], hw[e], lw[e]);
+        const uint32_t off = (uint32_t)((chunk >> 3) * kQHalf + r * 128 + (((chunk & 7) ^ (r & 7)) << 4));
         st_shared_v4(sbase + kOffQhi + off, hw[0], hw[1], hw[2], hw[3]);
         st_shared_v4(sbase + kOffQlo + off, lw[0], lw[1], lw[2], lw[3]);
       }
+      if (G > 1) asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory");  // the table is read
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(bar_q));
     }
+    float* xch = reinterpret_cast<float*>(smem + kSmemData + 256);  // [2 tiles][2 halves][128 rows]
     const int lim = len + min(tok, T - 1);
     float m_used = -INFINITY, l_sum = 0.f;
     bool ok = true;
+    // Every row thread runs every iteration and every pair barrier, whatever happens: a
+    // failed (timed-out) wait only clears `ok` and raises the abort flag, after which the
+    // remaining waits return at once and the work is skipped.  So the pair barriers, which
+    // cannot time out, always meet.
+    auto fail = [&]() {
+      ok = false;
+      *abort_flag = 1;
+    };
     for (int i = 0; i < nt; ++i) {
       // (waits are made warp-uniform: the TMEM accesses below are warp-collective)
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_s[i & 1]), (uint32_t)((i >> 1) & 1), abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sa[32], sb[32];
-      tmem_ld32(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys), sa);
-      tmem_ld32(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 32), sb);
-      tmem_wait_ld();
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_s[i & 1]), (uint32_t)((i >> 1) & 1), abort_flag)))
+        fail();
       const bool local = i >= nt_mem;
       const int key0 = local ? (i - nt_mem) * kKeys : i * kKeys;
       const int n_valid = local ? min(kKeys, n_local - key0) : min(kKeys, M - key0);
       float mx = -INFINITY;
-      float s[kKeys];
+      float sv[32];
+      if (ok) {
+        tc_fence_after();
+        uint32_t sa[32];
+        tmem_ld32(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 32 * hf), sa);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < kKeys; ++e) {
-        const int key = key0 + e;
-        const bool v = local ? key <= lim : key < M;
-        s[e] = v ? __uint_as_float(e < 32 ? sa[e] : sb[e - 32]) : -INFINITY;
-        mx = fmaxf(mx, s[e]);
+        for (int e = 0; e < 32; ++e) {
+          const int key = key0 + 32 * hf + e;
+          const bool v = local ? key <= lim : key < M;
+          sv[e] = v ? __uint_as_float(sa[e]) : -INFINITY;
+          mx = fmaxf(mx, sv[e]);
+        }
       }
-      const bool need = mx > m_used + kHeadroom;
+      xch[((i & 1) * 2 + hf) * kRows + r] = mx;
+      pair_sync();
+      mx = fmaxf(mx, xch[((i & 1) * 2 + (hf ^ 1)) * kRows + r]);
+      if (!ok) continue;
+      const bool need = mx > m_used + kHeadroom;  // (the same in both threads of the row)
       if (i > 0) {  // PV of the previous tile done: O is stable and the weight buffer free
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)((i - 1) & 1), abort_flag))) {
-          ok = false;
-          break;
+          fail();
+          continue;
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? exp2f(m_used - mx) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
+          for (int c = 0; c < 2; ++c) {  // this thread's 64 of the 128 output columns
             uint32_t o[32];
-            tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)(c * 32), o);
+            const uint32_t col = kColO + (uint32_t)(64 * hf + 32 * c);
+            tmem_ld32(tmem_base + lane_addr + col, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tmem_base + lane_addr + kColO + (uint32_t)(c * 32), o);
+            tmem_st32(tmem_base + lane_addr + col, o);
           }
           tmem_wait_st();
           if (need) l_sum *= alpha;
         }
       }
       if (need) m_used = mx;
-      // key rows past the valid count: zero their V rows (all four warps share the rows)
+      // key rows past the valid count: zero their V rows (all row threads share the rows)
       if (n_valid < kKeys) {
         const uint32_t vt = sbase + kOffRing + (i % kStages) * kTileBytes + 2 * kKVHalf;
-        for (int idx = r; idx < (kKeys - n_valid) * 16; idx += kRows) {
+        for (int idx = tid; idx < (kKeys - n_valid) * 16; idx += kRowWarps * 32) {
           const int row = n_valid + (idx >> 4), c16 = idx & 15;
           st_shared_v4(vt + (uint32_t)((c16 >> 3) * kKVHalf + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)), 0u, 0u, 0u,
                        0u);
@@ -340,17 +389,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float psum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kKeys / 8; ++c) {
+      for (int c = 0; c < 4; ++c) {  // keys 32 hf + 8c .. : chunk 4 hf + c of the weight row
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          p[e] = exp2f(s[8 * c + e] - m_used);
+          p[e] = exp2f(sv[8 * c + e] - m_used);
           psum += p[e];
         }
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) split2(p[2 * e], p[2 * e + 1], hw[e], lw[e]);
-        const uint32_t off = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+        const uint32_t off = (uint32_t)(r * 128 + (((4 * hf + c) ^ (r & 7)) << 4));
         st_shared_v4(sbase + kOffPhi + off, hw[0], hw[1], hw[2], hw[3]);
         st_shared_v4(sbase + kOffPlo + off, lw[0], lw[1], lw[2], lw[3]);
       }
@@ -362,18 +411,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && nt > 0 &&
         !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)((nt - 1) & 1), abort_flag)))
-      ok = false;
+      fail();
+    // the row's sum of weights: both halves (the exchange slot of tile nt is free)
+    xch[((nt & 1) * 2 + hf) * kRows + r] = l_sum;
+    pair_sync();
+    l_sum += xch[((nt & 1) * 2 + (hf ^ 1)) * kRows + r];
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const float inv = 1.0f / l_sum;
       __nv_bfloat16* dst = out + ((bl * T + tok) * Hq + (int64_t)h * G + hd) * kD;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)(c * 32), o);
+        const int col = 64 * hf + 32 * c;
+        tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)col, o);
         tmem_wait_ld();
         if (tok < T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + col);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             uint32_t w[4];
@@ -395,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc<false>(tmem_base, kTmemCols);
   }
