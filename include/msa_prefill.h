@@ -36,13 +36,14 @@ extern "C" {
  *           (msa_gather_kv output); mem_len DEVICE int32 [n_queries][n_layers]
  *   out     DEVICE bf16 [n_queries][n_layers][n_new][n_q_heads][head_dim]
  *   head_dim = 128; n_q_heads / n_kv_heads in {1, 2, 4, 8}; n_kv_heads <= 16;
- *   n_queries * n_layers <= 65535.  q, mem_kv, local_k, local_v, out 16-byte aligned.
+ *   n_queries * n_layers <= 65535.  q, k_new, v_new, mem_kv, local_k, local_v, out 16-byte
+ *   aligned.
  *   The caller owns every buffer; the call allocates nothing.
  * Three kernel launches on `stream` (append, attention, advance), asynchronous and
  * graph-capturable (every per-call quantity that changes is read on the device).  The
- * attention kernel takes one CTA per (query, layer, key head, 64 / G tokens): its four
- * warps each hold 16 (token, query head) rows, and K/V stream through shared memory in
- * tiles of 16 keys for the tensor cores.
+ * attention kernel runs on the tcgen05 tensor cores: one CTA per (query, layer, key head,
+ * 128 / G tokens), the 128 (token, query head) rows as the MMA's M, K/V streaming in tiles
+ * of 64 keys, scores and output in tensor memory.
  * A query whose cache cannot hold the whole block (local_len + n_new > local_cap) is
  * skipped (out and cache untouched, length not advanced) and sets MSA_DEVERR_LOCAL_FULL;
  * mem_len > max_mem_chunks is clamped with MSA_DEVERR_CAPACITY.  Host-checked argument

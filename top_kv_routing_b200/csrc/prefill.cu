@@ -24,37 +24,45 @@ constexpr int kHalf = 64;
 constexpr int kThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ void angle_cs(double pos, int j, double log2_theta, float* c, float* s) {
-  double u = pos * (exp2(-2.0 * (double)j / (double)kD * log2_theta) * 0.31830988618379067154);  // angle / pi
-  u -= 2.0 * rint(0.5 * u);                                                                   // in [-1, 1]
-  sincospif((float)u, s, c);
-}
 
-// (1) grid (n_new, H, B * L), 128 threads: rotate, round and append token i's key and value.
+// (1) grid (ceil(n_new / 8), H, B * L), 128 threads: 16 threads per token (4 rotation pairs
+// and 8 values each) rotate, round and append 8 tokens' keys and values; the 64 frequencies
+// are computed once per CTA.
+constexpr int kAppendTok = 8;
 __global__ void __launch_bounds__(kThreads) prefill_append_kernel(
     const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new, int T, int L, int H,
     __nv_bfloat16* __restrict__ local_k, __nv_bfloat16* __restrict__ local_v, const int32_t* __restrict__ local_len,
     int cap, const int32_t* __restrict__ mem_len, int M_max, int pos_off, double log2_theta, int32_t* dev_err) {
-  const int i = blockIdx.x, h = blockIdx.y;
+  __shared__ double s_w[kHalf];  // theta^(-2j/d) / pi
+  const int h = blockIdx.y;
   const int64_t bl = blockIdx.z;
   const int b = (int)(bl / L);
   const int tid = threadIdx.x;
   const int len = local_len[b];
   if (len < 0 || len + T > cap) {
-    if (i == 0 && h == 0 && (bl % L) == 0 && tid == 0) msa::set_err(dev_err, MSA_DEVERR_LOCAL_FULL);
+    if (blockIdx.x == 0 && h == 0 && (bl % L) == 0 && tid == 0) msa::set_err(dev_err, MSA_DEVERR_LOCAL_FULL);
     return;
   }
-  if (i == 0 && h == 0 && tid == 0 && mem_len[bl] > M_max) msa::set_err(dev_err, MSA_DEVERR_CAPACITY);
+  if (blockIdx.x == 0 && h == 0 && tid == 0 && mem_len[bl] > M_max) msa::set_err(dev_err, MSA_DEVERR_CAPACITY);
+  if (tid < kHalf) s_w[tid] = exp2(-2.0 * (double)tid / (double)kD * log2_theta) * 0.31830988618379067154;
+  __syncthreads();
+  const int i = blockIdx.x * kAppendTok + tid / 16, q16 = tid % 16;
+  if (i >= T) return;
   const int64_t src = ((bl * T + i) * H + h) * kD;
   const int64_t dst = ((bl * H + h) * (int64_t)cap + len + i) * kD;
-  if (tid < kHalf) {
-    float c, s;
-    angle_cs((double)pos_off + (double)(len + i), tid, log2_theta, &c, &s);
-    const float a = __bfloat162float(k_new[src + tid]), bb = __bfloat162float(k_new[src + tid + kHalf]);
-    local_k[dst + tid] = __float2bfloat16_rn(a * c - bb * s);
-    local_k[dst + tid + kHalf] = __float2bfloat16_rn(bb * c + a * s);
+  const double pos = (double)pos_off + (double)(len + i);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int j = 4 * q16 + e;
+    double u = pos * s_w[j];  // angle / pi, reduced to [-1, 1]
+    u -= 2.0 * rint(0.5 * u);
+    float c, sn;
+    sincospif((float)u, &sn, &c);
+    const float a = __bfloat162float(k_new[src + j]), bb = __bfloat162float(k_new[src + j + kHalf]);
+    local_k[dst + j] = __float2bfloat16_rn(a * c - bb * sn);
+    local_k[dst + j + kHalf] = __float2bfloat16_rn(bb * c + a * sn);
   }
-  local_v[dst + tid] = v_new[src + tid];
+  *reinterpret_cast<uint4*>(local_v + dst + 8 * q16) = *reinterpret_cast<const uint4*>(v_new + src + 8 * q16);
 }
 
 // (3) one thread per query: the length advances by the block (unless the cache was full).
@@ -82,9 +90,10 @@ extern "C" msa_status msa_sparse_prefill(const void* q, const void* k_new, const
       max_mem_chunks < 1)
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_queries * n_layers <= 65535)");
   if (!(rope_theta > 1.0f)) return msa_fail(MSA_ERR_INVALID_ARG, "rope_theta must be > 1");
-  if (!msa::aligned16(q) || !msa::aligned16(mem_kv) || !msa::aligned16(local_k) || !msa::aligned16(local_v) ||
+  if (!msa::aligned16(q) || !msa::aligned16(k_new) || !msa::aligned16(v_new) || !msa::aligned16(mem_kv) ||
+      !msa::aligned16(local_k) || !msa::aligned16(local_v) ||
       !msa::aligned16(out))
-    return msa_fail(MSA_ERR_INVALID_ARG, "16-byte alignment (q, mem_kv, local_k, local_v, out)");
+    return msa_fail(MSA_ERR_INVALID_ARG, "16-byte alignment (q, k_new, v_new, mem_kv, local_k, local_v, out)");
   const int arch = msa::current_device_is_sm100(nullptr);
   if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
   if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
@@ -92,7 +101,7 @@ extern "C" msa_status msa_sparse_prefill(const void* q, const void* k_new, const
   const double log2_theta = log2((double)rope_theta);
   const float qscale = softmax_scale * kLog2e;
   const int BL = n_queries * n_layers;
-  prefill_append_kernel<<<dim3(n_new, n_kv_heads, BL), kThreads, 0, s>>>(
+  prefill_append_kernel<<<dim3((n_new + kAppendTok - 1) / kAppendTok, n_kv_heads, BL), kThreads, 0, s>>>(
       (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_new, n_layers, n_kv_heads, (__nv_bfloat16*)local_k,
       (__nv_bfloat16*)local_v, local_len, local_cap, mem_len, max_mem_chunks, rope_pos_offset, log2_theta, dev_err);
   MSA_CUDA_TRY(cudaGetLastError());

@@ -355,6 +355,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       mx = fmaxf(mx, xch[((i & 1) * 2 + (hf ^ 1)) * kRows + r]);
       if (!ok) continue;
       const bool need = mx > m_used + kHeadroom;  // (the same in both threads of the row)
+      const float m_old = m_used;
+      if (need) m_used = mx;
+      // weights, split into bf16 + residual, before the wait for the previous PV (only the
+      // stores into the shared weight buffer and a rescale of O need it to be done)
+      uint32_t phw[16], plw[16];
+      float psum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float p0 = exp2f(sv[2 * e] - m_used), p1 = exp2f(sv[2 * e + 1] - m_used);
+        psum += p0 + p1;
+        split2(p0, p1, phw[e], plw[e]);
+      }
+      // key rows past the valid count: zero their V rows (this tile's stage; all row threads)
+      if (n_valid < kKeys) {
+        const uint32_t vt = sbase + kOffRing + (i % kStages) * kTileBytes + 2 * kKVHalf;
+        for (int idx = tid; idx < (kKeys - n_valid) * 16; idx += kRowWarps * 32) {
+          const int row = n_valid + (idx >> 4), c16 = idx & 15;
+          st_shared_v4(vt + (uint32_t)((c16 >> 3) * kKVHalf + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)), 0u, 0u, 0u,
+                       0u);
+        }
+      }
       if (i > 0) {  // PV of the previous tile done: O is stable and the weight buffer free
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)((i - 1) & 1), abort_flag))) {
           fail();
@@ -362,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? exp2f(m_used - mx) : 1.0f;
+          const float alpha = need ? exp2f(m_old - m_used) : 1.0f;
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {  // this thread's 64 of the 128 output columns
             uint32_t o[32];
@@ -377,31 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (need) l_sum *= alpha;
         }
       }
-      if (need) m_used = mx;
-      // key rows past the valid count: zero their V rows (all row threads share the rows)
-      if (n_valid < kKeys) {
-        const uint32_t vt = sbase + kOffRing + (i % kStages) * kTileBytes + 2 * kKVHalf;
-        for (int idx = tid; idx < (kKeys - n_valid) * 16; idx += kRowWarps * 32) {
-          const int row = n_valid + (idx >> 4), c16 = idx & 15;
-          st_shared_v4(vt + (uint32_t)((c16 >> 3) * kKVHalf + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)), 0u, 0u, 0u,
-                       0u);
-        }
-      }
-      float psum = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {  // keys 32 hf + 8c .. : chunk 4 hf + c of the weight row
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = exp2f(sv[8 * c + e] - m_used);
-          psum += p[e];
-        }
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) split2(p[2 * e], p[2 * e + 1], hw[e], lw[e]);
         const uint32_t off = (uint32_t)(r * 128 + (((4 * hf + c) ^ (r & 7)) << 4));
-        st_shared_v4(sbase + kOffPhi + off, hw[0], hw[1], hw[2], hw[3]);
-        st_shared_v4(sbase + kOffPlo + off, lw[0], lw[1], lw[2], lw[3]);
+        st_shared_v4(sbase + kOffPhi + off, phw[4 * c], phw[4 * c + 1], phw[4 * c + 2], phw[4 * c + 3]);
+        st_shared_v4(sbase + kOffPlo + off, plw[4 * c], plw[4 * c + 1], plw[4 * c + 2], plw[4 * c + 3]);
       }
       l_sum += psum;
       fence_async_smem();
