@@ -171,3 +171,23 @@ def test_prefill_memory_length_clamped(msa):
     worst_abs, worst_rel = case.prefill(msa, 0, 9, 16)
     assert worst_abs <= DEC_MAX_ABS and worst_rel <= DEC_REL_L2
     assert int(case.err.item()) == msa.MSA_DEVERR_CAPACITY
+
+
+def test_prefill_bench_shape_sampled_layers(msa):
+    # the benchmark's prefill: 256 tokens, 18 layers, GQA 32/8, 256 memory rows, empty
+    # prefix; two layers checked in full against the oracle, every layer's output finite
+    B, L, T, M = 1, 18, 256, 256
+    case = Case(B=B, L=L, M_max=M, mem_len=[[M] * L], len0=[0], cap=T, seed=19)
+    qb, kb, vb = prefill_inputs(19, 0, B, L, T, HQ, H)
+    out = torch.full((B, L, T, HQ, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    msa.msa_sparse_prefill(bf16_tensor(qb), bf16_tensor(kb), bf16_tensor(vb), T, B, L, HQ, H, D, case.d_lk,
+                           case.d_lv, case.d_len, T, case.d_mem, case.d_mlen, M, 16, THETA, case.scale, out, case.err)
+    torch.cuda.synchronize()
+    assert int(case.err.item()) == 0 and case.d_len.cpu().tolist() == [T]
+    got = bf16_to_np(out)
+    assert np.isfinite(got).all()
+    f = syn.bf16_bits_to_f32
+    for l in (0, 13):
+        ref = oracle.prefill(f(qb[0, l]), f(kb[0, l]), f(vb[0, l]), f(case.mem_bits[0, l]), M, case.o_lk[0, l],
+                             case.o_lv[0, l], 0, 16, THETA, case.scale)
+        assert np.abs(got[0, l] - ref).max() <= DEC_MAX_ABS and rel_l2(got[0, l], ref) <= DEC_REL_L2, l

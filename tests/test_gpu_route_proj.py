@@ -107,3 +107,49 @@ def test_projected_routing_launches_like_the_unfused_call(msa):
     # (E4M3 path: prep, projection, GEMM, top-k, rescore, final, and the five second-pass
     # kernels that return at once when every layer is certified)
     assert _case(msa, 6, [64], 128, 32, 3) == 11
+
+
+def test_projected_routing_bench_shape_sampled_layers(msa):
+    # the benchmark's projection shape: hidden 2560, 256 tokens, 18 layers, 32 heads; a
+    # 300-document bank keeps the oracle's routing short; layers 0 and 11 checked
+    L, T, hidden, Hq, k, n_docs = 18, 256, 2560, 32, 16, 300
+    lens = syn.doc_lengths_uniform(8, n_docs, 64, 900)
+    bank = syn.make_bank(8, n_docs, lens, L)
+    keys = _bank_keys(bank, L)
+    C = bank.n_chunks
+    targets = syn.pick_targets(8, n_docs, 16, sub=3)
+    tok_targets = np.asarray(targets)[np.arange(T) % 16]
+    h_bits, _ = _inputs(8, bank, T, hidden, Hq, 1, tok_targets)  # (the hidden states only)
+    # weights drawn on the device (377 MB); the host redraws the sampled layers' bits: noise
+    # as bf16, plus the identity block, rounded to bf16 once (as the device add does)
+    w_dev = torch.empty((L, Hq * D, hidden), dtype=torch.bfloat16, device="cuda")
+    syn.device_fill(w_dev, 8, syn.STREAM_KBAR, 92, 0, 0, L * Hq * D, hidden, 0.02)
+    w_dev.view(L, Hq, D, hidden)[..., :D] += torch.eye(D, dtype=torch.bfloat16, device="cuda")
+
+    def host_w(l):
+        noise = syn.fill(8, syn.STREAM_KBAR, 92, 0, l * Hq * D, Hq * D, hidden, sigma=0.02, dtype="bf16")
+        x = syn.bf16_bits_to_f32(noise).reshape(Hq, D, hidden)
+        x[:, np.arange(D), np.arange(D)] += 1.0
+        return syn.bf16_bits_to_f32(syn.f32_to_bf16_bits(x)).reshape(Hq * D, hidden)
+    d_keys = bf16_tensor(keys)
+    kr_f8 = torch.empty(keys.shape, dtype=torch.uint8, device="cuda")
+    msa.msa_route_filter_keys(d_keys, L, C, H, D, kr_f8)
+    coffs = torch.from_numpy(bank.doc_chunk_offsets).cuda()
+    ws = torch.empty(msa.msa_route_topk_workspace_size(L, 1, T, H, C, n_docs, k), dtype=torch.uint8, device="cuda")
+    ids = torch.full((1, L, k), -7, dtype=torch.int32, device="cuda")
+    sc = torch.full((1, L, k), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    msa.msa_route_topk_hidden(bf16_tensor(h_bits), w_dev, hidden, [0, T], d_keys, coffs, n_docs, C, L, Hq, H, D, k,
+                              ids, sc, ws, flags=msa.MSA_ROUTE_TENSOR_F8, dev_err=err, kr_f8=kr_f8)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    gi, gs = ids.cpu().numpy(), sc.cpu().numpy()
+    for l in range(L):
+        assert set(np.asarray(targets).tolist()) == set(gi[0, l].tolist()), l  # the 16 planted documents
+    f = syn.bf16_bits_to_f32
+    for l in (0, 11):
+        assert np.array_equal(w_dev[l].cpu().view(torch.int16).numpy().view(np.uint16),
+                              syn.f32_to_bf16_bits(host_w(l)))
+        q = oracle.router_project(f(h_bits), host_w(l), Hq)
+        _, _, ds, _ = oracle.route(q, f(keys[l]), bank.doc_chunk_offsets, k, grouped=True)
+        check_topk(gi[0, l], gs[0, l], ds, k)
