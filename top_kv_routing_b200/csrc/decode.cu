@@ -89,9 +89,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
   const int Hq = H * G;
   const int64_t bl = blockIdx.z;
   const int64_t uh = bl * H + h;
+  // inputs no earlier decode step writes (this step's q, k_new, v_new; the gathered memory's
+  // length) load before the wait for the previous grid: thread (head gg, m) takes q dims 2m,
+  // 2m+1 and their rotate-half partners 2m+64, 2m+65
+  const int gg = tid >> 5, mq = tid & 31;
+  uint32_t qlo = 0u, qhi = 0u;
+  if (gg < G) {
+    const __nv_bfloat16* qp = q + (bl * Hq + (int64_t)h * G + gg) * kD;
+    qlo = *reinterpret_cast<const uint32_t*>(qp + 2 * mq);
+    qhi = *reinterpret_cast<const uint32_t*>(qp + 2 * mq + kHalf);
+  }
+  float kx0 = 0.f, kx1 = 0.f;
+  __nv_bfloat16 vx = __float2bfloat16_rn(0.f);
+  if (tid < kHalf) {
+    kx0 = __bfloat162float(k_new[uh * kD + tid]);
+    kx1 = __bfloat162float(k_new[uh * kD + tid + kHalf]);
+  } else if (tid < kHalf + kD) {
+    vx = v_new[uh * kD + tid - kHalf];
+  }
+  int M = mem_len[bl];
+  // Launched as a programmatic dependent of the previous step: past this point that step
+  // (its cache row, the length it advanced, its counters) is complete and visible; the
+  // next step may then be scheduled onto SMs as this one's CTAs leave.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int len = local_len[b];
   const bool full = len < 0 || len >= cap;  // (a negative length is treated as unusable too)
-  int M = mem_len[bl];
   if (M > M_max) {
     if (tid == 0 && split == 0 && h == 0 && !full) msa::set_err(dev_err, MSA_DEVERR_CAPACITY);
     M = M_max;
@@ -105,24 +128,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     __syncthreads();
     if (tid == 0) arrived = arrive_release(&query_count[b]);
   } else {
-    // loads that depend on nothing else start first: thread (head gg, m) takes dims 2m,
-    // 2m+1 and their rotate-half partners 2m+64, 2m+65
-    const int gg = tid >> 5, mq = tid & 31;
-    uint32_t qlo = 0u, qhi = 0u;
-    if (gg < G) {
-      const __nv_bfloat16* qp = q + (bl * Hq + (int64_t)h * G + gg) * kD;
-      qlo = *reinterpret_cast<const uint32_t*>(qp + 2 * mq);
-      qhi = *reinterpret_cast<const uint32_t*>(qp + 2 * mq + kHalf);
-    }
-    float kx0 = 0.f, kx1 = 0.f;
-    __nv_bfloat16 vx = __float2bfloat16_rn(0.f);
-    if (tid < kHalf) {
-      kx0 = __bfloat162float(k_new[uh * kD + tid]);
-      kx1 = __bfloat162float(k_new[uh * kD + tid + kHalf]);
-    } else if (tid < kHalf + kD) {
-      vx = v_new[uh * kD + tid - kHalf];
-    }
-
     // ---- this warp's tiles (memory tiles, then local tiles; the new key, row len, rides
     // in the last local tile): the first ones are requested before anything else
     const int nt_mem = (M + kTileKeys - 1) / kTileKeys;
@@ -458,14 +463,27 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   const dim3 grid(splits, n_kv_heads, n_queries * n_layers);
   const double log2_theta = log2((double)rope_theta);
   const float qscale = softmax_scale * kLog2e;
+  // programmatic stream serialisation: the kernel may be scheduled before the previous
+  // kernel on the stream finishes and waits for it (griddepcontrol.wait) before reading
+  // what a previous step wrote
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kRingBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
 #define MSA_DECODE_LAUNCH(GG)                                                                                    \
   MSA_CUDA_TRY(cudaFuncSetAttribute(decode_mma_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
                                     kRingBytes));                                                                 \
-  decode_mma_kernel<GG><<<grid, kThreads, kRingBytes, s>>>(                                                       \
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, n_layers, n_kv_heads,     \
-      (__nv_bfloat16*)local_k, (__nv_bfloat16*)local_v, local_len, local_cap, (const __nv_bfloat16*)mem_kv,        \
-      mem_len, max_mem_chunks, rope_pos_offset, log2_theta, qscale, splits, part, stat, unit_count, query_count,  \
-      (__nv_bfloat16*)out, dev_err)
+  MSA_CUDA_TRY(cudaLaunchKernelEx(                                                                                \
+      &cfg, decode_mma_kernel<GG>, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k_new,                          \
+      (const __nv_bfloat16*)v_new, n_layers, n_kv_heads, (__nv_bfloat16*)local_k, (__nv_bfloat16*)local_v,        \
+      local_len, local_cap, (const __nv_bfloat16*)mem_kv, mem_len, max_mem_chunks, rope_pos_offset, log2_theta,  \
+      qscale, splits, part, stat, unit_count, query_count, (__nv_bfloat16*)out, dev_err))
   switch (G) {
     case 1: MSA_DECODE_LAUNCH(1); break;
     case 2: MSA_DECODE_LAUNCH(2); break;
