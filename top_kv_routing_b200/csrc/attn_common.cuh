@@ -1,6 +1,5 @@
-// Device helpers shared by the decode and prefill attention kernels: cp.async staging,
-// ldmatrix, mma.sync m16n8k16 (bf16 in, fp32 accumulate) and the bf16 value/residual
-// split of fp32 operands.
+// Device helpers of the decode attention kernel: cp.async staging, ldmatrix, mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate) and the bf16 value/residual split of fp32 operands.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
