@@ -12,7 +12,12 @@
 // One unit = (layer l, key head g, 128 tokens): a GEMM tile M = 128 tokens x N = 128 G
 // features (the G heads of the group) over K = hidden_size, bf16 operands, fp32 in TMEM.
 // The whole group's heads are in one accumulator, so the epilogue can normalise each head
-// and sum the group before anything leaves the SM; P itself is never stored.
+// and sum the group before anything leaves the SM; P itself is never stored.  With more
+// than 128 tokens, units of 256 tokens run on pairs of SMs (a 2-CTA cluster, tcgen05
+// cta_group::2, M = 256): each CTA loads its 128 token rows and half of every MMA's weight
+// rows, both CTAs' copies complete on the leader's barrier, the leader issues the MMAs and
+// its commits reach both CTAs, and each CTA's epilogue handles its own 128 tokens.  No load
+// uses cluster multicast.
 // Warp roles (192 threads, persistent, one CTA per SM):
 //   warp 0      TMA producer: A = 128 tokens x 128 B of h, B = 128 G features x 128 B of
 //               W (boxes of at most 256 rows), 128-byte swizzle, into a ring of stages
@@ -41,26 +46,27 @@ constexpr int kBK = 64;
 constexpr int kABytes = kBM * kRowBytes;
 constexpr int kThreads = 192;
 
-template <int G>
+template <int G, bool PAIR>
 struct Cfg {
   static constexpr int kN = kD * G;                    // features per unit
   static constexpr int kMmaN = kN < 256 ? kN : 256;    // N of one MMA
   static constexpr int kMmas = kN / kMmaN;             // MMAs per K step
-  static constexpr int kBox = kMmaN;                   // rows per TMA box of W
-  static constexpr int kBBytes = kN * kRowBytes;
+  static constexpr int kRows = PAIR ? 2 * kBM : kBM;   // tokens per unit (M of the MMA)
+  static constexpr int kBox = PAIR ? kMmaN / 2 : kMmaN;  // W rows per TMA box held by this CTA
+  static constexpr int kBBytes = kMmas * kBox * kRowBytes;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kStages = (200 * 1024) / kStage > 4 ? 4 : (200 * 1024) / kStage;
   static constexpr int kTmemCols = kN;                 // 128, 256 or 512: one accumulator
   static constexpr int kSmem = kStages * kStage + 1024 + 256;
 };
 
-template <int G>
+template <int G, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, int T, int kblocks,
                 int L, int Hq, int H, int m_tiles, int n_rows, const __grid_constant__ Layout lay,
                 float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16, __nv_bfloat16* __restrict__ qt_lo,
                 uint8_t* __restrict__ qt_f8, int32_t* __restrict__ redo, int32_t* dev_err) {
-  using K = Cfg<G>;
+  using K = Cfg<G, PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::kStages * K::kStage);
@@ -74,6 +80,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int units = L * H * m_tiles;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int first_unit = PAIR ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
+  const int unit_stride = PAIR ? (int)(gridDim.x / 2) : (int)gridDim.x;
   if (redo != nullptr && blockIdx.x == 0)
     for (int i = threadIdx.x; i < L; i += blockDim.x) redo[i] = 0;
 
@@ -83,18 +93,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(accf), 1);
-    mbar_init(smem_u32(acce), 4);
+    mbar_init(smem_u32(acce), PAIR ? 8 : 4);
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
-    tmem_alloc<false>(smem_u32(tmem_slot), K::kTmemCols);
-    tmem_relinquish<false>();
+    tmem_alloc<PAIR>(smem_u32(tmem_slot), K::kTmemCols);
+    tmem_relinquish<PAIR>();
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync_all();  // both CTAs' barriers initialised before any remote use
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -110,9 +121,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = first_unit; u < units && ok; u += unit_stride) {
         const int mt = u % m_tiles, g = (u / m_tiles) % H, l = u / (m_tiles * H);
-        const int row_w = (l * Hq + g * G) * kD;
+        const int row_h = mt * K::kRows + (int)rank * kBM;
+        const int row_w = (l * Hq + g * G) * kD + (int)rank * K::kBox;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
             ok = false;
@@ -120,11 +132,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t fb = smem_u32(&full[stage]);
           const uint32_t sa = smem_u32(smem + stage * K::kStage);
-          mbar_arrive_expect_tx(fb, K::kStage);
-          tma_load_2d(sa, &tm_h, fb, kb * kBK, mt * kBM, pol_h);
+          if (PAIR) {
+            const uint32_t fb_lead = map_to_rank(fb, 0);  // both CTAs' bytes land on the leader's barrier
+            if (leader) mbar_arrive_expect_tx(fb, 2 * K::kStage);
+            tma_load_2d_pair(sa, &tm_h, fb_lead, kb * kBK, row_h, pol_h);
 #pragma unroll
-          for (int i = 0; i < K::kMmas; ++i)
-            tma_load_2d(sa + kABytes + i * K::kBox * kRowBytes, &tm_w, fb, kb * kBK, row_w + i * K::kBox, pol_w);
+            for (int i = 0; i < K::kMmas; ++i)
+              tma_load_2d_pair(sa + kABytes + i * K::kBox * kRowBytes, &tm_w, fb_lead, kb * kBK,
+                               row_w + i * K::kMmaN, pol_w);
+          } else {
+            mbar_arrive_expect_tx(fb, K::kStage);
+            tma_load_2d(sa, &tm_h, fb, kb * kBK, row_h, pol_h);
+#pragma unroll
+            for (int i = 0; i < K::kMmas; ++i)
+              tma_load_2d(sa + kABytes + i * K::kBox * kRowBytes, &tm_w, fb, kb * kBK, row_w + i * K::kMmaN, pol_w);
+          }
           armed[stage] = (int)phase;
           if (++stage == K::kStages) {
             stage = 0;
@@ -135,18 +157,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
-        for (int s = 0; s < K::kStages; ++s)
-          if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
+        // let the copies this CTA issued land (the leader's barriers see both CTAs' bytes)
+        if (leader)
+          for (int s = 0; s < K::kStages; ++s)
+            if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      constexpr uint32_t idesc = idesc_make(kBM, K::kMmaN, false);
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the leader of a pair issues for both CTAs)
+      constexpr uint32_t idesc = idesc_make(K::kRows, K::kMmaN, false);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = first_unit; u < units && ok; u += unit_stride) {
         if (!mbar_wait(smem_u32(acce), acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -164,25 +188,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < kRowBytes / 32; ++k)  // 16 bf16 of K per MMA
 #pragma unroll
             for (int i = 0; i < K::kMmas; ++i)
-              umma<false, false>(tmem_base + (uint32_t)(i * K::kMmaN), da + (uint64_t)(2 * k),
-                                 sw128_desc(sa + kABytes + i * K::kBox * kRowBytes) + (uint64_t)(2 * k), idesc,
-                                 (kb | k) != 0 ? 1u : 0u);
+              umma<PAIR, false>(tmem_base + (uint32_t)(i * K::kMmaN), da + (uint64_t)(2 * k),
+                                sw128_desc(sa + kABytes + i * K::kBox * kRowBytes) + (uint64_t)(2 * k), idesc,
+                                (kb | k) != 0 ? 1u : 0u);
           issued = true;
-          umma_commit<false>(smem_u32(&empty[stage]));
+          umma_commit<PAIR>(smem_u32(&empty[stage]));
           if (++stage == K::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit<false>(smem_u32(accf));
+        umma_commit<PAIR>(smem_u32(accf));
         acc_phase ^= 1u;
       }
       if (!ok) {
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
         if (issued) {
-          umma_commit<false>(smem_u32(drain));
+          umma_commit<PAIR>(smem_u32(drain));  // arrives once every MMA issued so far has finished
           mbar_drain(smem_u32(drain), 0u);
         }
       }
@@ -192,11 +216,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int hd = H * kD;
     const float inv_hq = 1.0f / (float)Hq;
+    const uint32_t acce_lead = PAIR ? map_to_rank(smem_u32(acce), 0) : smem_u32(acce);
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = first_unit; u < units && ok; u += unit_stride) {
       const int mt = u % m_tiles, g = (u / m_tiles) % H, l = u / (m_tiles * H);
-      const int t = mt * kBM + quarter * 32 + lane;
+      const int t = mt * K::kRows + (int)rank * kBM + quarter * 32 + lane;
       int orow = -1;
       if (t < T) {
         int lo = 0, hi = lay.n_queries;  // largest b with off[b] <= t
@@ -289,7 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(acce));
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(acce_lead);
+        else mbar_arrive(acce_lead);
+      }
       acc_phase ^= 1u;
     }
     if (!ok && lane == 0) {
@@ -299,10 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync_all();  // no CTA exits while its peer may still signal its barriers
+  else __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc<false>(tmem_base, K::kTmemCols);
+    tmem_dealloc<PAIR>(tmem_base, K::kTmemCols);
   }
 }
 
@@ -336,26 +365,39 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G>
+template <int G, bool PAIR>
 int launch_g(const Args& a, cudaStream_t s, const char** why) {
-  using K = Cfg<G>;
+  using K = Cfg<G, PAIR>;
   CUtensorMap mh, mw;
   if (!make_map(&mh, a.hidden, (uint64_t)a.T, (uint64_t)a.hidden_size, kBM) ||
       !make_map(&mw, a.w, (uint64_t)a.L * a.Hq * kD, (uint64_t)a.hidden_size, K::kBox)) {
     *why = "cuTensorMapEncodeTiled failed";
     return 1;
   }
-  const int m_tiles = (a.T + kBM - 1) / kBM;
+  const int m_tiles = (a.T + K::kRows - 1) / K::kRows;
   const long long units = (long long)a.L * a.H * m_tiles;
-  int grid = msa::sm_count();
-  if (units < grid) grid = (int)units;
-  if (cudaFuncSetAttribute(proj_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) != cudaSuccess) {
+  const int per_unit = PAIR ? 2 : 1;
+  int grid = msa::sm_count() / per_unit * per_unit;
+  if (units * per_unit < grid) grid = (int)(units * per_unit);
+  if (cudaFuncSetAttribute(proj_kernel<G, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem) !=
+      cudaSuccess) {
     *why = "cudaFuncSetAttribute (shared memory)";
     return 1;
   }
-  proj_kernel<G><<<grid, kThreads, K::kSmem, s>>>(mh, mw, a.T, a.hidden_size / kBK, a.L, a.Hq, a.H, m_tiles, a.n_rows,
-                                                   a.lay, a.qt_f32, a.qt_bf16, a.qt_lo, a.qt_f8, a.redo, a.dev_err);
-  if (cudaGetLastError() != cudaSuccess) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = K::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = per_unit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, proj_kernel<G, PAIR>, mh, mw, a.T, a.hidden_size / kBK, a.L, a.Hq, a.H, m_tiles,
+                         a.n_rows, a.lay, a.qt_f32, a.qt_bf16, a.qt_lo, a.qt_f8, a.redo, a.dev_err) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
   }
@@ -379,10 +421,13 @@ int launch(const Args& a, cudaStream_t s, const char** why) {
     *why = "sizes beyond 32-bit TMA coordinates";
     return 1;
   }
+  // paired M = 256 tiles (two SMs per tile, each streaming half of the weight rows) once
+  // the tokens fill more than one 128-row tile
+  const bool pair = a.T > kBM;
   switch (a.Hq / a.H) {
-    case 1: return launch_g<1>(a, s, why);
-    case 2: return launch_g<2>(a, s, why);
-    default: return launch_g<4>(a, s, why);
+    case 1: return pair ? launch_g<1, true>(a, s, why) : launch_g<1, false>(a, s, why);
+    case 2: return pair ? launch_g<2, true>(a, s, why) : launch_g<2, false>(a, s, why);
+    default: return pair ? launch_g<4, true>(a, s, why) : launch_g<4, false>(a, s, why);
   }
 }
 
