@@ -50,6 +50,17 @@ def test_common_header_constants_match_binding(msa):
         assert getattr(msa, name) == int(re.search(rf"#define {name} (\d+)", text).group(1))
 
 
+def test_bank_header_constants_match_binding(msa):
+    text = open(os.path.join(ROOT, "include", "msa_bank.h")).read()
+    for name in ("MSA_BANK_KR", "MSA_BANK_KR_F8", "MSA_BANK_KV", "MSA_BANK_NORM"):
+        assert getattr(msa, name) == int(re.search(rf"#define {name} (\d+)u", text).group(1))
+    text = open(os.path.join(ROOT, "include", "msa_common.h")).read()
+    assert msa.MSA_ERR_IO == int(re.search(r"MSA_ERR_IO = (\d+)", text).group(1))
+    # the info struct as the header lays it out (4 int32, 2 int64, 1 uint32)
+    import ctypes
+    assert ctypes.sizeof(msa.MsaBankInfo) == 4 * 4 + 2 * 8 + 8
+
+
 def test_count_chunks_host(msa):
     n, offs = msa.msa_count_chunks(np.array([0, 64, 65, 65, 200]), 64)
     assert n == 1 + 1 + 0 + 3 and offs.tolist() == [0, 1, 2, 2, 5]

@@ -86,7 +86,7 @@ uint64_t align_up(uint64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool is_device(const void* p) {
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-    cudaGetLastError();  // clear the sticky-free error of a host pointer / no device
+    cudaGetLastError();  // (no device, or a pointer the runtime does not know: clear the error)
     return false;
   }
   return a.type == cudaMemoryTypeDevice;
