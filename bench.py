@@ -402,6 +402,65 @@ def time_projection(dev, bank, kr_hat, kr_f8):
             "route_hidden_ms_p50": round(sorted(whole)[len(whole) // 2], 3), "dev_err": int(err.item())}
 
 
+def time_tail_parts(eng, slot, dq, dk, dv, dev):
+    """Gather and decode timed apart on the slot's current selection (direct calls, CUDA
+    events, after the timed regions): the gather's GB/s against one large pinned
+    host-to-device copy (the PCIe ceiling), and decode microseconds per step with the key and
+    value bytes each step reads."""
+    import torch
+
+    import top_kv_routing_b200 as msa
+    L, H, D = eng.L, eng.H, eng.D
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    n = 256 << 20
+    src = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(n, dtype=torch.uint8, device=dev)
+    dst.copy_(src, non_blocking=True)
+    a, b = ev(), ev()
+    a.record()
+    dst.copy_(src, non_blocking=True)
+    b.record()
+    torch.cuda.synchronize(dev)
+    pcie = n / (a.elapsed_time(b) / 1e3) / 1e9
+    del src, dst
+    gms = []
+    for r in range(4):
+        a, b = ev(), ev()
+        torch.cuda._sleep(2_000_000)  # the GPU is busy while the host prepares the call
+        a.record()
+        msa.msa_gather_kv(eng.host_kv, eng.n_store, eng.doc_chunk_offsets, eng.doc_store_offsets, eng.n_docs,
+                          slot.ids, 1, L, eng.k, H, D, eng.M, slot.mem_kv, slot.mem_len, dev_err=slot.dev_err)
+        b.record()
+        torch.cuda.synchronize(dev)
+        if r:
+            gms.append(a.elapsed_time(b))
+    g_ms = sorted(gms)[len(gms) // 2]
+    mem_blocks = int(slot.mem_len.sum().item())
+    g_bytes = mem_blocks * 2 * H * D * 2
+    slot.local_len.copy_(slot.local_len0)
+    len0 = int(slot.local_len0.item())
+    steps = min(32, dq.shape[0], eng.cap - len0)
+    out = torch.empty((1, L, eng.Hq, D), dtype=torch.bfloat16, device=dev)
+    a, b = ev(), ev()
+    torch.cuda._sleep(20_000_000)  # all the steps are enqueued before the GPU reaches the start event
+    a.record()
+    for st in range(steps):
+        msa.msa_sparse_decode(dq[st], dk[st], dv[st], 1, L, eng.Hq, H, D, slot.local_k, slot.local_v, slot.local_len,
+                              eng.cap, slot.mem_kv, slot.mem_len, eng.M, eng.k, eng.theta, D ** -0.5, out, slot.dec_ws,
+                              dev_err=slot.dev_err)
+    b.record()
+    torch.cuda.synchronize(dev)
+    us = a.elapsed_time(b) * 1e3 / steps
+    # per step: every memory row and every local row (the new one included), K and V, bf16
+    d_bytes = (mem_blocks * H + L * H * (len0 + (steps + 1) / 2)) * 2 * D * 2
+    return {"gather": {"ms": round(g_ms, 4), "bytes": g_bytes, "gbs": round(g_bytes / g_ms / 1e6, 1),
+                       "pcie_h2d_gbs": round(pcie, 1), "frac_of_pcie_copy": round(g_bytes / g_ms / 1e6 / pcie, 4)},
+            "decode": {"us_per_step": round(us, 2), "steps": steps, "bytes_per_step": int(d_bytes),
+                       "gbs": round(d_bytes / (us / 1e6) / 1e9, 1),
+                       "note": "direct launches queued behind a GPU sleep, so back to back as in the graph; K/V "
+                               "are L2-resident after the first step"}}
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args):
@@ -594,6 +653,12 @@ def run_gpu(args):
     d2h = host["ids"][0].numel() * 4 + host["scores"][0].numel() * 4 + host["out"][0].numel() * 2
     # routing from hidden states (fused router projection), after the timed regions
     projection = time_projection(dev, bank, kr_hat, kr_f8) if (rank == 0 and not args.no_projection) else None
+    tail_parts = None
+    if rank == 0:
+        try:
+            tail_parts = time_tail_parts(eng, slot0, dq, dk, dv, dev)
+        except Exception as e:  # (a separate measurement: never at the cost of the line)
+            tail_parts = {"error": f"{type(e).__name__}: {e}"}
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
     if world > 1:
@@ -645,6 +710,7 @@ def run_gpu(args):
                                 "query i+1" if n_slots > 1 else "one query at a time"),
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "scan_gbs": round(achieved, 1),
+        "scan_frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
         "p50_route_decode_ms": round(p[len(p) // 2], 4),
         "p99_route_decode_ms": round(p[min(len(p) - 1, int(0.99 * len(p)))], 4),
         "p50_isolated_ms": round(iso_s[len(iso_s) // 2], 4),
@@ -672,6 +738,7 @@ def run_gpu(args):
         "pool": pool,
         "prefill": prefill,
         "router_projection": projection,
+        "tail_parts": tail_parts,
         "planted_recall": round(float(hits), 4),
         "dev_err": dev_err,
         "filter_keys_ms": None if f8_ms is None else round(f8_ms, 2),
