@@ -202,8 +202,9 @@ def prefill(q, k_new, v_new, mem_kv, mem_len: int, local_k, local_v, local_len: 
 
 
 def router_project(h, w, n_q_heads: int):
-    """Router query projection of one layer: h [T][hidden] times w [n_q_heads * d][hidden]
-    transposed.  Returns Q_r [T][n_q_heads][d] (double)."""
+    """Router query projection of one layer ("【MSA】突破100M Token 上下文：记忆稀疏注意力架构深度解析",
+    section 5.1: the decoupled, bias-free router_q_proj): h [T][hidden] times
+    w [n_q_heads * d][hidden] transposed.  Returns Q_r [T][n_q_heads][d] (double)."""
     h, w = _f32(h), _f32(w)
     T, hidden = h.shape
     F, hidden2 = w.shape
@@ -217,7 +218,13 @@ def layer_mean_topk(doc_scores, k: int):
     """Layer-aggregated selection: one top-k shared by every routing layer, ranking the
     documents by the mean over layers of their per-layer document scores (a document with
     no block scores -inf in every layer and so in the mean).  doc_scores [L][n_docs].
-    Returns (ids [k], scores [k], mean [n_docs])."""
+    Returns (ids [k], scores [k], mean [n_docs]).
+
+    The pages give the per-layer document score ("MSA端到端可训练记忆模型完整开源，支持亿级Token
+    上下文", section 架构: mean over heads, max over tokens) and one top-16 selection per query
+    (MSA paper reading notes, section 路由投影器 + Top-k 稀疏注意力); where one selection is to
+    serve all routing layers, this takes the plain reading that the layers' document scores
+    are averaged, and ranks as the per-layer top-k does (score descending, then id)."""
     ds = np.asarray(doc_scores, dtype=np.float64)
     L = ds.shape[0]
     mean = np.empty(ds.shape[1], dtype=np.float64)
@@ -230,6 +237,8 @@ def layer_mean_topk(doc_scores, k: int):
 
 def route_layer_mean(q_layers, kr_layers, doc_chunk_offsets, top_k: int):
     """Routing of one query with the layer-aggregated selection: q_layers [L][T][Hq][d],
-    kr_layers [L][C][H][d].  Returns (ids [k], scores [k], mean doc scores [n_docs])."""
+    kr_layers [L][C][H][d].  Each layer's document scores are the grouped routing form
+    (route(..., grouped=True)), then layer_mean_topk.  Returns (ids [k], scores [k], mean
+    doc scores [n_docs])."""
     per_layer = [route(q, kr, doc_chunk_offsets, top_k, grouped=True)[2] for q, kr in zip(q_layers, kr_layers)]
     return layer_mean_topk(np.stack(per_layer), top_k)

@@ -10,7 +10,7 @@
 //  [NOTES]   "MSA paper reading notes" (xiaohongrsx.github.io), sections 路由投影器 + Top-k 稀疏注意力,
 //            文档级 RoPE, KV 缓存压缩 + Memory Parallel, 推理全流程
 //  [DEEP]    "【MSA】突破100M Token 上下文：记忆稀疏注意力架构深度解析", sections 3.3.1, 3.3.2,
-//            5.2 (forward), 5.3 (map_tensor_to_group_ids)
+//            5.1 (router projectors), 5.2 (forward), 5.3 (map_tensor_to_group_ids)
 //
 // Readings where the pages are silent or garbled are listed beside each function.
 #include <math.h>
