@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_prefill.argtypes = [_p, _p, _p, _i32, _p, _i32, _i32, _p, _p, _i32, _i32, _i64, _dbl, _dbl,
                                         _i32, _i32, _i32, _p]
         _lib.oracle_prefill.restype = _i32
+        _lib.oracle_query_sums.argtypes = [_p, _i32, _i32, _i32, _i32, _p]
+        _lib.oracle_query_sums.restype = _i32
         _lib.oracle_router_project.argtypes = [_p, _i32, _i32, _p, _i32, _p]
         _lib.oracle_router_project.restype = None
     return _lib
@@ -137,6 +139,17 @@ def route(qr, kr, doc_chunk_offsets, top_k: int, grouped: bool = False):
     if r != 0:
         raise ValueError("oracle route: bad head counts")
     return ids, sc, doc_score, chunk_score
+
+
+def query_sums(qr, n_kv_heads: int):
+    """The grouped routing form's query operand: qr [T][Hq][d] -> qt [T][H][d] (double),
+    qt[t][g] = (1/Hq) sum of the unit query heads h with h / (Hq/H) == g."""
+    qr = _f32(qr)
+    T, Hq, d = qr.shape
+    out = np.empty((T, n_kv_heads, d), dtype=np.float64)
+    if lib().oracle_query_sums(_ptr(qr), T, Hq, n_kv_heads, d, _ptr(out)) != 0:
+        raise ValueError("oracle query_sums: bad head counts")
+    return out
 
 
 def gather(host_kv_bits, doc_chunk_offsets, ids, max_mem_chunks: int):

@@ -208,6 +208,29 @@ int32_t oracle_route_explicit(const float* qr, int32_t T, int32_t Hq, const floa
   return 0;
 }
 
+// The per-key-head query operand of the grouped form below, on its own:
+//   qt[t][g] = (1/Hq) sum over the G query heads h with h / G == g of
+//              Q_r[t][h] / max(||Q_r[t][h]||, 1e-8)
+// so that s[t][c] = sum_g <qt[t][g], Kbar_r[c][g]> / max(||Kbar_r[c][g]||, 1e-8).  The head
+// pairing h -> h / G is [DEEP] 5.1 (router_q: Hq heads, router_k: H heads, GQA).
+int32_t oracle_query_sums(const float* qr, int32_t T, int32_t Hq, int32_t H, int32_t d, double* qt) {
+  if (H <= 0 || Hq % H != 0) return -1;
+  const int32_t G = Hq / H;
+  for (size_t i = 0; i < (size_t)T * H * d; ++i) qt[i] = 0.0;
+  for (int32_t t = 0; t < T; ++t)
+    for (int32_t h = 0; h < Hq; ++h) {
+      double n = 0.0;
+      for (int32_t j = 0; j < d; ++j) {
+        const double x = qr[((size_t)t * Hq + h) * d + j];
+        n += x * x;
+      }
+      const double inv = 1.0 / std::max(sqrt(n), 1e-8);
+      for (int32_t j = 0; j < d; ++j)
+        qt[((size_t)t * H + h / G) * d + j] += qr[((size_t)t * Hq + h) * d + j] * inv / (double)Hq;
+    }
+  return 0;
+}
+
 // Step 2, grouped form of the same score, written separately (4x fewer products):
 //   qhat[t][h] = Q_r[t][h] / max(||Q_r[t][h]||, 1e-8)
 //   qsum[t][g] = sum over the G query heads h with h / G == g of qhat[t][h]

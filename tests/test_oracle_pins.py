@@ -241,6 +241,35 @@ def test_route_explicit_equals_grouped():
     assert list(a[0]) == list(b[0])
 
 
+def test_query_sums_hand_worked():
+    # 4 query heads, 2 key heads (G = 2): head 0 = (3, 4) -> (0.6, 0.8); head 1 = 2 e0 -> e0;
+    # head 2 = -5 e1 -> -e1; head 3 = e3; a zero head 4 of a second token stays zero
+    q = np.zeros((2, 4, 4), dtype=np.float32)
+    q[0, 0, :2] = [3, 4]
+    q[0, 1, 0] = 2
+    q[0, 2, 1] = -5
+    q[0, 3, 3] = 1
+    q[1, 0, 2] = 7
+    qt = oracle.query_sums(q, 2)
+    np.testing.assert_allclose(qt[0, 0], [1.6 / 4, 0.8 / 4, 0, 0], atol=1e-15)
+    np.testing.assert_allclose(qt[0, 1], [0, -0.25, 0, 0.25], atol=1e-15)
+    np.testing.assert_allclose(qt[1, 0], [0, 0, 0.25, 0], atol=1e-15)
+    np.testing.assert_allclose(qt[1, 1], 0, atol=0)
+
+
+def test_query_sums_give_the_explicit_routing_scores():
+    # sum_g <qt_g, k_g> / ||k_g|| is the explicit mean of the 32 cosines
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal((3, 32, 128)).astype(np.float32)
+    kr = rng.standard_normal((10, 8, 128)).astype(np.float32)
+    _, _, _, blk = oracle.route(q, kr, np.array([0, 10]), 1)
+    qt = oracle.query_sums(q, 8)
+    k = kr.astype(np.float64)
+    k /= np.linalg.norm(k, axis=2, keepdims=True)
+    s = np.einsum("tgd,cgd->tc", qt, k)
+    np.testing.assert_allclose(s.max(axis=0), blk, atol=1e-12)
+
+
 def test_topk_matches_python_sorted_with_ties():
     s = np.array([0.5, 0.9, 0.5, -1.0, 0.9, 0.1, -np.inf])
     ids, sc = oracle.topk(s, 5)
