@@ -56,8 +56,10 @@ typedef struct CUstream_st* msa_stream_t;
 #define MSA_DEVERR_LOCAL_FULL 4u  /* local cache has no room for the new token (skipped) */
 #define MSA_DEVERR_BAD_OFFSETS 8u /* offsets disagree with the declared counts           */
 #define MSA_DEVERR_TIMEOUT 16u    /* a bounded in-kernel wait ran out (work abandoned)    */
-#define MSA_DEVERR_UNCERTIFIED 32u /* tensor-core routing: the exactly rescored candidates do
-                                      not provably contain the exact top-k (see msa_route.h) */
+#define MSA_DEVERR_UNCERTIFIED 32u /* tensor-core routing: a selection whose certification
+                                      failed with no further stage to send it to (kept in
+                                      the ABI; the routing's last stage is an exact scan,
+                                      so msa_route_topk does not raise it) */
 
 /* Bytes of one memory block of one layer in a bf16 bank:
  * routing key H*d*2; content key + value 2*H*d*2. */

@@ -44,10 +44,16 @@ extern "C" {
  * path (AUTO picks it at any query length; with MSA_ROUTE_SCAN it is MSA_ERR_INVALID_ARG;
  * needs n_kv_heads = 8): the mean filter scores choose the candidates, every layer rescores
  * them exactly, and the final top-k is certified on the mean exact scores against the
- * best mean filter score left out (the same bounds as per layer: a mean of errors is
- * within the largest).  On the E4M3 path an uncertified query sends every layer to the
- * bf16 second pass. */
+ * best mean filter score left out by the mean of the layers' bounds (plus the fp32
+ * rounding of the means).  An uncertified query sends every layer through the same
+ * further stages as the per-layer selection (bf16 filter, widened rescoring, exact scan
+ * of every layer). */
 #define MSA_ROUTE_LAYER_MEAN 16
+/* OR-ed with MSA_ROUTE_TENSOR or MSA_ROUTE_TENSOR_F8 (not with the layer-aggregated
+ * variant): returns the top_k documents by the tensor-core FILTER score and those filter
+ * scores, without the exact rescoring.  The MSA pages have no counterpart; it exposes the
+ * filter whose error the certification bounds, so that the bound can be checked. */
+#define MSA_ROUTE_FILTER_SCORES 32
 
 /* Workspace bytes for one msa_route_topk call with these sizes. */
 msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, int32_t total_q_tokens,
@@ -83,15 +89,24 @@ msa_status msa_route_filter_keys(const void* kr_hat, int32_t n_layers, int64_t n
  *   1 <= top_k <= 64; 1 <= n_queries <= 256; n_kv_heads in {2, 4, 8, 16}; n_q_heads <= 64.
  *   out_ids, out_scores DEVICE [n_queries][n_layers][top_k] int32 / fp32.
  *   workspace        DEVICE, >= msa_route_topk_workspace_size bytes, 256-byte aligned.
- *   flags            MSA_ROUTE_AUTO / _SCAN / _TENSOR / _TENSOR_F8.
+ *   flags            MSA_ROUTE_AUTO / _SCAN / _TENSOR / _TENSOR_F8, optionally OR-ed with
+ *                    MSA_ROUTE_LAYER_MEAN or MSA_ROUTE_FILTER_SCORES.
  * The tensor paths score with low-precision operands as a filter, rescore the best
- * candidates exactly in fp32 and take the top_k from the exact scores.  A selection is
- * certified when its k-th exact score beats the best filter score left out by more than
- * the filter's error bound (1e-3 for bf16 operands, 2^-6 for E4M3).  On the E4M3 path,
- * layers that fail are filtered again with bf16 operands and rescored within the same
- * call (its kernels return at once when every layer is certified); a layer that fails
- * the bf16 bound sets MSA_DEVERR_UNCERTIFIED in dev_err, its ids being the best of the
- * rescored candidates (MSA_ROUTE_SCAN is exact).
+ * candidates (K2 = max(2 top_k, top_k + 32), at most 128) exactly and take the top_k
+ * from the exact scores.  A selection is certified when its k-th exact score beats the
+ * best filter score left out by more than a bound on |filter - exact| derived from the
+ * operands' rounding (Cauchy-Schwarz over each key head, computed per query token from the
+ * query's own operand rows and rounding residuals; the key side enters through its
+ * format: E4M3 keys at most 2^-4 relative per element, bf16 keys the nearest rounding of
+ * unit vectors).  That bound holds under two preconditions: kr_hat heads are the bf16
+ * rounding of unit vectors (or zero), as msa_pool_blocks writes them, and the tensor
+ * cores accumulate in fp32 (each addition rounded to nearest or toward zero).
+ * Layers that are not certified go, within the same call, through further stages, each
+ * of whose kernels return at once when no layer is marked for it: E4M3 filter -> bf16
+ * filter -> the 1024 best documents by bf16 filter score rescored exactly -> an exact
+ * scan of the layer.  The result is therefore always the exact top_k (up to the fp32
+ * rounding of the exact scores, about 1e-6); MSA_DEVERR_UNCERTIFIED is not raised.
+ * MSA_ROUTE_SCAN is exact from the start.
  * Asynchronous on stream; no host synchronisation. */
 msa_status msa_route_topk(const void* qr, msa_dtype q_dtype, const int32_t* q_offsets_host,
                           int32_t n_queries, const void* kr_hat, const void* kr_f8, const int64_t* doc_chunk_offsets,

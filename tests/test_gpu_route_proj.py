@@ -104,9 +104,11 @@ def test_projected_routing_short_query_takes_the_scan(msa):
 
 def test_projected_routing_launches_like_the_unfused_call(msa):
     # the projection replaces the query-preparation kernel one for one
-    # (E4M3 path: prep, projection, GEMM, top-k, rescore, final, and the five second-pass
-    # kernels that return at once when every layer is certified)
-    assert _case(msa, 6, [64], 128, 32, 3) == 11
+    # (E4M3 path: prep, projection, GEMM, top-k, rescore, final, the five bf16-pass kernels
+    # and the three of the widened rescoring, which return at once when every layer is
+    # certified; the bank has more documents than the first candidates and fewer than the
+    # widened ones, so no exact scan is enqueued)
+    assert _case(msa, 6, [64], 128, 32, 3) == 14
 
 
 def test_projected_routing_bench_shape_sampled_layers(msa):

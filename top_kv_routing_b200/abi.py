@@ -1,4 +1,4 @@
-"""Thin ctypes binding over the four C-ABI libraries in ``lib/`` (see ``include/*.h``).
+"""Thin ctypes binding over the six C-ABI libraries in ``lib/`` (see ``include/*.h``).
 
 Argument marshalling only; every step runs in the libraries' CUDA kernels.  PyTorch is
 used by callers for device memory and streams.  There is no CPU fallback: importing this
@@ -18,6 +18,7 @@ MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_CAPACITY
 MSA_F32, MSA_BF16 = 0, 1
 MSA_ROUTE_AUTO, MSA_ROUTE_SCAN, MSA_ROUTE_TENSOR, MSA_ROUTE_TENSOR_F8 = 0, 1, 2, 3
 MSA_ROUTE_LAYER_MEAN = 16  # OR-ed with a path: one selection for all layers
+MSA_ROUTE_FILTER_SCORES = 32  # OR-ed with a tensor path: the filter's own top-k and scores
 (MSA_DEVERR_CAPACITY, MSA_DEVERR_BAD_DOC, MSA_DEVERR_LOCAL_FULL, MSA_DEVERR_BAD_OFFSETS, MSA_DEVERR_TIMEOUT,
  MSA_DEVERR_UNCERTIFIED) = 1, 2, 4, 8, 16, 32
 

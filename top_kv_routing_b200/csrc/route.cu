@@ -27,11 +27,13 @@
 #include "common.cuh"
 #include "msa_route.h"
 #include "route_proj.cuh"
+#include "route_bound.cuh"
 #include "route_tc.cuh"
 
 MSA_DEFINE_LAST_ERROR(msa_route_last_error)
 
 namespace {
+using namespace route_bound;
 
 constexpr int kD = 128;
 constexpr int kMaxQueries = 256;
@@ -40,14 +42,7 @@ constexpr int kMaxCandidates = 128;  // documents rescored exactly after the ten
 constexpr int kTopkThreads = 512;
 constexpr int kMaxDocs = 1 << 20;    // documents per bank
 constexpr int kMaxBlocks = 64;       // docmax CTAs per (query, layer)
-// Error bound assumed for the tensor-core filter scores (bf16 operands, fp32 accumulate):
-// the observed error is ~1e-4 (3e-4 worst seen), this is ~10 standard deviations.  A
-// selection is certified when the k-th exact score beats the best filter score left out
-// by more than it.
-constexpr float kFilterErr = 1e-3f;
-// The same for the E4M3 filter (3 mantissa bits on both operands): rms error ~8e-4,
-// largest seen ~5e-3 over 8M (block, token) pairs of bank-like data; 2^-6 is ~19 rms.
-constexpr float kFilterErrF8 = 0.015625f;
+constexpr int kMaxWide = 1024;       // candidates of the widened rescoring
 
 // Candidates rescored exactly on the tensor-core path.
 int rescore_count(int32_t n_docs, int32_t k) {
@@ -55,6 +50,9 @@ int rescore_count(int32_t n_docs, int32_t k) {
   if (k2 > kMaxCandidates) k2 = kMaxCandidates;
   return n_docs < k2 ? n_docs : k2;
 }
+// Candidates of the widened rescoring (layers whose selection the bf16 filter could not
+// certify).
+int wide_count(int32_t n_docs) { return n_docs < kMaxWide ? n_docs : kMaxWide; }
 
 static thread_local int32_t g_launches = 0;
 static thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
@@ -84,10 +82,11 @@ int pow2_at_least(int n) {
 
 struct WsLayout {
   size_t qt_f32, qt_bf16, qt_lo, qt_f8, m, cand, apx, exact, redo, doc_score, block_doc, agg, apx_agg, exact_agg,
-      total;
+      etok, apx_w, exact_w, apx_agg_w, exact_agg_w, total;
   int n_pad;
   int nblk;
   int k2;
+  int kw;
 };
 
 // Upper bound of the padded operand rows for B queries of T_total tokens in all.
@@ -101,7 +100,9 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   w.n_pad = operand_rows_bound(T_total, B);
   w.nblk = topk_blocks(n_docs);
   w.k2 = rescore_count(n_docs, k);
+  w.kw = wide_count(n_docs);
   const int ksel = w.k2 > k ? w.k2 : k;
+  const size_t k2s = (size_t)(ksel > 0 ? ksel : 1), kws = (size_t)(w.kw > 0 ? w.kw : 1);
   size_t o = 0;
   w.qt_f32 = o;
   o += align256((size_t)L * T_total * H * kD * sizeof(float));
@@ -116,11 +117,11 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   w.cand = o;
   o += align256((size_t)B * L * w.nblk * ksel * sizeof(unsigned long long));
   w.apx = o;
-  o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(unsigned long long));
+  o += align256((size_t)B * L * k2s * sizeof(unsigned long long));
   w.exact = o;
-  o += align256((size_t)B * L * (w.k2 > 0 ? w.k2 : 1) * sizeof(float));
-  w.redo = o;
-  o += align256((size_t)L * sizeof(int32_t));
+  o += align256((size_t)B * L * k2s * sizeof(float));
+  w.redo = o;  // three layer masks: E4M3 pass failed, bf16 pass failed, widened pass failed
+  o += align256((size_t)3 * L * sizeof(int32_t));
   w.doc_score = o;
   o += align256((size_t)B * L * (size_t)(n_docs > 0 ? n_docs : 1) * sizeof(uint32_t));
   w.block_doc = o;
@@ -129,9 +130,21 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
   w.agg = o;
   o += align256((size_t)B * (size_t)(n_docs > 0 ? n_docs : 1) * sizeof(uint32_t));
   w.apx_agg = o;
-  o += align256((size_t)B * (w.k2 > 0 ? w.k2 : 1) * sizeof(unsigned long long));
+  o += align256((size_t)B * k2s * sizeof(unsigned long long));
   w.exact_agg = o;
-  o += align256((size_t)B * (w.k2 > 0 ? w.k2 : 1) * sizeof(uint32_t));
+  o += align256((size_t)B * k2s * sizeof(uint32_t));
+  // per (bound kind, layer, token) filter error bounds
+  w.etok = o;
+  o += align256((size_t)2 * L * T_total * sizeof(float));
+  // the widened rescoring's candidates
+  w.apx_w = o;
+  o += align256((size_t)B * L * kws * sizeof(unsigned long long));
+  w.exact_w = o;
+  o += align256((size_t)B * L * kws * sizeof(uint32_t));
+  w.apx_agg_w = o;
+  o += align256((size_t)B * kws * sizeof(unsigned long long));
+  w.exact_agg_w = o;
+  o += align256((size_t)B * kws * sizeof(uint32_t));
   w.total = o;
   return w;
 }
@@ -139,15 +152,20 @@ WsLayout ws_layout(int32_t L, int32_t B, int32_t T_total, int32_t H, int64_t C, 
 // ---------------------------------------------------------------------------- 1. q prep
 // grid (T_total, L); block 128 threads.  Hq <= 64.  The bf16 copy of token t of query b
 // goes to operand row row0[b] + (t - off[b]) of layer l (n_rows rows per layer).
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr, int q_is_bf16, int T_total,
                                                     int Hq, int H, int n_rows, QueryOffsets qo,
                                                     float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16,
                                                     __nv_bfloat16* __restrict__ qt_lo, uint8_t* __restrict__ qt_f8,
-                                                    int32_t* __restrict__ redo, int n_layers) {
+                                                    float* __restrict__ etok, int n_layers) {
   __shared__ float qhat[64][kD];
+  __shared__ float red[16][4][6];  // per key head, per warp: the six sums of the bounds
   const int t = blockIdx.x, l = blockIdx.y;
-  if (redo != nullptr && t == 0 && l == 0)
-    for (int i = threadIdx.x; i < n_layers; i += blockDim.x) redo[i] = 0;
   int qb = 0;
   {
     int lo = 0, hi = qo.n;  // largest b with off[b] <= t
@@ -182,6 +200,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
   __syncthreads();
   const int G = Hq / H;
   const float inv_hq = 1.0f / (float)Hq;
+  // (every thread runs the same number of iterations: H * 128 is a multiple of 128)
   for (int e = threadIdx.x; e < H * kD; e += blockDim.x) {
     const int g = e / kD, j = e % kD;
     float acc = 0.f;
@@ -189,12 +208,42 @@ __global__ void __launch_bounds__(128) qprep_kernel(const void* __restrict__ qr,
     acc *= inv_hq;
     if (qt_f32 != nullptr) qt_f32[((int64_t)l * T_total + t) * H * kD + e] = acc;
     const int64_t oi = ((int64_t)l * n_rows + orow) * H * kD + e;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
     if (qt_bf16 != nullptr) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
       qt_bf16[oi] = hi;
       if (qt_lo != nullptr) qt_lo[oi] = __float2bfloat16_rn(acc - __bfloat162float(hi));
     }
     if (qt_f8 != nullptr) qt_f8[oi] = __nv_cvt_float_to_fp8(acc * route_tc::kF8QueryScale, __NV_SATFINITE, __NV_E4M3);
+    if (etok != nullptr && g < 16) {
+      const float hf = __bfloat162float(hi), db = hf - acc;
+      const float a = acc * route_tc::kF8QueryScale, ah = e4m3_round(a), da = (ah - a) * (1.0f / route_tc::kF8QueryScale);
+      const float as = ah * (1.0f / route_tc::kF8QueryScale);
+      float v[6] = {acc * acc, db * db, hf * hf, as * as, da * da, fabsf(as)};
+#pragma unroll
+      for (int i = 0; i < 6; ++i) v[i] = warp_sum(v[i]);
+      if ((threadIdx.x & 31) == 0)
+#pragma unroll
+        for (int i = 0; i < 6; ++i) red[g][threadIdx.x >> 5][i] = v[i];
+    }
+  }
+  if (etok == nullptr) return;
+  __syncthreads();
+  // thread g < H: the bounds of key head g; then their sums over the heads
+  float2 eb = make_float2(0.f, 0.f);
+  if (threadIdx.x < H && threadIdx.x < 16) {
+    float v[6];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) v[i] = red[threadIdx.x][0][i] + red[threadIdx.x][1][i] + red[threadIdx.x][2][i] +
+                                     red[threadIdx.x][3][i];
+    eb = head_bounds(sqrtf(v[0]), sqrtf(v[1]), sqrtf(v[2]), sqrtf(v[3]), sqrtf(v[4]), v[5]);
+  }
+  if (threadIdx.x < 32) {
+    eb.x = warp_sum(eb.x);
+    eb.y = warp_sum(eb.y);
+    if (threadIdx.x == 0) {
+      etok[((int64_t)kBoundF8 * n_layers + l) * T_total + t] = eb.x * kBoundSlack + kBoundFloor;
+      etok[((int64_t)kBoundBf16 * n_layers + l) * T_total + t] = eb.y * kBoundSlack + kBoundFloor;
+    }
   }
 }
 
@@ -214,7 +263,8 @@ struct PadTargets {
 __global__ void route_prep_kernel(PadTargets pt, int n_rows, int L, QueryOffsets qo,
                                   const int64_t* __restrict__ doc_chunk_off, int n_docs,
                                   int32_t* __restrict__ block_doc, uint32_t* __restrict__ doc_score,
-                                  int64_t n_scores) {
+                                  int64_t n_scores, float* __restrict__ etok, int64_t n_etok,
+                                  int32_t* __restrict__ redo, int n_redo) {
   const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int k = 0; k < 3; ++k) {
@@ -237,6 +287,8 @@ __global__ void route_prep_kernel(PadTargets pt, int n_rows, int L, QueryOffsets
       for (int64_t c = doc_chunk_off[d]; c < doc_chunk_off[d + 1]; ++c) block_doc[c] = (int32_t)d;
   if (doc_score != nullptr)
     for (int64_t i = i0; i < n_scores; i += stride) doc_score[i] = kOrdNegInf;
+  for (int64_t i = i0; i < n_etok; i += stride) etok[i] = 0.f;  // (the projection adds into it)
+  for (int64_t i = i0; i < n_redo; i += stride) redo[i] = 0;
 }
 
 // grid (L, B): the document scores of the layers `only` marks back to -inf
@@ -345,12 +397,6 @@ __device__ __forceinline__ float lane_dot(const float4* __restrict__ qv, int lan
   return acc;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 // ---------------------------------------------------------------------------- 2a. scan
 // One warp per (layer, block) task: exact cosine scores of the block against every
 // query token, running max per query.
@@ -373,6 +419,55 @@ __global__ void __launch_bounds__(256) scan_kernel(const __nv_bfloat16* __restri
       float best = -INFINITY;
       for (int t = qo.off[b]; t < qo.off[b + 1]; ++t)
         best = fmaxf(best, warp_sum(lane_dot<NV>(reinterpret_cast<const float4*>(qbase + (int64_t)t * R), lane, kx)));
+      if (lane == 0) m[((int64_t)b * L + l) * C + c] = best;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- 2a'. exact fallback
+// The scan of the layers `only` marks (tensor path, 8 key heads), for every query: the
+// last resort when no filter could certify a layer's selection.  A token's query sum is
+// read as its bf16 operand row plus the bf16 residual row (about 16 mantissa bits; the
+// tensor path keeps no fp32 copy).  Returns at once when no layer is marked.
+__global__ void __launch_bounds__(256) scan_fallback_kernel(const __nv_bfloat16* __restrict__ kr_hat,
+                                                            const __nv_bfloat16* __restrict__ q_hi,
+                                                            const __nv_bfloat16* __restrict__ q_lo, int L, int64_t C,
+                                                            int n_rows, QueryOffsets qo, float* __restrict__ m,
+                                                            const int32_t* __restrict__ only) {
+  constexpr int NV = 4, R = NV * 256;
+  int any = 0;
+  for (int i = threadIdx.x; i < L; i += blockDim.x) any |= only[i] != 0;
+  if (!__syncthreads_or(any)) return;
+  const int lane = threadIdx.x % 32;
+  const int64_t warp_global = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
+  const int64_t n_warps = (int64_t)gridDim.x * blockDim.x / 32;
+  for (int64_t task = warp_global; task < (int64_t)L * C; task += n_warps) {
+    const int l = (int)(task / C);
+    if (only[l] == 0) continue;
+    const int64_t c = task % C;
+    float kx[NV][8];
+    load_unit_row<NV>(kr_hat + ((int64_t)l * C + c) * R, lane, kx);
+    for (int b = 0; b < qo.n; ++b) {
+      float best = -INFINITY;
+      const int T = qo.off[b + 1] - qo.off[b];
+      for (int t = 0; t < T; ++t) {
+        const int64_t row = (int64_t)l * n_rows + qo.row0[b] + t;
+        const uint4* hv = reinterpret_cast<const uint4*>(q_hi + row * R);
+        const uint4* lv = reinterpret_cast<const uint4*>(q_lo + row * R);
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const uint4 wh = __ldg(hv + lane + 32 * i), wl = __ldg(lv + lane + 32 * i);
+          const uint32_t h4[4] = {wh.x, wh.y, wh.z, wh.w}, l4[4] = {wl.x, wl.y, wl.z, wl.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 fh = msa::bf16x2_to_float2(h4[u]), fl = msa::bf16x2_to_float2(l4[u]);
+            acc = fmaf(kx[i][2 * u], fh.x + fl.x, acc);
+            acc = fmaf(kx[i][2 * u + 1], fh.y + fl.y, acc);
+          }
+        }
+        best = fmaxf(best, warp_sum(acc));
+      }
       if (lane == 0) m[((int64_t)b * L + l) * C + c] = best;
     }
   }
@@ -498,6 +593,7 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelBatch = 16;
 constexpr int kSelEqCap = 1024;
 
+template <int MAXC>
 __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* __restrict__ doc_score, int L,
                                                                 int n_docs, int k_sel,
                                                                 unsigned long long* __restrict__ out,
@@ -507,7 +603,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int s_need, s_gt, s_eq, s_taken;
   __shared__ int wsum[kSelThreads / 32];
-  __shared__ unsigned long long keys[kMaxCandidates];
+  __shared__ unsigned long long keys[MAXC];
   __shared__ int eq_docs[kSelEqCap];
   const int l = blockIdx.x, b = blockIdx.y;
   if (only != nullptr && only[l] == 0) return;
@@ -698,6 +794,7 @@ constexpr int kRsTile = 64;
 constexpr int kRsWarps = 8;
 constexpr size_t kRsSmem = (size_t)kRsTile * 8 * kD * 2;  // the staged keys
 
+template <int MAXC>
 __global__ void __launch_bounds__(kRsWarps * 32) rescore_mma_kernel(
     const __nv_bfloat16* __restrict__ kr_hat, const __nv_bfloat16* __restrict__ q_hi,
     const __nv_bfloat16* __restrict__ q_lo, int L, int64_t C, int n_rows, QueryOffsets qo,
@@ -706,21 +803,21 @@ __global__ void __launch_bounds__(kRsWarps * 32) rescore_mma_kernel(
   constexpr int kRowBytes = 8 * kD * 2;  // 2048
   extern __shared__ __align__(128) uint8_t ktile[];
   __shared__ float rho[kRsTile][8];
-  __shared__ int64_t cand_c0[kMaxCandidates];
-  __shared__ int cand_start[kMaxCandidates + 1];
+  __shared__ int64_t cand_c0[MAXC];
+  __shared__ int cand_start[MAXC + 1];
   __shared__ int row_rank[kRsTile];
   __shared__ uint32_t row_best[kRsTile];
-  __shared__ uint32_t best[kMaxCandidates];
+  __shared__ uint32_t best[MAXC];
   const int l = blockIdx.y, b = blockIdx.z;
   if (only != nullptr && only[l] == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t o = ((int64_t)b * L + l) * K2;
   // the candidates' block ranges, end to end
   if (warp == 0) {
-    int cnt[kMaxCandidates / 32];
     int run = 0;
-#pragma unroll
-    for (int i = 0; i < kMaxCandidates / 32; ++i) {
+#pragma unroll 4
+    for (int i = 0; i < MAXC / 32; ++i) {
+      if (32 * i >= K2) break;  // (uniform over the warp)
       const int r = 32 * i + lane;
       int n = 0;
       int64_t c0 = 0;
@@ -741,8 +838,7 @@ __global__ void __launch_bounds__(kRsWarps * 32) rescore_mma_kernel(
         if (lane >= off) incl += v;
       }
       if (r < K2) cand_start[r] = run + incl - n;
-      cnt[i] = __shfl_sync(0xffffffffu, incl, 31);
-      run += cnt[i];
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) cand_start[K2] = run;
   }
@@ -874,19 +970,38 @@ __global__ void __launch_bounds__(kRsWarps * 32) rescore_mma_kernel(
     if (best[r] != 0x007FFFFFu) atomicMax(&exact_bits[o + r], best[r]);
 }
 
+// The filter error bound of query b in layer l: the largest token bound of the query
+// (etok: one bound kind, [L][T_total]); 128-thread reduction, every thread gets it.
+__device__ float query_bound(const float* __restrict__ etok, int l, int T_total, const QueryOffsets& qo, int b,
+                             float* red) {
+  float e = 0.f;
+  for (int t = qo.off[b] + threadIdx.x; t < qo.off[b + 1]; t += blockDim.x) e = fmaxf(e, etok[(int64_t)l * T_total + t]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) e = fmaxf(e, __shfl_xor_sync(0xffffffffu, e, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = e;
+  __syncthreads();
+  e = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) e = fmaxf(e, red[w]);
+  return e;
+}
+
 // grid (L, B), 128 threads: final top-k of the K2 exactly rescored candidates.  The
 // selection is certified when the k-th exact score beats the best filter score left out
-// (the K2-th) by more than the filter's error bound.  Otherwise: with redo given (a first,
-// E4M3 pass) the layer is marked for the bf16 pass; without it MSA_DEVERR_UNCERTIFIED.
-// With only given, layers it does not mark are left as they are.
+// (the K2-th) by more than the (query, layer)'s filter error bound (query_bound).  An
+// uncertified layer is marked in redo_out for the next stage (MSA_DEVERR_UNCERTIFIED when
+// there is none).  With only given, layers it does not mark are left as they are.
+template <int MAXC>
 __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long long* __restrict__ apx,
                                                            const uint32_t* __restrict__ exact_bits, int K2, int k,
-                                                           int n_docs, int L, float err,
+                                                           int n_docs, int L, const float* __restrict__ etok,
+                                                           int T_total, QueryOffsets qo,
                                                            int32_t* __restrict__ out_ids,
                                                            float* __restrict__ out_scores, int32_t* dev_err,
-                                                           int32_t* __restrict__ redo,
+                                                           int32_t* __restrict__ redo_out,
                                                            const int32_t* __restrict__ only) {
-  __shared__ unsigned long long keys[kMaxCandidates];
+  __shared__ unsigned long long keys[MAXC];
+  __shared__ float red[4];
   const int l = blockIdx.x, b = blockIdx.y;
   if (only != nullptr && only[l] == 0) return;
   const int64_t base = ((int64_t)b * L + l) * K2;
@@ -901,7 +1016,7 @@ __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long l
     }
     keys[i] = key;
   }
-  __syncthreads();
+  const float err = query_bound(etok, l, T_total, qo, b, red);  // (its barriers order the stores above)
   block_sort_desc(keys, n_pow2);
   for (int r = threadIdx.x; r < k; r += blockDim.x) {
     int doc;
@@ -916,7 +1031,7 @@ __global__ void __launch_bounds__(128) select_final_kernel(const unsigned long l
     split_key(apx[base + K2 - 1], &d_left, &s_left);
     split_key(keys[k - 1], &d_kth, &s_kth);
     if (!(s_kth > s_left + err)) {
-      if (redo != nullptr) redo[l] = 1;
+      if (redo_out != nullptr) redo_out[l] = 1;
       else msa::set_err(dev_err, MSA_DEVERR_UNCERTIFIED);
     }
   }
@@ -963,13 +1078,16 @@ __global__ void replicate_candidates_kernel(const unsigned long long* __restrict
 
 // grid (B): the final top-k of the shared candidates by the mean over layers of their
 // exact scores, written to every layer; certified when the k-th exact mean beats the best
-// mean filter score left out by more than err (else the redo mark on all layers, or
+// mean filter score left out by more than the mean over layers of the query's bounds plus
+// the fp32 rounding of the two means (else the mark on every layer in redo_out, or
 // MSA_DEVERR_UNCERTIFIED).
+template <int MAXC>
 __global__ void __launch_bounds__(128) select_final_mean_kernel(
     const unsigned long long* __restrict__ apx_agg, const uint32_t* __restrict__ exact_bits, int K2, int k, int n_docs,
-    int L, float err, int32_t* __restrict__ out_ids, float* __restrict__ out_scores, int32_t* dev_err,
-    int32_t* __restrict__ redo, const int32_t* __restrict__ gate) {
-  __shared__ unsigned long long keys[kMaxCandidates];
+    int L, const float* __restrict__ etok, int T_total, QueryOffsets qo, int32_t* __restrict__ out_ids,
+    float* __restrict__ out_scores, int32_t* dev_err, int32_t* __restrict__ redo_out, const int32_t* __restrict__ gate) {
+  __shared__ unsigned long long keys[MAXC];
+  __shared__ float red[4];
   if (gate != nullptr && gate[0] == 0) return;
   const int b = blockIdx.x;
   const int n_pow2 = K2 <= 1 ? 1 : (1 << (32 - __clz(K2 - 1)));
@@ -988,7 +1106,9 @@ __global__ void __launch_bounds__(128) select_final_mean_kernel(
     }
     keys[i] = key;
   }
-  __syncthreads();
+  float err = 0.f;
+  for (int l = 0; l < L; ++l) err += query_bound(etok, l, T_total, qo, b, red);
+  err = err * inv_l * kBoundSlack + (float)(L + 1) * (1.0f / 4194304);  // + (L + 1) 2^-22
   block_sort_desc(keys, n_pow2);
   for (int e = threadIdx.x; e < L * k; e += blockDim.x) {
     const int l = e / k, r = e % k;
@@ -1004,11 +1124,56 @@ __global__ void __launch_bounds__(128) select_final_mean_kernel(
     split_key(apx_agg[(int64_t)b * K2 + K2 - 1], &d_left, &s_left);
     split_key(keys[k - 1], &d_kth, &s_kth);
     if (!(s_kth > s_left + err)) {
-      if (redo != nullptr)
-        for (int l = 0; l < L; ++l) redo[l] = 1;
+      if (redo_out != nullptr)
+        for (int l = 0; l < L; ++l) redo_out[l] = 1;
       else
         msa::set_err(dev_err, MSA_DEVERR_UNCERTIFIED);
     }
+  }
+}
+
+// grid (L, B): exact document scores from the fallback scan's block scores m, as ordered
+// bits into doc_score (layers `only` marks).
+__global__ void doc_exact_kernel(const float* __restrict__ m, const int64_t* __restrict__ doc_chunk_off, int n_docs,
+                                 int64_t C, int L, uint32_t* __restrict__ doc_score, const int32_t* __restrict__ only) {
+  const int l = blockIdx.x, b = blockIdx.y;
+  if (only[l] == 0) return;
+  const float* mb = m + ((int64_t)b * L + l) * C;
+  uint32_t* out = doc_score + ((int64_t)b * L + l) * n_docs;
+  for (int d = threadIdx.x; d < n_docs; d += blockDim.x) {
+    float s = -INFINITY;
+    for (int64_t c = doc_chunk_off[d]; c < doc_chunk_off[d + 1]; ++c) s = fmaxf(s, mb[c]);
+    out[d] = float_to_ord(s);
+  }
+}
+
+// grid (B): the keys of query b's final selection (best first) written as ids / scores to
+// every layer (gate: only when gate[0] != 0).
+__global__ void keys_to_layers_kernel(const unsigned long long* __restrict__ keys, int k, int L,
+                                      int32_t* __restrict__ out_ids, float* __restrict__ out_scores,
+                                      const int32_t* __restrict__ gate) {
+  if (gate != nullptr && gate[0] == 0) return;
+  const int b = blockIdx.x;
+  for (int e = threadIdx.x; e < L * k; e += blockDim.x) {
+    const int l = e / k, r = e % k;
+    int doc;
+    float s;
+    split_key(keys[(int64_t)b * k + r], &doc, &s);
+    out_ids[((int64_t)b * L + l) * k + r] = doc;
+    out_scores[((int64_t)b * L + l) * k + r] = s;
+  }
+}
+
+// grid (L, B): keys [B][L][k] (best first) split into ids / scores.
+__global__ void keys_to_out_kernel(const unsigned long long* __restrict__ keys, int k, int L,
+                                   int32_t* __restrict__ out_ids, float* __restrict__ out_scores) {
+  const int64_t o = ((int64_t)blockIdx.y * L + blockIdx.x) * k;
+  for (int r = threadIdx.x; r < k; r += blockDim.x) {
+    int doc;
+    float s;
+    split_key(keys[o + r], &doc, &s);
+    out_ids[o + r] = doc;
+    out_scores[o + r] = s;
   }
 }
 
@@ -1100,10 +1265,13 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
     return msa_fail(MSA_ERR_INVALID_ARG, "bad counts (n_docs <= 2^20)");
   if (!project && q_dtype != MSA_F32 && q_dtype != MSA_BF16) return msa_fail(MSA_ERR_UNSUPPORTED, "q_dtype");
   const bool layer_mean = (flags & MSA_ROUTE_LAYER_MEAN) != 0;
-  flags &= ~MSA_ROUTE_LAYER_MEAN;
+  const bool filter_only = (flags & MSA_ROUTE_FILTER_SCORES) != 0;
+  flags &= ~(MSA_ROUTE_LAYER_MEAN | MSA_ROUTE_FILTER_SCORES);
   if (flags < MSA_ROUTE_AUTO || flags > MSA_ROUTE_TENSOR_F8) return msa_fail(MSA_ERR_INVALID_ARG, "flags");
   if (layer_mean && flags == MSA_ROUTE_SCAN)
     return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_LAYER_MEAN runs on the tensor path, not MSA_ROUTE_SCAN");
+  if (filter_only && (layer_mean || (flags != MSA_ROUTE_TENSOR && flags != MSA_ROUTE_TENSOR_F8)))
+    return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_FILTER_SCORES takes MSA_ROUTE_TENSOR or _TENSOR_F8 alone");
   if (flags == MSA_ROUTE_TENSOR_F8 && !kr_f8)
     return msa_fail(MSA_ERR_INVALID_ARG, "MSA_ROUTE_TENSOR_F8 needs the E4M3 keys (msa_route_filter_keys)");
   if (!msa::aligned16(qr) || !msa::aligned16(kr_hat) || !msa::aligned16(kr_f8) ||
@@ -1148,13 +1316,19 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   }
   const bool tensor = (path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && n_chunks > 0;
   const bool f8 = tensor && path == MSA_ROUTE_TENSOR_F8;
-  const float filter_err = f8 ? kFilterErrF8 : kFilterErr;
 
   uint8_t* qt_f8 = reinterpret_cast<uint8_t*>(ws + w.qt_f8);
   uint32_t* doc_score = reinterpret_cast<uint32_t*>(ws + w.doc_score);
   int32_t* block_doc = reinterpret_cast<int32_t*>(ws + w.block_doc);
   __nv_bfloat16* qt_lo = reinterpret_cast<__nv_bfloat16*>(ws + w.qt_lo);
-  int32_t* redo = reinterpret_cast<int32_t*>(ws + w.redo);
+  // layer masks: redo1 = the E4M3 pass could not certify, redo2 = nor the bf16 pass,
+  // redo3 = nor the widened rescoring (exact scan); etok = the per-token filter bounds
+  int32_t* redo1 = reinterpret_cast<int32_t*>(ws + w.redo);
+  int32_t* redo2 = redo1 + n_layers;
+  int32_t* redo3 = redo2 + n_layers;
+  float* etok = reinterpret_cast<float*>(ws + w.etok);
+  const float* etok_f8 = etok + (size_t)kBoundF8 * n_layers * T_total;
+  const float* etok_bf16 = etok + (size_t)kBoundBf16 * n_layers * T_total;
   if (tensor) {
     // operand rows: bf16 (GEMM, and the high half of the exact rescoring), its residual
     // (the low half) and, on the E4M3 path, E4M3
@@ -1167,7 +1341,8 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
     pt.words_per_row[2] = H * kD / 16;
     route_prep_kernel<<<msa::sm_count() * 4, 256, 0, s>>>(pt, n_rows, n_layers, qo, doc_chunk_offsets, n_docs,
                                                            block_doc, doc_score,
-                                                           (int64_t)n_queries * n_layers * n_docs);
+                                                           (int64_t)n_queries * n_layers * n_docs, etok,
+                                                           (int64_t)2 * n_layers * T_total, redo1, 3 * n_layers);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
   }
@@ -1192,7 +1367,7 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
     pa.qt_bf16 = tensor ? qt_bf16 : nullptr;
     pa.qt_lo = tensor ? qt_lo : nullptr;
     pa.qt_f8 = f8 ? qt_f8 : nullptr;
-    pa.redo = f8 ? redo : nullptr;
+    pa.etok = tensor ? etok : nullptr;
     pa.dev_err = dev_err;
     const char* why = nullptr;
     if (route_proj::launch(pa, s, &why) != 0)
@@ -1201,7 +1376,7 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
     qprep_kernel<<<dim3(T_total, n_layers), 128, 0, s>>>(qr, q_dtype == MSA_BF16, T_total, n_q_heads, H, n_rows, qo,
                                                         tensor ? nullptr : qt_f32, tensor ? qt_bf16 : nullptr,
                                                         tensor ? qt_lo : nullptr, f8 ? qt_f8 : nullptr,
-                                                        f8 ? redo : nullptr, n_layers);
+                                                        tensor ? etok : nullptr, n_layers);
   }
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
@@ -1259,102 +1434,204 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   const size_t tk_smem = (size_t)doc_pow2 * sizeof(unsigned long long);
   if (tk_smem > 48 * 1024)
     MSA_CUDA_TRY(cudaFuncSetAttribute(docmax_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tk_smem));
-  if (!tensor || n_docs == 0) {
-    // scan path (exact scores): per-block top-k, then one merge straight to the outputs
-    const int mg_pow2 = pow2_at_least(w.nblk * top_k);
-    const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
-    if (mg_smem > 48 * 1024)
-      MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
+  const int mg_pow2 = pow2_at_least(w.nblk * top_k);
+  const size_t mg_smem = (size_t)mg_pow2 * sizeof(unsigned long long);
+  if (mg_smem > 48 * 1024)
+    MSA_CUDA_TRY(cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mg_smem));
+  // exact per-block scores m -> per-CTA best documents -> top_k (only: the layers marked)
+  auto docmax_merge = [&](const int32_t* only) -> msa_status {
     docmax_topk_kernel<<<dim3(w.nblk, n_layers, n_queries), kTopkThreads, tk_smem, s>>>(
-        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, top_k, doc_pow2, cand, nullptr);
+        m, doc_chunk_offsets, n_docs, n_chunks, n_layers, top_k, doc_pow2, cand, only);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     merge_topk_kernel<<<dim3(n_layers, n_queries), kTopkThreads, mg_smem, s>>>(cand, w.nblk, n_layers, top_k, mg_pow2,
-                                                                            nullptr, out_ids, out_scores, nullptr);
-    ++g_launches;
-    MSA_CUDA_TRY(cudaGetLastError());
-    return msa_ok();
-  }
-  // tensor path: the GEMM scores are a filter; the K2 best documents by those scores are
-  // rescored exactly (fp32 cosines) and the final top-k is taken from the exact scores
-  const int K2 = w.k2;
-  unsigned long long* apx = reinterpret_cast<unsigned long long*>(ws + w.apx);
-  uint32_t* exact = reinterpret_cast<uint32_t*>(ws + w.exact);
-  MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRsSmem));
-  // CTAs per (query, layer) of the rescoring: about two per SM in all, at most 8
-  int rs_x = (2 * msa::sm_count() + n_layers * n_queries - 1) / (n_layers * n_queries);
-  rs_x = rs_x < 1 ? 1 : (rs_x > 8 ? 8 : rs_x);
-  // candidates -> exact rescoring -> final top-k (+ certification), on the layers `only`
-  // marks; uncertified layers go to redo_out when given
-  auto select = [&](float err, int32_t* redo_out, const int32_t* only) -> msa_status {
-    topk_docs_kernel<<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs, K2, apx, exact,
-                                                                      only);
-    ++g_launches;
-    MSA_CUDA_TRY(cudaGetLastError());
-    rescore_mma_kernel<<<dim3(rs_x, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
-        (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx, K2,
-        exact, only);
-    ++g_launches;
-    MSA_CUDA_TRY(cudaGetLastError());
-    select_final_kernel<<<dim3(n_layers, n_queries), 128, 0, s>>>(apx, exact, K2, top_k, n_docs, n_layers, err,
-                                                                 out_ids, out_scores, dev_err, redo_out, only);
+                                                                            nullptr, out_ids, out_scores, only);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     return msa_ok();
   };
+  if (!tensor || n_docs == 0) return docmax_merge(nullptr);  // scan path: exact scores
+
+  unsigned long long* apx = reinterpret_cast<unsigned long long*>(ws + w.apx);
+  uint32_t* exact = reinterpret_cast<uint32_t*>(ws + w.exact);
+  if (filter_only) {
+    // the documents' filter scores themselves (no rescoring): for measuring the filter
+    topk_docs_kernel<kMaxCandidates><<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs,
+                                                                                      top_k, apx, exact, nullptr);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    keys_to_out_kernel<<<dim3(n_layers, n_queries), 64, 0, s>>>(apx, top_k, n_layers, out_ids, out_scores);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    return msa_ok();
+  }
+
+  // tensor path: the GEMM scores are a filter; the K2 best documents by those scores are
+  // rescored exactly (fp32 cosines) and the final top-k is taken from the exact scores
+  const int K2 = w.k2, KW = w.kw;
+  unsigned long long* apx_w = reinterpret_cast<unsigned long long*>(ws + w.apx_w);
+  uint32_t* exact_w = reinterpret_cast<uint32_t*>(ws + w.exact_w);
+  MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_mma_kernel<kMaxCandidates>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kRsSmem));
+  MSA_CUDA_TRY(cudaFuncSetAttribute(rescore_mma_kernel<kMaxWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kRsSmem));
+  // CTAs per (query, layer) of the rescoring: about two per SM in all, at most 8; the
+  // widened rescoring (rarely more than a few layers) up to 32
+  const int lb = n_layers * n_queries;
+  int rs_x = (2 * msa::sm_count() + lb - 1) / lb;
+  rs_x = rs_x < 1 ? 1 : (rs_x > 8 ? 8 : rs_x);
+  int rs_xw = (4 * msa::sm_count() + lb - 1) / lb;
+  rs_xw = rs_xw < 1 ? 1 : (rs_xw > 32 ? 32 : rs_xw);
+  // K best documents by filter score -> exact rescoring -> final top-k + certification,
+  // on the layers `only` marks; uncertified layers go to redo_out
+  auto select = [&](bool wide, const float* eb, int32_t* redo_out, const int32_t* only) -> msa_status {
+    if (!wide) {
+      topk_docs_kernel<kMaxCandidates><<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs,
+                                                                                        K2, apx, exact, only);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      rescore_mma_kernel<kMaxCandidates><<<dim3(rs_x, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
+          (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx, K2,
+          exact, only);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      select_final_kernel<kMaxCandidates><<<dim3(n_layers, n_queries), 128, 0, s>>>(
+          apx, exact, K2, top_k, n_docs, n_layers, eb, T_total, qo, out_ids, out_scores, dev_err, redo_out, only);
+    } else {
+      topk_docs_kernel<kMaxWide><<<dim3(n_layers, n_queries), kSelThreads, 0, s>>>(doc_score, n_layers, n_docs, KW,
+                                                                                  apx_w, exact_w, only);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      rescore_mma_kernel<kMaxWide><<<dim3(rs_xw, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
+          (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx_w, KW,
+          exact_w, only);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      select_final_kernel<kMaxWide><<<dim3(n_layers, n_queries), 128, 0, s>>>(
+          apx_w, exact_w, KW, top_k, n_docs, n_layers, eb, T_total, qo, out_ids, out_scores, dev_err, redo_out, only);
+    }
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    return msa_ok();
+  };
+  // the exact scan of the layers `only` marks, for every query (block scores into m)
+  int64_t fb_blocks = ((int64_t)n_layers * n_chunks + 7) / 8;
+  if (fb_blocks > (int64_t)msa::sm_count() * 8) fb_blocks = (int64_t)msa::sm_count() * 8;
+  if (fb_blocks < 1) fb_blocks = 1;
+  auto exact_scan = [&](const int32_t* only) -> msa_status {
+    scan_fallback_kernel<<<(unsigned)fb_blocks, 256, 0, s>>>((const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers,
+                                                             n_chunks, n_rows, qo, m, only);
+    ++g_launches;
+    MSA_CUDA_TRY(cudaGetLastError());
+    return msa_ok();
+  };
+  msa_status st;
+  if (!layer_mean) {
+    // E4M3 pass -> (its uncertified layers) bf16 pass -> (uncertified) widened rescoring
+    // -> (uncertified) exact scan; each stage's kernels return at once when no layer is
+    // marked for them
+    if (f8) {
+      if ((st = select(false, etok_f8, redo1, nullptr)) != MSA_OK) return st;
+      doc_reset_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(doc_score, n_layers, n_docs, redo1);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      if ((st = gemm(false, redo1)) != MSA_OK) return st;
+      if ((st = select(false, etok_bf16, redo2, redo1)) != MSA_OK) return st;
+    } else {
+      if ((st = select(false, etok_bf16, redo2, nullptr)) != MSA_OK) return st;
+    }
+    if (n_docs <= K2) return msa_ok();  // every document was rescored: nothing left to certify
+    if ((st = select(true, etok_bf16, redo3, redo2)) != MSA_OK) return st;
+    if (n_docs <= KW) return msa_ok();
+    if ((st = exact_scan(redo3)) != MSA_OK) return st;
+    return docmax_merge(redo3);
+  }
+
   // the layer-aggregated variant: shared candidates from the mean filter scores, exact
-  // rescoring in every layer, final top-k on the mean exact scores (gate: the second
-  // pass runs these only when the first marked the layers)
+  // rescoring in every layer, final top-k on the mean exact scores (gate: the later
+  // stages run only when the earlier one marked the layers; every layer is marked alike)
   unsigned long long* apx_agg = reinterpret_cast<unsigned long long*>(ws + w.apx_agg);
   uint32_t* agg = reinterpret_cast<uint32_t*>(ws + w.agg);
   uint32_t* exact_agg = reinterpret_cast<uint32_t*>(ws + w.exact_agg);
-  auto select_mean = [&](float err, int32_t* redo_out, const int32_t* gate) -> msa_status {
-    const int64_t n_agg = (int64_t)n_queries * n_docs;
-    const int mean_blocks = (int)((n_agg + 255) / 256 < msa::sm_count() * 4 ? (n_agg + 255) / 256 : msa::sm_count() * 4);
+  unsigned long long* apx_agg_w = reinterpret_cast<unsigned long long*>(ws + w.apx_agg_w);
+  uint32_t* exact_agg_w = reinterpret_cast<uint32_t*>(ws + w.exact_agg_w);
+  const int64_t n_agg = (int64_t)n_queries * n_docs;
+  const int mean_blocks =
+      (int)((n_agg + 255) / 256 < msa::sm_count() * 4 ? (n_agg + 255) / 256 : msa::sm_count() * 4);
+  auto layer_mean_scores = [&](const int32_t* gate) -> msa_status {
     layer_mean_kernel<<<mean_blocks > 0 ? mean_blocks : 1, 256, 0, s>>>(doc_score, n_queries, n_layers, n_docs, agg,
                                                                         gate);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
-    topk_docs_kernel<<<dim3(1, n_queries), kSelThreads, 0, s>>>(agg, 1, n_docs, K2, apx_agg, exact_agg, gate);
+    return msa_ok();
+  };
+  auto select_mean = [&](bool wide, const float* eb, int32_t* redo_out, const int32_t* gate) -> msa_status {
+    msa_status r = layer_mean_scores(gate);
+    if (r != MSA_OK) return r;
+    const int K = wide ? KW : K2;
+    unsigned long long* aa = wide ? apx_agg_w : apx_agg;
+    unsigned long long* ap = wide ? apx_w : apx;
+    uint32_t* ex = wide ? exact_w : exact;
+    if (wide)
+      topk_docs_kernel<kMaxWide><<<dim3(1, n_queries), kSelThreads, 0, s>>>(agg, 1, n_docs, K, aa, exact_agg_w, gate);
+    else
+      topk_docs_kernel<kMaxCandidates><<<dim3(1, n_queries), kSelThreads, 0, s>>>(agg, 1, n_docs, K, aa, exact_agg,
+                                                                                 gate);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
-    const int64_t n_rep = (int64_t)n_queries * n_layers * K2;
-    replicate_candidates_kernel<<<(int)((n_rep + 255) / 256), 256, 0, s>>>(apx_agg, n_queries, n_layers, K2, apx,
-                                                                          exact, gate);
+    const int64_t n_rep = (int64_t)n_queries * n_layers * K;
+    replicate_candidates_kernel<<<(int)((n_rep + 255) / 256), 256, 0, s>>>(aa, n_queries, n_layers, K, ap, ex, gate);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
-    rescore_mma_kernel<<<dim3(rs_x, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
-        (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, apx, K2,
-        exact, gate);
-    ++g_launches;
-    MSA_CUDA_TRY(cudaGetLastError());
-    select_final_mean_kernel<<<n_queries, 128, 0, s>>>(apx_agg, exact, K2, top_k, n_docs, n_layers, err, out_ids,
-                                                       out_scores, dev_err, redo_out, gate);
+    if (wide) {
+      rescore_mma_kernel<kMaxWide><<<dim3(rs_xw, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
+          (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, ap, K, ex,
+          gate);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      select_final_mean_kernel<kMaxWide><<<n_queries, 128, 0, s>>>(aa, ex, K, top_k, n_docs, n_layers, eb, T_total, qo,
+                                                                  out_ids, out_scores, dev_err, redo_out, gate);
+    } else {
+      rescore_mma_kernel<kMaxCandidates><<<dim3(rs_x, n_layers, n_queries), kRsWarps * 32, kRsSmem, s>>>(
+          (const __nv_bfloat16*)kr_hat, qt_bf16, qt_lo, n_layers, n_chunks, n_rows, qo, doc_chunk_offsets, ap, K, ex,
+          gate);
+      ++g_launches;
+      MSA_CUDA_TRY(cudaGetLastError());
+      select_final_mean_kernel<kMaxCandidates><<<n_queries, 128, 0, s>>>(aa, ex, K, top_k, n_docs, n_layers, eb,
+                                                                        T_total, qo, out_ids, out_scores, dev_err,
+                                                                        redo_out, gate);
+    }
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
     return msa_ok();
   };
-  if (layer_mean) {
-    msa_status st = select_mean(filter_err, f8 ? redo : nullptr, nullptr);
-    if (st != MSA_OK || !f8) return st;
-    doc_reset_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(doc_score, n_layers, n_docs, redo);
+  if (f8) {
+    if ((st = select_mean(false, etok_f8, redo1, nullptr)) != MSA_OK) return st;
+    doc_reset_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(doc_score, n_layers, n_docs, redo1);
     ++g_launches;
     MSA_CUDA_TRY(cudaGetLastError());
-    st = gemm(false, redo);
-    if (st != MSA_OK) return st;
-    return select_mean(kFilterErr, nullptr, redo);
+    if ((st = gemm(false, redo1)) != MSA_OK) return st;
+    if ((st = select_mean(false, etok_bf16, redo2, redo1)) != MSA_OK) return st;
+  } else {
+    if ((st = select_mean(false, etok_bf16, redo2, nullptr)) != MSA_OK) return st;
   }
-  msa_status st = select(filter_err, f8 ? redo : nullptr, nullptr);
-  if (st != MSA_OK || !f8) return st;
-  // E4M3 layers that could not be certified: bf16 filter over them, then the same steps
-  // with the bf16 error bound (every kernel returns at once on certified layers)
-  doc_reset_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(doc_score, n_layers, n_docs, redo);
+  if (n_docs <= K2) return msa_ok();
+  if ((st = select_mean(true, etok_bf16, redo3, redo2)) != MSA_OK) return st;
+  if (n_docs <= KW) return msa_ok();
+  // exact scan of every layer, exact document scores, their mean, top_k to every layer
+  if ((st = exact_scan(redo3)) != MSA_OK) return st;
+  doc_exact_kernel<<<dim3(n_layers, n_queries), 256, 0, s>>>(m, doc_chunk_offsets, n_docs, n_chunks, n_layers,
+                                                            doc_score, redo3);
   ++g_launches;
   MSA_CUDA_TRY(cudaGetLastError());
-  st = gemm(false, redo);
-  if (st != MSA_OK) return st;
-  st = select(kFilterErr, nullptr, redo);
-  if (st != MSA_OK) return st;
+  if ((st = layer_mean_scores(redo3)) != MSA_OK) return st;
+  topk_docs_kernel<kMaxCandidates><<<dim3(1, n_queries), kSelThreads, 0, s>>>(agg, 1, n_docs, top_k, apx_agg,
+                                                                             exact_agg, redo3);
+  ++g_launches;
+  MSA_CUDA_TRY(cudaGetLastError());
+  keys_to_layers_kernel<<<n_queries, 128, 0, s>>>(apx_agg, top_k, n_layers, out_ids, out_scores, redo3);
+  ++g_launches;
+  MSA_CUDA_TRY(cudaGetLastError());
   return msa_ok();
 }
 

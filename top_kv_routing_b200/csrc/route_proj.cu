@@ -32,6 +32,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "route_bound.cuh"
 #include "route_proj.cuh"
 #include "tc_common.cuh"
 
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, int T, int kblocks,
                 int L, int Hq, int H, int m_tiles, int n_rows, const __grid_constant__ Layout lay,
                 float* __restrict__ qt_f32, __nv_bfloat16* __restrict__ qt_bf16, __nv_bfloat16* __restrict__ qt_lo,
-                uint8_t* __restrict__ qt_f8, int32_t* __restrict__ redo, int32_t* dev_err) {
+                uint8_t* __restrict__ qt_f8, float* __restrict__ etok, int32_t* dev_err) {
   using K = Cfg<G, PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -84,8 +85,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int first_unit = PAIR ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
   const int unit_stride = PAIR ? (int)(gridDim.x / 2) : (int)gridDim.x;
-  if (redo != nullptr && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < L; i += blockDim.x) redo[i] = 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < K::kStages; ++s) {
@@ -252,7 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         inv[h] = 1.0f / fmaxf(sqrtf(ss), 1e-8f);
       }
-      // pass 2: (1/Hq) * sum of the unit heads, 32 columns at a time
+      // pass 2: (1/Hq) * sum of the unit heads, 32 columns at a time (and the norms of
+      // the filter error bounds: q, its bf16 rounding and residual, its E4M3 operand and residual)
+      float bsum[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         float acc[32];
@@ -269,6 +270,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] *= inv_hq;
         if (orow < 0) continue;
+        if (etok != nullptr) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float hf = __bfloat162float(__float2bfloat16_rn(acc[i])), db = hf - acc[i];
+            const float a = acc[i] * route_tc::kF8QueryScale, ah = route_bound::e4m3_round(a);
+            const float as = ah * (1.0f / route_tc::kF8QueryScale), da = (ah - a) * (1.0f / route_tc::kF8QueryScale);
+            bsum[0] = fmaf(acc[i], acc[i], bsum[0]);
+            bsum[1] = fmaf(db, db, bsum[1]);
+            bsum[2] = fmaf(hf, hf, bsum[2]);
+            bsum[3] = fmaf(as, as, bsum[3]);
+            bsum[4] = fmaf(da, da, bsum[4]);
+            bsum[5] += fabsf(as);
+          }
+        }
         const int e0 = g * kD + c * 32;
         if (qt_f32 != nullptr) {
           float4* dst = reinterpret_cast<float4*>(qt_f32 + ((int64_t)l * T + t) * hd + e0);
@@ -311,6 +326,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           df[0] = make_uint4(fw[0], fw[1], fw[2], fw[3]);
           df[1] = make_uint4(fw[4], fw[5], fw[6], fw[7]);
         }
+      }
+      if (etok != nullptr && orow >= 0) {
+        // this key head's share of the token's bounds
+        const float2 eb = route_bound::head_bounds(sqrtf(bsum[0]), sqrtf(bsum[1]), sqrtf(bsum[2]), sqrtf(bsum[3]),
+                                                   sqrtf(bsum[4]), bsum[5]);
+        atomicAdd(etok + ((int64_t)route_bound::kBoundF8 * L + l) * T + t,
+                  eb.x * route_bound::kBoundSlack + route_bound::kBoundFloor);
+        atomicAdd(etok + ((int64_t)route_bound::kBoundBf16 * L + l) * T + t,
+                  eb.y * route_bound::kBoundSlack + route_bound::kBoundFloor);
       }
       tc_fence_before();
       __syncwarp();
@@ -397,7 +421,7 @@ int launch_g(const Args& a, cudaStream_t s, const char** why) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, proj_kernel<G, PAIR>, mh, mw, a.T, a.hidden_size / kBK, a.L, a.Hq, a.H, m_tiles,
-                         a.n_rows, a.lay, a.qt_f32, a.qt_bf16, a.qt_lo, a.qt_f8, a.redo, a.dev_err) != cudaSuccess) {
+                         a.n_rows, a.lay, a.qt_f32, a.qt_bf16, a.qt_lo, a.qt_f8, a.etok, a.dev_err) != cudaSuccess) {
     *why = "kernel launch";
     return 1;
   }

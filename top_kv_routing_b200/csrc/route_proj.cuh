@@ -24,7 +24,8 @@ struct Args {
   __nv_bfloat16* qt_bf16;      // [L][n_rows][H * 128] or null (with qt_lo)
   __nv_bfloat16* qt_lo;
   uint8_t* qt_f8;              // [L][n_rows][H * 128] or null
-  int32_t* redo;               // L entries set to 0, or null
+  float* etok;                 // [2][L][T] filter error bounds per token (zeroed by the
+                               // caller; each key head's share is added), or null
   int32_t* dev_err;
 };
 
