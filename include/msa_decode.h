@@ -53,7 +53,10 @@ msa_status msa_sparse_decode_workspace_size(int32_t n_queries, int32_t n_layers,
  * A query whose cache is full (local_len >= local_cap) is skipped (out untouched, length
  * not advanced) and sets MSA_DEVERR_LOCAL_FULL; mem_len > max_mem_chunks is clamped with
  * MSA_DEVERR_CAPACITY.  One kernel launch, asynchronous on stream, graph-capturable
- * (every per-step quantity is read on the device). */
+ * (every per-step quantity is read on the device).  The kernel is launched as a
+ * programmatic dependent of the kernel before it on the stream: it may be scheduled while
+ * that kernel finishes, and it reads every input only after waiting for it, so inputs that
+ * the preceding kernel or copy writes (msa_gather_kv's mem_len, this step's q) are seen. */
 msa_status msa_sparse_decode(const void* q, const void* k_new, const void* v_new, int32_t n_queries,
                              int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                              void* local_k, void* local_v, int32_t* local_len, int32_t local_cap,
@@ -66,7 +69,9 @@ msa_status msa_sparse_decode(const void* q, const void* k_new, const void* v_new
  * a host that hands the library only the buffers it already owns, or code running where
  * allocation is forbidden mid-stream).  The scratch is a fixed array inside this library,
  * MSA_DECODE_STATIC_SCRATCH_BYTES in size, which every GPU that loads the library keeps
- * until the process exits; sizes that need more fail with MSA_ERR_CAPACITY.  The first
+ * until the process exits; sizes that need more fail with MSA_ERR_CAPACITY.  A call needs
+ * n_queries * n_layers * n_kv_heads * (2080 * G + 4) + 4 * n_queries bytes (G = n_q_heads /
+ * n_kv_heads): at 18 layers, 8 key heads and G = 4, six queries fit.  The first
  * call on a device looks the array's device address up (issue that first call before any
  * stream capture).  Each call clears the part that must start at zero with one
  * cudaMemsetAsync on `stream` and allocates nothing.  All calls share the one array:

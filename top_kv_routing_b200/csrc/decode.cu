@@ -62,6 +62,11 @@ size_t ws_bytes(int B, int L, int Hq, int H) {
   return ws_floats(B, L, Hq, H) * sizeof(float) + ((size_t)B * L * H + (size_t)B) * sizeof(int);
 }
 
+// RoPE frequencies of one call: w_j / pi = theta^(-2j/128) / pi, j < 64 (fp64).
+struct RopeFreq {
+  double w_over_pi[kHalf];
+};
+
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
@@ -69,7 +74,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     // rows [0, len) are read; row len is written by split 0 and read by nobody here
     __nv_bfloat16* local_k, __nv_bfloat16* local_v, int32_t* local_len, int cap,
     const __nv_bfloat16* __restrict__ mem_kv, const int32_t* __restrict__ mem_len, int M_max, int pos_off,
-    double log2_theta, float qscale, int splits, float* part, float2* stat, int* unit_count, int* query_count,
+    const __grid_constant__ RopeFreq rf, float qscale, int splits, float* part, float2* stat, int* unit_count,
+    int* query_count,
     __nv_bfloat16* __restrict__ out, int32_t* dev_err) {
   extern __shared__ __align__(128) unsigned char ring[];
   // query fragments in MMA order: row g*4 + t holds thread (g, t)'s 8 k-steps x 4 words,
@@ -89,9 +95,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
   const int Hq = H * G;
   const int64_t bl = blockIdx.z;
   const int64_t uh = bl * H + h;
-  // inputs no earlier decode step writes (this step's q, k_new, v_new; the gathered memory's
-  // length) load before the wait for the previous grid: thread (head gg, m) takes q dims 2m,
-  // 2m+1 and their rotate-half partners 2m+64, 2m+65
+  // Launched as a programmatic dependent of the kernel before it on the stream (the
+  // previous decode step, or whatever kernel or copy wrote this step's inputs: the gather
+  // writes mem_len, a copy may write q): every input is read after the wait, past which that
+  // grid's writes are complete and visible.  The next step may then be scheduled onto SMs as
+  // this one's CTAs leave.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // thread (head gg, m) takes q dims 2m, 2m+1 and their rotate-half partners 2m+64, 2m+65
   const int gg = tid >> 5, mq = tid & 31;
   uint32_t qlo = 0u, qhi = 0u;
   if (gg < G) {
@@ -108,11 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     vx = v_new[uh * kD + tid - kHalf];
   }
   int M = mem_len[bl];
-  // Launched as a programmatic dependent of the previous step: past this point that step
-  // (its cache row, the length it advanced, its counters) is complete and visible; the
-  // next step may then be scheduled onto SMs as this one's CTAs leave.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int len = local_len[b];
   const bool full = len < 0 || len >= cap;  // (a negative length is treated as unusable too)
   if (M > M_max) {
@@ -185,11 +191,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
       cp_async_commit();
     }
 
-    // ---- RoPE angles of this step's position: w_j / pi in fp64, the product reduced
-    // modulo 2 pi in fp64, fp32 sincospif
+    // ---- RoPE angles of this step's position: p * w_j / pi in fp64 (w_j / pi computed once
+    // per call on the host), reduced modulo 2 pi in fp64, fp32 sincospif
     const double pos = (double)pos_off + (double)len;
     if (tid < kHalf) {
-      double u = pos * (exp2(-2.0 * (double)tid / (double)kD * log2_theta) * 0.31830988618379067154);
+      double u = pos * rf.w_over_pi[tid];
       u -= 2.0 * rint(0.5 * u);  // in [-1, 1]
       float sn, c;
       sincospif((float)u, &sn, &c);
@@ -427,13 +433,13 @@ extern "C" msa_status msa_sparse_decode_workspace_size(int32_t n_queries, int32_
   return msa_ok();
 }
 
-extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const void* v_new, int32_t n_queries,
-                                        int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
-                                        void* local_k, void* local_v, int32_t* local_len, int32_t local_cap,
-                                        const void* mem_kv, const int32_t* mem_len, int32_t max_mem_chunks,
-                                        int32_t rope_pos_offset, float rope_theta, float softmax_scale, void* out,
-                                        void* workspace, size_t workspace_bytes, int32_t* dev_err,
-                                        msa_stream_t stream) {
+namespace {
+// Host-side argument and device checks of a decode call (nothing is enqueued).
+msa_status check_decode(const void* q, const void* k_new, const void* v_new, int32_t n_queries, int32_t n_layers,
+                        int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, const void* local_k,
+                        const void* local_v, const int32_t* local_len, int32_t local_cap, const void* mem_kv,
+                        const int32_t* mem_len, int32_t max_mem_chunks, float rope_theta, const void* out,
+                        const void* workspace, size_t workspace_bytes) {
   if (!q || !k_new || !v_new || !local_k || !local_v || !local_len || !mem_kv || !mem_len || !out || !workspace)
     return msa_fail(MSA_ERR_INVALID_ARG, "null pointer");
   if (head_dim != kD) return msa_fail(MSA_ERR_INVALID_ARG, "head_dim must be 128");
@@ -453,6 +459,16 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   const int arch = msa::current_device_is_sm100(nullptr);
   if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
   if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
+  return msa_ok();
+}
+
+// Enqueues the decode kernel (arguments already checked).
+msa_status launch_decode(const void* q, const void* k_new, const void* v_new, int32_t n_queries, int32_t n_layers,
+                         int32_t n_q_heads, int32_t n_kv_heads, void* local_k, void* local_v, int32_t* local_len,
+                         int32_t local_cap, const void* mem_kv, const int32_t* mem_len, int32_t max_mem_chunks,
+                         int32_t rope_pos_offset, float rope_theta, float softmax_scale, void* out, void* workspace,
+                         int32_t* dev_err, msa_stream_t stream) {
+  const int G = n_q_heads / n_kv_heads;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t units = (int64_t)n_queries * n_layers * n_kv_heads;
   const int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, msa::sm_count() / units));
@@ -461,11 +477,13 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   int* unit_count = reinterpret_cast<int*>(part + ws_floats(n_queries, n_layers, n_q_heads, n_kv_heads));
   int* query_count = unit_count + units;
   const dim3 grid(splits, n_kv_heads, n_queries * n_layers);
+  RopeFreq rf;
   const double log2_theta = log2((double)rope_theta);
+  for (int j = 0; j < kHalf; ++j) rf.w_over_pi[j] = exp2(-2.0 * (double)j / (double)kD * log2_theta) / M_PI;
   const float qscale = softmax_scale * kLog2e;
   // programmatic stream serialisation: the kernel may be scheduled before the previous
   // kernel on the stream finishes and waits for it (griddepcontrol.wait) before reading
-  // what a previous step wrote
+  // any input
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -482,7 +500,7 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
   MSA_CUDA_TRY(cudaLaunchKernelEx(                                                                                \
       &cfg, decode_mma_kernel<GG>, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k_new,                          \
       (const __nv_bfloat16*)v_new, n_layers, n_kv_heads, (__nv_bfloat16*)local_k, (__nv_bfloat16*)local_v,        \
-      local_len, local_cap, (const __nv_bfloat16*)mem_kv, mem_len, max_mem_chunks, rope_pos_offset, log2_theta,  \
+      local_len, local_cap, (const __nv_bfloat16*)mem_kv, mem_len, max_mem_chunks, rope_pos_offset, rf,          \
       qscale, splits, part, stat, unit_count, query_count, (__nv_bfloat16*)out, dev_err))
   switch (G) {
     case 1: MSA_DECODE_LAUNCH(1); break;
@@ -493,6 +511,23 @@ extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const 
 #undef MSA_DECODE_LAUNCH
   MSA_CUDA_TRY(cudaGetLastError());
   return msa_ok();
+}
+}  // namespace
+
+extern "C" msa_status msa_sparse_decode(const void* q, const void* k_new, const void* v_new, int32_t n_queries,
+                                        int32_t n_layers, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                        void* local_k, void* local_v, int32_t* local_len, int32_t local_cap,
+                                        const void* mem_kv, const int32_t* mem_len, int32_t max_mem_chunks,
+                                        int32_t rope_pos_offset, float rope_theta, float softmax_scale, void* out,
+                                        void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                                        msa_stream_t stream) {
+  const msa_status st = check_decode(q, k_new, v_new, n_queries, n_layers, n_q_heads, n_kv_heads, head_dim, local_k,
+                                     local_v, local_len, local_cap, mem_kv, mem_len, max_mem_chunks, rope_theta, out,
+                                     workspace, workspace_bytes);
+  if (st != MSA_OK) return st;
+  return launch_decode(q, k_new, v_new, n_queries, n_layers, n_q_heads, n_kv_heads, local_k, local_v, local_len,
+                       local_cap, mem_kv, mem_len, max_mem_chunks, rope_pos_offset, rope_theta, softmax_scale, out,
+                       workspace, dev_err, stream);
 }
 
 // ---------------------------------------------------------------------------- no-allocation entry
@@ -521,6 +556,9 @@ extern "C" msa_status msa_sparse_decode_static(const void* q, const void* k_new,
   if (need > MSA_DECODE_STATIC_SCRATCH_BYTES)
     return msa_fail(MSA_ERR_CAPACITY, "static decode scratch holds %u bytes, these sizes need %zu",
                     MSA_DECODE_STATIC_SCRATCH_BYTES, need);
+  const int arch = msa::current_device_is_sm100(nullptr);
+  if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
+  if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
   int dev = 0;
   MSA_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return msa_fail(MSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
@@ -534,12 +572,18 @@ extern "C" msa_status msa_sparse_decode_static(const void* q, const void* k_new,
     }
     scratch = g_scratch_addr[dev];
   }
+  // every check before anything is enqueued: a rejected call leaves the stream (and a
+  // graph being captured) untouched
+  const msa_status st = check_decode(q, k_new, v_new, n_queries, n_layers, n_q_heads, n_kv_heads, head_dim, local_k,
+                                     local_v, local_len, local_cap, mem_kv, mem_len, max_mem_chunks, rope_theta, out,
+                                     scratch, MSA_DECODE_STATIC_SCRATCH_BYTES);
+  if (st != MSA_OK) return st;
   // the arrival counters must start at zero: their place depends on the sizes, and the
   // array keeps whatever the previous call left there
   const size_t counters_at = ws_floats(n_queries, n_layers, n_q_heads, n_kv_heads) * sizeof(float);
   MSA_CUDA_TRY(cudaMemsetAsync(static_cast<unsigned char*>(scratch) + counters_at, 0, need - counters_at,
                                reinterpret_cast<cudaStream_t>(stream)));
-  return msa_sparse_decode(q, k_new, v_new, n_queries, n_layers, n_q_heads, n_kv_heads, head_dim, local_k, local_v,
-                           local_len, local_cap, mem_kv, mem_len, max_mem_chunks, rope_pos_offset, rope_theta,
-                           softmax_scale, out, scratch, MSA_DECODE_STATIC_SCRATCH_BYTES, dev_err, stream);
+  return launch_decode(q, k_new, v_new, n_queries, n_layers, n_q_heads, n_kv_heads, local_k, local_v, local_len,
+                       local_cap, mem_kv, mem_len, max_mem_chunks, rope_pos_offset, rope_theta, softmax_scale, out,
+                       scratch, dev_err, stream);
 }
