@@ -29,6 +29,7 @@
 #include "route_proj.cuh"
 #include "route_bound.cuh"
 #include "route_tc.cuh"
+#include "tc_common.cuh"
 
 MSA_DEFINE_LAST_ERROR(msa_route_last_error)
 
@@ -424,6 +425,249 @@ __global__ void __launch_bounds__(256) scan_kernel(const __nv_bfloat16* __restri
   }
 }
 
+__device__ __forceinline__ void rs_ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void rs_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------- 2a. scan (streaming, tensor cores)
+// The streaming scan of few-token queries (T_total <= 4 tokens, all queries of the call;
+// H <= 8 key heads).  Persistent, one CTA per SM, thirteen warps.  Warp 12 streams tiles
+// of 16 consecutive blocks of one layer into 6 shared-memory stages, one cp.async.bulk per
+// block row issued by lanes 0..15 (rows padded by 16 bytes, so that ldmatrix reads them
+// without bank conflicts; completion on mbarriers, every wait bounded).  Warps 0..11 are
+// six pairs; pair p takes the tiles p, p + 6, ..., always in the stage only it reads (so
+// no warp waits on a stage's next fill before the previous one), each warp of the pair
+// half of the key heads.  Per key head, on the tensor cores (mma.sync m16n8k16, fp32
+// accumulation, even and odd k-steps in two chains): A = 16 key rows x 16 dims (the stored
+// bf16 keys, exact); B = the query sums of up to 4 tokens as 8 columns, the bf16 value of
+// each token in columns 0..3 and its bf16 residual in 4..7 (about 16 mantissa bits).  The
+// rows' squared norms are summed in fp32 from the same A fragments; each head's dot is
+// scaled by 1 / max(||k||, 1e-8) and the heads summed, the second warp's half through
+// shared memory; the maximum over each query's tokens goes to m.  On a timeout the kernel
+// sets MSA_DEVERR_TIMEOUT, waits (bounded) for its own copies in flight and returns.
+constexpr int kScanPairs = 6;
+constexpr int kScanConsumers = 2 * kScanPairs;
+constexpr int kScanThreads = 32 * (kScanConsumers + 1);
+constexpr int kScanTile = 16;
+constexpr int kScanStages = kScanPairs;
+constexpr int kScanMmaTokens = 4;
+
+__device__ __forceinline__ void scan_bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+template <int H>
+struct ScanCfg {
+  static constexpr int kHW = H / 2;                       // key heads per warp
+  static constexpr int kRowBytes = H * kD * 2;
+  static constexpr int kStride = kRowBytes + 16;          // padded row in shared memory
+  static constexpr int kStageBytes = kScanTile * kStride;
+  static constexpr int kSmem = kScanStages * kStageBytes + kScanPairs * 2 * 32 * 16;  // + the pairs' exchange
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo_elem, float hi_elem) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int H>
+__global__ void __launch_bounds__(kScanThreads, 1) scan_mma_kernel(const __nv_bfloat16* __restrict__ kr_hat,
+                                                                   const float* __restrict__ qt, int L, int64_t C,
+                                                                   int T_total,
+                                                                   const __grid_constant__ QueryOffsets qo,
+                                                                   float* __restrict__ m, int32_t* dev_err) {
+  using K = ScanCfg<H>;
+  constexpr int R = H * kD;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ __align__(8) uint64_t full[kScanStages], empty[kScanStages];
+  __shared__ int abort_flag;
+  __shared__ int pair_ok[kScanPairs][2][2];  // per pair, tile parity, warp: its wait succeeded
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tpl = (C + kScanTile - 1) / kScanTile;  // tiles per layer
+  const int64_t tiles = (int64_t)L * tpl;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kScanStages; ++i) {
+      tc::mbar_init(tc::smem_u32(&full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&empty[i]), 2);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const uint32_t ring_base = tc::smem_u32(ring);
+
+  if (warp == kScanConsumers) {
+    // ------------------------------------------------------------ producer: lane 0 waits for
+    // a free stage and arms its barrier, then lanes 0..15 issue one row copy each
+    uint32_t armed = 0u, armed_phase = 0u;  // stages with copies issued, and their phase bit
+    bool ok = true;
+    int64_t i = 0;
+    for (int64_t u = blockIdx.x; u < tiles; u += gridDim.x, ++i) {
+      const int st = (int)(i % kScanStages);
+      const uint32_t ph = (uint32_t)((i / kScanStages) & 1);
+      bool got = true;
+      if (lane == 0) got = tc::mbar_wait(tc::smem_u32(&empty[st]), ph ^ 1u, &abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        ok = false;
+        break;
+      }
+      const int l = (int)(u / tpl);
+      const int64_t c0 = (u % tpl) * kScanTile;
+      const int n = (int)min((int64_t)kScanTile, C - c0);
+      const uint32_t fb = tc::smem_u32(&full[st]);
+      if (lane == 0) tc::mbar_arrive_expect_tx(fb, (uint32_t)n * K::kRowBytes);
+      __syncwarp();  // armed before any copy can complete on it
+      if (lane < n)
+        scan_bulk_copy(ring_base + st * K::kStageBytes + lane * K::kStride,
+                       kr_hat + ((int64_t)l * C + c0 + lane) * R, K::kRowBytes, fb);
+      armed |= 1u << st;
+      armed_phase = (armed_phase & ~(1u << st)) | (ph << st);
+    }
+    if (lane == 0) {
+      if (!ok) {
+        abort_flag = 1;
+        msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+      }
+      // no copy may still be writing this CTA's shared memory when it exits
+      for (int k = 0; k < kScanStages; ++k)
+        if ((armed >> k) & 1u) tc::mbar_drain(tc::smem_u32(&full[k]), (armed_phase >> k) & 1u);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int pair = warp >> 1, sub = warp & 1;
+  const int g = lane >> 2, t = lane & 3;
+  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lhalf = lane >> 4;
+  float4* xch = reinterpret_cast<float4*>(ring + kScanStages * K::kStageBytes) + pair * 2 * 32;
+  uint32_t bq[K::kHW][8][2];  // B fragments of this warp's heads (values in columns 0..3, residuals 4..7)
+  int cur_l = -1;
+  int64_t i = pair;  // this CTA's tile index
+  for (int64_t u = blockIdx.x + (int64_t)pair * gridDim.x, k = 0; u < tiles;
+       u += (int64_t)kScanPairs * gridDim.x, i += kScanPairs, ++k) {
+    const int l = (int)(u / tpl);
+    const int64_t c0 = (u % tpl) * kScanTile;
+    const int n = (int)min((int64_t)kScanTile, C - c0);
+    if (l != cur_l) {
+      // column g of B: token g & 3, its bf16 value (g < 4) or residual (g >= 4); rows
+      // k = 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1) of each 16-dim slice
+      const int tok = g & 3;
+      const bool lo = g >= 4;
+      const float* qrow = qt + ((int64_t)l * T_total + tok) * R;
+#pragma unroll
+      for (int j = 0; j < K::kHW; ++j)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          float x[4] = {0.f, 0.f, 0.f, 0.f};
+          if (tok < T_total) {
+            const int d0 = (sub * K::kHW + j) * kD + 16 * ks + 2 * t;
+            const float2 p = __ldg(reinterpret_cast<const float2*>(qrow + d0));
+            const float2 p8 = __ldg(reinterpret_cast<const float2*>(qrow + d0 + 8));
+            x[0] = p.x; x[1] = p.y; x[2] = p8.x; x[3] = p8.y;
+          }
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float hi = __bfloat162float(__float2bfloat16_rn(x[e]));
+            v[e] = lo ? x[e] - hi : x[e];
+          }
+          bq[j][ks][0] = pack_bf16x2(v[0], v[1]);
+          bq[j][ks][1] = pack_bf16x2(v[2], v[3]);
+        }
+      cur_l = l;
+    }
+    const int st = (int)(i % kScanStages);
+    const uint32_t ph = (uint32_t)((i / kScanStages) & 1);
+    // (warp-uniform; a failed wait raises the abort flag, the pair still meets at its
+    // barrier below, and both warps leave on the flags they exchange there)
+    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tc::smem_u32(&full[st]), ph, &abort_flag));
+    if (!ok) abort_flag = 1;
+    float tot[4] = {0.f, 0.f, 0.f, 0.f};  // rows g, g (tokens 2(t&1), +1), rows g+8, g+8
+    if (ok) {
+      const uint32_t arow = ring_base + st * K::kStageBytes + lrow * K::kStride + lhalf * 16;
+#pragma unroll
+      for (int j = 0; j < K::kHW; ++j) {
+        const int hh = sub * K::kHW + j;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd k-steps
+        float ss0 = 0.f, ss1 = 0.f;  // squared norms of rows g, g + 8 (this lane's elements)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t a[4];
+          rs_ldsm_x4(arow + (uint32_t)((hh * kD + 16 * ks) * 2), a);
+          if (ks & 1) rs_mma(acc2, a, bq[j][ks][0], bq[j][ks][1]);
+          else rs_mma(acc, a, bq[j][ks][0], bq[j][ks][1]);
+          const float2 f0 = msa::bf16x2_to_float2(a[0]), f1 = msa::bf16x2_to_float2(a[1]);
+          const float2 f2 = msa::bf16x2_to_float2(a[2]), f3 = msa::bf16x2_to_float2(a[3]);
+          ss0 = fmaf(f0.x, f0.x, ss0); ss0 = fmaf(f0.y, f0.y, ss0); ss0 = fmaf(f2.x, f2.x, ss0); ss0 = fmaf(f2.y, f2.y, ss0);
+          ss1 = fmaf(f1.x, f1.x, ss1); ss1 = fmaf(f1.y, f1.y, ss1); ss1 = fmaf(f3.x, f3.x, ss1); ss1 = fmaf(f3.y, f3.y, ss1);
+        }
+        ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);  // the row's 4 lanes t
+        ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
+        ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
+        ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
+        const float r0 = 1.0f / fmaxf(sqrtf(ss0), 1e-8f), r1 = 1.0f / fmaxf(sqrtf(ss1), 1e-8f);
+        // columns 2t, 2t+1: lanes t < 2 hold the values, lanes t >= 2 the residuals of the
+        // same tokens; the pair sum is the ~16-bit dot
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[e] += acc2[e];
+          acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 2);
+        }
+        tot[0] = fmaf(r0, acc[0], tot[0]);
+        tot[1] = fmaf(r0, acc[1], tot[1]);
+        tot[2] = fmaf(r1, acc[2], tot[2]);
+        tot[3] = fmaf(r1, acc[3], tot[3]);
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tc::smem_u32(&empty[st]));  // done with the stage
+    }
+    // the second warp's half of the heads, through shared memory (double-buffered by the
+    // pair's tile count, so one barrier per tile orders writes and reads)
+    if (sub == 1) xch[(k & 1) * 32 + lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
+    if (lane == 0) pair_ok[pair][k & 1][sub] = ok ? 1 : 0;
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory");
+    if (!(pair_ok[pair][k & 1][0] && pair_ok[pair][k & 1][1])) break;  // (the same in both warps)
+    if (sub == 1) continue;
+    const float4 o = xch[(k & 1) * 32 + lane];
+    tot[0] += o.x;
+    tot[1] += o.y;
+    tot[2] += o.z;
+    tot[3] += o.w;
+    // lane (g, t): tokens 2(t&1), 2(t&1)+1 of rows g, g+8; the other pair from lane t ^ 1
+    float oth[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oth[e] = __shfl_xor_sync(0xffffffffu, tot[e], 1);
+    if (t == 0) {
+      const float s0[4] = {tot[0], tot[1], oth[0], oth[1]};  // row g, tokens 0..3
+      const float s1[4] = {tot[2], tot[3], oth[2], oth[3]};  // row g + 8
+      for (int b = 0; b < qo.n; ++b) {
+        float b0 = -INFINITY, b1 = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kScanMmaTokens; ++q)
+          if (q >= qo.off[b] && q < qo.off[b + 1]) {
+            b0 = fmaxf(b0, s0[q]);
+            b1 = fmaxf(b1, s1[q]);
+          }
+        float* mrow = m + ((int64_t)b * L + l) * C + c0;
+        if (g < n) mrow[g] = b0;
+        if (g + 8 < n) mrow[g + 8] = b1;
+      }
+    }
+  }
+  if (lane == 0 && abort_flag) msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+}
+
 // ---------------------------------------------------------------------------- 2a'. exact fallback
 // The scan of the layers `only` marks (tensor path, 8 key heads), for every query: the
 // last resort when no filter could certify a layer's selection.  A token's query sum is
@@ -770,19 +1014,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_docs_kernel(const uint32_t* 
 // so every thread reads each query token with 16-byte loads; the key tile is written to
 // shared memory in the same order (rows of 64 k-steps x 32 bytes, 16-byte chunks XOR-
 // swizzled by row for conflict-free ldmatrix).
-
-__device__ __forceinline__ void rs_ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void rs_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 // grid (x, L, B), 256 threads: the blocks of all K2 candidates of (b, l), laid end to
 // end, are cut into tiles of kRsTile blocks; CTA x takes tiles x, x + gridDim.x, ...
@@ -1177,6 +1408,33 @@ __global__ void keys_to_out_kernel(const unsigned long long* __restrict__ keys, 
   }
 }
 
+// Query tokens (all queries of a call) the tensor-core streaming scan takes: up to 4 (its
+// B operand holds each token's bf16 value and residual in 8 columns), for 2, 4 or 8 key
+// heads (each warp of a pair keeps half of the heads' B fragments in registers).
+int scan_mma_tokens(int H) { return (H == 2 || H == 4 || H == 8) ? kScanMmaTokens : 0; }
+
+template <int H>
+msa_status launch_scan_mma_h(const __nv_bfloat16* kr, const float* qt, int L, int64_t C, int T_total,
+                             const QueryOffsets& qo, float* m, int32_t* dev_err, cudaStream_t s) {
+  using K = ScanCfg<H>;
+  MSA_CUDA_TRY(cudaFuncSetAttribute(scan_mma_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::kSmem));
+  const int64_t tiles = (int64_t)L * ((C + kScanTile - 1) / kScanTile);
+  const int grid = (int)(tiles < msa::sm_count() ? tiles : msa::sm_count());
+  scan_mma_kernel<H><<<grid, kScanThreads, K::kSmem, s>>>(kr, qt, L, C, T_total, qo, m, dev_err);
+  MSA_CUDA_TRY(cudaGetLastError());
+  return msa_ok();
+}
+
+// The tensor-core streaming scan for H <= 8 key heads and T_total <= scan_mma_tokens(H).
+msa_status launch_scan_mma(int H, int T_total, const __nv_bfloat16* kr, const float* qt, int L, int64_t C,
+                           const QueryOffsets& qo, float* m, int32_t* dev_err, cudaStream_t s) {
+  switch (H) {
+    case 2: return launch_scan_mma_h<2>(kr, qt, L, C, T_total, qo, m, dev_err, s);
+    case 4: return launch_scan_mma_h<4>(kr, qt, L, C, T_total, qo, m, dev_err, s);
+    default: return launch_scan_mma_h<8>(kr, qt, L, C, T_total, qo, m, dev_err, s);
+  }
+}
+
 }  // namespace
 
 extern "C" msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_queries, int32_t total_q_tokens,
@@ -1190,6 +1448,19 @@ extern "C" msa_status msa_route_topk_workspace_size(int32_t n_layers, int32_t n_
 }
 
 extern "C" int32_t msa_route_last_launch_count(void) { return g_launches; }
+
+extern "C" msa_status msa_route_wait_selftest(int64_t wait_ns, int32_t release_first, int32_t* dev_err,
+                                              msa_stream_t stream) {
+  if (!dev_err) return msa_fail(MSA_ERR_INVALID_ARG, "null pointer");
+  if (wait_ns < 1 || wait_ns > 10000000000ll) return msa_fail(MSA_ERR_INVALID_ARG, "wait_ns in [1, 1e10]");
+  const int arch = msa::current_device_is_sm100(nullptr);
+  if (arch < 0) return msa_fail(MSA_ERR_CUDA, "no CUDA device");
+  if (arch == 0) return msa_fail(MSA_ERR_UNSUPPORTED, "device is not sm_100");
+  if (route_tc::launch_wait_selftest((unsigned long long)wait_ns, release_first, dev_err,
+                                     reinterpret_cast<cudaStream_t>(stream)) != 0)
+    return msa_fail(MSA_ERR_CUDA, "self-test launch");
+  return msa_ok();
+}
 
 extern "C" msa_status msa_route_set_pair_mode(int32_t enabled) {
   g_pair_mode = enabled != 0;
@@ -1303,12 +1574,13 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + w.cand);
   const int H = n_kv_heads;
 
-  // Path: the CUDA-core scan while the query is a handful of tokens, tensor cores beyond
-  // (on the E4M3 keys when the caller has them).
+  // Path: the streaming scan while the query is a handful of tokens (those its tensor-core
+  // form takes), the tcgen05 filter GEMM beyond (on the E4M3 keys when the caller has them).
   int path = flags;
   if (path == MSA_ROUTE_AUTO)
-    path = (T_total <= route_tc::kScanMaxTokens && !layer_mean) ? MSA_ROUTE_SCAN
-                                                                 : (kr_f8 ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
+    path = (T_total <= scan_mma_tokens(n_kv_heads) && !layer_mean)
+               ? MSA_ROUTE_SCAN
+               : (kr_f8 ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
   if ((path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && !route_tc::supported(H)) {
     if (flags != MSA_ROUTE_AUTO || layer_mean)
       return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
@@ -1410,7 +1682,12 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
 
   if (n_chunks > 0) {
     if (g_prof_start) MSA_CUDA_TRY(cudaEventRecord(g_prof_start, s));
-    if (!tensor) {
+    if (!tensor && T_total <= scan_mma_tokens(H)) {
+      const msa_status st = launch_scan_mma(H, T_total, (const __nv_bfloat16*)kr_hat, qt_f32, n_layers, n_chunks,
+                                            qo, m, dev_err, s);
+      if (st != MSA_OK) return st;
+      ++g_launches;
+    } else if (!tensor) {
       int64_t warps = (int64_t)n_layers * n_chunks;
       int64_t blocks = (warps + 7) / 8;
       const int64_t cap = (int64_t)msa::sm_count() * 8;
