@@ -138,6 +138,15 @@ msa_status msa_route_topk_hidden(const void* hidden, const void* w_router_q, int
                                  void* workspace, size_t workspace_bytes, int32_t flags, int32_t* dev_err,
                                  msa_stream_t stream);
 
+/* Self test of the bounded waits that every tensor-core routing kernel uses (the MSA
+ * pages have no counterpart).  Enqueues one small kernel that takes tensor memory as those
+ * kernels do and waits on a barrier that nothing completes (unless release_first != 0,
+ * which completes it first), the wait bounded by wait_ns on the GPU's global timer.  On
+ * expiry the kernel ORs MSA_DEVERR_TIMEOUT into *dev_err (DEVICE int32), frees its tensor
+ * memory and returns, leaving the context usable: the exit path of the routing kernels,
+ * whose own limit is 2 s.  1 <= wait_ns <= 1e10.  Asynchronous on stream. */
+msa_status msa_route_wait_selftest(int64_t wait_ns, int32_t release_first, int32_t* dev_err, msa_stream_t stream);
+
 /* Number of kernel launches the last successful msa_route_topk on this thread enqueued
  * (for launch accounting). */
 int32_t msa_route_last_launch_count(void);

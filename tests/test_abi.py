@@ -111,3 +111,60 @@ def test_workspace_size_grows_with_bank(msa):
     a = msa.msa_route_topk_workspace_size(18, 1, 256, 8, 1000, 100, 16)
     b = msa.msa_route_topk_workspace_size(18, 1, 256, 8, 2000, 100, 16)
     assert b - a >= 18 * 1000 * 4 - 256
+
+
+# ----------------------------------------------------------------------------- prototypes
+_CTYPE = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "float": ctypes.c_float, "double": ctypes.c_double,
+          "size_t": ctypes.c_size_t, "msa_dtype": ctypes.c_int32, "msa_stream_t": ctypes.c_void_p}
+
+
+def _prototypes(header):
+    """{name: [parameter C types]} of every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", header)).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(msa_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",")]
+        params = [] if params == ["void"] or params == [""] else params
+        # a parameter's type: the declaration without its trailing name
+        out[m.group(1)] = [re.sub(r"\s*\b[A-Za-z_][A-Za-z_0-9]*$", "", p).strip() for p in params]
+    return out
+
+
+def _expected_ctype(c_type: str):
+    t = c_type.replace("const ", "").strip()
+    if "*" in t:
+        return ctypes.c_void_p
+    return _CTYPE[t]
+
+
+@pytest.mark.parametrize("lib", sorted(HEADERS))
+def test_binding_argtypes_follow_the_header_prototypes(msa, lib):
+    # every entry point the binding declares takes the header's parameters in the header's
+    # order and widths (pointers as c_void_p; char* and struct* count as pointers)
+    import top_kv_routing_b200.abi as abi
+    dll = getattr(abi, f"{lib}_lib")
+    protos = _prototypes(HEADERS[lib])
+    checked = 0
+    for name, params in protos.items():
+        fn = getattr(dll, name)
+        if fn.argtypes is None:
+            continue
+        got = [a if a not in (ctypes.c_char_p,) else ctypes.c_void_p for a in fn.argtypes]
+        want = [_expected_ctype(p) for p in params]
+        assert len(got) == len(want), (name, len(got), len(want))
+        for i, (g, w) in enumerate(zip(got, want)):
+            ok = g == w or (w is ctypes.c_void_p and (g is ctypes.c_void_p or isinstance(g, type) and
+                                                      issubclass(g, (ctypes._Pointer, ctypes.c_char_p))))
+            assert ok, (name, i, params[i], g, w)
+        checked += 1
+    assert checked >= 1
+
+
+def test_c_caller_compiled_against_the_headers(msa, tmp_path):
+    # a C program built against include/*.h calls every entry point through the headers'
+    # own prototypes with arguments the host checks must reject, and checks the statuses
+    exe = tmp_path / "abi_check"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), "-o",
+                    str(exe), os.path.join(ROOT, "tests", "abi_check.c"), "-ldl"], check=True)
+    out = subprocess.run([str(exe), msa.LIB_DIR], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout

@@ -69,6 +69,8 @@ route_lib.msa_route_filter_keys.restype = _i32
 route_lib.msa_route_topk.restype = _i32
 route_lib.msa_route_last_launch_count.restype = _i32
 route_lib.msa_route_last_error.restype = ctypes.c_char_p
+route_lib.msa_route_wait_selftest.argtypes = [_i64, _i32, _p, _p]
+route_lib.msa_route_wait_selftest.restype = _i32
 route_lib.msa_route_set_pair_mode.argtypes = [_i32]
 route_lib.msa_route_set_pair_mode.restype = _i32
 route_lib.msa_route_set_profile_events.argtypes = [_p, _p]
@@ -233,6 +235,12 @@ def msa_route_filter_keys(kr_hat, n_layers: int, n_chunks: int, n_kv_heads: int,
     st = route_lib.msa_route_filter_keys(_ptr(kr_hat), n_layers, n_chunks, n_kv_heads, head_dim, _ptr(kr_f8),
                                          _stream(stream))
     _check(st, "msa_route_filter_keys", route_lib, "msa_route_last_error")
+
+
+def msa_route_wait_selftest(wait_ns: int, release_first: bool, dev_err, stream=None) -> None:
+    """The bounded-wait self test of the routing library (include/msa_route.h)."""
+    st = route_lib.msa_route_wait_selftest(int(wait_ns), 1 if release_first else 0, _ptr(dev_err), _stream(stream))
+    _check(st, "msa_route_wait_selftest", route_lib, "msa_route_last_error")
 
 
 def msa_route_set_pair_mode(enabled: bool) -> None:

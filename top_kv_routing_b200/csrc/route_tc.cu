@@ -446,4 +446,47 @@ int launch(const LaunchArgs& a, cudaStream_t s, int* launches, const char** why)
   return r;
 }
 
+namespace {
+// One CTA of 64 threads, the set-up and exit path of the tensor-core kernels on their
+// own: warp 0 takes 32 columns of tensor memory, thread 0 waits on a barrier of count 1
+// that nothing arrives on (unless release_first), bounded by limit_ns on the global timer;
+// on expiry it sets MSA_DEVERR_TIMEOUT, and the tensor memory is freed before the kernel
+// returns.
+__global__ void __launch_bounds__(64) wait_selftest_kernel(unsigned long long limit_ns, int release_first,
+                                                           int32_t* dev_err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x / 32;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(tc::smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    tc::tmem_alloc<false>(tc::smem_u32(&tmem_slot), 32);
+    tc::tmem_relinquish<false>();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (threadIdx.x == 0) {
+    if (release_first) tc::mbar_arrive(tc::smem_u32(&bar));
+    if (!tc::mbar_wait(tc::smem_u32(&bar), 0, &abort_flag, limit_ns)) {
+      abort_flag = 1;
+      msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 0) tc::tmem_dealloc<false>(tmem_slot, 32);
+}
+}  // namespace
+
+int launch_wait_selftest(unsigned long long limit_ns, int release_first, int32_t* dev_err, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 64, 0, s>>>(limit_ns, release_first, dev_err);
+  return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
 }  // namespace route_tc

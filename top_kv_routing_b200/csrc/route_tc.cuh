@@ -70,4 +70,7 @@ struct LaunchArgs {
 // Enqueues the score kernel; returns 0 on success (launches += kernels enqueued).
 int launch(const LaunchArgs& a, cudaStream_t s, int* launches, const char** why);
 
+// Enqueues the bounded-wait self test (see msa_route_wait_selftest); 0 on success.
+int launch_wait_selftest(unsigned long long limit_ns, int release_first, int32_t* dev_err, cudaStream_t s);
+
 }  // namespace route_tc
