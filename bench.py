@@ -156,31 +156,26 @@ def set_bank_size(n_docs: int) -> None:
     N_DOCS, N_TOKENS = n_docs, n_docs * TOKENS_PER_DOC
 
 
-def make_workload(dev, host_store_chunks: int, f8: bool):
+def build_keys(dev, seed: int, bank, f8: bool):
+    """Routing keys of every layer on the device: pooled-level draws (topic + noise/8) made
+    unit per head by the pool kernel with 1-token blocks (no rotation), plus the E4M3
+    filter copy.  Returns (kr_hat, kr_f8 or None, filter-key ms or None, topic)."""
     import torch
 
     import msa_synth as syn
     import top_kv_routing_b200 as msa
-
-    t0 = time.time()
-    lens = syn.doc_lengths_exact_total(SEED, N_DOCS, N_TOKENS)
-    bank = syn.make_bank(SEED, N_DOCS, lens, L)
     C = bank.n_chunks
     coffs = bank.doc_chunk_offsets
     topic = torch.from_numpy(bank.topic).to(dev)
-    # routing keys: pooled-level draws (topic + noise/8), made unit per head by the pool
-    # kernel with 1-token blocks (no rotation)
     kr_hat = torch.empty((L, C, H, D), dtype=torch.bfloat16, device=dev)
     scratch = torch.empty((C, H, D), dtype=torch.bfloat16, device=dev)
     row_topic = torch.from_numpy(syn.chunk_docs(coffs)).to(dev)
     ones = torch.arange(C + 1, dtype=torch.int64, device=dev)
     for l in range(L):
-        syn.device_fill(scratch, SEED, syn.STREAM_KRBAR, l, 0, 0, C, H * D, syn.POOLED_NOISE, topic, row_topic)
+        syn.device_fill(scratch, seed, syn.STREAM_KRBAR, l, 0, 0, C, H * D, syn.POOLED_NOISE, topic, row_topic)
         msa.msa_pool_blocks(None, None, scratch, ones, ones, C, C, H, D, 1, 0.0, None, None, kr_hat[l], None, None,
                             in_dtype=msa.MSA_BF16)
     del scratch, row_topic, ones
-    torch.cuda.synchronize(dev)
-    log(f"routing keys ready: {C} blocks x {L} layers ({kr_hat.numel() * 2 / 1e9:.1f} GB) in {time.time() - t0:.1f}s")
     kr_f8, f8_ms = None, None
     if f8:
         # the E4M3 filter copy of the keys (built once per bank, like the keys themselves)
@@ -191,22 +186,79 @@ def make_workload(dev, host_store_chunks: int, f8: bool):
         e1.record()
         torch.cuda.synchronize(dev)
         f8_ms = e0.elapsed_time(e1)
+    torch.cuda.synchronize(dev)
+    return kr_hat, kr_f8, f8_ms, topic
+
+
+def mem_available_gb() -> float | None:
+    """MemAvailable of this host (GB), or None where /proc/meminfo is absent."""
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    return int(line.split()[1]) * 1024 / 1e9
+    except OSError:
+        return None
+    return None
+
+
+def host_cores() -> dict:
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        aff = None
+    return {"nproc": aff or os.cpu_count(), "cpu_count": os.cpu_count()}
+
+
+def store_blocks_to_use(requested: int | None, C: int) -> tuple[int, str]:
+    """Physical blocks per layer of the page-locked content store: the whole bank (every
+    document at its own blocks) when the host has room for it with 24 GB to spare, else a
+    smaller store read at hashed per-document offsets (the same bytes move per query)."""
+    if requested is not None:
+        return min(requested, C), "requested on the command line"
+    need = L * C * 2 * H * D * 2 / 1e9
+    avail = mem_available_gb()
+    if avail is None or avail >= need + 24:
+        return C, f"whole bank ({need:.1f} GB; host MemAvailable {avail if avail is None else round(avail, 1)} GB)"
+    P = 163_840
+    return min(P, C), (f"host MemAvailable {avail:.1f} GB < {need:.1f} GB + 24 GB: {P} blocks per layer at "
+                       "hashed document offsets")
+
+
+def make_workload(dev, host_store_chunks: int | None, f8: bool):
+    import torch
+
+    import msa_synth as syn
+
+    t0 = time.time()
+    lens = syn.doc_lengths_exact_total(SEED, N_DOCS, N_TOKENS)
+    bank = syn.make_bank(SEED, N_DOCS, lens, L)
+    C = bank.n_chunks
+    coffs = bank.doc_chunk_offsets
+    kr_hat, kr_f8, f8_ms, topic = build_keys(dev, SEED, bank, f8)
+    log(f"routing keys ready: {C} blocks x {L} layers ({kr_hat.numel() * 2 / 1e9:.1f} GB) in {time.time() - t0:.1f}s")
+    if f8_ms is not None:
         log(f"E4M3 filter keys: {kr_f8.numel() / 1e9:.1f} GB in {f8_ms:.1f} ms")
-    # content store: host_store_chunks physical blocks per layer; document d reads the
+    # content store: P physical blocks per layer; with P < C document d reads the
     # contiguous physical range starting at a hashed offset (same bytes per selection)
-    P = min(host_store_chunks, C)
+    P, why = store_blocks_to_use(host_store_chunks, C)
     per_doc = np.diff(coffs)
     h = syn.hashes(syn.tensor_key(SEED, syn.STREAM_TARGETS, 0, 99), np.arange(N_DOCS, dtype=np.uint64))
     store_off = (h % np.uint64(max(1, P - int(per_doc.max())))).astype(np.int64) if P < C else coffs[:-1].copy()
+    t1 = time.time()
     host_kv = torch.empty((L, P, 2, H, D), dtype=torch.bfloat16, pin_memory=True)
+    pin_s = time.time() - t1
     stage = torch.empty((2, P, H * D), dtype=torch.bfloat16, device=dev)
     for l in range(L):
         syn.device_fill(stage[0], SEED, syn.STREAM_KBAR, l, 0, 0, P, H * D, syn.POOLED_NOISE)
         syn.device_fill(stage[1], SEED, syn.STREAM_VBAR, l, 0, 0, P, H * D, syn.POOLED_NOISE)
         host_kv[l].copy_(stage.permute(1, 0, 2).reshape(P, 2, H, D))
     del stage
-    log(f"host content store: {P} blocks x {L} layers ({host_kv.numel() * 2 / 1e9:.1f} GB pinned)")
-    return bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic
+    torch.cuda.empty_cache()
+    store = {"blocks_per_layer": int(P), "gb_pinned": round(host_kv.numel() * 2 / 1e9, 1), "choice": why,
+             "pin_s": round(pin_s, 1), "fill_s": round(time.time() - t1 - pin_s, 1)}
+    log(f"host content store: {P} blocks x {L} layers ({store['gb_pinned']} GB pinned in {pin_s:.1f} s)")
+    return bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic, store
 
 
 def make_queries(dev, bank, topic, n_queries: int):
@@ -461,6 +513,229 @@ def time_tail_parts(eng, slot, dq, dk, dv, dev):
                                "are L2-resident after the first step"}}
 
 
+def _route_timed(msa, dev, qr, q_off, kr_hat, kr_f8, coffs, n_docs, C, k, flags, ws, reps=4, warm=2):
+    """Direct route calls: median device time of the whole call and of its score kernel
+    (the library's events around the scan or the GEMM), plus the last ids / dev_err."""
+    import torch
+    B = len(q_off) - 1
+    ids = torch.empty((B, L, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, L, k), device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    g1.record()
+    torch.cuda.synchronize(dev)
+    whole, score = [], []
+    msa.msa_route_set_profile_events(g0, g1)
+    try:
+        for r in range(warm + reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(1_000_000)  # the GPU is busy while the host prepares the call
+            a.record()
+            msa.msa_route_topk(qr, q_off, kr_hat, coffs, n_docs, C, L, HQ, H, D, k, ids, sc, ws, flags=flags,
+                               dev_err=err, kr_f8=kr_f8)
+            b.record()
+            torch.cuda.synchronize(dev)
+            if r >= warm:
+                whole.append(a.elapsed_time(b))
+                score.append(g0.elapsed_time(g1))
+    finally:
+        msa.msa_route_set_profile_events(None, None)
+    return sorted(whole)[len(whole) // 2], sorted(score)[len(score) // 2], ids, int(err.item())
+
+
+def _roof(C: int, T: int, ms: float, elem: int, f8: bool):
+    """Algorithmic bytes / flops of one routing pass over C blocks x L layers for a T-token
+    query, and the fractions of the measured peaks they reach in ms (tensor peak: bf16
+    burst, x 2 for E4M3 operands, the nominal dense ratio)."""
+    hbm, bf16_burst, _, src = measured_peaks()
+    by = L * C * H * D * elem
+    fl = 2.0 * T * H * D * L * C
+    gbs = by / ms / 1e6
+    tf = fl / ms / 1e9
+    tc_peak = bf16_burst * (2.0 if f8 else 1.0)
+    return {"ms": round(ms, 4), "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 4),
+            "frac_of_nominal_8tbs": round(gbs / 8000.0, 4), "tflops": round(tf, 1),
+            "tensor_frac_of_burst": round(tf / tc_peak, 4), "peaks": src}
+
+
+def time_bf16_filter(dev, eng, qs):
+    """The step's route with the bf16 filter (MSA_ROUTE_TENSOR) instead of E4M3, on the same
+    bank and query, timed by direct calls: whole route and its GEMM."""
+    import top_kv_routing_b200 as msa
+    slot = eng.slots[0]
+    slot.qr.copy_(qs[0])
+    whole, gemm, ids, err = _route_timed(msa, dev, slot.qr, [0, T], eng.kr_hat, None, eng.doc_chunk_offsets,
+                                         eng.n_docs, eng.C, eng.k, msa.MSA_ROUTE_TENSOR, slot.ws)
+    out = {"route_ms": round(whole, 4), "gemm": _roof(eng.C, T, gemm, 2, False), "dev_err": err,
+           "timing": "direct calls, CUDA events (library hook around the GEMM); median of 4 after 2 warm-up"}
+    return out
+
+
+SWEEP_T = (1, 2, 4, 8, 64, 256, 1024)  # the workload's sweep {1, 8, 64, 256, 1024} plus 2 and 4
+
+
+def time_sweep(dev, f8: bool):
+    """Query-length sweep on the 10M-token bank (10,000 documents, lognormal lengths, seed
+    2): for every T the scan (T <= 64), the bf16 GEMM filter and the E4M3 GEMM filter, each
+    timed as a whole route and as its score kernel, with the planted documents' recall;
+    and which path MSA_ROUTE_AUTO takes."""
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+    seed, n_docs = 2, 10_000
+    lens = syn.doc_lengths_lognormal(seed, n_docs)
+    bank = syn.make_bank(seed, n_docs, lens, L)
+    C = bank.n_chunks
+    kr_hat, kr_f8, _, topic = build_keys(dev, seed, bank, f8)
+    coffs = torch.from_numpy(bank.doc_chunk_offsets).to(dev)
+    targets = syn.pick_targets(seed, n_docs, TOPK, sub=0)
+    points = []
+    for Tq in SWEEP_T:
+        q = torch.empty((L, Tq, HQ, D), dtype=torch.bfloat16, device=dev)
+        rt = torch.from_numpy(np.repeat(targets[np.arange(Tq) % TOPK], HQ).astype(np.int32)).to(dev)
+        for l in range(L):
+            syn.device_fill(q[l], seed, syn.STREAM_QR, l, 0, 0, Tq * HQ, D, 0.5, topic, rt)
+        ws = torch.empty(msa.msa_route_topk_workspace_size(L, 1, Tq, H, C, n_docs, TOPK), dtype=torch.uint8,
+                         device=dev)
+        want = set(targets[:min(Tq, TOPK)].tolist())
+        row = {"T": Tq, "auto_path": "scan" if Tq <= 4 else ("tensor_e4m3" if f8 else "tensor_bf16")}
+        paths = [("scan", msa.MSA_ROUTE_SCAN, None, 2, False)] if Tq <= 64 else []
+        paths += [("tensor_bf16", msa.MSA_ROUTE_TENSOR, None, 2, False)]
+        if f8:
+            paths += [("tensor_e4m3", msa.MSA_ROUTE_TENSOR_F8, kr_f8, 1, True)]
+        for name, flags, f8k, elem, is_f8 in paths:
+            whole, score, ids, err = _route_timed(msa, dev, q, [0, Tq], kr_hat, f8k, coffs, n_docs, C, TOPK, flags, ws)
+            got = ids.cpu().numpy()[0]
+            rec = float(np.mean([len(want & set(got[l].tolist())) / len(want) for l in range(L)]))
+            row[name] = {"route_ms": round(whole, 4), "score_kernel": _roof(C, Tq, score, elem, is_f8),
+                         "planted_recall": round(rec, 4), "dev_err": err}
+        points.append(row)
+        del q, ws
+    # crossover: the smallest T at which a tensor path's whole route beats the scan's
+    cross = None
+    for row in points:
+        if "scan" in row:
+            best_t = min(row[n]["route_ms"] for n in ("tensor_bf16", "tensor_e4m3") if n in row)
+            if best_t < row["scan"]["route_ms"] and cross is None:
+                cross = row["T"]
+    del kr_hat, kr_f8
+    torch.cuda.empty_cache()
+    return {"bank": f"10M-token bank: {n_docs} documents, lognormal lengths (median 900, sigma 0.5), {C} blocks x "
+                    f"{L} layers", "blocks": C, "points": points,
+            "first_T_where_tensor_route_beats_scan": cross,
+            "timing": "direct calls, CUDA events; score_kernel = the scan or GEMM alone (library hook)"}
+
+
+def time_interleave(dev, host_kv, f8: bool):
+    """Multi-round interleave on the 10M-token bank: 64 queries of 128 router tokens, each
+    planted with a chain of three documents A -> B -> C (the router vectors of the first
+    128 tokens carry A); round r routes over all of each query's tokens so far (128 + 512 r),
+    gathers the selections for all 64 queries, decodes 32 tokens; between rounds 512 local
+    tokens are appended per query whose router vectors carry the next chain document.
+    Reports per round the route, gather and decode device times and the chain recovery
+    (fraction of (query, layer) selections holding the chain so far)."""
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+    seed, n_docs, B, T0, A, R, DEC_R, k = 4, 10_000, 64, 128, 512, 3, 32, 16
+    lens = syn.doc_lengths_lognormal(2, n_docs)
+    bank = syn.make_bank(2, n_docs, lens, L)
+    C = bank.n_chunks
+    coffs_np = bank.doc_chunk_offsets
+    kr_hat, kr_f8, _, topic = build_keys(dev, 2, bank, f8)
+    coffs = torch.from_numpy(coffs_np).to(dev)
+    P = host_kv.shape[1]
+    per_doc = np.diff(coffs_np)
+    h = syn.hashes(syn.tensor_key(seed, syn.STREAM_TARGETS, 0, 98), np.arange(n_docs, dtype=np.uint64))
+    store_off = torch.from_numpy((h % np.uint64(max(1, P - int(per_doc.max())))).astype(np.int64)).to(dev)
+    chains = [syn.pick_targets(seed, n_docs, 3, sub=b) for b in range(B)]
+    cap = T0 + R * DEC_R + (R - 1) * A
+    M = k * int(per_doc.max())
+    mem = torch.zeros((B, L, 2, H, M, D), dtype=torch.bfloat16, device=dev)
+    mem_len = torch.zeros((B, L), dtype=torch.int32, device=dev)
+    lk = torch.zeros((B, L, H, cap, D), dtype=torch.bfloat16, device=dev)
+    lv = torch.zeros_like(lk)
+    llen = torch.zeros(B, dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_dec = torch.zeros(msa.msa_sparse_decode_workspace_size(B, L, HQ, H), dtype=torch.uint8, device=dev)
+    seg = torch.empty((L * H * A, D), dtype=torch.bfloat16, device=dev)
+    dq = torch.empty((DEC_R, B, L, HQ, D), dtype=torch.bfloat16, device=dev)
+    dk = torch.empty((DEC_R, B, L, H, D), dtype=torch.bfloat16, device=dev)
+    dv = torch.empty_like(dk)
+    out = torch.empty((B, L, HQ, D), dtype=torch.bfloat16, device=dev)
+
+    def append_local(r, n):
+        for b in range(B):
+            pos = int(llen[b].item())
+            for stream, cache in ((syn.STREAM_LOCAL_K, lk), (syn.STREAM_LOCAL_V, lv)):
+                syn.device_fill(seg[:L * H * n], seed, stream, r, b, 0, L * H * n, D)
+                cache[b, :, :, pos:pos + n] = seg[:L * H * n].view(L, H, n, D)
+            llen[b] += n
+
+    def fill_q(dst, b, tok0, n, doc):
+        rt = torch.full((n * HQ,), int(doc), dtype=torch.int32, device=dev)
+        for l in range(L):
+            syn.device_fill(dst[l], seed, syn.STREAM_QR, l, b, tok0 * HQ, n * HQ, D, 0.5, topic, rt)
+
+    append_local(0, T0)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    rounds = []
+    for r in range(R):
+        Tq = T0 + r * A
+        qr = torch.empty((L, B * Tq, HQ, D), dtype=torch.bfloat16, device=dev)
+        for b in range(B):
+            fill_q(qr[:, b * Tq:b * Tq + T0], b, 0, T0, chains[b][0])
+            for rr in range(1, r + 1):
+                t0 = T0 + (rr - 1) * A
+                fill_q(qr[:, b * Tq + t0:b * Tq + t0 + A], b, t0, A, chains[b][rr])
+        offs = [b * Tq for b in range(B + 1)]
+        ws = torch.empty(msa.msa_route_topk_workspace_size(L, B, B * Tq, H, C, n_docs, k), dtype=torch.uint8,
+                         device=dev)
+        ids = torch.empty((B, L, k), dtype=torch.int32, device=dev)
+        sc = torch.empty((B, L, k), device=dev)
+        for s_ in range(DEC_R):
+            step = r * DEC_R + s_
+            syn.device_fill(dq[s_], seed, syn.STREAM_DEC_Q, step, 0, 0, B * L * HQ, D)
+            syn.device_fill(dk[s_], seed, syn.STREAM_DEC_K, step, 0, 0, B * L * H, D)
+            syn.device_fill(dv[s_], seed, syn.STREAM_DEC_V, step, 0, 0, B * L * H, D)
+        torch.cuda.synchronize(dev)
+        e = [ev() for _ in range(4)]
+        e[0].record()
+        msa.msa_route_topk(qr, offs, kr_hat, coffs, n_docs, C, L, HQ, H, D, k, ids, sc, ws, dev_err=err, kr_f8=kr_f8)
+        e[1].record()
+        msa.msa_gather_kv(host_kv, P, coffs, store_off, n_docs, ids, B, L, k, H, D, M, mem, mem_len, dev_err=err)
+        e[2].record()
+        for s_ in range(DEC_R):
+            msa.msa_sparse_decode(dq[s_], dk[s_], dv[s_], B, L, HQ, H, D, lk, lv, llen, cap, mem, mem_len, M, k, THETA,
+                                  D ** -0.5, out, ws_dec, dev_err=err)
+        e[3].record()
+        torch.cuda.synchronize(dev)
+        got = ids.cpu().numpy()
+        rec = float(np.mean([set(chains[b][:r + 1].tolist()) <= set(got[b, l].tolist())
+                             for b in range(B) for l in range(L)]))
+        g_bytes = int(mem_len.sum().item()) * 2 * H * D * 2
+        g_ms = e[1].elapsed_time(e[2])
+        rounds.append({"round": r, "router_tokens_per_query": Tq, "route_ms": round(e[0].elapsed_time(e[1]), 3),
+                       "gather_ms": round(g_ms, 3), "gather_gbs": round(g_bytes / g_ms / 1e6, 1),
+                       "decode_ms": round(e[2].elapsed_time(e[3]), 3),
+                       "decode_us_per_step": round(e[2].elapsed_time(e[3]) * 1e3 / DEC_R, 2),
+                       "round_ms": round(e[0].elapsed_time(e[3]), 3), "chain_recovery": round(rec, 4),
+                       "dev_err": int(err.item())})
+        del qr, ws
+        if r + 1 < R:
+            append_local(r + 1, A)
+    del kr_hat, kr_f8, mem, lk, lv, seg
+    torch.cuda.empty_cache()
+    return {"bank": f"10M-token bank ({n_docs} documents, {C} blocks x {L} layers)", "queries": B,
+            "first_tokens": T0, "appended_per_round": A, "decode_per_round": DEC_R, "rounds": rounds,
+            "filter": "E4M3" if f8 else "bf16",
+            "store": f"page-locked host store of {P} blocks per layer at hashed document offsets",
+            "timing": "CUDA events around one route (64 queries), one gather, 32 decode launches per round"}
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args):
@@ -480,8 +755,9 @@ def run_gpu(args):
     prefill = time_prefill(dev) if (rank == 0 and not args.no_prefill) else None
     torch.cuda.empty_cache()
     f8 = args.filter == "e4m3"
-    bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic = make_workload(dev, args.host_store_blocks, f8)
+    bank, kr_hat, kr_f8, f8_ms, host_kv, store_off, topic, store = make_workload(dev, args.host_store_blocks, f8)
     qs, targets = make_queries(dev, bank, topic, args.queries)
+    n_distinct = len(qs)
     dq, dk, dv, pk, pv = make_decode_inputs(dev)
     n_slots = args.pipeline
     dec_inputs = [(dq.clone(), dk.clone(), dv.clone(), torch.empty((DEC, 1, L, HQ, D), dtype=torch.bfloat16,
@@ -653,12 +929,25 @@ def run_gpu(args):
     d2h = host["ids"][0].numel() * 4 + host["scores"][0].numel() * 4 + host["out"][0].numel() * 2
     # routing from hidden states (fused router projection), after the timed regions
     projection = time_projection(dev, bank, kr_hat, kr_f8) if (rank == 0 and not args.no_projection) else None
-    tail_parts = None
+    tail_parts = bf16_filter = sweep = interleave = None
     if rank == 0:
-        try:
-            tail_parts = time_tail_parts(eng, slot0, dq, dk, dv, dev)
-        except Exception as e:  # (a separate measurement: never at the cost of the line)
-            tail_parts = {"error": f"{type(e).__name__}: {e}"}
+        def guarded(fn, *a):
+            try:
+                return fn(*a)
+            except Exception as e:  # (a separate measurement: never at the cost of the line)
+                return {"error": f"{type(e).__name__}: {e}"}
+        tail_parts = guarded(time_tail_parts, eng, slot0, dq, dk, dv, dev)
+        if f8 and not args.no_bf16_filter:
+            bf16_filter = guarded(time_bf16_filter, dev, eng, qs)
+    # the 100M bank's device buffers go before the 10M-bank measurements (the host store stays)
+    del eng, slot0, kr_hat, kr_f8, qs, dec_inputs, stage_in, stage_out
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    if rank == 0:
+        if not args.no_sweep:
+            sweep = guarded(time_sweep, dev, f8)
+        if not args.no_interleave:
+            interleave = guarded(time_interleave, dev, host_kv, f8)
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
     if world > 1:
@@ -676,8 +965,8 @@ def run_gpu(args):
     flops = 2.0 * T * H * D * L * bank.n_chunks
     tflops = flops / (gemm_avg / 1e3) / 1e12
     # tensor peak of the operand type: E4M3 = 2 x the measured bf16 figure (the nominal
-    # dense ratio); sustained, as the GEMM runs for milliseconds back to back
-    tc_peak = (bf16_sus or bf16_peak) * (2.0 if f8 else 1.0)
+    # dense ratio); the burst figure, as the GEMM is timed by isolated direct calls
+    tc_peak = bf16_peak * (2.0 if f8 else 1.0)
     t_hbm = algo_bytes / (hbm_peak * 1e9)
     t_tc = flops / (tc_peak * 1e12)
     bound = "tensor" if t_tc > t_hbm else "hbm"
@@ -703,7 +992,8 @@ def run_gpu(args):
                               "bf16 keys, tcgen05 kind::f16; top candidates rescored exactly in fp32"),
                    "n_docs": N_DOCS, "n_tokens": N_TOKENS, "n_blocks": bank.n_chunks,
                    "layers": L, "kv_heads": H, "q_heads": HQ, "head_dim": D, "query_tokens": T, "top_k": TOPK,
-                   "decode_tokens": DEC, "distinct_queries": len(qs), "host_store_blocks": int(host_kv.shape[1]),
+                   "decode_tokens": DEC, "distinct_queries": n_distinct, "host_store_blocks": int(host_kv.shape[1]),
+                   "host_store": store,
                    "l2": f"inputs larger than L2 ({algo_bytes / 1e9:.1f} GB of routing keys stream through every step)",
                    "graph": "per query two CUDA graphs: route; gather + 128 decode steps",
                    "pipeline": (f"{n_slots} query slots: the gather+decode of query i overlaps the route of "
@@ -719,9 +1009,13 @@ def run_gpu(args):
                      "peak": round(tc_peak if bound == "tensor" else hbm_peak, 1),
                      "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
                      "frac": round(tflops / tc_peak if bound == "tensor" else achieved / hbm_peak, 4),
-                     "peak_source": (f"{peak_src}: " + ("sustained bf16 x 2 (E4M3/bf16 nominal ratio)" if f8 else
-                                                        "sustained bf16") if bound == "tensor" else
+                     "peak_source": (f"{peak_src}: " + ("bf16 burst x 2 (E4M3/bf16 nominal ratio)" if f8 else
+                                                        "bf16 burst") if bound == "tensor" else
                                      f"{peak_src}: HBM copy"),
+                     "timing": "score GEMM alone, direct calls between steps (CUDA events the route library "
+                               "records around it); burst peak for an isolated kernel",
+                     "tensor_frac_of_sustained": round(tflops / (bf16_sus * (2.0 if f8 else 1.0)), 4)
+                     if bf16_sus else None,
                      "traffic": None if traffic_pbl is None else round(traffic_pbl * L * bank.n_chunks),
                      "traffic_source": ("ncu dram bytes of a 2M-token launch scaled by blocks" if traffic_pbl
                                         else "not captured for this kernel yet"),
@@ -743,6 +1037,11 @@ def run_gpu(args):
         "dev_err": dev_err,
         "filter_keys_ms": None if f8_ms is None else round(f8_ms, 2),
         "ids_match_bf16_filter": same_as_bf16,
+        "bf16_filter": bf16_filter,
+        "sweep": sweep,
+        "interleave": interleave,
+        "host": dict(host_cores(), mem_available_gb=None if mem_available_gb() is None else
+                     round(mem_available_gb(), 1)),
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -783,13 +1082,28 @@ def cpu_baseline(seconds: float):
     value = nb * 64 / L / dt
     return {"value": round(value, 3), "unit": "bank tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"layer 0 of 18, first {nb} of 1,562,500 blocks, T=256 query, explicit cosine form "
-                      f"({dt:.1f} s); rate scaled to all 18 layers", "setup_s": round(t0 - t_probe, 1)}
+                      f"({dt:.1f} s); rate scaled to all 18 layers", "setup_s": round(t0 - t_probe, 1),
+            "host_nproc": host_cores()["nproc"]}
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    """The oracle on a bounded sample, on rank 0; with several ranks (gloo, host only) the
+    others wait for it at a barrier and print nothing."""
+    world, rank, _ = rank_env()
+    if world > 1:
+        import torch.distributed as dist
+        init_ranks("gloo", timeout_s=1800)
+        try:
+            if rank == 0:
+                _reference_line(args, world)
+            dist.barrier()
+        finally:
+            dist.destroy_process_group()
         return
+    _reference_line(args, 1)
+
+
+def _reference_line(args, world: int):
     vals = []
     for _ in range(args.warmup):
         cpu_baseline(min(2.0, args.cpu_seconds))
@@ -799,12 +1113,12 @@ def run_reference(args):
     step_ms = (time.time() - t0) * 1e3 / max(1, args.steps)
     v = float(np.mean([x["value"] for x in vals]))
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "bank tokens/s",
-            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(step_ms, 1), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD},
             "cpu_baseline": {"value": round(v, 3), "unit": "bank tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": vals[0]["sample"]},
+                             "sample": vals[0]["sample"], "host_nproc": host_cores()["nproc"]},
             "e2e": {"value": round(v, 3), "unit": "bank tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -816,9 +1130,14 @@ def main():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--queries", type=int, default=4, help="distinct synthetic queries cycled over the steps")
-    ap.add_argument("--host-store-blocks", type=int, default=163_840,
-                    help="physical blocks per layer in the page-locked content store")
+    ap.add_argument("--queries", type=int, default=16, help="distinct synthetic queries cycled over the steps")
+    ap.add_argument("--host-store-blocks", type=int, default=None,
+                    help="physical blocks per layer in the page-locked content store (default: the whole bank "
+                         "when the host has room for it)")
+    ap.add_argument("--no-bf16-filter", action="store_true", help="skip the bf16-filter route measurement")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the query-length sweep on the 10M-token bank")
+    ap.add_argument("--no-interleave", action="store_true",
+                    help="skip the multi-round interleave measurement on the 10M-token bank")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool", action="store_true", help="skip the separate pooling measurement")
@@ -832,11 +1151,30 @@ def main():
     ap.add_argument("--docs", type=int, default=N_DOCS,
                     help="documents in the bank (x1000 tokens); smaller banks serve profiling captures")
     args = ap.parse_args()
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(spawn_ranks(args.gpus))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        log(f"bench.py: --gpus {args.gpus} but the launcher started {world} ranks")
+        sys.exit(2)
     set_bank_size(args.docs)
     if args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
+
+
+def spawn_ranks(n: int) -> int:
+    """--gpus N without a launcher: starts N local ranks of this same command under
+    torch.distributed.run (rendezvous on 127.0.0.1); rank 0 prints the line.  Returns the
+    launcher's exit status."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 if __name__ == "__main__":
