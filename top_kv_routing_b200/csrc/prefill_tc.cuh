@@ -6,6 +6,11 @@
 
 namespace prefill_tc {
 
+// RoPE frequencies of one call, theta^(-2j/128) / pi for j < 64 (fp64), computed on the host.
+struct RopeW {
+  double w_over_pi[64];
+};
+
 struct Args {
   const __nv_bfloat16* q;       // [B][L][T][H*G][128]
   __nv_bfloat16* out;           // [B][L][T][H*G][128]
