@@ -628,6 +628,48 @@ def time_sweep(dev, f8: bool):
             "timing": "direct calls, CUDA events; score_kernel = the scan or GEMM alone (library hook)"}
 
 
+def time_scan(dev, n_blocks: int = 1_000_000, calls: int = 3):
+    """The streaming scan alone on one layer of n_blocks blocks x 8 key heads (2 GB of bf16
+    routing keys at 1M blocks, larger than L2): a one-token query, documents of 10 blocks,
+    MSA_ROUTE_SCAN, `calls` whole routes timed with CUDA events.  The workload of the scan
+    kernel's ncu capture."""
+    import torch
+
+    import msa_synth as syn
+    import top_kv_routing_b200 as msa
+    C, seed = n_blocks, 5
+    kr = torch.empty((1, C, H, D), dtype=torch.bfloat16, device=dev)
+    scratch = torch.empty((C, H, D), dtype=torch.bfloat16, device=dev)
+    syn.device_fill(scratch, seed, syn.STREAM_KRBAR, 0, 0, 0, C, H * D, syn.POOLED_NOISE)
+    ones = torch.arange(C + 1, dtype=torch.int64, device=dev)
+    msa.msa_pool_blocks(None, None, scratch, ones, ones, C, C, H, D, 1, 0.0, None, None, kr[0], None, None,
+                        in_dtype=msa.MSA_BF16)
+    del scratch, ones
+    n_docs = C // 10
+    coffs = torch.arange(0, C + 1, 10, dtype=torch.int64, device=dev)
+    q = torch.from_numpy(syn.fill(seed, syn.STREAM_QR, 0, 0, 0, HQ, D).reshape(1, 1, HQ, D).astype(np.float32)).to(dev)
+    ws = torch.empty(msa.msa_route_topk_workspace_size(1, 1, 1, H, C, n_docs, TOPK), dtype=torch.uint8, device=dev)
+    ids = torch.empty((1, 1, TOPK), dtype=torch.int32, device=dev)
+    sc = torch.empty((1, 1, TOPK), dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ms = []
+    for _ in range(calls):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        n = msa.msa_route_topk(q, [0, 1], kr, coffs, n_docs, C, 1, HQ, H, D, TOPK, ids, sc, ws,
+                               flags=msa.MSA_ROUTE_SCAN, dev_err=err)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    key_bytes = C * H * D * 2
+    best = min(ms)
+    out = {"blocks": C, "key_bytes": key_bytes, "route_ms": [round(x, 4) for x in ms], "launches": n,
+           "route_GBps_best": round(key_bytes / best / 1e6, 1), "dev_err": int(err.item())}
+    del kr, q, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_interleave(dev, host_kv, f8: bool):
     """Multi-round interleave on the 10M-token bank: 64 queries of 128 router tokens, each
     planted with a chain of three documents A -> B -> C (the router vectors of the first

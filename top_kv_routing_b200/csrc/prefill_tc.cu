@@ -6,19 +6,19 @@
 // times the values.  Follows "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", section
 // 推理流水线, and the MSA paper reading notes, section 推理全流程.
 //
-// One CTA (320 threads) per 128 rows: 128 / G tokens x the G query heads of key head h.
-//   warp 9, one thread   TMA producer: tiles of 64 keys (K as two 64-column boxes, then V
+// One CTA (576 threads) per 128 rows: 128 / G tokens x the G query heads of key head h.
+//   warp 17, one thread  TMA producer: tiles of 64 keys (K as two 64-column boxes, then V
 //                        the same), 128-byte swizzle, a 3-stage ring; memory tiles first,
 //                        then local tiles up to the CTA's last token
-//   warp 8, one thread   MMA issuer: S_i = Q K_i^T (M = 128, N = 64, K = 128) into one of two
+//   warp 16, one thread  MMA issuer: S_i = Q K_i^T (M = 128, N = 64, K = 128) into one of two
 //                        TMEM score buffers, then O += P_{i-1} V_{i-1} (M = 128, N = 128,
 //                        K = 64) into the TMEM output, with P read from tensor memory (it
 //                        replaces the scores it was computed from) and V read MN-major
 //                        straight from its [key][d] rows.  The rotated queries and the
 //                        weights are each a bf16 value plus a bf16 residual (two MMAs); keys
 //                        and values exact bf16; fp32 accumulation
-//   warps 0..7           two threads per row (TMEM lane), each with half of the row's dims
-//                        and half of every tile's keys: build the rotated, scaled query row
+//   warps 0..15          four threads per row (TMEM lane), each with a quarter of the row's
+//                        dims and of every tile's keys: build the rotated, scaled query row
 //                        in shared memory; per tile read the score row, mask it (memory keys
 //                        < M, local keys <= its own local index), keep a running maximum
 //                        that is raised (and O rescaled in TMEM) only when a score exceeds
@@ -46,37 +46,58 @@ constexpr int kD = 128;
 constexpr int kHalf = 64;
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kStages = 3;
-constexpr int kRowWarps = 8;                  // two threads per row: 32 keys of a tile each
+constexpr int kStages = 4;
+constexpr int kRowWarps = 16;                 // four threads per row: 16 keys of a tile each
+constexpr int kParts = kRowWarps / 4;
 constexpr int kMmaWarp = kRowWarps, kTmaWarp = kRowWarps + 1;
 constexpr int kThreads = (kRowWarps + 2) * 32;
-constexpr int kQHalf = kRows * 128;      // 16 KB: 64 bf16 of every row
-constexpr int kQBytes = 2 * kQHalf;      // 32 KB: one bf16 copy of the CTA's queries
 constexpr int kKVHalf = kKeys * 128;     // 8 KB: 64 keys x 64 elements
 constexpr int kTileBytes = 4 * kKVHalf;  // K (two halves) then V (two halves)
-constexpr int kOffQ = 0;                 // values
-constexpr int kOffQlo = kQBytes;         // residuals
-constexpr int kOffRing = 2 * kQBytes;
-constexpr int kOffTab = kOffRing + kStages * kTileBytes;  // cos / sin of the block's tokens (G > 1)
-constexpr int kTabBytes = 64 * kHalf * 8;                 // up to 64 tokens x 64 angles x float2
+constexpr int kOffRing = 0;
+constexpr int kQBoxHalf = kRows * 128;                    // 16 KB: 64 dims of the CTA's 128 rows
+constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // the queries as loaded; later the output rows
+constexpr int kOffTab = kOffQraw + 2 * kQBoxHalf;          // cos / sin of the block's tokens (G > 1)
+constexpr int kTabStride = kHalf + 1;                     // (a token's 64 angles + 1: the G-row groups of
+                                                           // a warp read 8 tokens in distinct banks)
+constexpr int kTabBytes = 64 * kTabStride * 8;             // up to 64 tokens x 64 angles x float2
 constexpr int kSmemData = kOffTab + kTabBytes;
-constexpr int kSmem = kSmemData + 1024 + 256 + 4 * 128 * 4;  // + barriers, the row pairs' exchange buffer
-constexpr uint32_t kTmemCols = 256;  // S0 / P0 [0, 64) | S1 / P1 [64, 128) | O [128, 256)
-constexpr uint32_t kColPlo = 32;     // residuals of a tile's weights, after its 32 value columns
+constexpr int kOffXch = 256;                                 // after the barriers: the rows' exchange buffer
+constexpr int kOffW = kOffXch + 2 * kParts * kRows * 4;      // then the RoPE frequencies (64 x 8 bytes)
+constexpr int kSmem = kSmemData + 1024 + kOffW + kHalf * 8;  // (+ alignment of the dynamic base)
+// S0 / P0 [0, 64) | S1 / P1 [64, 128) | O [128, 256) | Q [256, 320) | Q residual [320, 384)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColPlo = 32;  // residuals of a tile's weights, after its 32 value columns
 constexpr uint32_t kColO = 128;
+constexpr uint32_t kColQ = 256;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
+constexpr uint32_t kColQlo = 320;
 constexpr float kHeadroom = 8.0f;    // log2 growth of a row's maximum tolerated before rescaling
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// x = value + residual, both bf16: the value is x with its low 16 bits cleared (exact), the
+// residual x - value (exact in fp32, at most 2^-7 |x|) rounded to bf16, so |error| <= 2^-16 |x|.
+// Packed in pairs (x0 in the low half); one float-to-bf16 conversion per pair.
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
+  const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+  hi = __byte_perm(b0, b1, 0x7632);
   const __nv_bfloat162 l =
-      __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
+      __floats2bfloat162_rn(x0 - __uint_as_float(b0 & 0xFFFF0000u), x1 - __uint_as_float(b1 & 0xFFFF0000u));
   lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// cos / sin of the RoPE angle of position p at frequency step s (2^-64 turns per position):
+// the top 32 bits of p * s mod 2^64, read as signed, are the angle / pi in [-1, 1) x 2^31.
+__device__ __forceinline__ void rope_cs(unsigned long long p, unsigned long long s, float& cs, float& sn) {
+  const int top = (int)((p * s) >> 32);
+  sincospif((float)top * 4.656612873077392578125e-10f, &sn, &cs);  // x 2^-31
 }
 
 __device__ __forceinline__ uint32_t pack2(float x0, float x1) {
@@ -95,22 +116,48 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// 4D tiled TMA load (no multicast) completing on an mbarrier of this CTA: the box of a
+// CTA's query rows, [128 / G tokens][G heads][64 dims].
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z,
+                                            int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
+}
+
+// The matching 4D tiled TMA store (elements outside the tensor are not written).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int x, int y, int z, int w) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
 }
 
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_mem, const __grid_constant__ CUtensorMap tm_lk,
-                      const __grid_constant__ CUtensorMap tm_lv, const __nv_bfloat16* __restrict__ q, int T, int L,
+                      const __grid_constant__ CUtensorMap tm_lv, const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_out, int T, int L,
                       int H, const int32_t* __restrict__ local_len, int cap, const int32_t* __restrict__ mem_len,
                       int M_max, int pos_off, const __grid_constant__ RopeW rw, float qscale,
-                      __nv_bfloat16* __restrict__ out, int32_t* dev_err) {
+                      int32_t* dev_err) {
   constexpr int kTok = kRows / G;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -122,18 +169,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_p = bar_s + 2;           // weights ready (8 warps)
   uint64_t* bar_pv = bar_p + 1;          // PV done
   uint64_t* drain = bar_pv + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* bar_qraw = drain + 1;        // the query box has landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  unsigned long long* wsm = reinterpret_cast<unsigned long long*>(smem + kSmemData + kOffW);
 
   const int h = blockIdx.y;
   const int64_t bl = blockIdx.z;
   const int b = (int)(bl / L);
   const int tok0 = blockIdx.x * kTok;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Hq = H * G;
   const int len = local_len[b];
-  if (len < 0 || len + T > cap) return;  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
   int M = mem_len[bl];
+  if (len < 0 || len + T > cap) return;  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
   M = M < 0 ? 0 : (M > M_max ? M_max : M);
   const int tok_last = min(T, tok0 + kTok) - 1;
   const int n_local = len + tok_last + 1;
@@ -151,10 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(bar_p), kRowWarps);
     mbar_init(smem_u32(bar_pv), 1);
     mbar_init(smem_u32(drain), 1);
+    mbar_init(smem_u32(bar_qraw), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
   }
+  if (tid < kHalf) wsm[tid] = rw.step[tid];  // (indexed per lane: read from shared memory below)
   if (warp == kMmaWarp) {
     tmem_alloc<false>(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish<false>();
@@ -171,8 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lk)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lv)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_out)) : "memory");
+      mbar_arrive_expect_tx(smem_u32(bar_qraw), 2 * kQBoxHalf);
+      tma_load_4d(sbase + kOffQraw, &tm_q, smem_u32(bar_qraw), 0, h * G, tok0, (int)bl);
+      tma_load_4d(sbase + kOffQraw + kQBoxHalf, &tm_q, smem_u32(bar_qraw), kHalf, h * G, tok0, (int)bl);
       const uint64_t pol = policy_evict_last();
-      int armed[kStages] = {-1, -1, -1};
+      int armed[kStages];
+#pragma unroll
+      for (int st = 0; st < kStages; ++st) armed[st] = -1;
       bool ok = true;
       for (int i = 0; i < nt && ok; ++i) {
         const int stage = i % kStages;
@@ -205,44 +262,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
         for (int s = 0; s < kStages; ++s)
           if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
+        mbar_drain(smem_u32(bar_qraw), 0u);
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      // ---------------- MMA issuer (tensor-core operations from this thread run in order,
-      // so S_{i+2}, written over P_i, follows the PV that reads P_i)
-      constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
-      constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
-      bool ok = mbar_wait(smem_u32(bar_q), 0u, abort_flag), issued = false;
-      tc_fence_after();
-      for (int i = 0; i <= nt && ok; ++i) {
-        if (i < nt) {
-          const int stage = i % kStages;
-          if (!mbar_wait(smem_u32(&full[stage]), (uint32_t)((i / kStages) & 1), abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+    // ---------------- MMA issuer: the warp waits together, one elected lane issues (the
+    // tensor-core operations of that lane run in order, so S_{i+2}, written over P_i,
+    // follows the PV that reads P_i)
+    const bool leader = elect_one();
+    constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
+    constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), 0u, abort_flag)), issued = false;
+    tc_fence_after();
+    for (int i = 0; i <= nt && ok; ++i) {
+      if (i < nt) {
+        const int stage = i % kStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((i / kStages) & 1), abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
           const uint32_t kt = sbase + kOffRing + stage * kTileBytes;
           const uint32_t d_s = tmem_base + (uint32_t)((i & 1) * kKeys);
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = (uint32_t)((ks >> 2) * kQHalf);
             const uint64_t kdesc = sw128_desc(kt + (uint32_t)((ks >> 2) * kKVHalf)) + (uint64_t)(2 * (ks & 3));
-            umma<false, false>(d_s, sw128_desc(sbase + kOffQ + off) + (uint64_t)(2 * (ks & 3)), kdesc, idesc_s,
-                               ks > 0 ? 1u : 0u);
-            umma<false, false>(d_s, sw128_desc(sbase + kOffQlo + off) + (uint64_t)(2 * (ks & 3)), kdesc, idesc_s, 1u);
+            umma_ts(d_s, tmem_base + kColQ + (uint32_t)(8 * ks), kdesc, idesc_s, ks > 0 ? 1u : 0u);
+            umma_ts(d_s, tmem_base + kColQlo + (uint32_t)(8 * ks), kdesc, idesc_s, 1u);
           }
-          issued = true;
           umma_commit<false>(smem_u32(&bar_s[i & 1]));
         }
-        if (i >= 1) {
-          const int j = i - 1, stage = j % kStages;
-          if (!mbar_wait(smem_u32(bar_p), (uint32_t)(j & 1), abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        issued = true;
+        __syncwarp();
+      }
+      if (i >= 1) {
+        const int j = i - 1, stage = j % kStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_p), (uint32_t)(j & 1), abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
           const uint32_t vt = sbase + kOffRing + stage * kTileBytes + 2 * kKVHalf;
           const uint32_t p_tmem = tmem_base + (uint32_t)((j & 1) * kKeys);  // P_j: 64 bf16 in 32 columns
 #pragma unroll
@@ -254,49 +315,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit<false>(smem_u32(bar_pv));
           umma_commit<false>(smem_u32(&empty[stage]));
         }
+        __syncwarp();
       }
-      if (!ok) {
+    }
+    if (!ok) {
+      if (lane == 0) {
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
-        if (issued) {
-          umma_commit<false>(smem_u32(drain));
-          mbar_drain(smem_u32(drain), 0u);
-        }
+      }
+      if (issued) {
+        if (leader) umma_commit<false>(smem_u32(drain));
+        __syncwarp();
+        mbar_drain(smem_u32(drain), 0u);
       }
     }
   } else {
-    // ---------------- rows (warps 0..7): thread (row r = TMEM lane, half hf) takes the row's
-    // dims 32 hf .. 32 hf + 31 and 64 + 32 hf .. 95 + 32 hf of the query, and keys
-    // 32 hf .. 32 hf + 31 of every tile; the pair meets in shared memory (warps w, w + 4)
+    // ---------------- rows (warps 0..15): thread (row r = TMEM lane, part hf of 4) takes the
+    // row's dims 16 hf .. 16 hf + 15 and 64 + 16 hf .. 79 + 16 hf of the query, and keys
+    // 16 hf .. 16 hf + 15 of every tile; the four meet in shared memory (warps w, w + 4,
+    // w + 8, w + 12)
     const int r = tid & (kRows - 1), hf = tid >> 7;
-    const int tl = r / G, hd = r % G;
+    const int tl = r / G;
     const int tok = tok0 + tl;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    const int pair_bar = 1 + (warp & 3);  // named barrier of warps w and w + 4
-    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
-    {  // rotated, scaled query row (bf16 value and residual), 128-byte swizzled, 8 dims (and
+    const int pair_bar = 1 + (warp & 3);  // named barrier of the row's four warps
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(pair_bar) : "memory"); };
+    bool ok = true;
+    // Every row thread runs every iteration and every barrier, whatever happens: a failed
+    // (timed-out) wait only clears `ok` and raises the abort flag, after which the remaining
+    // waits return at once and the work is skipped.  So the named barriers, which cannot time
+    // out, always meet.
+    auto fail = [&]() {
+      ok = false;
+      *abort_flag = 1;
+    };
+    {  // rotated, scaled query row (bf16 value and residual) into tensor memory, 8 dims (and
        // their partners) at a time; with G > 1 the cos / sin of each token are computed once
        // into a table its G rows share
-      const __nv_bfloat16* src = q + ((bl * T + tok) * Hq + (int64_t)h * G + hd) * kD;
-      const double pos = (double)pos_off + (double)(len + tok);
+      const unsigned long long pos = (unsigned long long)((long long)pos_off + len + tok);
       float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
       if (G > 1) {
         for (int e = tid; e < kTok * kHalf; e += kRowWarps * 32) {
           const int t2 = e / kHalf, j = e % kHalf;
-          double u = ((double)pos_off + (double)(len + tok0 + t2)) * rw.w_over_pi[j];
-          u -= 2.0 * rint(0.5 * u);
           float sn, cs;
-          sincospif((float)u, &sn, &cs);
-          tab[e] = make_float2(cs, sn);
+          rope_cs((unsigned long long)((long long)pos_off + len + tok0 + t2), wsm[j], cs, sn);
+          tab[t2 * kTabStride + j] = make_float2(cs, sn);
         }
         asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory");
       }
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float xa[8], xb[8];  // dims 32 hf + 8c + e and 64 + 32 hf + 8c + e
-        if (tok < T) {
-          const uint4 wa = __ldg(reinterpret_cast<const uint4*>(src + 32 * hf + 8 * c));
-          const uint4 wb = __ldg(reinterpret_cast<const uint4*>(src + kHalf + 32 * hf + 8 * c));
+      // the query box (TMA, 128-byte swizzle): row r's 16-byte chunk c of each 64-dim half at
+      // 128 r + 16 (c ^ (r & 7))
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_qraw), 0u, abort_flag))) fail();
+      uint32_t qh[16], ql[16];  // bf16 pairs of the row's dims (values, residuals)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float xa[8], xb[8];  // dims 16 hf + 8c + e and 64 + 16 hf + 8c + e
+        if (tok < T && ok) {
+          const uint32_t qoff = sbase + kOffQraw + (uint32_t)(r * 128 + (((2 * hf + c) ^ (r & 7)) << 4));
+          const uint4 wa = ld_shared_v4(qoff), wb = ld_shared_v4(qoff + kQBoxHalf);
           const uint32_t va[4] = {wa.x, wa.y, wa.z, wa.w}, vb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -309,13 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 8; ++e) {
             float sn, cs;
             if (G > 1) {
-              const float2 t2 = tab[tl * kHalf + 32 * hf + 8 * c + e];
+              const float2 t2 = tab[tl * kTabStride + 16 * hf + 8 * c + e];
               cs = t2.x;
               sn = t2.y;
             } else {
-              double u = pos * rw.w_over_pi[32 * hf + 8 * c + e];
-              u -= 2.0 * rint(0.5 * u);
-              sincospif((float)u, &sn, &cs);
+              rope_cs(pos, wsm[16 * hf + 8 * c + e], cs, sn);
             }
             const float a = xa[e], bb = xb[e];
             xa[e] = (a * cs - bb * sn) * qscale;
@@ -325,37 +399,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
         }
-        // chunk 4 hf + c of the first half, 8 + 4 hf + c of the second
-        const int ca = 4 * hf + c, cb = 8 + 4 * hf + c;
-        const uint32_t oa = (uint32_t)((ca >> 3) * kQHalf + r * 128 + (((ca & 7) ^ (r & 7)) << 4));
-        const uint32_t ob = (uint32_t)((cb >> 3) * kQHalf + r * 128 + (((cb & 7) ^ (r & 7)) << 4));
-        uint32_t ha[4], la[4], hb[4], lb[4];
+        // dims 16 hf + 8c .. + 7 -> columns 8 hf + 4c .. + 3 (and 32 further for the second half)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          split2(xa[2 * e], xa[2 * e + 1], ha[e], la[e]);
-          split2(xb[2 * e], xb[2 * e + 1], hb[e], lb[e]);
+          split2(xa[2 * e], xa[2 * e + 1], qh[4 * c + e], ql[4 * c + e]);
+          split2(xb[2 * e], xb[2 * e + 1], qh[8 + 4 * c + e], ql[8 + 4 * c + e]);
         }
-        st_shared_v4(sbase + kOffQ + oa, ha[0], ha[1], ha[2], ha[3]);
-        st_shared_v4(sbase + kOffQlo + oa, la[0], la[1], la[2], la[3]);
-        st_shared_v4(sbase + kOffQ + ob, hb[0], hb[1], hb[2], hb[3]);
-        st_shared_v4(sbase + kOffQlo + ob, lb[0], lb[1], lb[2], lb[3]);
       }
-      fence_async_smem();
+      tmem_st8(tmem_base + lane_addr + kColQ + (uint32_t)(8 * hf), *reinterpret_cast<const uint32_t(*)[8]>(qh));
+      tmem_st8(tmem_base + lane_addr + kColQ + 32 + (uint32_t)(8 * hf), *reinterpret_cast<const uint32_t(*)[8]>(qh + 8));
+      tmem_st8(tmem_base + lane_addr + kColQlo + (uint32_t)(8 * hf), *reinterpret_cast<const uint32_t(*)[8]>(ql));
+      tmem_st8(tmem_base + lane_addr + kColQlo + 32 + (uint32_t)(8 * hf),
+               *reinterpret_cast<const uint32_t(*)[8]>(ql + 8));
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(bar_q));
     }
-    float* xch = reinterpret_cast<float*>(smem + kSmemData + 256);  // [2 tiles][2 halves][128 rows]
+    float* xch = reinterpret_cast<float*>(smem + kSmemData + kOffXch);  // [2 tiles][4 parts][128 rows]
     const int lim = len + min(tok, T - 1);
     float m_used = -INFINITY, l_sum = 0.f;
-    bool ok = true;
-    // Every row thread runs every iteration and every pair barrier, whatever happens: a
-    // failed (timed-out) wait only clears `ok` and raises the abort flag, after which the
-    // remaining waits return at once and the work is skipped.  So the pair barriers, which
-    // cannot time out, always meet.
-    auto fail = [&]() {
-      ok = false;
-      *abort_flag = 1;
-    };
     // PV_{i-1} done (the bar_pv phases are waited one by one, in order)
     auto wait_pv = [&](int j) {
       if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)(j & 1), abort_flag))) fail();
@@ -369,25 +432,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key0 = local ? (i - nt_mem) * kKeys : i * kKeys;
       const int n_valid = local ? min(kKeys, n_local - key0) : min(kKeys, M - key0);
       float mx = -INFINITY;
-      float sv[32];
+      float sv[16];
       if (ok) {
         tc_fence_after();
-        uint32_t sa[32];
-        tmem_ld32(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 32 * hf), sa);
+        uint32_t sa[16];
+        tmem_ld16(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 16 * hf), sa);
         tmem_wait_ld();
-        // this thread's 32 keys: all visible (a memory tile's first keys below M, or local
+        // this thread's 16 keys: all visible (a memory tile's first keys below M, or local
         // keys up to the row's limit), or masked one by one
-        const int kfirst = key0 + 32 * hf;
-        const bool all_in = local ? kfirst + 31 <= lim : kfirst + 31 < M;
+        const int kfirst = key0 + 16 * hf;
+        const bool all_in = local ? kfirst + 15 <= lim : kfirst + 15 < M;
         if (all_in) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          for (int e = 0; e < 16; ++e) {
             sv[e] = __uint_as_float(sa[e]);
             mx = fmaxf(mx, sv[e]);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          for (int e = 0; e < 16; ++e) {
             const int key = kfirst + e;
             const bool v = local ? key <= lim : key < M;
             sv[e] = v ? __uint_as_float(sa[e]) : -INFINITY;
@@ -395,17 +458,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      xch[((i & 1) * 2 + hf) * kRows + r] = mx;
-      pair_sync();  // (also: both threads of the row have read the score row before either writes P)
-      mx = fmaxf(mx, xch[((i & 1) * 2 + (hf ^ 1)) * kRows + r]);
+      xch[((i & 1) * kParts + hf) * kRows + r] = mx;
+      pair_sync();  // (also: the row's four threads have read the score row before any writes P)
+#pragma unroll
+      for (int o = 1; o < kParts; ++o) mx = fmaxf(mx, xch[((i & 1) * kParts + ((hf + o) & 3)) * kRows + r]);
       if (!ok) continue;
       const bool need = mx > m_used + kHeadroom;  // (the same in both threads of the row)
       const float m_old = m_used;
       if (need) m_used = mx;
-      uint32_t pw[16], plw[16];
+      uint32_t pw[8], plw[8];
       float psum = 0.f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
+      for (int e = 0; e < 8; ++e) {
         const float p0 = exp2f(sv[2 * e] - m_used), p1 = exp2f(sv[2 * e + 1] - m_used);
         psum += p0 + p1;
         split2(p0, p1, pw[e], plw[e]);
@@ -424,10 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         wait_pv(i - 1);
         if (!ok) continue;
         const float alpha = need ? exp2f(m_old - m_used) : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {  // this thread's 64 of the 128 output columns
+        {  // this thread's 32 of the 128 output columns
           uint32_t o[32];
-          const uint32_t col = kColO + (uint32_t)(64 * hf + 32 * c);
+          const uint32_t col = kColO + (uint32_t)(32 * hf);
           tmem_ld32(tmem_base + lane_addr + col, o);
           tmem_wait_ld();
 #pragma unroll
@@ -436,10 +499,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (need) l_sum *= alpha;
       }
-      // P_i over the scores it came from: values in columns 16 hf .. 16 hf + 15 of the
-      // tile's buffer, residuals 32 columns further
-      tmem_st16(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 16 * hf), pw);
-      tmem_st16(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + kColPlo + 16 * hf), plw);
+      // P_i over the scores it came from: values in columns 8 hf .. 8 hf + 7 of the tile's
+      // buffer, residuals 32 columns further
+      tmem_st8(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 8 * hf), pw);
+      tmem_st8(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + kColPlo + 8 * hf), plw);
       tmem_wait_st();
       l_sum += psum;
       fence_async_smem();
@@ -449,35 +512,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i > 0 && !rescale) wait_pv(i - 1);  // (one wait per tile, in order)
     }
     if (nt > 0) wait_pv(nt - 1);
-    // the row's sum of weights: both halves (the exchange slot of tile nt is free)
-    xch[((nt & 1) * 2 + hf) * kRows + r] = l_sum;
+    // the row's sum of weights: all four parts (the exchange slot of tile nt is free)
+    xch[((nt & 1) * kParts + hf) * kRows + r] = l_sum;
     pair_sync();
-    l_sum += xch[((nt & 1) * 2 + (hf ^ 1)) * kRows + r];
+#pragma unroll
+    for (int o = 1; o < kParts; ++o) l_sum += xch[((nt & 1) * kParts + ((hf + o) & 3)) * kRows + r];
     ok = __all_sync(0xffffffffu, ok);
+    // the output rows, bf16, into the query box's space (read long ago) in the layout of the
+    // query box, then one TMA store per 64-dim half (rows past the block's last token fall
+    // outside the tensor and are not written)
+    const uint32_t stage_o = sbase + kOffQraw;
     if (ok) {
       const float inv = 1.0f / l_sum;
-      __nv_bfloat16* dst = out + ((bl * T + tok) * Hq + (int64_t)h * G + hd) * kD;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t o[32];
-        const int col = 64 * hf + 32 * c;
-        tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)col, o);
-        tmem_wait_ld();
-        if (tok < T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + col);
+      uint32_t o[32];
+      tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)(32 * hf), o);
+      tmem_wait_ld();
+      const uint32_t half = stage_o + (uint32_t)((hf >> 1) * kQBoxHalf) + (uint32_t)(r * 128);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint32_t w[4];
+      for (int e = 0; e < 4; ++e) {
+        uint32_t w[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              w[u] = pack2(__uint_as_float(o[8 * e + 2 * u]) * inv, __uint_as_float(o[8 * e + 2 * u + 1]) * inv);
-            d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+        for (int u = 0; u < 4; ++u)
+          w[u] = pack2(__uint_as_float(o[8 * e + 2 * u]) * inv, __uint_as_float(o[8 * e + 2 * u + 1]) * inv);
+        const int c = 4 * (hf & 1) + e;
+        st_shared_v4(half + (uint32_t)((c ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
       }
+      fence_async_smem();
     } else {
       *abort_flag = 1;
       if (lane == 0) msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+    }
+    asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory");
+    if (tid == 0 && !*abort_flag) {
+      tma_store_4d(&tm_out, stage_o, 0, h * G, tok0, (int)bl);
+      tma_store_4d(&tm_out, stage_o + kQBoxHalf, kHalf, h * G, tok0, (int)bl);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the box has been read out
     }
   }
 
@@ -519,13 +589,28 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [B*L][T][Hq][128] (queries or outputs), box [128 / G tokens][G heads][64 dims],
+// 128-byte swizzle; coordinates (dim, head, token, b*L + l)
+bool make_rows_map(CUtensorMap* m, const void* base, int Hq, int T, int BL, int G) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)BL};
+  const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)Hq * kD * 2, (cuuint64_t)T * Hq * kD * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)kHalf, (cuuint32_t)G, (cuuint32_t)(kRows / G), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int G>
 int launch_g(const Args& a, cudaStream_t s, const char** why) {
-  CUtensorMap tm_mem, tm_lk, tm_lv;
+  CUtensorMap tm_mem, tm_lk, tm_lv, tm_q, tm_out;
   const uint64_t mem_rows = (uint64_t)a.B * a.L * 2 * a.H * a.M_max;
   const uint64_t loc_rows = (uint64_t)a.B * a.L * a.H * a.cap;
   if (!make_map(&tm_mem, a.mem_kv, mem_rows) || !make_map(&tm_lk, a.local_k, loc_rows) ||
-      !make_map(&tm_lv, a.local_v, loc_rows)) {
+      !make_map(&tm_lv, a.local_v, loc_rows) || !make_rows_map(&tm_q, a.q, a.H * G, a.T, a.B * a.L, G) ||
+      !make_rows_map(&tm_out, a.out, a.H * G, a.T, a.B * a.L, G)) {
     *why = "cuTensorMapEncodeTiled failed";
     return 1;
   }
@@ -535,10 +620,13 @@ int launch_g(const Args& a, cudaStream_t s, const char** why) {
   }
   const int tiles = (a.T + kRows / G - 1) / (kRows / G);
   RopeW rw;
-  for (int j = 0; j < kHalf; ++j) rw.w_over_pi[j] = exp2(-2.0 * (double)j / (double)kD * a.log2_theta) / M_PI;
+  for (int j = 0; j < kHalf; ++j) {
+    const long double turns = exp2l(-2.0L * j / kD * (long double)a.log2_theta) / (2.0L * 3.14159265358979323846264338L);
+    rw.step[j] = (unsigned long long)llroundl(ldexpl(turns, 64));
+  }
   prefill_tc_kernel<G><<<dim3(tiles, a.H, a.B * a.L), kThreads, kSmem, s>>>(
-      tm_mem, tm_lk, tm_lv, a.q, a.T, a.L, a.H, a.local_len, a.cap, a.mem_len, a.M_max, a.pos_off, rw, a.qscale,
-      a.out, a.dev_err);
+      tm_mem, tm_lk, tm_lv, tm_q, tm_out, a.T, a.L, a.H, a.local_len, a.cap, a.mem_len, a.M_max, a.pos_off, rw,
+      a.qscale, a.dev_err);
   if (cudaGetLastError() != cudaSuccess) {
     *why = "kernel launch";
     return 1;

@@ -6,9 +6,12 @@
 
 namespace prefill_tc {
 
-// RoPE frequencies of one call, theta^(-2j/128) / pi for j < 64 (fp64), computed on the host.
+// RoPE frequencies of one call in fixed point, computed on the host: step[j] =
+// round(2^64 * theta^(-2j/128) / (2 pi)), the rotation of frequency j per position in units
+// of 2^-64 turns.  The angle of position p is then p * step[j] mod 2^64 turns (exact integer
+// arithmetic, no range reduction needed).
 struct RopeW {
-  double w_over_pi[64];
+  unsigned long long step[64];
 };
 
 struct Args {
