@@ -21,10 +21,11 @@
 // (b, l, h) to arrive (a self-resetting counter) merges them.  The last CTA of query b
 // advances local_len[b].  The rotated new key (rounded to the cache's bf16) and the new
 // value go to the cache (split 0) and into the zero-filled row of the last local tile
-// in shared memory, so they are scored like every other key.  RoPE angles: p * w_j with
-// w_j / pi in fp64, the product reduced modulo 2 pi in fp64, fp32 sincospif.  The query
-// fragments are built once per CTA in shared memory in MMA order (the kernel's per-launch
-// path is kept short: it runs with a cold instruction cache on every launch).
+// in shared memory, so they are scored like every other key.  RoPE angles: position times
+// a 64-bit fixed-point step per frequency (turns, modulo 1 by integer wrap-around), fp32
+// sincospif.  The query fragments are built once per CTA in shared memory in MMA order (the
+// kernel's per-launch path is kept short: it runs with a cold instruction cache on every
+// launch).
 #include "attn_common.cuh"
 #include "common.cuh"
 #include "msa_decode.h"
@@ -62,9 +63,11 @@ size_t ws_bytes(int B, int L, int Hq, int H) {
   return ws_floats(B, L, Hq, H) * sizeof(float) + ((size_t)B * L * H + (size_t)B) * sizeof(int);
 }
 
-// RoPE frequencies of one call: w_j / pi = theta^(-2j/128) / pi, j < 64 (fp64).
+// RoPE frequencies of one call in fixed point: step[j] = round(2^64 theta^(-2j/128) / (2 pi)),
+// the rotation of frequency j per position in units of 2^-64 turns, so that the angle of
+// position p is p * step[j] mod 2^64 turns (exact integer arithmetic, no range reduction).
 struct RopeFreq {
-  double w_over_pi[kHalf];
+  unsigned long long step[kHalf];
 };
 
 template <int G>
@@ -126,13 +129,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     M = M_max;
   }
   if (M < 0) M = 0;
-  int arrived = 0;  // tid 0: arrivals on query_count[b] before this CTA's
+  // once every thread has read local_len[b], lane 0 of the last warp announces it (arrivals
+  // before this CTA's are counted in `arrived`); the last CTA of the query to arrive
+  // advances the length at its end.  That lane loads no new key or value and has no tile
+  // copy pending yet, so the release costs it little, and nothing waits for the atomic's
+  // result until the end.
+  constexpr int kAnnouncer = kThreads - 32;
+  static_assert(kAnnouncer >= kHalf + kD, "the announcer loads no new key or value");
+  int arrived = 0;
+  __syncthreads();
+  if (tid == kAnnouncer) arrived = arrive_release(&query_count[b]);
 
   if (full) {
     if (tid == 0 && split == 0 && h == 0 && (bl % L) == 0) msa::set_err(dev_err, MSA_DEVERR_LOCAL_FULL);
     if (splits > 1 && tid < G) stat[(uh * kMaxSplits + split) * G + tid] = make_float2(-INFINITY, -1.f);
-    __syncthreads();
-    if (tid == 0) arrived = arrive_release(&query_count[b]);
   } else {
     // ---- this warp's tiles (memory tiles, then local tiles; the new key, row len, rides
     // in the last local tile): the first ones are requested before anything else
@@ -191,20 +201,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
       cp_async_commit();
     }
 
-    // ---- RoPE angles of this step's position: p * w_j / pi in fp64 (w_j / pi computed once
-    // per call on the host), reduced modulo 2 pi in fp64, fp32 sincospif
-    const double pos = (double)pos_off + (double)len;
+    // ---- RoPE angles of this step's position p: the top 32 bits of p * step[j] mod 2^64,
+    // read as signed, are the angle / pi in [-1, 1) x 2^31; fp32 sincospif
     if (tid < kHalf) {
-      double u = pos * rf.w_over_pi[tid];
-      u -= 2.0 * rint(0.5 * u);  // in [-1, 1]
+      const unsigned long long pos = (unsigned long long)((long long)pos_off + len);
+      const int top = (int)((pos * rf.step[tid]) >> 32);
       float sn, c;
-      sincospif((float)u, &sn, &c);
+      sincospif((float)top * 4.656612873077392578125e-10f, &sn, &c);  // x 2^-31
       cs[tid] = make_float2(c, sn);
     }
     __syncthreads();
-    // every thread has read local_len[b]: announce it (the last CTA of the query to
-    // arrive advances the length at its end)
-    if (tid == 0) arrived = arrive_release(&query_count[b]);
     {  // rotated, scaled query pairs -> MMA fragments (bf16 value and bf16 residual)
       float r[4] = {0.f, 0.f, 0.f, 0.f};  // dims 2m, 2m+1, 2m+64, 2m+65
       if (gg < G) {
@@ -416,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     }
   }
   // every CTA of query b arrived after reading local_len[b]; the last one advances it
-  if (tid == 0 && arrived == L * H * splits - 1) {
+  if (tid == kAnnouncer && arrived == L * H * splits - 1) {
     if (!full) local_len[b] = len + 1;
     query_count[b] = 0;  // ready for the next call
   }
@@ -478,8 +484,11 @@ msa_status launch_decode(const void* q, const void* k_new, const void* v_new, in
   int* query_count = unit_count + units;
   const dim3 grid(splits, n_kv_heads, n_queries * n_layers);
   RopeFreq rf;
-  const double log2_theta = log2((double)rope_theta);
-  for (int j = 0; j < kHalf; ++j) rf.w_over_pi[j] = exp2(-2.0 * (double)j / (double)kD * log2_theta) / M_PI;
+  const long double log2_theta = log2l((long double)rope_theta);
+  for (int j = 0; j < kHalf; ++j) {
+    const long double turns = exp2l(-2.0L * j / kD * log2_theta) / (2.0L * 3.14159265358979323846264338L);
+    rf.step[j] = (unsigned long long)llroundl(ldexpl(turns, 64));
+  }
   const float qscale = softmax_scale * kLog2e;
   // programmatic stream serialisation: the kernel may be scheduled before the previous
   // kernel on the stream finishes and waits for it (griddepcontrol.wait) before reading
