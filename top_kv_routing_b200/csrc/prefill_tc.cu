@@ -94,10 +94,12 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
 }
 
 // cos / sin of the RoPE angle of position p at frequency step s (2^-64 turns per position):
-// the top 32 bits of p * s mod 2^64, read as signed, are the angle / pi in [-1, 1) x 2^31.
+// the top 32 bits of p * s mod 2^64, read as signed, are the angle in [-pi, pi) x 2^31 / pi.
+// The hardware sine / cosine is used on that reduced angle (absolute error about 2^-21 on
+// [-pi, pi], far below the query's value + residual precision of 2^-16).
 __device__ __forceinline__ void rope_cs(unsigned long long p, unsigned long long s, float& cs, float& sn) {
   const int top = (int)((p * s) >> 32);
-  sincospif((float)top * 4.656612873077392578125e-10f, &sn, &cs);  // x 2^-31
+  __sincosf((float)top * 1.4629180792671596e-09f, &sn, &cs);  // x pi / 2^31
 }
 
 __device__ __forceinline__ uint32_t pack2(float x0, float x1) {
@@ -179,15 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = (int)(bl / L);
   const int tok0 = blockIdx.x * kTok;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int len = local_len[b];
-  int M = mem_len[bl];
-  if (len < 0 || len + T > cap) return;  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
-  M = M < 0 ? 0 : (M > M_max ? M_max : M);
-  const int tok_last = min(T, tok0 + kTok) - 1;
-  const int n_local = len + tok_last + 1;
-  const int nt_mem = (M + kKeys - 1) / kKeys;
-  const int nt = nt_mem + (n_local + kKeys - 1) / kKeys;
+  const uint32_t sbase = smem_u32(smem);
 
+  // thread 0: the barriers, then at once the query box (it does not depend on the lengths)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
@@ -203,7 +199,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
+    mbar_arrive_expect_tx(smem_u32(bar_qraw), 2 * kQBoxHalf);
+    tma_load_4d(sbase + kOffQraw, &tm_q, smem_u32(bar_qraw), 0, h * G, tok0, (int)bl);
+    tma_load_4d(sbase + kOffQraw + kQBoxHalf, &tm_q, smem_u32(bar_qraw), kHalf, h * G, tok0, (int)bl);
   }
+  const int len = local_len[b];
+  int M = mem_len[bl];
+  if (len < 0 || len + T > cap) {  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
+    if (tid == 0) mbar_drain(smem_u32(bar_qraw), 0u);  // the query box lands before the CTA leaves
+    return;
+  }
+  M = M < 0 ? 0 : (M > M_max ? M_max : M);
+  const int tok_last = min(T, tok0 + kTok) - 1;
+  const int n_local = len + tok_last + 1;
+  const int nt_mem = (M + kKeys - 1) / kKeys;
+  const int nt = nt_mem + (n_local + kKeys - 1) / kKeys;
   if (tid < kHalf) wsm[tid] = rw.step[tid];  // (indexed per lane: read from shared memory below)
   if (warp == kMmaWarp) {
     tmem_alloc<false>(smem_u32(tmem_slot), kTmemCols);
@@ -213,7 +223,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t sbase = smem_u32(smem);
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
@@ -221,11 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lk)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lv)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_out)) : "memory");
-      mbar_arrive_expect_tx(smem_u32(bar_qraw), 2 * kQBoxHalf);
-      tma_load_4d(sbase + kOffQraw, &tm_q, smem_u32(bar_qraw), 0, h * G, tok0, (int)bl);
-      tma_load_4d(sbase + kOffQraw + kQBoxHalf, &tm_q, smem_u32(bar_qraw), kHalf, h * G, tok0, (int)bl);
       const uint64_t pol = policy_evict_last();
       int armed[kStages];
 #pragma unroll
