@@ -46,7 +46,7 @@ constexpr int kD = 128;
 constexpr int kHalf = 64;
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kRowWarps = 16;                 // four threads per row: 16 keys of a tile each
 constexpr int kParts = kRowWarps / 4;
 constexpr int kMmaWarp = kRowWarps, kTmaWarp = kRowWarps + 1;
@@ -55,8 +55,9 @@ constexpr int kKVHalf = kKeys * 128;     // 8 KB: 64 keys x 64 elements
 constexpr int kTileBytes = 4 * kKVHalf;  // K (two halves) then V (two halves)
 constexpr int kOffRing = 0;
 constexpr int kQBoxHalf = kRows * 128;                    // 16 KB: 64 dims of the CTA's 128 rows
-constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // the queries as loaded; later the output rows
-constexpr int kOffTab = kOffQraw + 2 * kQBoxHalf;          // cos / sin of the block's tokens (G > 1)
+constexpr int kQBox = 2 * kQBoxHalf;                      // 32 KB: one unit's query rows
+constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // per unit: its queries as loaded, later its output
+constexpr int kOffTab = kOffQraw + 2 * kQBox;              // cos / sin of a unit's tokens (G > 1)
 constexpr int kTabStride = kHalf + 1;                     // (a token's 64 angles + 1: the G-row groups of
                                                            // a warp read 8 tokens in distinct banks)
 constexpr int kTabBytes = 64 * kTabStride * 8;             // up to 64 tokens x 64 angles x float2
@@ -64,12 +65,14 @@ constexpr int kSmemData = kOffTab + kTabBytes;
 constexpr int kOffXch = 256;                                 // after the barriers: the rows' exchange buffer
 constexpr int kOffW = kOffXch + 2 * kParts * kRows * 4;      // then the RoPE frequencies (64 x 8 bytes)
 constexpr int kSmem = kSmemData + 1024 + kOffW + kHalf * 8;  // (+ alignment of the dynamic base)
-// S0 / P0 [0, 64) | S1 / P1 [64, 128) | O [128, 256) | Q [256, 320) | Q residual [320, 384)
+// S0 / P0 [0, 64) | S1 / P1 [64, 128) | O [128, 256) | unit 0's query value [256, 320) and
+// residual [320, 384) | unit 1's [384, 448) and [448, 512)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColPlo = 32;  // residuals of a tile's weights, after its 32 value columns
 constexpr uint32_t kColO = 128;
 constexpr uint32_t kColQ = 256;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
 constexpr uint32_t kColQlo = 320;
+constexpr uint32_t kColQUnit = 128;  // the second unit's query, further on
 constexpr float kHeadroom = 8.0f;    // log2 growth of a row's maximum tolerated before rescaling
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -166,24 +169,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
-  uint64_t* bar_q = empty + kStages;     // queries written (8 warps)
+  uint64_t* bar_q = empty + kStages;     // a unit's queries written (16 warps; one phase per unit)
   uint64_t* bar_s = bar_q + 1;           // [2] scores ready
-  uint64_t* bar_p = bar_s + 2;           // weights ready (8 warps)
+  uint64_t* bar_p = bar_s + 2;           // weights ready (16 warps)
   uint64_t* bar_pv = bar_p + 1;          // PV done
   uint64_t* drain = bar_pv + 1;
-  uint64_t* bar_qraw = drain + 1;        // the query box has landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 1);
+  uint64_t* bar_qraw = drain + 1;        // [2] a unit's query box has landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   unsigned long long* wsm = reinterpret_cast<unsigned long long*>(smem + kSmemData + kOffW);
 
+  // two units of 128 rows per CTA: token tiles j and n_tiles - 1 - j of (b, l, h), a short
+  // and a long one under the causal mask (one unit when they coincide)
   const int h = blockIdx.y;
   const int64_t bl = blockIdx.z;
   const int b = (int)(bl / L);
-  const int tok0 = blockIdx.x * kTok;
+  const int n_tiles = (T + kTok - 1) / kTok;
+  const int n_units = (int)blockIdx.x == n_tiles - 1 - (int)blockIdx.x ? 1 : 2;
+  const int tok0_u[2] = {(int)blockIdx.x * kTok, (n_tiles - 1 - (int)blockIdx.x) * kTok};
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
 
-  // thread 0: the barriers, then at once the query box (it does not depend on the lengths)
+  // thread 0: the barriers, then at once the units' query boxes (they do not depend on the
+  // lengths)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
@@ -195,25 +203,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(bar_p), kRowWarps);
     mbar_init(smem_u32(bar_pv), 1);
     mbar_init(smem_u32(drain), 1);
-    mbar_init(smem_u32(bar_qraw), 1);
+    mbar_init(smem_u32(&bar_qraw[0]), 1);
+    mbar_init(smem_u32(&bar_qraw[1]), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
-    mbar_arrive_expect_tx(smem_u32(bar_qraw), 2 * kQBoxHalf);
-    tma_load_4d(sbase + kOffQraw, &tm_q, smem_u32(bar_qraw), 0, h * G, tok0, (int)bl);
-    tma_load_4d(sbase + kOffQraw + kQBoxHalf, &tm_q, smem_u32(bar_qraw), kHalf, h * G, tok0, (int)bl);
+    for (int u = 0; u < n_units; ++u) {
+      const uint32_t qb = smem_u32(&bar_qraw[u]), dst = sbase + kOffQraw + (uint32_t)(u * kQBox);
+      mbar_arrive_expect_tx(qb, kQBox);
+      tma_load_4d(dst, &tm_q, qb, 0, h * G, tok0_u[u], (int)bl);
+      tma_load_4d(dst + kQBoxHalf, &tm_q, qb, kHalf, h * G, tok0_u[u], (int)bl);
+    }
   }
   const int len = local_len[b];
   int M = mem_len[bl];
   if (len < 0 || len + T > cap) {  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
-    if (tid == 0) mbar_drain(smem_u32(bar_qraw), 0u);  // the query box lands before the CTA leaves
+    if (tid == 0)  // the query boxes land before the CTA leaves
+      for (int u = 0; u < n_units; ++u) mbar_drain(smem_u32(&bar_qraw[u]), 0u);
     return;
   }
   M = M < 0 ? 0 : (M > M_max ? M_max : M);
-  const int tok_last = min(T, tok0 + kTok) - 1;
-  const int n_local = len + tok_last + 1;
   const int nt_mem = (M + kKeys - 1) / kKeys;
-  const int nt = nt_mem + (n_local + kKeys - 1) / kKeys;
+  // per unit: local keys up to its last token, tiles; the units' tiles are numbered on from
+  // one to the next (g = unit 0's 0 .. nt[0] - 1, then unit 1's)
+  int n_local[2], nt[2];
+  for (int u = 0; u < 2; ++u) {
+    n_local[u] = len + min(T, tok0_u[u] + kTok);
+    nt[u] = nt_mem + (n_local[u] + kKeys - 1) / kKeys;
+  }
+  const int nt_all = nt[0] + (n_units == 2 ? nt[1] : 0);
   if (tid < kHalf) wsm[tid] = rw.step[tid];  // (indexed per lane: read from shared memory below)
   if (warp == kMmaWarp) {
     tmem_alloc<false>(smem_u32(tmem_slot), kTmemCols);
@@ -226,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- TMA producer: every tile of unit 0, then of unit 1
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lk)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lv)) : "memory");
@@ -236,9 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int st = 0; st < kStages; ++st) armed[st] = -1;
       bool ok = true;
-      for (int i = 0; i < nt && ok; ++i) {
-        const int stage = i % kStages;
-        const uint32_t ph = (uint32_t)((i / kStages) & 1);
+      for (int g = 0; g < nt_all && ok; ++g) {
+        const int i = g < nt[0] ? g : g - nt[0];  // the unit's own tile
+        const int stage = g % kStages;
+        const uint32_t ph = (uint32_t)((g / kStages) & 1);
         if (!mbar_wait(smem_u32(&empty[stage]), ph ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -267,42 +286,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
         for (int s = 0; s < kStages; ++s)
           if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
-        mbar_drain(smem_u32(bar_qraw), 0u);
+        for (int u = 0; u < n_units; ++u) mbar_drain(smem_u32(&bar_qraw[u]), 0u);
       }
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer: the warp waits together, one elected lane issues (the
-    // tensor-core operations of that lane run in order, so S_{i+2}, written over P_i,
-    // follows the PV that reads P_i)
+    // tensor-core operations of that lane run in order, so S_{g+2}, written over P_g,
+    // follows the PV that reads P_g).  A unit's first score tile waits for its queries.
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
     constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), 0u, abort_flag)), issued = false;
-    tc_fence_after();
-    for (int i = 0; i <= nt && ok; ++i) {
-      if (i < nt) {
-        const int stage = i % kStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((i / kStages) & 1), abort_flag))) {
+    bool ok = true, issued = false;
+    for (int g = 0; g <= nt_all && ok; ++g) {
+      if (g < nt_all) {
+        const int u = g < nt[0] ? 0 : 1, i = g - (u ? nt[0] : 0);
+        if (i == 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), (uint32_t)u, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int stage = g % kStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((g / kStages) & 1), abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (leader) {
           const uint32_t kt = sbase + kOffRing + stage * kTileBytes;
-          const uint32_t d_s = tmem_base + (uint32_t)((i & 1) * kKeys);
+          const uint32_t d_s = tmem_base + (uint32_t)((g & 1) * kKeys);
+          const uint32_t q_t = tmem_base + kColQ + (uint32_t)u * kColQUnit;
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint64_t kdesc = sw128_desc(kt + (uint32_t)((ks >> 2) * kKVHalf)) + (uint64_t)(2 * (ks & 3));
-            umma_ts(d_s, tmem_base + kColQ + (uint32_t)(8 * ks), kdesc, idesc_s, ks > 0 ? 1u : 0u);
-            umma_ts(d_s, tmem_base + kColQlo + (uint32_t)(8 * ks), kdesc, idesc_s, 1u);
+            umma_ts(d_s, q_t + (uint32_t)(8 * ks), kdesc, idesc_s, ks > 0 ? 1u : 0u);
+            umma_ts(d_s, q_t + (kColQlo - kColQ) + (uint32_t)(8 * ks), kdesc, idesc_s, 1u);
           }
-          umma_commit<false>(smem_u32(&bar_s[i & 1]));
+          umma_commit<false>(smem_u32(&bar_s[g & 1]));
         }
         issued = true;
         __syncwarp();
       }
-      if (i >= 1) {
-        const int j = i - 1, stage = j % kStages;
+      if (g >= 1) {
+        const int j = g - 1, stage = j % kStages;
+        const int jj = j < nt[0] ? j : j - nt[0];  // its index in its unit: 0 starts the unit's O
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_p), (uint32_t)(j & 1), abort_flag))) {
           ok = false;
           break;
@@ -314,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int ks = 0; ks < kKeys / 16; ++ks) {
             const uint64_t vdesc = sw128_desc_mn(vt + (uint32_t)(ks * 2048), kKVHalf, 1024);
-            umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
             umma_ts(tmem_base + kColO, p_tmem + kColPlo + (uint32_t)(8 * ks), vdesc, idesc_pv, 1u);
           }
           umma_commit<false>(smem_u32(bar_pv));
@@ -338,13 +366,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- rows (warps 0..15): thread (row r = TMEM lane, part hf of 4) takes the
     // row's dims 16 hf .. 16 hf + 15 and 64 + 16 hf .. 79 + 16 hf of the query, and keys
     // 16 hf .. 16 hf + 15 of every tile; the four meet in shared memory (warps w, w + 4,
-    // w + 8, w + 12)
+    // w + 8, w + 12).  Order: unit 0's queries and tiles; unit 1's queries (so that its first
+    // score tiles run under what follows); unit 0's output; unit 1's tiles and output.
     const int r = tid & (kRows - 1), hf = tid >> 7;
     const int tl = r / G;
-    const int tok = tok0 + tl;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const int pair_bar = 1 + (warp & 3);  // named barrier of the row's four warps
     auto pair_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(pair_bar) : "memory"); };
+    auto rows_sync = [&]() { asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory"); };
     bool ok = true;
     // Every row thread runs every iteration and every barrier, whatever happens: a failed
     // (timed-out) wait only clears `ok` and raises the abort flag, after which the remaining
@@ -354,9 +383,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = false;
       *abort_flag = 1;
     };
-    {  // rotated, scaled query row (bf16 value and residual) into tensor memory, 8 dims (and
-       // their partners) at a time; with G > 1 the cos / sin of each token are computed once
-       // into a table its G rows share
+    float* xch = reinterpret_cast<float*>(smem + kSmemData + kOffXch);  // [2 tiles][4 parts][128 rows]
+    // PV_g done (the bar_pv phases are waited one by one, in order)
+    auto wait_pv = [&](int g) {
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)(g & 1), abort_flag))) fail();
+      if (ok) tc_fence_after();
+    };
+
+    // rotated, scaled query rows of unit u (bf16 value and residual) into its tensor-memory
+    // columns, 8 dims (and their partners) at a time; with G > 1 the cos / sin of each token
+    // are computed once into a table its G rows share
+    auto stage_q = [&](int u) {
+      const int tok0 = tok0_u[u], tok = tok0 + tl;
       const unsigned long long pos = (unsigned long long)((long long)pos_off + len + tok);
       float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
       if (G > 1) {
@@ -366,17 +404,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           rope_cs((unsigned long long)((long long)pos_off + len + tok0 + t2), wsm[j], cs, sn);
           tab[t2 * kTabStride + j] = make_float2(cs, sn);
         }
-        asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory");
+        rows_sync();
       }
       // the query box (TMA, 128-byte swizzle): row r's 16-byte chunk c of each 64-dim half at
       // 128 r + 16 (c ^ (r & 7))
-      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_qraw), 0u, abort_flag))) fail();
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_qraw[u]), 0u, abort_flag))) fail();
+      const uint32_t qbox = sbase + kOffQraw + (uint32_t)(u * kQBox);
       uint32_t qh[16], ql[16];  // bf16 pairs of the row's dims (values, residuals)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float xa[8], xb[8];  // dims 16 hf + 8c + e and 64 + 16 hf + 8c + e
         if (tok < T && ok) {
-          const uint32_t qoff = sbase + kOffQraw + (uint32_t)(r * 128 + (((2 * hf + c) ^ (r & 7)) << 4));
+          const uint32_t qoff = qbox + (uint32_t)(r * 128 + (((2 * hf + c) ^ (r & 7)) << 4));
           const uint4 wa = ld_shared_v4(qoff), wb = ld_shared_v4(qoff + kQBoxHalf);
           const uint32_t va[4] = {wa.x, wa.y, wa.z, wa.w}, vb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
@@ -411,149 +450,169 @@ __global__ void __launch_bounds__(kThreads, 1)
           split2(xb[2 * e], xb[2 * e + 1], qh[8 + 4 * c + e], ql[8 + 4 * c + e]);
         }
       }
-      tmem_st8(tmem_base + lane_addr + kColQ + (uint32_t)(8 * hf), *reinterpret_cast<const uint32_t(*)[8]>(qh));
-      tmem_st8(tmem_base + lane_addr + kColQ + 32 + (uint32_t)(8 * hf), *reinterpret_cast<const uint32_t(*)[8]>(qh + 8));
-      tmem_st8(tmem_base + lane_addr + kColQlo + (uint32_t)(8 * hf), *reinterpret_cast<const uint32_t(*)[8]>(ql));
-      tmem_st8(tmem_base + lane_addr + kColQlo + 32 + (uint32_t)(8 * hf),
-               *reinterpret_cast<const uint32_t(*)[8]>(ql + 8));
+      const uint32_t qcol = tmem_base + lane_addr + kColQ + (uint32_t)u * kColQUnit + (uint32_t)(8 * hf);
+      tmem_st8(qcol, *reinterpret_cast<const uint32_t(*)[8]>(qh));
+      tmem_st8(qcol + 32, *reinterpret_cast<const uint32_t(*)[8]>(qh + 8));
+      tmem_st8(qcol + (kColQlo - kColQ), *reinterpret_cast<const uint32_t(*)[8]>(ql));
+      tmem_st8(qcol + (kColQlo - kColQ) + 32, *reinterpret_cast<const uint32_t(*)[8]>(ql + 8));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(bar_q));
-    }
-    float* xch = reinterpret_cast<float*>(smem + kSmemData + kOffXch);  // [2 tiles][4 parts][128 rows]
-    const int lim = len + min(tok, T - 1);
-    float m_used = -INFINITY, l_sum = 0.f;
-    // PV_{i-1} done (the bar_pv phases are waited one by one, in order)
-    auto wait_pv = [&](int j) {
-      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)(j & 1), abort_flag))) fail();
-      if (ok) tc_fence_after();
     };
-    for (int i = 0; i < nt; ++i) {
-      // (waits are made warp-uniform: the TMEM accesses below are warp-collective)
-      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_s[i & 1]), (uint32_t)((i >> 1) & 1), abort_flag)))
-        fail();
-      const bool local = i >= nt_mem;
-      const int key0 = local ? (i - nt_mem) * kKeys : i * kKeys;
-      const int n_valid = local ? min(kKeys, n_local - key0) : min(kKeys, M - key0);
-      float mx = -INFINITY;
-      float sv[16];
-      if (ok) {
-        tc_fence_after();
-        uint32_t sa[16];
-        tmem_ld16(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 16 * hf), sa);
-        tmem_wait_ld();
-        // this thread's 16 keys: all visible (a memory tile's first keys below M, or local
-        // keys up to the row's limit), or masked one by one
-        const int kfirst = key0 + 16 * hf;
-        const bool all_in = local ? kfirst + 15 <= lim : kfirst + 15 < M;
-        if (all_in) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            sv[e] = __uint_as_float(sa[e]);
-            mx = fmaxf(mx, sv[e]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int key = kfirst + e;
-            const bool v = local ? key <= lim : key < M;
-            sv[e] = v ? __uint_as_float(sa[e]) : -INFINITY;
-            mx = fmaxf(mx, sv[e]);
-          }
-        }
-      }
-      xch[((i & 1) * kParts + hf) * kRows + r] = mx;
-      pair_sync();  // (also: the row's four threads have read the score row before any writes P)
-#pragma unroll
-      for (int o = 1; o < kParts; ++o) mx = fmaxf(mx, xch[((i & 1) * kParts + ((hf + o) & 3)) * kRows + r]);
-      if (!ok) continue;
-      const bool need = mx > m_used + kHeadroom;  // (the same in both threads of the row)
-      const float m_old = m_used;
-      if (need) m_used = mx;
-      uint32_t pw[8], plw[8];
-      float psum = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float p0 = exp2f(sv[2 * e] - m_used), p1 = exp2f(sv[2 * e + 1] - m_used);
-        psum += p0 + p1;
-        split2(p0, p1, pw[e], plw[e]);
-      }
-      // key rows past the valid count: zero their V rows (this tile's stage; all row threads)
-      if (n_valid < kKeys) {
-        const uint32_t vt = sbase + kOffRing + (i % kStages) * kTileBytes + 2 * kKVHalf;
-        for (int idx = tid; idx < (kKeys - n_valid) * 16; idx += kRowWarps * 32) {
-          const int row = n_valid + (idx >> 4), c16 = idx & 15;
-          st_shared_v4(vt + (uint32_t)((c16 >> 3) * kKVHalf + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)), 0u, 0u, 0u,
-                       0u);
-        }
-      }
-      const bool rescale = __any_sync(0xffffffffu, need);
-      if (i > 0 && rescale) {  // O must be stable: PV_{i-1} done before it is rescaled
-        wait_pv(i - 1);
-        if (!ok) continue;
-        const float alpha = need ? exp2f(m_old - m_used) : 1.0f;
-        {  // this thread's 32 of the 128 output columns
-          uint32_t o[32];
-          const uint32_t col = kColO + (uint32_t)(32 * hf);
-          tmem_ld32(tmem_base + lane_addr + col, o);
+
+    // unit u's tiles (global numbers g0 ..): masked scores, weights into tensor memory, the
+    // running maximum and sum; the wait for its last PV is left to its output step
+    float m_used, l_sum;
+    auto run_tiles = [&](int u) {
+      const int g0 = u ? nt[0] : 0, ntu = nt[u];
+      const int tok = tok0_u[u] + tl;
+      const int lim = len + min(tok, T - 1);
+      m_used = -INFINITY;
+      l_sum = 0.f;
+      for (int i = 0; i < ntu; ++i) {
+        const int g = g0 + i;
+        // (waits are made warp-uniform: the TMEM accesses below are warp-collective)
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_s[g & 1]), (uint32_t)((g >> 1) & 1), abort_flag)))
+          fail();
+        const bool local = i >= nt_mem;
+        const int key0 = local ? (i - nt_mem) * kKeys : i * kKeys;
+        const int n_valid = local ? min(kKeys, n_local[u] - key0) : min(kKeys, M - key0);
+        float mx = -INFINITY;
+        float sv[16];
+        if (ok) {
+          tc_fence_after();
+          uint32_t sa[16];
+          tmem_ld16(tmem_base + lane_addr + (uint32_t)((g & 1) * kKeys + 16 * hf), sa);
           tmem_wait_ld();
+          // this thread's 16 keys: all visible (a memory tile's first keys below M, or local
+          // keys up to the row's limit), or masked one by one
+          const int kfirst = key0 + 16 * hf;
+          const bool all_in = local ? kfirst + 15 <= lim : kfirst + 15 < M;
+          if (all_in) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tmem_base + lane_addr + col, o);
+            for (int e = 0; e < 16; ++e) {
+              sv[e] = __uint_as_float(sa[e]);
+              mx = fmaxf(mx, sv[e]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int key = kfirst + e;
+              const bool v = local ? key <= lim : key < M;
+              sv[e] = v ? __uint_as_float(sa[e]) : -INFINITY;
+              mx = fmaxf(mx, sv[e]);
+            }
+          }
         }
-        if (need) l_sum *= alpha;
+        xch[((g & 1) * kParts + hf) * kRows + r] = mx;
+        pair_sync();  // (also: the row's four threads have read the score row before any writes P)
+#pragma unroll
+        for (int o = 1; o < kParts; ++o) mx = fmaxf(mx, xch[((g & 1) * kParts + ((hf + o) & 3)) * kRows + r]);
+        if (!ok) continue;
+        const bool need = mx > m_used + kHeadroom;  // (the same in the four threads of the row)
+        const float m_old = m_used;
+        if (need) m_used = mx;
+        uint32_t pw[8], plw[8];
+        float psum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float p0 = exp2f(sv[2 * e] - m_used), p1 = exp2f(sv[2 * e + 1] - m_used);
+          psum += p0 + p1;
+          split2(p0, p1, pw[e], plw[e]);
+        }
+        // key rows past the valid count: zero their V rows (this tile's stage; all row threads)
+        if (n_valid < kKeys) {
+          const uint32_t vt = sbase + kOffRing + (g % kStages) * kTileBytes + 2 * kKVHalf;
+          for (int idx = tid; idx < (kKeys - n_valid) * 16; idx += kRowWarps * 32) {
+            const int row = n_valid + (idx >> 4), c16 = idx & 15;
+            st_shared_v4(vt + (uint32_t)((c16 >> 3) * kKVHalf + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)), 0u, 0u,
+                         0u, 0u);
+          }
+        }
+        const bool rescale = __any_sync(0xffffffffu, need);
+        if (i > 0 && rescale) {  // O must be stable: PV_{g-1} done before it is rescaled
+          wait_pv(g - 1);
+          if (!ok) continue;
+          const float alpha = need ? exp2f(m_old - m_used) : 1.0f;
+          {  // this thread's 32 of the 128 output columns
+            uint32_t o[32];
+            const uint32_t col = kColO + (uint32_t)(32 * hf);
+            tmem_ld32(tmem_base + lane_addr + col, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tmem_base + lane_addr + col, o);
+          }
+          if (need) l_sum *= alpha;
+        }
+        // P_g over the scores it came from: values in columns 8 hf .. 8 hf + 7 of the tile's
+        // buffer, residuals 32 columns further
+        tmem_st8(tmem_base + lane_addr + (uint32_t)((g & 1) * kKeys + 8 * hf), pw);
+        tmem_st8(tmem_base + lane_addr + (uint32_t)((g & 1) * kKeys + kColPlo + 8 * hf), plw);
+        tmem_wait_st();
+        l_sum += psum;
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(bar_p));
+        if (i > 0 && !rescale) wait_pv(g - 1);  // (one wait per tile, in order)
       }
-      // P_i over the scores it came from: values in columns 8 hf .. 8 hf + 7 of the tile's
-      // buffer, residuals 32 columns further
-      tmem_st8(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + 8 * hf), pw);
-      tmem_st8(tmem_base + lane_addr + (uint32_t)((i & 1) * kKeys + kColPlo + 8 * hf), plw);
-      tmem_wait_st();
-      l_sum += psum;
-      fence_async_smem();
+    };
+
+    // unit u's output: its last PV, the row sums, O / sum as bf16 into the unit's query-box
+    // space (read long ago) in the layout of that box, then one TMA store per 64-dim half
+    // (rows past the block's last token fall outside the tensor and are not written)
+    auto output = [&](int u) {
+      const int g_end = (u ? nt[0] : 0) + nt[u];
+      wait_pv(g_end - 1);
+      // the row's sum of weights: all four parts (the exchange slot of tile g_end is free)
+      xch[((g_end & 1) * kParts + hf) * kRows + r] = l_sum;
+      pair_sync();
+      float sum = l_sum;
+#pragma unroll
+      for (int o = 1; o < kParts; ++o) sum += xch[((g_end & 1) * kParts + ((hf + o) & 3)) * kRows + r];
+      ok = __all_sync(0xffffffffu, ok);
+      const uint32_t stage_o = sbase + kOffQraw + (uint32_t)(u * kQBox);
+      if (ok) {
+        const float inv = 1.0f / sum;
+        uint32_t o[32];
+        tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)(32 * hf), o);
+        tmem_wait_ld();
+        const uint32_t half = stage_o + (uint32_t)((hf >> 1) * kQBoxHalf) + (uint32_t)(r * 128);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t w[4];
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            w[v] = pack2(__uint_as_float(o[8 * e + 2 * v]) * inv, __uint_as_float(o[8 * e + 2 * v + 1]) * inv);
+          const int c = 4 * (hf & 1) + e;
+          st_shared_v4(half + (uint32_t)((c ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+        }
+        fence_async_smem();
+      } else {
+        *abort_flag = 1;
+        if (lane == 0) msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+      }
+      // (O is read: from here the next unit's first PV may overwrite it)
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(bar_p));
-      if (i > 0 && !rescale) wait_pv(i - 1);  // (one wait per tile, in order)
-    }
-    if (nt > 0) wait_pv(nt - 1);
-    // the row's sum of weights: all four parts (the exchange slot of tile nt is free)
-    xch[((nt & 1) * kParts + hf) * kRows + r] = l_sum;
-    pair_sync();
-#pragma unroll
-    for (int o = 1; o < kParts; ++o) l_sum += xch[((nt & 1) * kParts + ((hf + o) & 3)) * kRows + r];
-    ok = __all_sync(0xffffffffu, ok);
-    // the output rows, bf16, into the query box's space (read long ago) in the layout of the
-    // query box, then one TMA store per 64-dim half (rows past the block's last token fall
-    // outside the tensor and are not written)
-    const uint32_t stage_o = sbase + kOffQraw;
-    if (ok) {
-      const float inv = 1.0f / l_sum;
-      uint32_t o[32];
-      tmem_ld32(tmem_base + lane_addr + kColO + (uint32_t)(32 * hf), o);
-      tmem_wait_ld();
-      const uint32_t half = stage_o + (uint32_t)((hf >> 1) * kQBoxHalf) + (uint32_t)(r * 128);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        uint32_t w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          w[u] = pack2(__uint_as_float(o[8 * e + 2 * u]) * inv, __uint_as_float(o[8 * e + 2 * u + 1]) * inv);
-        const int c = 4 * (hf & 1) + e;
-        st_shared_v4(half + (uint32_t)((c ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+      rows_sync();
+      if (tid == 0 && !*abort_flag) {
+        tma_store_4d(&tm_out, stage_o, 0, h * G, tok0_u[u], (int)bl);
+        tma_store_4d(&tm_out, stage_o + kQBoxHalf, kHalf, h * G, tok0_u[u], (int)bl);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
-      fence_async_smem();
-    } else {
-      *abort_flag = 1;
-      if (lane == 0) msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+    };
+
+    stage_q(0);
+    run_tiles(0);
+    if (n_units == 2) stage_q(1);
+    output(0);
+    if (n_units == 2) {
+      run_tiles(1);
+      output(1);
     }
-    asm volatile("bar.sync 5, %0;" ::"n"(kRowWarps * 32) : "memory");
-    if (tid == 0 && !*abort_flag) {
-      tma_store_4d(&tm_out, stage_o, 0, h * G, tok0, (int)bl);
-      tma_store_4d(&tm_out, stage_o + kQBoxHalf, kHalf, h * G, tok0, (int)bl);
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the box has been read out
-    }
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the boxes are read out
   }
 
   tc_fence_before();
@@ -624,12 +683,13 @@ int launch_g(const Args& a, cudaStream_t s, const char** why) {
     return 1;
   }
   const int tiles = (a.T + kRows / G - 1) / (kRows / G);
+  const int ctas_x = (tiles + 1) / 2;  // two token tiles per CTA (tile j with tile tiles - 1 - j)
   RopeW rw;
   for (int j = 0; j < kHalf; ++j) {
     const long double turns = exp2l(-2.0L * j / kD * (long double)a.log2_theta) / (2.0L * 3.14159265358979323846264338L);
     rw.step[j] = (unsigned long long)llroundl(ldexpl(turns, 64));
   }
-  prefill_tc_kernel<G><<<dim3(tiles, a.H, a.B * a.L), kThreads, kSmem, s>>>(
+  prefill_tc_kernel<G><<<dim3(ctas_x, a.H, a.B * a.L), kThreads, kSmem, s>>>(
       tm_mem, tm_lk, tm_lv, tm_q, tm_out, a.T, a.L, a.H, a.local_len, a.cap, a.mem_len, a.M_max, a.pos_off, rw,
       a.qscale, a.dev_err);
   if (cudaGetLastError() != cudaSuccess) {
