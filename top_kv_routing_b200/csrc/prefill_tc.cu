@@ -34,6 +34,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "prefill_tc.cuh"
 #include "tc_common.cuh"
@@ -56,8 +58,9 @@ constexpr int kTileBytes = 4 * kKVHalf;  // K (two halves) then V (two halves)
 constexpr int kOffRing = 0;
 constexpr int kQBoxHalf = kRows * 128;                    // 16 KB: 64 dims of the CTA's 128 rows
 constexpr int kQBox = 2 * kQBoxHalf;                      // 32 KB: one unit's query rows
-constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // per unit: its queries as loaded, later its output
-constexpr int kOffTab = kOffQraw + 2 * kQBox;              // cos / sin of a unit's tokens (G > 1)
+constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // a unit's queries as loaded
+constexpr int kOffOut = kOffQraw + kQBox;                  // a unit's output rows on their way out
+constexpr int kOffTab = kOffOut + kQBox;                   // cos / sin of a unit's tokens (G > 1)
 constexpr int kTabStride = kHalf + 1;                     // (a token's 64 angles + 1: the G-row groups of
                                                            // a warp read 8 tokens in distinct banks)
 constexpr int kTabBytes = 64 * kTabStride * 8;             // up to 64 tokens x 64 angles x float2
@@ -155,13 +158,66 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t sr
                : "memory");
 }
 
+// The CTA's work, in order: the valid units of the tile pairs p = blockIdx.x, + gridDim.x, ...
+// of the grid's (query, layer, key head) x pair list.  Pair j of (b, l, h) holds token tiles j
+// and n_tiles - 1 - j (a short and a long one under the causal mask; one unit when they
+// coincide).  Every role walks the same sequence; a pair whose cache cannot take the block
+// is skipped by all of them.
+struct UnitWalk {
+  int T, L, H, cap, M_max, n_tiles, pairs_x, n_pairs, kTok;
+  const int32_t* local_len;
+  const int32_t* mem_len;
+  // the current unit
+  int p, k, nu;       // pair, unit within it, units in it
+  int64_t bl;
+  int h, len, M, tok0, nt_mem, n_local, nt;
+  __device__ bool load_pair() {  // from p: the first pair whose cache takes the block
+    for (; p < n_pairs; p += gridDim.x) {
+      const int j = p % pairs_x;
+      h = (p / pairs_x) % H;
+      bl = p / (pairs_x * H);
+      len = local_len[bl / L];
+      if (len < 0 || len + T > cap) continue;  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
+      const int m = mem_len[bl];
+      M = m < 0 ? 0 : (m > M_max ? M_max : m);
+      nt_mem = (M + kKeys - 1) / kKeys;
+      nu = j == n_tiles - 1 - j ? 1 : 2;
+      k = 0;
+      return true;
+    }
+    return false;
+  }
+  __device__ void set_unit() {
+    const int j = p % pairs_x;
+    tok0 = (k == 0 ? j : n_tiles - 1 - j) * kTok;
+    n_local = len + min(T, tok0 + kTok);
+    nt = nt_mem + (n_local + kKeys - 1) / kKeys;
+  }
+  __device__ bool first() {
+    p = blockIdx.x;
+    if (!load_pair()) return false;
+    set_unit();
+    return true;
+  }
+  __device__ bool next() {
+    if (++k < nu) {
+      set_unit();
+      return true;
+    }
+    p += gridDim.x;
+    if (!load_pair()) return false;
+    set_unit();
+    return true;
+  }
+};
+
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_mem, const __grid_constant__ CUtensorMap tm_lk,
                       const __grid_constant__ CUtensorMap tm_lv, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_out, int T, int L,
                       int H, const int32_t* __restrict__ local_len, int cap, const int32_t* __restrict__ mem_len,
-                      int M_max, int pos_off, const __grid_constant__ RopeW rw, float qscale,
+                      int M_max, int pos_off, const __grid_constant__ RopeW rw, float qscale, int n_bl,
                       int32_t* dev_err) {
   constexpr int kTok = kRows / G;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -169,29 +225,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
-  uint64_t* bar_q = empty + kStages;     // a unit's queries written (16 warps; one phase per unit)
+  uint64_t* bar_q = empty + kStages;     // a unit's queries in tensor memory (16 warps; a phase per unit)
   uint64_t* bar_s = bar_q + 1;           // [2] scores ready
   uint64_t* bar_p = bar_s + 2;           // weights ready (16 warps)
   uint64_t* bar_pv = bar_p + 1;          // PV done
   uint64_t* drain = bar_pv + 1;
-  uint64_t* bar_qraw = drain + 1;        // [2] a unit's query box has landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 2);
+  uint64_t* bar_qraw = drain + 1;        // a unit's query box has landed (a phase per unit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   unsigned long long* wsm = reinterpret_cast<unsigned long long*>(smem + kSmemData + kOffW);
 
-  // two units of 128 rows per CTA: token tiles j and n_tiles - 1 - j of (b, l, h), a short
-  // and a long one under the causal mask (one unit when they coincide)
-  const int h = blockIdx.y;
-  const int64_t bl = blockIdx.z;
-  const int b = (int)(bl / L);
-  const int n_tiles = (T + kTok - 1) / kTok;
-  const int n_units = (int)blockIdx.x == n_tiles - 1 - (int)blockIdx.x ? 1 : 2;
-  const int tok0_u[2] = {(int)blockIdx.x * kTok, (n_tiles - 1 - (int)blockIdx.x) * kTok};
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
+  const int n_tiles = (T + kTok - 1) / kTok;
+  const int pairs_x = (n_tiles + 1) / 2;
+  UnitWalk walk{T, L, H, cap, M_max, n_tiles, pairs_x, pairs_x * H * n_bl, kTok, local_len, mem_len};
 
-  // thread 0: the barriers, then at once the units' query boxes (they do not depend on the
-  // lengths)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
@@ -203,35 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(bar_p), kRowWarps);
     mbar_init(smem_u32(bar_pv), 1);
     mbar_init(smem_u32(drain), 1);
-    mbar_init(smem_u32(&bar_qraw[0]), 1);
-    mbar_init(smem_u32(&bar_qraw[1]), 1);
+    mbar_init(smem_u32(bar_qraw), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
-    for (int u = 0; u < n_units; ++u) {
-      const uint32_t qb = smem_u32(&bar_qraw[u]), dst = sbase + kOffQraw + (uint32_t)(u * kQBox);
-      mbar_arrive_expect_tx(qb, kQBox);
-      tma_load_4d(dst, &tm_q, qb, 0, h * G, tok0_u[u], (int)bl);
-      tma_load_4d(dst + kQBoxHalf, &tm_q, qb, kHalf, h * G, tok0_u[u], (int)bl);
-    }
   }
-  const int len = local_len[b];
-  int M = mem_len[bl];
-  if (len < 0 || len + T > cap) {  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
-    if (tid == 0)  // the query boxes land before the CTA leaves
-      for (int u = 0; u < n_units; ++u) mbar_drain(smem_u32(&bar_qraw[u]), 0u);
-    return;
-  }
-  M = M < 0 ? 0 : (M > M_max ? M_max : M);
-  const int nt_mem = (M + kKeys - 1) / kKeys;
-  // per unit: local keys up to its last token, tiles; the units' tiles are numbered on from
-  // one to the next (g = unit 0's 0 .. nt[0] - 1, then unit 1's)
-  int n_local[2], nt[2];
-  for (int u = 0; u < 2; ++u) {
-    n_local[u] = len + min(T, tok0_u[u] + kTok);
-    nt[u] = nt_mem + (n_local[u] + kKeys - 1) / kKeys;
-  }
-  const int nt_all = nt[0] + (n_units == 2 ? nt[1] : 0);
   if (tid < kHalf) wsm[tid] = rw.step[tid];  // (indexed per lane: read from shared memory below)
   if (warp == kMmaWarp) {
     tmem_alloc<false>(smem_u32(tmem_slot), kTmemCols);
@@ -244,7 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
-      // ---------------- TMA producer: every tile of unit 0, then of unit 1
+      // ---------------- TMA producer: per unit its query box (once the previous unit's
+      // queries have been read out of the box's space), then its K / V tiles
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lk)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lv)) : "memory");
@@ -253,60 +280,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       int armed[kStages];
 #pragma unroll
       for (int st = 0; st < kStages; ++st) armed[st] = -1;
+      int qarmed = -1;
       bool ok = true;
-      for (int g = 0; g < nt_all && ok; ++g) {
-        const int i = g < nt[0] ? g : g - nt[0];  // the unit's own tile
-        const int stage = g % kStages;
-        const uint32_t ph = (uint32_t)((g / kStages) & 1);
-        if (!mbar_wait(smem_u32(&empty[stage]), ph ^ 1u, abort_flag)) {
+      int g = 0, vu = 0;
+      for (bool more = walk.first(); more && ok; more = walk.next(), ++vu) {
+        if (vu > 0 && !mbar_wait(smem_u32(bar_q), (uint32_t)((vu - 1) & 1), abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t fb = smem_u32(&full[stage]);
-        const uint32_t dst = sbase + kOffRing + stage * kTileBytes;
-        mbar_arrive_expect_tx(fb, kTileBytes);
-        if (i < nt_mem) {
-          const int rk = (int)((((bl * 2 + 0) * H + h) * (int64_t)M_max) + i * kKeys);
-          const int rv = (int)((((bl * 2 + 1) * H + h) * (int64_t)M_max) + i * kKeys);
-          tma_load_2d(dst, &tm_mem, fb, 0, rk, pol);
-          tma_load_2d(dst + kKVHalf, &tm_mem, fb, kHalf, rk, pol);
-          tma_load_2d(dst + 2 * kKVHalf, &tm_mem, fb, 0, rv, pol);
-          tma_load_2d(dst + 3 * kKVHalf, &tm_mem, fb, kHalf, rv, pol);
-        } else {
-          const int r = (int)((bl * H + h) * (int64_t)cap + (int64_t)(i - nt_mem) * kKeys);
-          tma_load_2d(dst, &tm_lk, fb, 0, r, pol);
-          tma_load_2d(dst + kKVHalf, &tm_lk, fb, kHalf, r, pol);
-          tma_load_2d(dst + 2 * kKVHalf, &tm_lv, fb, 0, r, pol);
-          tma_load_2d(dst + 3 * kKVHalf, &tm_lv, fb, kHalf, r, pol);
+        const uint32_t qb = smem_u32(bar_qraw);
+        mbar_arrive_expect_tx(qb, kQBox);
+        tma_load_4d(sbase + kOffQraw, &tm_q, qb, 0, walk.h * G, walk.tok0, (int)walk.bl);
+        tma_load_4d(sbase + kOffQraw + kQBoxHalf, &tm_q, qb, kHalf, walk.h * G, walk.tok0, (int)walk.bl);
+        qarmed = vu & 1;
+        for (int i = 0; i < walk.nt; ++i, ++g) {
+          const int stage = g % kStages;
+          const uint32_t ph = (uint32_t)((g / kStages) & 1);
+          if (!mbar_wait(smem_u32(&empty[stage]), ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[stage]);
+          const uint32_t dst = sbase + kOffRing + stage * kTileBytes;
+          mbar_arrive_expect_tx(fb, kTileBytes);
+          if (i < walk.nt_mem) {
+            const int rk = (int)((((walk.bl * 2 + 0) * H + walk.h) * (int64_t)M_max) + i * kKeys);
+            const int rv = (int)((((walk.bl * 2 + 1) * H + walk.h) * (int64_t)M_max) + i * kKeys);
+            tma_load_2d(dst, &tm_mem, fb, 0, rk, pol);
+            tma_load_2d(dst + kKVHalf, &tm_mem, fb, kHalf, rk, pol);
+            tma_load_2d(dst + 2 * kKVHalf, &tm_mem, fb, 0, rv, pol);
+            tma_load_2d(dst + 3 * kKVHalf, &tm_mem, fb, kHalf, rv, pol);
+          } else {
+            const int r = (int)((walk.bl * H + walk.h) * (int64_t)cap + (int64_t)(i - walk.nt_mem) * kKeys);
+            tma_load_2d(dst, &tm_lk, fb, 0, r, pol);
+            tma_load_2d(dst + kKVHalf, &tm_lk, fb, kHalf, r, pol);
+            tma_load_2d(dst + 2 * kKVHalf, &tm_lv, fb, 0, r, pol);
+            tma_load_2d(dst + 3 * kKVHalf, &tm_lv, fb, kHalf, r, pol);
+          }
+          armed[stage] = (int)ph;
         }
-        armed[stage] = (int)ph;
       }
       if (!ok) {
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
         for (int s = 0; s < kStages; ++s)
           if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
-        for (int u = 0; u < n_units; ++u) mbar_drain(smem_u32(&bar_qraw[u]), 0u);
+        if (qarmed >= 0) mbar_drain(smem_u32(bar_qraw), (uint32_t)qarmed);
       }
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer: the warp waits together, one elected lane issues (the
     // tensor-core operations of that lane run in order, so S_{g+2}, written over P_g,
-    // follows the PV that reads P_g).  A unit's first score tile waits for its queries.
+    // follows the PV that reads P_g).  A unit's first score tile waits for its queries;
+    // unit v's queries sit in tensor-memory columns 256 + 128 (v & 1).
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
     constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
     bool ok = true, issued = false;
-    for (int g = 0; g <= nt_all && ok; ++g) {
-      if (g < nt_all) {
-        const int u = g < nt[0] ? 0 : 1, i = g - (u ? nt[0] : 0);
-        if (i == 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), (uint32_t)u, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+    int g = 0, vu = 0;
+    bool prev_first = false;  // tile g - 1 starts its unit's O
+    auto pv = [&](int j, bool starts) {  // PV of tile j
+      const int stage = j % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_p), (uint32_t)(j & 1), abort_flag))) return false;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t vt = sbase + kOffRing + stage * kTileBytes + 2 * kKVHalf;
+        const uint32_t p_tmem = tmem_base + (uint32_t)((j & 1) * kKeys);  // P_j: 64 bf16 in 32 columns
+#pragma unroll
+        for (int ks = 0; ks < kKeys / 16; ++ks) {
+          const uint64_t vdesc = sw128_desc_mn(vt + (uint32_t)(ks * 2048), kKVHalf, 1024);
+          umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (!starts || ks > 0) ? 1u : 0u);
+          umma_ts(tmem_base + kColO, p_tmem + kColPlo + (uint32_t)(8 * ks), vdesc, idesc_pv, 1u);
         }
+        umma_commit<false>(smem_u32(bar_pv));
+        umma_commit<false>(smem_u32(&empty[stage]));
+      }
+      __syncwarp();
+      return true;
+    };
+    for (bool more = walk.first(); more && ok; more = walk.next(), ++vu) {
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), (uint32_t)(vu & 1), abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t q_t = tmem_base + kColQ + (uint32_t)(vu & 1) * kColQUnit;
+      for (int i = 0; i < walk.nt; ++i, ++g) {
         const int stage = g % kStages;
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((g / kStages) & 1), abort_flag))) {
           ok = false;
@@ -316,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           const uint32_t kt = sbase + kOffRing + stage * kTileBytes;
           const uint32_t d_s = tmem_base + (uint32_t)((g & 1) * kKeys);
-          const uint32_t q_t = tmem_base + kColQ + (uint32_t)u * kColQUnit;
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint64_t kdesc = sw128_desc(kt + (uint32_t)((ks >> 2) * kKVHalf)) + (uint64_t)(2 * (ks & 3));
@@ -327,30 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         issued = true;
         __syncwarp();
-      }
-      if (g >= 1) {
-        const int j = g - 1, stage = j % kStages;
-        const int jj = j < nt[0] ? j : j - nt[0];  // its index in its unit: 0 starts the unit's O
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_p), (uint32_t)(j & 1), abort_flag))) {
+        if (g >= 1 && !pv(g - 1, prev_first)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (leader) {
-          const uint32_t vt = sbase + kOffRing + stage * kTileBytes + 2 * kKVHalf;
-          const uint32_t p_tmem = tmem_base + (uint32_t)((j & 1) * kKeys);  // P_j: 64 bf16 in 32 columns
-#pragma unroll
-          for (int ks = 0; ks < kKeys / 16; ++ks) {
-            const uint64_t vdesc = sw128_desc_mn(vt + (uint32_t)(ks * 2048), kKVHalf, 1024);
-            umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
-            umma_ts(tmem_base + kColO, p_tmem + kColPlo + (uint32_t)(8 * ks), vdesc, idesc_pv, 1u);
-          }
-          umma_commit<false>(smem_u32(bar_pv));
-          umma_commit<false>(smem_u32(&empty[stage]));
-        }
-        __syncwarp();
+        prev_first = i == 0;
       }
     }
+    if (ok && g >= 1 && !pv(g - 1, prev_first)) ok = false;  // the last tile's PV
     if (!ok) {
       if (lane == 0) {
         *abort_flag = 1;
@@ -366,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- rows (warps 0..15): thread (row r = TMEM lane, part hf of 4) takes the
     // row's dims 16 hf .. 16 hf + 15 and 64 + 16 hf .. 79 + 16 hf of the query, and keys
     // 16 hf .. 16 hf + 15 of every tile; the four meet in shared memory (warps w, w + 4,
-    // w + 8, w + 12).  Order: unit 0's queries and tiles; unit 1's queries (so that its first
-    // score tiles run under what follows); unit 0's output; unit 1's tiles and output.
+    // w + 8, w + 12).  Per unit: its queries (so that its first score tiles run under what
+    // follows), the previous unit's output, its tiles.
     const int r = tid & (kRows - 1), hf = tid >> 7;
     const int tl = r / G;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
@@ -390,32 +432,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) tc_fence_after();
     };
 
-    // rotated, scaled query rows of unit u (bf16 value and residual) into its tensor-memory
+    // unit v's rotated, scaled query rows (bf16 value and residual) into its tensor-memory
     // columns, 8 dims (and their partners) at a time; with G > 1 the cos / sin of each token
     // are computed once into a table its G rows share
-    auto stage_q = [&](int u) {
-      const int tok0 = tok0_u[u], tok = tok0 + tl;
-      const unsigned long long pos = (unsigned long long)((long long)pos_off + len + tok);
+    auto stage_q = [&](const UnitWalk& w, int v) {
+      const int tok0 = w.tok0, tok = tok0 + tl;
+      const unsigned long long pos = (unsigned long long)((long long)pos_off + w.len + tok);
       float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
       if (G > 1) {
         for (int e = tid; e < kTok * kHalf; e += kRowWarps * 32) {
           const int t2 = e / kHalf, j = e % kHalf;
           float sn, cs;
-          rope_cs((unsigned long long)((long long)pos_off + len + tok0 + t2), wsm[j], cs, sn);
+          rope_cs((unsigned long long)((long long)pos_off + w.len + tok0 + t2), wsm[j], cs, sn);
           tab[t2 * kTabStride + j] = make_float2(cs, sn);
         }
         rows_sync();
       }
       // the query box (TMA, 128-byte swizzle): row r's 16-byte chunk c of each 64-dim half at
       // 128 r + 16 (c ^ (r & 7))
-      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_qraw[u]), 0u, abort_flag))) fail();
-      const uint32_t qbox = sbase + kOffQraw + (uint32_t)(u * kQBox);
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_qraw), (uint32_t)(v & 1), abort_flag))) fail();
       uint32_t qh[16], ql[16];  // bf16 pairs of the row's dims (values, residuals)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float xa[8], xb[8];  // dims 16 hf + 8c + e and 64 + 16 hf + 8c + e
         if (tok < T && ok) {
-          const uint32_t qoff = qbox + (uint32_t)(r * 128 + (((2 * hf + c) ^ (r & 7)) << 4));
+          const uint32_t qoff = sbase + kOffQraw + (uint32_t)(r * 128 + (((2 * hf + c) ^ (r & 7)) << 4));
           const uint4 wa = ld_shared_v4(qoff), wb = ld_shared_v4(qoff + kQBoxHalf);
           const uint32_t va[4] = {wa.x, wa.y, wa.z, wa.w}, vb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
@@ -450,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           split2(xb[2 * e], xb[2 * e + 1], qh[8 + 4 * c + e], ql[8 + 4 * c + e]);
         }
       }
-      const uint32_t qcol = tmem_base + lane_addr + kColQ + (uint32_t)u * kColQUnit + (uint32_t)(8 * hf);
+      const uint32_t qcol = tmem_base + lane_addr + kColQ + (uint32_t)(v & 1) * kColQUnit + (uint32_t)(8 * hf);
       tmem_st8(qcol, *reinterpret_cast<const uint32_t(*)[8]>(qh));
       tmem_st8(qcol + 32, *reinterpret_cast<const uint32_t(*)[8]>(qh + 8));
       tmem_st8(qcol + (kColQlo - kColQ), *reinterpret_cast<const uint32_t(*)[8]>(ql));
@@ -461,23 +502,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(smem_u32(bar_q));
     };
 
-    // unit u's tiles (global numbers g0 ..): masked scores, weights into tensor memory, the
+    // a unit's tiles (global numbers g0 ..): masked scores, weights into tensor memory, the
     // running maximum and sum; the wait for its last PV is left to its output step
-    float m_used, l_sum;
-    auto run_tiles = [&](int u) {
-      const int g0 = u ? nt[0] : 0, ntu = nt[u];
-      const int tok = tok0_u[u] + tl;
-      const int lim = len + min(tok, T - 1);
+    float m_used = -INFINITY, l_sum = 0.f;
+    auto run_tiles = [&](const UnitWalk& w, int g0) {
+      const int tok = w.tok0 + tl;
+      const int lim = w.len + min(tok, T - 1);
       m_used = -INFINITY;
       l_sum = 0.f;
-      for (int i = 0; i < ntu; ++i) {
+      for (int i = 0; i < w.nt; ++i) {
         const int g = g0 + i;
         // (waits are made warp-uniform: the TMEM accesses below are warp-collective)
         if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_s[g & 1]), (uint32_t)((g >> 1) & 1), abort_flag)))
           fail();
-        const bool local = i >= nt_mem;
-        const int key0 = local ? (i - nt_mem) * kKeys : i * kKeys;
-        const int n_valid = local ? min(kKeys, n_local[u] - key0) : min(kKeys, M - key0);
+        const bool local = i >= w.nt_mem;
+        const int key0 = local ? (i - w.nt_mem) * kKeys : i * kKeys;
+        const int n_valid = local ? min(kKeys, w.n_local - key0) : min(kKeys, w.M - key0);
         float mx = -INFINITY;
         float sv[16];
         if (ok) {
@@ -488,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // this thread's 16 keys: all visible (a memory tile's first keys below M, or local
           // keys up to the row's limit), or masked one by one
           const int kfirst = key0 + 16 * hf;
-          const bool all_in = local ? kfirst + 15 <= lim : kfirst + 15 < M;
+          const bool all_in = local ? kfirst + 15 <= lim : kfirst + 15 < w.M;
           if (all_in) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -499,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int key = kfirst + e;
-              const bool v = local ? key <= lim : key < M;
-              sv[e] = v ? __uint_as_float(sa[e]) : -INFINITY;
+              const bool vis = local ? key <= lim : key < w.M;
+              sv[e] = vis ? __uint_as_float(sa[e]) : -INFINITY;
               mx = fmaxf(mx, sv[e]);
             }
           }
@@ -560,20 +600,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 
-    // unit u's output: its last PV, the row sums, O / sum as bf16 into the unit's query-box
-    // space (read long ago) in the layout of that box, then one TMA store per 64-dim half
-    // (rows past the block's last token fall outside the tensor and are not written)
-    auto output = [&](int u) {
-      const int g_end = (u ? nt[0] : 0) + nt[u];
+    // a unit's output: its last PV (tile g_end - 1), the row sums, O / sum as bf16 into the
+    // output box's space in the layout of the query box (once the previous unit's store has
+    // read it), then one TMA store per 64-dim half (rows past the block's last token fall
+    // outside the tensor and are not written)
+    auto output = [&](int64_t obl, int oh, int otok0, int g_end, float sum) {
       wait_pv(g_end - 1);
       // the row's sum of weights: all four parts (the exchange slot of tile g_end is free)
-      xch[((g_end & 1) * kParts + hf) * kRows + r] = l_sum;
+      xch[((g_end & 1) * kParts + hf) * kRows + r] = sum;
       pair_sync();
-      float sum = l_sum;
 #pragma unroll
       for (int o = 1; o < kParts; ++o) sum += xch[((g_end & 1) * kParts + ((hf + o) & 3)) * kRows + r];
       ok = __all_sync(0xffffffffu, ok);
-      const uint32_t stage_o = sbase + kOffQraw + (uint32_t)(u * kQBox);
+      if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the previous store
+      rows_sync();
+      const uint32_t stage_o = sbase + kOffOut;
       if (ok) {
         const float inv = 1.0f / sum;
         uint32_t o[32];
@@ -582,12 +623,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t half = stage_o + (uint32_t)((hf >> 1) * kQBoxHalf) + (uint32_t)(r * 128);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          uint32_t w[4];
+          uint32_t wd[4];
 #pragma unroll
           for (int v = 0; v < 4; ++v)
-            w[v] = pack2(__uint_as_float(o[8 * e + 2 * v]) * inv, __uint_as_float(o[8 * e + 2 * v + 1]) * inv);
+            wd[v] = pack2(__uint_as_float(o[8 * e + 2 * v]) * inv, __uint_as_float(o[8 * e + 2 * v + 1]) * inv);
           const int c = 4 * (hf & 1) + e;
-          st_shared_v4(half + (uint32_t)((c ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+          st_shared_v4(half + (uint32_t)((c ^ (r & 7)) << 4), wd[0], wd[1], wd[2], wd[3]);
         }
         fence_async_smem();
       } else {
@@ -598,21 +639,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       rows_sync();
       if (tid == 0 && !*abort_flag) {
-        tma_store_4d(&tm_out, stage_o, 0, h * G, tok0_u[u], (int)bl);
-        tma_store_4d(&tm_out, stage_o + kQBoxHalf, kHalf, h * G, tok0_u[u], (int)bl);
+        tma_store_4d(&tm_out, stage_o, 0, oh * G, otok0, (int)obl);
+        tma_store_4d(&tm_out, stage_o + kQBoxHalf, kHalf, oh * G, otok0, (int)obl);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
     };
 
-    stage_q(0);
-    run_tiles(0);
-    if (n_units == 2) stage_q(1);
-    output(0);
-    if (n_units == 2) {
-      run_tiles(1);
-      output(1);
+    bool have_prev = false;
+    int64_t prev_bl = 0;
+    int prev_h = 0, prev_tok0 = 0, g = 0, vu = 0;
+    for (bool more = walk.first(); more; more = walk.next(), ++vu) {
+      stage_q(walk, vu);
+      if (have_prev) output(prev_bl, prev_h, prev_tok0, g, l_sum);
+      run_tiles(walk, g);
+      g += walk.nt;
+      have_prev = true;
+      prev_bl = walk.bl;
+      prev_h = walk.h;
+      prev_tok0 = walk.tok0;
     }
-    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the boxes are read out
+    if (have_prev) output(prev_bl, prev_h, prev_tok0, g, l_sum);
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the last box is read out
   }
 
   tc_fence_before();
@@ -683,15 +730,18 @@ int launch_g(const Args& a, cudaStream_t s, const char** why) {
     return 1;
   }
   const int tiles = (a.T + kRows / G - 1) / (kRows / G);
-  const int ctas_x = (tiles + 1) / 2;  // two token tiles per CTA (tile j with tile tiles - 1 - j)
+  // persistent: at most one CTA per SM, each walking its share of the (tile pair, key head,
+  // query x layer) list
+  const int64_t pairs = (int64_t)(tiles + 1) / 2 * a.H * a.B * a.L;
+  const int ctas = (int)std::min<int64_t>(pairs, std::max(1, msa::sm_count()));
   RopeW rw;
   for (int j = 0; j < kHalf; ++j) {
     const long double turns = exp2l(-2.0L * j / kD * (long double)a.log2_theta) / (2.0L * 3.14159265358979323846264338L);
     rw.step[j] = (unsigned long long)llroundl(ldexpl(turns, 64));
   }
-  prefill_tc_kernel<G><<<dim3(ctas_x, a.H, a.B * a.L), kThreads, kSmem, s>>>(
+  prefill_tc_kernel<G><<<dim3(ctas, 1, 1), kThreads, kSmem, s>>>(
       tm_mem, tm_lk, tm_lv, tm_q, tm_out, a.T, a.L, a.H, a.local_len, a.cap, a.mem_len, a.M_max, a.pos_off, rw,
-      a.qscale, a.dev_err);
+      a.qscale, a.B * a.L, a.dev_err);
   if (cudaGetLastError() != cudaSuccess) {
     *why = "kernel launch";
     return 1;
