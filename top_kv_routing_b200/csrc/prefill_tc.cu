@@ -226,10 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
   uint64_t* bar_q = empty + kStages;     // a unit's queries in tensor memory (16 warps; a phase per unit)
-  uint64_t* bar_s = bar_q + 1;           // [2] scores ready
-  uint64_t* bar_p = bar_s + 2;           // weights ready (16 warps)
-  uint64_t* bar_pv = bar_p + 1;          // PV done
-  uint64_t* drain = bar_pv + 1;
+  // scores ready, weights ready (16 warps) and PV done, one of each per score buffer: tile
+  // g's phase is g / 2 of barrier g % 2, so neither side can complete a phase the other has
+  // not waited for yet
+  uint64_t* bar_s = bar_q + 1;           // [2]
+  uint64_t* bar_p = bar_s + 2;           // [2]
+  uint64_t* bar_pv = bar_p + 2;          // [2]
+  uint64_t* drain = bar_pv + 2;
   uint64_t* bar_qraw = drain + 1;        // a unit's query box has landed (a phase per unit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -247,10 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(bar_q), kRowWarps);
-    mbar_init(smem_u32(&bar_s[0]), 1);
-    mbar_init(smem_u32(&bar_s[1]), 1);
-    mbar_init(smem_u32(bar_p), kRowWarps);
-    mbar_init(smem_u32(bar_pv), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bar_s[s]), 1);
+      mbar_init(smem_u32(&bar_p[s]), kRowWarps);
+      mbar_init(smem_u32(&bar_pv[s]), 1);
+    }
     mbar_init(smem_u32(drain), 1);
     mbar_init(smem_u32(bar_qraw), 1);
     *abort_flag = 0;
@@ -341,7 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool prev_first = false;  // tile g - 1 starts its unit's O
     auto pv = [&](int j, bool starts) {  // PV of tile j
       const int stage = j % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_p), (uint32_t)(j & 1), abort_flag))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_p[j & 1]), (uint32_t)((j >> 1) & 1), abort_flag)))
+        return false;
       tc_fence_after();
       if (leader) {
         const uint32_t vt = sbase + kOffRing + stage * kTileBytes + 2 * kKVHalf;
@@ -352,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (!starts || ks > 0) ? 1u : 0u);
           umma_ts(tmem_base + kColO, p_tmem + kColPlo + (uint32_t)(8 * ks), vdesc, idesc_pv, 1u);
         }
-        umma_commit<false>(smem_u32(bar_pv));
+        umma_commit<false>(smem_u32(&bar_pv[j & 1]));
         umma_commit<false>(smem_u32(&empty[stage]));
       }
       __syncwarp();
@@ -426,9 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
     };
     float* xch = reinterpret_cast<float*>(smem + kSmemData + kOffXch);  // [2 tiles][4 parts][128 rows]
-    // PV_g done (the bar_pv phases are waited one by one, in order)
+    // PV_g done (the PV phases are waited one by one, in order)
     auto wait_pv = [&](int g) {
-      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_pv), (uint32_t)(g & 1), abort_flag))) fail();
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_pv[g & 1]), (uint32_t)((g >> 1) & 1), abort_flag)))
+        fail();
       if (ok) tc_fence_after();
     };
 
@@ -595,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(bar_p));
+        if (lane == 0) mbar_arrive(smem_u32(&bar_p[g & 1]));
         if (i > 0 && !rescale) wait_pv(g - 1);  // (one wait per tile, in order)
       }
     };
