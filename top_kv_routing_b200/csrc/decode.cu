@@ -195,8 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
         cp_async16(st + row * kRowBytes + ((chunk ^ (row & 7)) << 4), src, ok ? 16u : 0u);
       }
     };
+    // all three stages requested at once (a stage is refilled as soon as its tile is used)
 #pragma unroll
-    for (int p = 0; p < kStages - 1; ++p) {
+    for (int p = 0; p < kStages; ++p) {
       if (p < my_n) issue(p);
       cp_async_commit();
     }
@@ -269,10 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     float m = -INFINITY, lsum = 0.f;
     for (int i = 0; i < my_n; ++i) {
-      __syncwarp();  // every lane is done with the stage about to be refilled
-      if (i + kStages - 1 < my_n) issue(i + kStages - 1);
-      cp_async_commit();
-      cp_async_wait<kStages - 1>();
+      cp_async_wait<kStages - 1>();  // (3 + i groups committed: tile i has landed)
       __syncwarp();
       const Tile tl = tile(i);
       const uint32_t st = my_ring + (i % kStages) * kStageBytes;
@@ -344,6 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
         mma_bf16(o[2 * i2], pa, v0, v1);
         mma_bf16(o[2 * i2 + 1], pa, v2, v3);
       }
+      __syncwarp();  // every lane is done with the stage: refill it with tile i + 3
+      if (i + kStages < my_n) issue(i + kStages);
+      cp_async_commit();
     }
     cp_async_wait<0>();
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
