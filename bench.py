@@ -572,7 +572,7 @@ def time_bf16_filter(dev, eng, qs):
     return out
 
 
-SWEEP_T = (1, 2, 4, 8, 64, 256, 1024)  # the workload's sweep {1, 8, 64, 256, 1024} plus 2 and 4
+SWEEP_T = (1, 2, 4, 8, 16, 32, 64, 256, 1024)  # the workload's sweep {1, 8, 64, 256, 1024} plus 2, 4, 16, 32
 
 
 def time_sweep(dev, f8: bool):
