@@ -41,9 +41,10 @@ extern "C" {
  *   The caller owns every buffer; the call allocates nothing.
  * Three kernel launches on `stream` (append, attention, advance), asynchronous and
  * graph-capturable (every per-call quantity that changes is read on the device).  The
- * attention kernel runs on the tcgen05 tensor cores: one CTA per (query, layer, key head,
- * 128 / G tokens), the 128 (token, query head) rows as the MMA's M, K/V streaming in tiles
- * of 64 keys, scores and output in tensor memory.
+ * attention kernel runs on the tcgen05 tensor cores: at most one CTA per SM, each walking
+ * units of 128 (token, query head) rows (the MMA's M) of its share of the (query, layer,
+ * key head, token tile) list, K/V streaming in tiles of 64 keys, the query, scores,
+ * weights and output in tensor memory.
  * A query whose cache cannot hold the whole block (local_len + n_new > local_cap) is
  * skipped (out and cache untouched, length not advanced) and sets MSA_DEVERR_LOCAL_FULL;
  * mem_len > max_mem_chunks is clamped with MSA_DEVERR_CAPACITY.  Host-checked argument

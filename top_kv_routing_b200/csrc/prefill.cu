@@ -9,8 +9,8 @@
 //
 // Three launches: (1) the new keys are rotated (RoPE at position offset + local index),
 // rounded to the cache's bf16 and appended with the new values; (2) attention on the
-// tcgen05 tensor cores (prefill_tc.cu), 128 (token, query head) rows per CTA; (3)
-// local_len += n_new.
+// tcgen05 tensor cores (prefill_tc.cu), persistent CTAs taking 128 (token, query head)
+// rows at a time; (3) local_len += n_new.
 #include "common.cuh"
 #include "msa_prefill.h"
 #include "prefill_tc.cuh"
