@@ -6,35 +6,27 @@
 // times the values.  Follows "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", section
 // 推理流水线, and the MSA paper reading notes, section 推理全流程.
 //
-// Persistent CTAs of 576 threads, at most one per SM.  A unit is 128 rows: 128 / G tokens x
-// the G query heads of key head h.  CTA c walks the tile pairs c, c + gridDim.x, ... of the
-// (query x layer, key head, pair) list, pair j holding token tiles j and n_tiles - 1 - j (a
-// short and a long one under the causal mask), one unit at a time:
-//   warp 17, one thread  TMA producer: per unit its query rows as a 4D box (once the
-//                        previous unit's queries are in tensor memory), then its tiles of
-//                        64 keys (K as two 64-column boxes, then V the same), 128-byte
-//                        swizzle, a 3-stage ring; memory tiles first, then local tiles up to
-//                        the unit's last token
-//   warp 16              MMA issuer (the warp waits, one elected lane issues): S_g = Q K_g^T
-//                        (M = 128, N = 64, K = 128, the query read from tensor memory) into
-//                        score buffer g % 2, then O += P_{g-1} V_{g-1} (M = 128, N = 128,
-//                        K = 64) into the TMEM output, P read from tensor memory (it replaces
-//                        the scores it was computed from), V read MN-major from its [key][d]
-//                        rows.  The rotated queries and the weights are each a bf16 value
-//                        plus a bf16 residual (two MMAs); keys and values exact bf16; fp32
-//                        accumulation.  g runs on from unit to unit.
+// One CTA (576 threads) per 128 rows: 128 / G tokens x the G query heads of key head h.
+//   warp 17, one thread  TMA producer: tiles of 64 keys (K as two 64-column boxes, then V
+//                        the same), 128-byte swizzle, a 3-stage ring; memory tiles first,
+//                        then local tiles up to the CTA's last token
+//   warp 16, one thread  MMA issuer: S_i = Q K_i^T (M = 128, N = 64, K = 128) into one of two
+//                        TMEM score buffers, then O += P_{i-1} V_{i-1} (M = 128, N = 128,
+//                        K = 64) into the TMEM output, with P read from tensor memory (it
+//                        replaces the scores it was computed from) and V read MN-major
+//                        straight from its [key][d] rows.  The rotated queries and the
+//                        weights are each a bf16 value plus a bf16 residual (two MMAs); keys
+//                        and values exact bf16; fp32 accumulation
 //   warps 0..15          four threads per row (TMEM lane), each with a quarter of the row's
-//                        dims and of every tile's keys.  Per unit: rotate and scale the
-//                        query rows into tensor memory (RoPE table of the unit's tokens,
-//                        64-bit fixed-point angles); then the previous unit's output: O /
-//                        sum as bf16 through a shared-memory box, one TMA store; then per
-//                        tile read the score row, mask it (memory keys < M, local keys <= its
-//                        own local index), keep a running maximum that is raised (and O
-//                        rescaled in TMEM) only when a score exceeds it by more than 2^8,
-//                        and write the weights exp2(s - m) into the tile's score columns
-//                        (values in the first 32, residuals in the last 32).
+//                        dims and of every tile's keys: build the rotated, scaled query row
+//                        in shared memory; per tile read the score row, mask it (memory keys
+//                        < M, local keys <= its own local index), keep a running maximum
+//                        that is raised (and O rescaled in TMEM) only when a score exceeds
+//                        it by more than 2^8, write the weights exp2(s - m) into the tile's
+//                        score columns (values in the first 32, residuals in the last 32),
+//                        and at the end divide O by the running sum.
 // Weights of a tile are written while the previous tile's PV runs: the row threads wait
-// for PV_{g-1} after releasing P_g (before, only when O must be rescaled).  Key rows past a
+// for PV_{i-1} after releasing P_i (before, only when O must be rescaled).  Key rows past a
 // tile's valid count are zeroed in shared memory before the PV that reads them (the cache
 // rows beyond the valid length may hold anything).  Every wait is bounded (2 s); a timeout
 // sets MSA_DEVERR_TIMEOUT and the CTA drains and frees its TMEM.
@@ -76,14 +68,14 @@ constexpr int kSmemData = kOffTab + kTabBytes;
 constexpr int kOffXch = 256;                                 // after the barriers: the rows' exchange buffer
 constexpr int kOffW = kOffXch + 2 * kParts * kRows * 4;      // then the RoPE frequencies (64 x 8 bytes)
 constexpr int kSmem = kSmemData + 1024 + kOffW + kHalf * 8;  // (+ alignment of the dynamic base)
-// S0 / P0 [0, 64) | S1 / P1 [64, 128) | O [128, 256) | unit 0's query value [256, 320) and
-// residual [320, 384) | unit 1's [384, 448) and [448, 512)
+// S0 / P0 [0, 64) | S1 / P1 [64, 128) | S2 / P2 [128, 192) | O [192, 320) | the unit's query
+// value [320, 384) and residual [384, 448)
+constexpr int kSBufs = 3;         // score buffers: the MMA runs up to two tiles ahead of the weights
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColPlo = 32;  // residuals of a tile's weights, after its 32 value columns
-constexpr uint32_t kColO = 128;
-constexpr uint32_t kColQ = 256;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
-constexpr uint32_t kColQlo = 320;
-constexpr uint32_t kColQUnit = 128;  // the second unit's query, further on
+constexpr uint32_t kColO = 192;
+constexpr uint32_t kColQ = 320;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
+constexpr uint32_t kColQlo = 384;
 constexpr float kHeadroom = 8.0f;    // log2 growth of a row's maximum tolerated before rescaling
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -234,13 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
   uint64_t* bar_q = empty + kStages;     // a unit's queries in tensor memory (16 warps; a phase per unit)
-  // scores ready, weights ready (16 warps) and PV done, one of each per score buffer: tile
-  // g's phase is g / 2 of barrier g % 2, so neither side can complete a phase the other has
-  // not waited for yet
-  uint64_t* bar_s = bar_q + 1;           // [2]
-  uint64_t* bar_p = bar_s + 2;           // [2]
-  uint64_t* bar_pv = bar_p + 2;          // [2]
-  uint64_t* drain = bar_pv + 2;
+  uint64_t* bar_s = bar_q + 1;           // [kSBufs] scores ready
+  // weights ready (16 warps) and PV done, one of each per score buffer: tile g's phases are
+  // g / 3 of barrier g % 3, so neither side can complete a phase the other has not waited
+  // for yet (the MMA thread issues scores up to two tiles ahead)
+  uint64_t* bar_p = bar_s + kSBufs;      // [kSBufs]
+  uint64_t* bar_pv = bar_p + kSBufs;     // [kSBufs]
+  uint64_t* drain = bar_pv + kSBufs;
   uint64_t* bar_qraw = drain + 1;        // a unit's query box has landed (a phase per unit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -258,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(bar_q), kRowWarps);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(smem_u32(&bar_s[s]), 1);
       mbar_init(smem_u32(&bar_p[s]), kRowWarps);
       mbar_init(smem_u32(&bar_pv[s]), 1);
@@ -341,71 +333,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    // ---------------- MMA issuer: the warp waits together, one elected lane issues (the
-    // tensor-core operations of that lane run in order, so S_{g+2}, written over P_g,
-    // follows the PV that reads P_g).  A unit's first score tile waits for its queries;
-    // unit v's queries sit in tensor-memory columns 256 + 128 (v & 1).
+    // ---------------- MMA issuer: the warp waits together, one elected lane issues.  The
+    // tensor-core operations of that lane run in order.  S_g goes to score buffer g % 3 as
+    // soon as its tile has landed and PV_{g-2} has been issued (so that S_g, written over
+    // P_{g-3}, follows the PV that reads it): the scores run up to two tiles ahead of the
+    // weights.  A unit's first score tile waits for its queries, and only after the PVs the
+    // rows wait for inside the previous unit have been issued (PV up to its second last).
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
     constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
     bool ok = true, issued = false;
-    int g = 0, vu = 0;
-    bool prev_first = false;  // tile g - 1 starts its unit's O
-    auto pv = [&](int j, bool starts) {  // PV of tile j
-      const int stage = j % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_p[j & 1]), (uint32_t)((j >> 1) & 1), abort_flag)))
+    // score side: the walk is one unit ahead of the PV side at most
+    UnitWalk sw = walk, pw = walk;
+    bool s_more = sw.first(), p_more = pw.first();
+    int s_i = 0, s_vu = 0, g_s = 0;  // next S: tile s_i of unit s_vu (global g_s)
+    int p_i = 0, g_pv = 0;           // next PV: tile p_i of the PV side's unit (global g_pv)
+    auto issue_s = [&]() -> bool {
+      if (s_i == 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), (uint32_t)(s_vu & 1), abort_flag))) return false;
+        tc_fence_after();
+      }
+      const int stage = g_s % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((g_s / kStages) & 1), abort_flag)))
+        return false;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t kt = sbase + kOffRing + stage * kTileBytes;
+        const uint32_t d_s = tmem_base + (uint32_t)((g_s % kSBufs) * kKeys);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint64_t kdesc = sw128_desc(kt + (uint32_t)((ks >> 2) * kKVHalf)) + (uint64_t)(2 * (ks & 3));
+          umma_ts(d_s, tmem_base + kColQ + (uint32_t)(8 * ks), kdesc, idesc_s, ks > 0 ? 1u : 0u);
+          umma_ts(d_s, tmem_base + kColQlo + (uint32_t)(8 * ks), kdesc, idesc_s, 1u);
+        }
+        umma_commit<false>(smem_u32(&bar_s[g_s % kSBufs]));
+      }
+      issued = true;
+      __syncwarp();
+      ++g_s;
+      if (++s_i == sw.nt) {
+        s_i = 0;
+        ++s_vu;
+        s_more = sw.next();
+      }
+      return true;
+    };
+    auto issue_pv = [&]() -> bool {
+      const int j = g_pv, stage = j % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_p[j % kSBufs]), (uint32_t)((j / kSBufs) & 1), abort_flag)))
         return false;
       tc_fence_after();
       if (leader) {
         const uint32_t vt = sbase + kOffRing + stage * kTileBytes + 2 * kKVHalf;
-        const uint32_t p_tmem = tmem_base + (uint32_t)((j & 1) * kKeys);  // P_j: 64 bf16 in 32 columns
+        const uint32_t p_tmem = tmem_base + (uint32_t)((j % kSBufs) * kKeys);  // P_j: 64 bf16 in 32 columns
 #pragma unroll
         for (int ks = 0; ks < kKeys / 16; ++ks) {
           const uint64_t vdesc = sw128_desc_mn(vt + (uint32_t)(ks * 2048), kKVHalf, 1024);
-          umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (!starts || ks > 0) ? 1u : 0u);
+          umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (p_i > 0 || ks > 0) ? 1u : 0u);
           umma_ts(tmem_base + kColO, p_tmem + kColPlo + (uint32_t)(8 * ks), vdesc, idesc_pv, 1u);
         }
-        umma_commit<false>(smem_u32(&bar_pv[j & 1]));
+        umma_commit<false>(smem_u32(&bar_pv[j % kSBufs]));
         umma_commit<false>(smem_u32(&empty[stage]));
       }
       __syncwarp();
+      ++g_pv;
+      if (++p_i == pw.nt) {
+        p_i = 0;
+        p_more = pw.next();
+      }
       return true;
     };
-    for (bool more = walk.first(); more && ok; more = walk.next(), ++vu) {
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), (uint32_t)(vu & 1), abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t q_t = tmem_base + kColQ + (uint32_t)(vu & 1) * kColQUnit;
-      for (int i = 0; i < walk.nt; ++i, ++g) {
-        const int stage = g % kStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((g / kStages) & 1), abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (leader) {
-          const uint32_t kt = sbase + kOffRing + stage * kTileBytes;
-          const uint32_t d_s = tmem_base + (uint32_t)((g & 1) * kKeys);
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint64_t kdesc = sw128_desc(kt + (uint32_t)((ks >> 2) * kKVHalf)) + (uint64_t)(2 * (ks & 3));
-            umma_ts(d_s, q_t + (uint32_t)(8 * ks), kdesc, idesc_s, ks > 0 ? 1u : 0u);
-            umma_ts(d_s, q_t + (kColQlo - kColQ) + (uint32_t)(8 * ks), kdesc, idesc_s, 1u);
-          }
-          umma_commit<false>(smem_u32(&bar_s[g & 1]));
-        }
-        issued = true;
-        __syncwarp();
-        if (g >= 1 && !pv(g - 1, prev_first)) {
-          ok = false;
-          break;
-        }
-        prev_first = i == 0;
-      }
+    while (ok && p_more) {
+      // scores first while allowed: up to two ahead of the next PV; a unit's first one only
+      // once the PV before the previous unit's last tile has been issued (g_pv >= g_s - 1)
+      while (ok && s_more && g_s <= g_pv + 2 && (s_i != 0 || g_s == 0 || g_s <= g_pv + 1))
+        ok = issue_s();
+      if (ok) ok = issue_pv();
     }
-    if (ok && g >= 1 && !pv(g - 1, prev_first)) ok = false;  // the last tile's PV
     if (!ok) {
       if (lane == 0) {
         *abort_flag = 1;
@@ -441,7 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* xch = reinterpret_cast<float*>(smem + kSmemData + kOffXch);  // [2 tiles][4 parts][128 rows]
     // PV_g done (the PV phases are waited one by one, in order)
     auto wait_pv = [&](int g) {
-      if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_pv[g & 1]), (uint32_t)((g >> 1) & 1), abort_flag)))
+      if (ok && !__all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&bar_pv[g % kSBufs]), (uint32_t)((g / kSBufs) & 1), abort_flag)))
         fail();
       if (ok) tc_fence_after();
     };
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           split2(xb[2 * e], xb[2 * e + 1], qh[8 + 4 * c + e], ql[8 + 4 * c + e]);
         }
       }
-      const uint32_t qcol = tmem_base + lane_addr + kColQ + (uint32_t)(v & 1) * kColQUnit + (uint32_t)(8 * hf);
+      const uint32_t qcol = tmem_base + lane_addr + kColQ + (uint32_t)(8 * hf);
       tmem_st8(qcol, *reinterpret_cast<const uint32_t(*)[8]>(qh));
       tmem_st8(qcol + 32, *reinterpret_cast<const uint32_t(*)[8]>(qh + 8));
       tmem_st8(qcol + (kColQlo - kColQ), *reinterpret_cast<const uint32_t(*)[8]>(ql));
@@ -527,7 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < w.nt; ++i) {
         const int g = g0 + i;
         // (waits are made warp-uniform: the TMEM accesses below are warp-collective)
-        if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_s[g & 1]), (uint32_t)((g >> 1) & 1), abort_flag)))
+        if (ok && !__all_sync(0xffffffffu,
+                              mbar_wait(smem_u32(&bar_s[g % kSBufs]), (uint32_t)((g / kSBufs) & 1), abort_flag)))
           fail();
         const bool local = i >= w.nt_mem;
         const int key0 = local ? (i - w.nt_mem) * kKeys : i * kKeys;
@@ -537,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           tc_fence_after();
           uint32_t sa[16];
-          tmem_ld16(tmem_base + lane_addr + (uint32_t)((g & 1) * kKeys + 16 * hf), sa);
+          tmem_ld16(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + 16 * hf), sa);
           tmem_wait_ld();
           // this thread's 16 keys: all visible (a memory tile's first keys below M, or local
           // keys up to the row's limit), or masked one by one
@@ -602,15 +608,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P_g over the scores it came from: values in columns 8 hf .. 8 hf + 7 of the tile's
         // buffer, residuals 32 columns further
-        tmem_st8(tmem_base + lane_addr + (uint32_t)((g & 1) * kKeys + 8 * hf), pw);
-        tmem_st8(tmem_base + lane_addr + (uint32_t)((g & 1) * kKeys + kColPlo + 8 * hf), plw);
+        tmem_st8(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + 8 * hf), pw);
+        tmem_st8(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + kColPlo + 8 * hf), plw);
         tmem_wait_st();
         l_sum += psum;
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_p[g & 1]));
-        if (i > 0 && !rescale) wait_pv(g - 1);  // (one wait per tile, in order)
+        if (lane == 0) mbar_arrive(smem_u32(&bar_p[g % kSBufs]));
+        // (no wait for PV_{g-1} here: the rows wait for a PV only before a rescale of O and
+        // before the output; PV_t's barrier cannot complete its next phase, PV_{t+3}, before
+        // the rows have released P_{t+3}, so skipping the phases in between is safe)
       }
     };
 
