@@ -6,30 +6,39 @@
 // times the values.  Follows "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", section
 // 推理流水线, and the MSA paper reading notes, section 推理全流程.
 //
-// One CTA (576 threads) per 128 rows: 128 / G tokens x the G query heads of key head h.
-//   warp 17, one thread  TMA producer: tiles of 64 keys (K as two 64-column boxes, then V
-//                        the same), 128-byte swizzle, a 3-stage ring; memory tiles first,
-//                        then local tiles up to the CTA's last token
-//   warp 16, one thread  MMA issuer: S_i = Q K_i^T (M = 128, N = 64, K = 128) into one of two
-//                        TMEM score buffers, then O += P_{i-1} V_{i-1} (M = 128, N = 128,
-//                        K = 64) into the TMEM output, with P read from tensor memory (it
-//                        replaces the scores it was computed from) and V read MN-major
-//                        straight from its [key][d] rows.  The rotated queries and the
+// Persistent CTAs of 576 threads, at most one per SM.  A unit is 128 rows: 128 / G tokens x
+// the G query heads of key head h.  CTA c walks the tile pairs c, c + gridDim.x, ... of the
+// (query x layer, key head, pair) list, pair j holding token tiles j and n_tiles - 1 - j (a
+// short and a long one under the causal mask), one unit at a time:
+//   warp 17, one thread  TMA producer: per unit its query rows as a 4D box (once the
+//                        previous unit's queries are in tensor memory), then its tiles of
+//                        64 keys (K as two 64-column boxes, then V the same), 128-byte
+//                        swizzle, a 3-stage ring; memory tiles first, then local tiles up to
+//                        the unit's last token
+//   warp 16              MMA issuer (the warp waits, one elected lane issues): S_g = Q K_g^T
+//                        (M = 128, N = 64, K = 128, the query read from tensor memory) into
+//                        score buffer g % 3, up to two tiles ahead of the weights; O +=
+//                        P_g V_g (M = 128, N = 128, K = 64) into the TMEM output, P read from
+//                        tensor memory (it replaces the scores it was computed from), V read
+//                        MN-major from its [key][d] rows.  The rotated queries and the
 //                        weights are each a bf16 value plus a bf16 residual (two MMAs); keys
-//                        and values exact bf16; fp32 accumulation
+//                        and values exact bf16; fp32 accumulation.  g runs on from unit to
+//                        unit.
 //   warps 0..15          four threads per row (TMEM lane), each with a quarter of the row's
-//                        dims and of every tile's keys: build the rotated, scaled query row
-//                        in shared memory; per tile read the score row, mask it (memory keys
-//                        < M, local keys <= its own local index), keep a running maximum
-//                        that is raised (and O rescaled in TMEM) only when a score exceeds
-//                        it by more than 2^8, write the weights exp2(s - m) into the tile's
-//                        score columns (values in the first 32, residuals in the last 32),
-//                        and at the end divide O by the running sum.
-// Weights of a tile are written while the previous tile's PV runs: the row threads wait
-// for PV_{i-1} after releasing P_i (before, only when O must be rescaled).  Key rows past a
-// tile's valid count are zeroed in shared memory before the PV that reads them (the cache
-// rows beyond the valid length may hold anything).  Every wait is bounded (2 s); a timeout
-// sets MSA_DEVERR_TIMEOUT and the CTA drains and frees its TMEM.
+//                        dims and of every tile's keys.  Per unit: rotate and scale the
+//                        query rows into tensor memory (RoPE table of the unit's tokens,
+//                        64-bit fixed-point angles); then the previous unit's output: O /
+//                        sum as bf16 through a shared-memory box, one TMA store; then per
+//                        tile read the score row, mask it (memory keys < M, local keys <= its
+//                        own local index), keep a running maximum that is raised (and O
+//                        rescaled in TMEM) only when a score exceeds it by more than 2^8,
+//                        and write the weights exp2(s - m) into the tile's score columns
+//                        (values in the first 32, residuals in the last 32).
+// The row threads wait for a PV only before rescaling O and before the output; one score,
+// weight and PV barrier per score buffer keeps every wait's phase unambiguous.  Key rows
+// past a tile's valid count are zeroed in shared memory before the PV that reads them (the
+// cache rows beyond the valid length may hold anything).  Every wait is bounded (2 s); a
+// timeout sets MSA_DEVERR_TIMEOUT and the CTA drains and frees its TMEM.
 #include <cuda.h>
 
 #include <math.h>
