@@ -346,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tensor-core operations of that lane run in order.  S_g goes to score buffer g % 3 as
     // soon as its tile has landed and PV_{g-2} has been issued (so that S_g, written over
     // P_{g-3}, follows the PV that reads it): the scores run up to two tiles ahead of the
-    // weights.  A unit's first score tile waits for its queries, and only after the PVs the
-    // rows wait for inside the previous unit have been issued (PV up to its second last).
+    // weights.  A unit's first score tile waits for its queries, and only after every PV of
+    // the previous unit has been issued.
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
     constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
@@ -414,8 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     while (ok && p_more) {
       // scores first while allowed: up to two ahead of the next PV; a unit's first one only
-      // once the PV before the previous unit's last tile has been issued (g_pv >= g_s - 1)
-      while (ok && s_more && g_s <= g_pv + 2 && (s_i != 0 || g_s == 0 || g_s <= g_pv + 1))
+      // once every PV of the previous unit has been issued (g_pv >= g_s), so that the last
+      // PV, which the previous unit's output waits for, does not queue behind the next
+      // unit's scores
+      while (ok && s_more && g_s <= g_pv + 2 && (s_i != 0 || g_s <= g_pv))
         ok = issue_s();
       if (ok) ok = issue_pv();
     }
