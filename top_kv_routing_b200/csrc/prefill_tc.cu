@@ -57,7 +57,6 @@ constexpr int kD = 128;
 constexpr int kHalf = 64;
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kStages = 3;
 constexpr int kRowWarps = 16;                 // four threads per row: 16 keys of a tile each
 constexpr int kParts = kRowWarps / 4;
 constexpr int kMmaWarp = kRowWarps, kTmaWarp = kRowWarps + 1;
@@ -67,16 +66,26 @@ constexpr int kTileBytes = 4 * kKVHalf;  // K (two halves) then V (two halves)
 constexpr int kOffRing = 0;
 constexpr int kQBoxHalf = kRows * 128;                    // 16 KB: 64 dims of the CTA's 128 rows
 constexpr int kQBox = 2 * kQBoxHalf;                      // 32 KB: one unit's query rows
-constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // a unit's queries as loaded
-constexpr int kOffOut = kOffQraw + kQBox;                  // a unit's output rows on their way out
-constexpr int kOffTab = kOffOut + kQBox;                   // cos / sin of a unit's tokens (G > 1)
+
 constexpr int kTabStride = kHalf + 1;                     // (a token's 64 angles + 1: the G-row groups of
                                                            // a warp read 8 tokens in distinct banks)
-constexpr int kTabBytes = 64 * kTabStride * 8;             // up to 64 tokens x 64 angles x float2
-constexpr int kSmemData = kOffTab + kTabBytes;
 constexpr int kOffXch = 256;                                 // after the barriers: the rows' exchange buffer
 constexpr int kOffW = kOffXch + 2 * kParts * kRows * 4;      // then the RoPE frequencies (64 x 8 bytes)
-constexpr int kSmem = kSmemData + 1024 + kOffW + kHalf * 8;  // (+ alignment of the dynamic base)
+// Shared memory per group size: the K / V ring, a unit's query box, its output box, the
+// RoPE table of its 128 / G tokens (none for G = 1), then barriers, exchange buffer and the
+// frequencies.  Four ring stages where they fit (all but G = 2), else three.
+template <int G>
+struct Lay {
+  static constexpr int kTabBytes = G > 1 ? (kRows / G) * kTabStride * 8 : 0;
+  static constexpr int kTail = 1024 + kOffW + kHalf * 8;  // (+ alignment of the dynamic base)
+  static constexpr int kStages = 4 * kTileBytes + 2 * kQBox + kTabBytes + kTail <= 227 * 1024 ? 4 : 3;
+  static constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // a unit's queries as loaded
+  static constexpr int kOffOut = kOffQraw + kQBox;                  // a unit's output rows on their way out
+  static constexpr int kOffTab = kOffOut + kQBox;                   // cos / sin of a unit's tokens (G > 1)
+  static constexpr int kSmemData = kOffTab + kTabBytes;
+  static constexpr int kSmem = kSmemData + kTail;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
 // S0 / P0 [0, 64) | S1 / P1 [64, 128) | S2 / P2 [128, 192) | O [192, 320) | the unit's query
 // value [320, 384) and residual [384, 448)
 constexpr int kSBufs = 3;         // score buffers: the MMA runs up to two tiles ahead of the weights
@@ -229,6 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       int M_max, int pos_off, const __grid_constant__ RopeW rw, float qscale, int n_bl,
                       int32_t* dev_err) {
   constexpr int kTok = kRows / G;
+  constexpr int kStages = Lay<G>::kStages, kOffQraw = Lay<G>::kOffQraw, kOffOut = Lay<G>::kOffOut;
+  constexpr int kOffTab = Lay<G>::kOffTab, kSmemData = Lay<G>::kSmemData;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
@@ -758,6 +769,7 @@ int launch_g(const Args& a, cudaStream_t s, const char** why) {
     *why = "cuTensorMapEncodeTiled failed";
     return 1;
   }
+  constexpr int kSmem = Lay<G>::kSmem;
   if (cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) {
     *why = "cudaFuncSetAttribute (shared memory)";
     return 1;
