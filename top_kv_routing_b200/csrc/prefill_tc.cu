@@ -117,6 +117,14 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+// 2^x by the hardware approximation (relative error about 2^-22, results below 2^-126
+// flushed to zero, 2^-inf = 0): the weights exp2(s - m), with s - m <= 8 or -inf.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // cos / sin of the RoPE angle of position p at frequency step s (2^-64 turns per position):
 // the top 32 bits of p * s mod 2^64, read as signed, are the angle in [-pi, pi) x 2^31 / pi.
 // The hardware sine / cosine is used on that reduced angle (absolute error about 2^-21 on
@@ -599,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float psum = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float p0 = exp2f(sv[2 * e] - m_used), p1 = exp2f(sv[2 * e + 1] - m_used);
+          const float p0 = ex2_ftz(sv[2 * e] - m_used), p1 = ex2_ftz(sv[2 * e + 1] - m_used);
           psum += p0 + p1;
           split2(p0, p1, pw[e], plw[e]);
         }
