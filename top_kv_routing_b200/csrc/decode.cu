@@ -70,6 +70,14 @@ struct RopeFreq {
   unsigned long long step[kHalf];
 };
 
+// 2^x by the hardware approximation (relative error about 2^-22, results below 2^-126
+// flushed to zero, 2^-inf = 0): the weights exp2(s - m) with s <= m, and the rescale factors.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
@@ -317,10 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m, mx);
-      const float alpha = exp2f(m - m_new);  // 0 while m is still -inf
+      const float alpha = ex2_ftz(m - m_new);  // 0 while m is still -inf
       float pr[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) pr[u] = exp2f(sc[u] - m_new);
+      for (int u = 0; u < 4; ++u) pr[u] = ex2_ftz(sc[u] - m_new);
       lsum = fmaf(lsum, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
       m = m_new;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
