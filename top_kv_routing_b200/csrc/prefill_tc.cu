@@ -60,7 +60,8 @@ constexpr int kKeys = 64;
 constexpr int kRowWarps = 16;                 // four threads per row: 16 keys of a tile each
 constexpr int kParts = kRowWarps / 4;
 constexpr int kMmaWarp = kRowWarps, kTmaWarp = kRowWarps + 1;
-constexpr int kThreads = (kRowWarps + 2) * 32;
+constexpr int kTabWarp = kRowWarps + 2;  // the next unit's RoPE table, off the row warps' path
+constexpr int kThreads = (kRowWarps + 3) * 32;
 constexpr int kKVHalf = kKeys * 128;     // 8 KB: 64 keys x 64 elements
 constexpr int kTileBytes = 4 * kKVHalf;  // K (two halves) then V (two halves)
 constexpr int kOffRing = 0;
@@ -262,7 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_pv = bar_p + kSBufs;     // [kSBufs]
   uint64_t* drain = bar_pv + kSBufs;
   uint64_t* bar_qraw = drain + 1;        // a unit's query box has landed (a phase per unit)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qraw + 1);
+  uint64_t* bar_tab = bar_qraw + 1;      // a unit's RoPE table is written (a phase per unit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tab + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   unsigned long long* wsm = reinterpret_cast<unsigned long long*>(smem + kSmemData + kOffW);
 
@@ -285,6 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(drain), 1);
     mbar_init(smem_u32(bar_qraw), 1);
+    mbar_init(smem_u32(bar_tab), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
@@ -451,6 +454,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(smem_u32(drain), 0u);
       }
     }
+  } else if (warp == kTabWarp) {
+    // ---------------- RoPE table (G > 1): per unit the cos / sin of its 128 / G tokens at
+    // the 64 frequencies, written once the rows have staged the previous unit's queries
+    if (G > 1) {
+      float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
+      int vu = 0;
+      for (bool more = walk.first(); more; more = walk.next(), ++vu) {
+        if (vu > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_q), (uint32_t)((vu - 1) & 1), abort_flag))) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
+          }
+          break;
+        }
+        for (int e = lane; e < kTok * kHalf; e += 32) {
+          const int t2 = e / kHalf, j = e % kHalf;
+          float sn, cs;
+          rope_cs((unsigned long long)((long long)pos_off + walk.len + walk.tok0 + t2), wsm[j], cs, sn);
+          tab[t2 * kTabStride + j] = make_float2(cs, sn);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(bar_tab));
+      }
+    }
   } else {
     // ---------------- rows (warps 0..15): thread (row r = TMEM lane, part hf of 4) takes the
     // row's dims 16 hf .. 16 hf + 15 and 64 + 16 hf .. 79 + 16 hf of the query, and keys
@@ -487,16 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage_q = [&](const UnitWalk& w, int v) {
       const int tok0 = w.tok0, tok = tok0 + tl;
       const unsigned long long pos = (unsigned long long)((long long)pos_off + w.len + tok);
-      float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
-      if (G > 1) {
-        for (int e = tid; e < kTok * kHalf; e += kRowWarps * 32) {
-          const int t2 = e / kHalf, j = e % kHalf;
-          float sn, cs;
-          rope_cs((unsigned long long)((long long)pos_off + w.len + tok0 + t2), wsm[j], cs, sn);
-          tab[t2 * kTabStride + j] = make_float2(cs, sn);
-        }
-        rows_sync();
-      }
+      const float2* tab = reinterpret_cast<const float2*>(smem + kOffTab);
+      if (G > 1 && ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_tab), (uint32_t)(v & 1), abort_flag)))
+        fail();  // (the table warp has written the unit's table)
       // the query box (TMA, 128-byte swizzle): row r's 16-byte chunk c of each 64-dim half at
       // 128 r + 16 (c ^ (r & 7))
       if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_qraw), (uint32_t)(v & 1), abort_flag))) fail();
