@@ -13,27 +13,31 @@
 //   warp 17, one thread  TMA producer: per unit its query rows as a 4D box (once the
 //                        previous unit's queries are in tensor memory), then its tiles of
 //                        64 keys (K as two 64-column boxes, then V the same), 128-byte
-//                        swizzle, a 3-stage ring; memory tiles first, then local tiles up to
-//                        the unit's last token
+//                        swizzle, a ring of 4 stages (3 where shared memory is short, G = 2);
+//                        memory tiles first, then local tiles up to the unit's last token
 //   warp 16              MMA issuer (the warp waits, one elected lane issues): S_g = Q K_g^T
 //                        (M = 128, N = 64, K = 128, the query read from tensor memory) into
 //                        score buffer g % 3, up to two tiles ahead of the weights; O +=
 //                        P_g V_g (M = 128, N = 128, K = 64) into the TMEM output, P read from
 //                        tensor memory (it replaces the scores it was computed from), V read
-//                        MN-major from its [key][d] rows.  The rotated queries and the
-//                        weights are each a bf16 value plus a bf16 residual (two MMAs); keys
-//                        and values exact bf16; fp32 accumulation.  g runs on from unit to
-//                        unit.
+//                        MN-major from its [key][d] rows.  The rotated queries are a bf16
+//                        value plus a bf16 residual (two MMAs); the weights are bf16, rounded
+//                        to nearest, and the row sums are taken over the rounded weights, so
+//                        numerator and denominator use the same ones; keys and values exact
+//                        bf16; fp32 accumulation.  g runs on from unit to unit.
+//   warp 18              (G > 1) the RoPE table of a unit's 128 / G tokens (64-bit
+//                        fixed-point angles, hardware sin / cos of the reduced angle), written
+//                        once the rows have staged the previous unit's queries
 //   warps 0..15          four threads per row (TMEM lane), each with a quarter of the row's
 //                        dims and of every tile's keys.  Per unit: rotate and scale the
-//                        query rows into tensor memory (RoPE table of the unit's tokens,
-//                        64-bit fixed-point angles); then the previous unit's output: O /
+//                        query rows into tensor memory (from the table; G = 1 computes its
+//                        one token's angles in place); then the previous unit's output: O /
 //                        sum as bf16 through a shared-memory box, one TMA store; then per
 //                        tile read the score row, mask it (memory keys < M, local keys <= its
 //                        own local index), keep a running maximum that is raised (and O
 //                        rescaled in TMEM) only when a score exceeds it by more than 2^8,
-//                        and write the weights exp2(s - m) into the tile's score columns
-//                        (values in the first 32, residuals in the last 32).
+//                        and write the weights exp2(s - m) as bf16 into the first 32 of the
+//                        tile's score columns.
 // The row threads wait for a PV only before rescaling O and before the output; one score,
 // weight and PV barrier per score buffer keeps every wait's phase unambiguous.  Key rows
 // past a tile's valid count are zeroed in shared memory before the PV that reads them (the
@@ -91,7 +95,6 @@ struct Lay {
 // value [320, 384) and residual [384, 448)
 constexpr int kSBufs = 3;         // score buffers: the MMA runs up to two tiles ahead of the weights
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColPlo = 32;  // residuals of a tile's weights, after its 32 value columns
 constexpr uint32_t kColO = 192;
 constexpr uint32_t kColQ = 320;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
 constexpr uint32_t kColQlo = 384;
@@ -421,7 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < kKeys / 16; ++ks) {
           const uint64_t vdesc = sw128_desc_mn(vt + (uint32_t)(ks * 2048), kKVHalf, 1024);
           umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (p_i > 0 || ks > 0) ? 1u : 0u);
-          umma_ts(tmem_base + kColO, p_tmem + kColPlo + (uint32_t)(8 * ks), vdesc, idesc_pv, 1u);
         }
         umma_commit<false>(smem_u32(&bar_pv[j % kSBufs]));
         umma_commit<false>(smem_u32(&empty[stage]));
@@ -623,13 +625,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool need = mx > m_used + kHeadroom;  // (the same in the four threads of the row)
         const float m_old = m_used;
         if (need) m_used = mx;
-        uint32_t pw[8], plw[8];
+        // the weights rounded to bf16 (the PV's A operand); the row sum adds the rounded values
+        uint32_t pw[8];
         float psum = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float p0 = ex2_ftz(sv[2 * e] - m_used), p1 = ex2_ftz(sv[2 * e + 1] - m_used);
-          psum += p0 + p1;
-          split2(p0, p1, pw[e], plw[e]);
+          const __nv_bfloat162 pb =
+              __floats2bfloat162_rn(ex2_ftz(sv[2 * e] - m_used), ex2_ftz(sv[2 * e + 1] - m_used));
+          const float2 pr = __bfloat1622float2(pb);
+          psum += pr.x + pr.y;
+          pw[e] = *reinterpret_cast<const uint32_t*>(&pb);
         }
         // key rows past the valid count: zero their V rows (this tile's stage; all row threads)
         if (n_valid < kKeys) {
@@ -656,10 +661,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (need) l_sum *= alpha;
         }
-        // P_g over the scores it came from: values in columns 8 hf .. 8 hf + 7 of the tile's
-        // buffer, residuals 32 columns further
+        // P_g over the scores it came from: columns 8 hf .. 8 hf + 7 of the tile's buffer
         tmem_st8(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + 8 * hf), pw);
-        tmem_st8(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + kColPlo + 8 * hf), plw);
         tmem_wait_st();
         l_sum += psum;
         fence_async_smem();
