@@ -6,38 +6,41 @@
 // times the values.  Follows "MSA端到端可训练记忆模型完整开源，支持亿级Token上下文", section
 // 推理流水线, and the MSA paper reading notes, section 推理全流程.
 //
-// Persistent CTAs of 576 threads, at most one per SM.  A unit is 128 rows: 128 / G tokens x
+// Persistent CTAs of 608 threads, at most one per SM.  A unit is 128 rows: 128 / G tokens x
 // the G query heads of key head h.  CTA c walks the tile pairs c, c + gridDim.x, ... of the
 // (query x layer, key head, pair) list, pair j holding token tiles j and n_tiles - 1 - j (a
 // short and a long one under the causal mask), one unit at a time:
 //   warp 17, one thread  TMA producer: per unit its query rows as a 4D box (once the
 //                        previous unit's queries are in tensor memory), then its tiles of
-//                        64 keys (K as two 64-column boxes, then V the same), 128-byte
-//                        swizzle, a ring of 4 stages (3 where shared memory is short, G = 2);
-//                        memory tiles first, then local tiles up to the unit's last token
+//                        128 keys (memory tiles first, then local tiles up to the unit's last
+//                        token) as 64-key boxes, 128-byte swizzle, into a ring of two slots:
+//                        the K of tile g once the scores of tile g - 2 have read that slot's
+//                        K, then the V of tile g - 1 once PV_{g-3} has read its V.  A tile
+//                        with at most 64 valid keys is loaded as one box.
 //   warp 16              MMA issuer (the warp waits, one elected lane issues): S_g = Q K_g^T
-//                        (M = 128, N = 64, K = 128, the query read from tensor memory) into
-//                        score buffer g % 3, up to two tiles ahead of the weights; O +=
-//                        P_g V_g (M = 128, N = 128, K = 64) into the TMEM output, P read from
-//                        tensor memory (it replaces the scores it was computed from), V read
-//                        MN-major from its [key][d] rows.  The rotated queries are a bf16
-//                        value plus a bf16 residual (two MMAs); the weights are bf16, rounded
-//                        to nearest, and the row sums are taken over the rounded weights, so
-//                        numerator and denominator use the same ones; keys and values exact
-//                        bf16; fp32 accumulation.  g runs on from unit to unit.
-//   warp 18              (G > 1) the RoPE table of a unit's 128 / G tokens (64-bit
+//                        (M = 128, N = 128, or 64 for a half tile, K = 128, the query read
+//                        from tensor memory) into score buffer g % 2, one tile ahead of the
+//                        weights; O += P_g V_g (M = 128, N = 128, K = the tile's keys) into
+//                        the TMEM output, P read from tensor memory (it replaces the scores
+//                        it was computed from), V read MN-major from its [key][d] rows.  The
+//                        rotated queries are a bf16 value plus a bf16 residual (two MMAs);
+//                        the weights are bf16, rounded to nearest, and the row sums are taken
+//                        over the rounded weights, so numerator and denominator use the same
+//                        ones; keys and values exact bf16; fp32 accumulation.  g runs on from
+//                        unit to unit.
+//   warp 18              (G >= 4) the RoPE table of a unit's 128 / G tokens (64-bit
 //                        fixed-point angles, hardware sin / cos of the reduced angle), written
 //                        once the rows have staged the previous unit's queries
 //   warps 0..15          four threads per row (TMEM lane), each with a quarter of the row's
-//                        dims and of every tile's keys.  Per unit: rotate and scale the
-//                        query rows into tensor memory (from the table; G = 1 computes its
-//                        one token's angles in place); then the previous unit's output: O /
-//                        sum as bf16 through a shared-memory box, one TMA store; then per
-//                        tile read the score row, mask it (memory keys < M, local keys <= its
-//                        own local index), keep a running maximum that is raised (and O
-//                        rescaled in TMEM) only when a score exceeds it by more than 2^8,
-//                        and write the weights exp2(s - m) as bf16 into the first 32 of the
-//                        tile's score columns.
+//                        dims and 32 keys of every tile.  Per unit: rotate and scale the
+//                        query rows into tensor memory (from the table; G <= 2 computes the
+//                        angles in place); then the previous unit's output: O / sum as bf16
+//                        through a shared-memory box, one TMA store; then per tile read the
+//                        score row, mask it (memory keys < M, local keys <= its own local
+//                        index), keep a running maximum that is raised (and O rescaled in
+//                        TMEM) only when a score exceeds it by more than 2^8, and write the
+//                        weights exp2(s - m) as bf16 over the first 64 of the tile's score
+//                        columns.
 // The row threads wait for a PV only before rescaling O and before the output; one score,
 // weight and PV barrier per score buffer keeps every wait's phase unambiguous.  Key rows
 // past a tile's valid count are zeroed in shared memory before the PV that reads them (the
@@ -60,14 +63,16 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr int kHalf = 64;
 constexpr int kRows = 128;
-constexpr int kKeys = 64;
+constexpr int kKeys = 64;   // keys per TMA box (half a tile)
+constexpr int kTile = 128;  // keys per score tile
 constexpr int kRowWarps = 16;                 // four threads per row: 16 keys of a tile each
 constexpr int kParts = kRowWarps / 4;
 constexpr int kMmaWarp = kRowWarps, kTmaWarp = kRowWarps + 1;
 constexpr int kTabWarp = kRowWarps + 2;  // the next unit's RoPE table, off the row warps' path
 constexpr int kThreads = (kRowWarps + 3) * 32;
-constexpr int kKVHalf = kKeys * 128;     // 8 KB: 64 keys x 64 elements
-constexpr int kTileBytes = 4 * kKVHalf;  // K (two halves) then V (two halves)
+constexpr int kKVHalf = kTile * 128;     // 16 KB: a tile's 128 keys x 64 elements
+constexpr int kTileBytes = 4 * kKVHalf;  // 64 KB: K (two 64-dim halves) then V (two halves)
+constexpr int kSlots = 2;                // ring slots of one tile
 constexpr int kOffRing = 0;
 constexpr int kQBoxHalf = kRows * 128;                    // 16 KB: 64 dims of the CTA's 128 rows
 constexpr int kQBox = 2 * kQBoxHalf;                      // 32 KB: one unit's query rows
@@ -76,28 +81,28 @@ constexpr int kTabStride = kHalf + 1;                     // (a token's 64 angle
                                                            // a warp read 8 tokens in distinct banks)
 constexpr int kOffXch = 256;                                 // after the barriers: the rows' exchange buffer
 constexpr int kOffW = kOffXch + 2 * kParts * kRows * 4;      // then the RoPE frequencies (64 x 8 bytes)
-// Shared memory per group size: the K / V ring, a unit's query box, its output box, the
-// RoPE table of its 128 / G tokens (none for G = 1), then barriers, exchange buffer and the
-// frequencies.  Four ring stages where they fit (all but G = 2), else three.
+// Shared memory per group size: the K / V ring (two tiles), a unit's query box, its output
+// box, the RoPE table of its 128 / G tokens (G >= 4; smaller groups compute their angles in
+// place), then barriers, exchange buffer and the frequencies.
 template <int G>
 struct Lay {
-  static constexpr int kTabBytes = G > 1 ? (kRows / G) * kTabStride * 8 : 0;
+  static constexpr bool kUseTab = G >= 4;
+  static constexpr int kTabBytes = kUseTab ? (kRows / G) * kTabStride * 8 : 0;
   static constexpr int kTail = 1024 + kOffW + kHalf * 8;  // (+ alignment of the dynamic base)
-  static constexpr int kStages = 4 * kTileBytes + 2 * kQBox + kTabBytes + kTail <= 227 * 1024 ? 4 : 3;
-  static constexpr int kOffQraw = kOffRing + kStages * kTileBytes;  // a unit's queries as loaded
+  static constexpr int kOffQraw = kOffRing + kSlots * kTileBytes;  // a unit's queries as loaded
   static constexpr int kOffOut = kOffQraw + kQBox;                  // a unit's output rows on their way out
-  static constexpr int kOffTab = kOffOut + kQBox;                   // cos / sin of a unit's tokens (G > 1)
+  static constexpr int kOffTab = kOffOut + kQBox;                   // cos / sin of a unit's tokens (G >= 4)
   static constexpr int kSmemData = kOffTab + kTabBytes;
   static constexpr int kSmem = kSmemData + kTail;
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
-// S0 / P0 [0, 64) | S1 / P1 [64, 128) | S2 / P2 [128, 192) | O [192, 320) | the unit's query
-// value [320, 384) and residual [384, 448)
-constexpr int kSBufs = 3;         // score buffers: the MMA runs up to two tiles ahead of the weights
+// S0 / P0 [0, 128) | S1 / P1 [128, 256) | O [256, 384) | the unit's query value [384, 448) and
+// residual [448, 512)
+constexpr int kSBufs = 2;         // score buffers: the MMA runs one tile ahead of the weights
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 192;
-constexpr uint32_t kColQ = 320;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
-constexpr uint32_t kColQlo = 384;
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kColQ = 384;   // the rotated, scaled query rows: dims 2c, 2c + 1 in column c
+constexpr uint32_t kColQlo = 448;
 constexpr float kHeadroom = 8.0f;    // log2 growth of a row's maximum tolerated before rescaling
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -169,6 +174,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // 4D tiled TMA load (no multicast) completing on an mbarrier of this CTA: the box of a
 // CTA's query rows, [128 / G tokens][G heads][64 dims].
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z,
@@ -210,7 +224,7 @@ struct UnitWalk {
       if (len < 0 || len + T > cap) continue;  // (the append kernel has set MSA_DEVERR_LOCAL_FULL)
       const int m = mem_len[bl];
       M = m < 0 ? 0 : (m > M_max ? M_max : m);
-      nt_mem = (M + kKeys - 1) / kKeys;
+      nt_mem = (M + kTile - 1) / kTile;
       nu = j == n_tiles - 1 - j ? 1 : 2;
       k = 0;
       return true;
@@ -221,7 +235,13 @@ struct UnitWalk {
     const int j = p % pairs_x;
     tok0 = (k == 0 ? j : n_tiles - 1 - j) * kTok;
     n_local = len + min(T, tok0 + kTok);
-    nt = nt_mem + (n_local + kKeys - 1) / kKeys;
+    nt = nt_mem + (n_local + kTile - 1) / kTile;
+  }
+  // tile i of the unit: its first key (within the memory rows or the local rows) and its
+  // number of valid keys (a tile with at most 64 is loaded, scored and summed half-size)
+  __device__ int key0(int i) const { return i >= nt_mem ? (i - nt_mem) * kTile : i * kTile; }
+  __device__ int n_valid(int i) const {
+    return i >= nt_mem ? min(kTile, n_local - key0(i)) : min(kTile, M - key0(i));
   }
   __device__ bool first() {
     p = blockIdx.x;
@@ -250,14 +270,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                       int M_max, int pos_off, const __grid_constant__ RopeW rw, float qscale, int n_bl,
                       int32_t* dev_err) {
   constexpr int kTok = kRows / G;
-  constexpr int kStages = Lay<G>::kStages, kOffQraw = Lay<G>::kOffQraw, kOffOut = Lay<G>::kOffOut;
+  constexpr int kStages = kSlots, kOffQraw = Lay<G>::kOffQraw, kOffOut = Lay<G>::kOffOut;
+  constexpr bool kUseTab = Lay<G>::kUseTab;
   constexpr int kOffTab = Lay<G>::kOffTab, kSmemData = Lay<G>::kSmemData;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
-  uint64_t* full = bars;                 // [kStages]
-  uint64_t* empty = bars + kStages;      // [kStages]
-  uint64_t* bar_q = empty + kStages;     // a unit's queries in tensor memory (16 warps; a phase per unit)
+  // per ring slot: its K landed / read by the score MMAs, its V landed / read by the PV MMAs
+  uint64_t* full_k = bars;               // [kStages]
+  uint64_t* empty_k = bars + kStages;    // [kStages]
+  uint64_t* full_v = bars + 2 * kStages;   // [kStages]
+  uint64_t* empty_v = bars + 3 * kStages;  // [kStages]
+  uint64_t* bar_q = bars + 4 * kStages;  // a unit's queries in tensor memory (16 warps; a phase per unit)
   uint64_t* bar_s = bar_q + 1;           // [kSBufs] scores ready
   // weights ready (16 warps) and PV done, one of each per score buffer: tile g's phases are
   // g / 3 of barrier g % 3, so neither side can complete a phase the other has not waited
@@ -279,8 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
+      mbar_init(smem_u32(&full_k[s]), 1);
+      mbar_init(smem_u32(&empty_k[s]), 1);
+      mbar_init(smem_u32(&full_v[s]), 1);
+      mbar_init(smem_u32(&empty_v[s]), 1);
     }
     mbar_init(smem_u32(bar_q), kRowWarps);
     for (int s = 0; s < kSBufs; ++s) {
@@ -308,18 +334,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kTmaWarp) {
     if (lane == 0) {
       // ---------------- TMA producer: per unit its query box (once the previous unit's
-      // queries have been read out of the box's space), then its K / V tiles
+      // queries have been read out of the box's space), then its tiles in 64-key boxes: the
+      // K of tile g once S_{g-2} has read the slot's K, then the V of tile g - 1 once
+      // PV_{g-3} has read that slot's V (so a tile's keys land a softmax step before its
+      // scores are due, and its values a step later still)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_mem)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lk)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_lv)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_out)) : "memory");
       const uint64_t pol = policy_evict_last();
-      int armed[kStages];
+      int armed_k[kStages], armed_v[kStages];
 #pragma unroll
-      for (int st = 0; st < kStages; ++st) armed[st] = -1;
+      for (int st = 0; st < kStages; ++st) armed_k[st] = armed_v[st] = -1;
       int qarmed = -1;
       bool ok = true;
+      // a tile's source: the memory rows (K and V in one tensor) or the local cache's
+      struct Src {
+        int g, krow, vrow, boxes;
+        bool mem;
+      };
+      // its K (is_v false) or V into slot g % 2: `boxes` 64-key boxes of both 64-dim halves
+      auto load = [&](const Src& t, bool is_v) -> bool {
+        const int stage = t.g % kStages;
+        const uint32_t ph = (uint32_t)((t.g / kStages) & 1);
+        if (!mbar_wait(smem_u32(is_v ? &empty_v[stage] : &empty_k[stage]), ph ^ 1u, abort_flag)) return false;
+        const uint32_t fb = smem_u32(is_v ? &full_v[stage] : &full_k[stage]);
+        const CUtensorMap* map = t.mem ? &tm_mem : (is_v ? &tm_lv : &tm_lk);
+        const int row = is_v ? t.vrow : t.krow;
+        const uint32_t dst = sbase + kOffRing + stage * kTileBytes + (is_v ? 2 * kKVHalf : 0);
+        mbar_arrive_expect_tx(fb, t.boxes * (kTileBytes / 4));
+        for (int hb = 0; hb < t.boxes; ++hb) {
+          const uint32_t d = dst + (uint32_t)(hb * kKeys * 128);
+          tma_load_2d(d, map, fb, 0, row + hb * kKeys, pol);
+          tma_load_2d(d + kKVHalf, map, fb, kHalf, row + hb * kKeys, pol);
+        }
+        (is_v ? armed_v : armed_k)[stage] = (int)ph;
+        return true;
+      };
+      Src prev{0, 0, 0, 0, false};
+      bool have_prev = false;
       int g = 0, vu = 0;
       for (bool more = walk.first(); more && ok; more = walk.next(), ++vu) {
         if (vu > 0 && !mbar_wait(smem_u32(bar_q), (uint32_t)((vu - 1) & 1), abort_flag)) {
@@ -331,50 +385,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sbase + kOffQraw, &tm_q, qb, 0, walk.h * G, walk.tok0, (int)walk.bl);
         tma_load_4d(sbase + kOffQraw + kQBoxHalf, &tm_q, qb, kHalf, walk.h * G, walk.tok0, (int)walk.bl);
         qarmed = vu & 1;
-        for (int i = 0; i < walk.nt; ++i, ++g) {
-          const int stage = g % kStages;
-          const uint32_t ph = (uint32_t)((g / kStages) & 1);
-          if (!mbar_wait(smem_u32(&empty[stage]), ph ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = smem_u32(&full[stage]);
-          const uint32_t dst = sbase + kOffRing + stage * kTileBytes;
-          mbar_arrive_expect_tx(fb, kTileBytes);
-          if (i < walk.nt_mem) {
-            const int rk = (int)((((walk.bl * 2 + 0) * H + walk.h) * (int64_t)M_max) + i * kKeys);
-            const int rv = (int)((((walk.bl * 2 + 1) * H + walk.h) * (int64_t)M_max) + i * kKeys);
-            tma_load_2d(dst, &tm_mem, fb, 0, rk, pol);
-            tma_load_2d(dst + kKVHalf, &tm_mem, fb, kHalf, rk, pol);
-            tma_load_2d(dst + 2 * kKVHalf, &tm_mem, fb, 0, rv, pol);
-            tma_load_2d(dst + 3 * kKVHalf, &tm_mem, fb, kHalf, rv, pol);
+        for (int i = 0; i < walk.nt && ok; ++i, ++g) {
+          Src t;
+          t.g = g;
+          t.boxes = walk.n_valid(i) > kKeys ? 2 : 1;
+          t.mem = i < walk.nt_mem;
+          if (t.mem) {
+            t.krow = (int)((((walk.bl * 2 + 0) * H + walk.h) * (int64_t)M_max) + i * kTile);
+            t.vrow = (int)((((walk.bl * 2 + 1) * H + walk.h) * (int64_t)M_max) + i * kTile);
           } else {
-            const int r = (int)((walk.bl * H + walk.h) * (int64_t)cap + (int64_t)(i - walk.nt_mem) * kKeys);
-            tma_load_2d(dst, &tm_lk, fb, 0, r, pol);
-            tma_load_2d(dst + kKVHalf, &tm_lk, fb, kHalf, r, pol);
-            tma_load_2d(dst + 2 * kKVHalf, &tm_lv, fb, 0, r, pol);
-            tma_load_2d(dst + 3 * kKVHalf, &tm_lv, fb, kHalf, r, pol);
+            t.krow = t.vrow = (int)((walk.bl * H + walk.h) * (int64_t)cap + (int64_t)(i - walk.nt_mem) * kTile);
           }
-          armed[stage] = (int)ph;
+          ok = load(t, false);
+          if (ok && have_prev) ok = load(prev, true);
+          prev = t;
+          have_prev = true;
         }
       }
+      if (ok && have_prev) ok = load(prev, true);
       if (!ok) {
         *abort_flag = 1;
         msa::set_err(dev_err, MSA_DEVERR_TIMEOUT);
-        for (int s = 0; s < kStages; ++s)
-          if (armed[s] >= 0) mbar_drain(smem_u32(&full[s]), (uint32_t)armed[s]);
+        for (int s = 0; s < kStages; ++s) {
+          if (armed_k[s] >= 0) mbar_drain(smem_u32(&full_k[s]), (uint32_t)armed_k[s]);
+          if (armed_v[s] >= 0) mbar_drain(smem_u32(&full_v[s]), (uint32_t)armed_v[s]);
+        }
         if (qarmed >= 0) mbar_drain(smem_u32(bar_qraw), (uint32_t)qarmed);
       }
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer: the warp waits together, one elected lane issues.  The
-    // tensor-core operations of that lane run in order.  S_g goes to score buffer g % 3 as
-    // soon as its tile has landed and PV_{g-2} has been issued (so that S_g, written over
-    // P_{g-3}, follows the PV that reads it): the scores run up to two tiles ahead of the
-    // weights.  A unit's first score tile waits for its queries, and only after every PV of
-    // the previous unit has been issued.
+    // tensor-core operations of that lane run in order.  S_g goes to score buffer g % 2 as
+    // soon as its tile has landed and PV_{g-2} has been issued (S_g is written over P_{g-2}
+    // and follows the PV that reads it): the scores run one tile ahead of the weights.  A
+    // tile of at most 64 valid keys is scored with N = 64 and summed over its first 64 keys.
+    // A unit's first score tile waits for its queries, and only after every PV of the
+    // previous unit has been issued.
     const bool leader = elect_one();
-    constexpr uint32_t idesc_s = idesc_make(kRows, kKeys, false);
+    constexpr uint32_t idesc_s = idesc_make(kRows, kTile, false), idesc_s_half = idesc_make(kRows, kKeys, false);
     constexpr uint32_t idesc_pv = idesc_make_bmn(kRows, kD);
     bool ok = true, issued = false;
     // score side: the walk is one unit ahead of the PV side at most
@@ -388,19 +436,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       const int stage = g_s % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[stage]), (uint32_t)((g_s / kStages) & 1), abort_flag)))
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_k[stage]), (uint32_t)((g_s / kStages) & 1), abort_flag)))
         return false;
       tc_fence_after();
       if (leader) {
         const uint32_t kt = sbase + kOffRing + stage * kTileBytes;
-        const uint32_t d_s = tmem_base + (uint32_t)((g_s % kSBufs) * kKeys);
+        const uint32_t d_s = tmem_base + (uint32_t)((g_s % kSBufs) * kTile);
+        const uint32_t idesc = sw.n_valid(s_i) > kKeys ? idesc_s : idesc_s_half;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint64_t kdesc = sw128_desc(kt + (uint32_t)((ks >> 2) * kKVHalf)) + (uint64_t)(2 * (ks & 3));
-          umma_ts(d_s, tmem_base + kColQ + (uint32_t)(8 * ks), kdesc, idesc_s, ks > 0 ? 1u : 0u);
-          umma_ts(d_s, tmem_base + kColQlo + (uint32_t)(8 * ks), kdesc, idesc_s, 1u);
+          umma_ts(d_s, tmem_base + kColQ + (uint32_t)(8 * ks), kdesc, idesc, ks > 0 ? 1u : 0u);
+          umma_ts(d_s, tmem_base + kColQlo + (uint32_t)(8 * ks), kdesc, idesc, 1u);
         }
         umma_commit<false>(smem_u32(&bar_s[g_s % kSBufs]));
+        umma_commit<false>(smem_u32(&empty_k[stage]));
       }
       issued = true;
       __syncwarp();
@@ -416,17 +466,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = g_pv, stage = j % kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_p[j % kSBufs]), (uint32_t)((j / kSBufs) & 1), abort_flag)))
         return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_v[stage]), (uint32_t)((j / kStages) & 1), abort_flag)))
+        return false;
       tc_fence_after();
       if (leader) {
         const uint32_t vt = sbase + kOffRing + stage * kTileBytes + 2 * kKVHalf;
-        const uint32_t p_tmem = tmem_base + (uint32_t)((j % kSBufs) * kKeys);  // P_j: 64 bf16 in 32 columns
-#pragma unroll
-        for (int ks = 0; ks < kKeys / 16; ++ks) {
+        const uint32_t p_tmem = tmem_base + (uint32_t)((j % kSBufs) * kTile);  // P_j: 128 bf16 in 64 columns
+        const int n_ks = pw.n_valid(p_i) > kKeys ? kTile / 16 : kKeys / 16;
+        for (int ks = 0; ks < n_ks; ++ks) {
           const uint64_t vdesc = sw128_desc_mn(vt + (uint32_t)(ks * 2048), kKVHalf, 1024);
           umma_ts(tmem_base + kColO, p_tmem + (uint32_t)(8 * ks), vdesc, idesc_pv, (p_i > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit<false>(smem_u32(&bar_pv[j % kSBufs]));
-        umma_commit<false>(smem_u32(&empty[stage]));
+        umma_commit<false>(smem_u32(&empty_v[stage]));
       }
       __syncwarp();
       ++g_pv;
@@ -437,11 +489,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     while (ok && p_more) {
-      // scores first while allowed: up to two ahead of the next PV; a unit's first one only
+      // scores first while allowed: up to one ahead of the next PV; a unit's first one only
       // once every PV of the previous unit has been issued (g_pv >= g_s), so that the last
       // PV, which the previous unit's output waits for, does not queue behind the next
       // unit's scores
-      while (ok && s_more && g_s <= g_pv + 2 && (s_i != 0 || g_s <= g_pv))
+      while (ok && s_more && g_s <= g_pv + 1 && (s_i != 0 || g_s <= g_pv))
         ok = issue_s();
       if (ok) ok = issue_pv();
     }
@@ -457,9 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kTabWarp) {
-    // ---------------- RoPE table (G > 1): per unit the cos / sin of its 128 / G tokens at
+    // ---------------- RoPE table (G >= 4): per unit the cos / sin of its 128 / G tokens at
     // the 64 frequencies, written once the rows have staged the previous unit's queries
-    if (G > 1) {
+    if (kUseTab) {
       float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
       int vu = 0;
       for (bool more = walk.first(); more; more = walk.next(), ++vu) {
@@ -511,13 +563,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // unit v's rotated, scaled query rows (bf16 value and residual) into its tensor-memory
-    // columns, 8 dims (and their partners) at a time; with G > 1 the cos / sin of each token
-    // are computed once into a table its G rows share
+    // columns, 8 dims (and their partners) at a time; with G >= 4 the cos / sin of each token
+    // come from the table the table warp has written for the G rows that share them
     auto stage_q = [&](const UnitWalk& w, int v) {
       const int tok0 = w.tok0, tok = tok0 + tl;
       const unsigned long long pos = (unsigned long long)((long long)pos_off + w.len + tok);
       const float2* tab = reinterpret_cast<const float2*>(smem + kOffTab);
-      if (G > 1 && ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_tab), (uint32_t)(v & 1), abort_flag)))
+      if (kUseTab && ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(bar_tab), (uint32_t)(v & 1), abort_flag)))
         fail();  // (the table warp has written the unit's table)
       // the query box (TMA, 128-byte swizzle): row r's 16-byte chunk c of each 64-dim half at
       // 128 r + 16 (c ^ (r & 7))
@@ -540,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             float sn, cs;
-            if (G > 1) {
+            if (kUseTab) {
               const float2 t2 = tab[tl * kTabStride + 16 * hf + 8 * c + e];
               cs = t2.x;
               sn = t2.y;
@@ -588,34 +640,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                               mbar_wait(smem_u32(&bar_s[g % kSBufs]), (uint32_t)((g / kSBufs) & 1), abort_flag)))
           fail();
         const bool local = i >= w.nt_mem;
-        const int key0 = local ? (i - w.nt_mem) * kKeys : i * kKeys;
-        const int n_valid = local ? min(kKeys, w.n_local - key0) : min(kKeys, w.M - key0);
+        const int key0 = w.key0(i), n_valid = w.n_valid(i);
+        const int n_keys = n_valid > kKeys ? kTile : kKeys;  // keys scored and summed
+        const uint32_t s_col = tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kTile);
+        // this thread's 32 keys: none valid (left out: weights 0), all visible (a memory
+        // tile's first keys below M, or local keys up to the row's limit), or masked one by one
+        const bool none = 32 * hf >= n_valid;  // (the same in the whole warp)
+        const int kfirst = key0 + 32 * hf;
+        const bool all_in = local ? kfirst + 31 <= lim : kfirst + 31 < w.M;
+        uint32_t sv[32];  // (fp32 bits; a masked key is -inf)
         float mx = -INFINITY;
-        float sv[16];
-        if (ok) {
+        if (ok && !none) {
           tc_fence_after();
-          uint32_t sa[16];
-          tmem_ld16(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + 16 * hf), sa);
+          tmem_ld32(s_col + (uint32_t)(32 * hf), sv);
           tmem_wait_ld();
-          // this thread's 16 keys: all visible (a memory tile's first keys below M, or local
-          // keys up to the row's limit), or masked one by one
-          const int kfirst = key0 + 16 * hf;
-          const bool all_in = local ? kfirst + 15 <= lim : kfirst + 15 < w.M;
-          if (all_in) {
+          if (!all_in) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              sv[e] = __uint_as_float(sa[e]);
-              mx = fmaxf(mx, sv[e]);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 32; ++e) {
               const int key = kfirst + e;
-              const bool vis = local ? key <= lim : key < w.M;
-              sv[e] = vis ? __uint_as_float(sa[e]) : -INFINITY;
-              mx = fmaxf(mx, sv[e]);
+              if (!(local ? key <= lim : key < w.M)) sv[e] = 0xFF800000u;
             }
           }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
         }
         xch[((g & 1) * kParts + hf) * kRows + r] = mx;
         pair_sync();  // (also: the row's four threads have read the score row before any writes P)
@@ -625,53 +672,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool need = mx > m_used + kHeadroom;  // (the same in the four threads of the row)
         const float m_old = m_used;
         if (need) m_used = mx;
-        // the weights rounded to bf16 (the PV's A operand); the row sum adds the rounded values
-        uint32_t pw[8];
-        float psum = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const __nv_bfloat162 pb =
-              __floats2bfloat162_rn(ex2_ftz(sv[2 * e] - m_used), ex2_ftz(sv[2 * e + 1] - m_used));
-          const float2 pr = __bfloat1622float2(pb);
-          psum += pr.x + pr.y;
-          pw[e] = *reinterpret_cast<const uint32_t*>(&pb);
-        }
-        // key rows past the valid count: zero their V rows (this tile's stage; all row threads)
-        if (n_valid < kKeys) {
+        // key rows past the valid count, up to the keys summed: zero their V rows (this
+        // tile's slot; all row threads)
+        if (n_valid < n_keys) {
+          // (once the tile's values have landed)
+          if (ok && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_v[g % kStages]), (uint32_t)((g / kStages) & 1),
+                                                       abort_flag)))
+            fail();
           const uint32_t vt = sbase + kOffRing + (g % kStages) * kTileBytes + 2 * kKVHalf;
-          for (int idx = tid; idx < (kKeys - n_valid) * 16; idx += kRowWarps * 32) {
+          for (int idx = tid; idx < (n_keys - n_valid) * 16; idx += kRowWarps * 32) {
             const int row = n_valid + (idx >> 4), c16 = idx & 15;
             st_shared_v4(vt + (uint32_t)((c16 >> 3) * kKVHalf + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)), 0u, 0u,
                          0u, 0u);
           }
+          fence_async_smem();
         }
         const bool rescale = __any_sync(0xffffffffu, need);
         if (i > 0 && rescale) {  // O must be stable: PV_{g-1} done before it is rescaled
           wait_pv(g - 1);
           if (!ok) continue;
           const float alpha = need ? exp2f(m_old - m_used) : 1.0f;
-          {  // this thread's 32 of the 128 output columns
-            uint32_t o[32];
-            const uint32_t col = kColO + (uint32_t)(32 * hf);
-            tmem_ld32(tmem_base + lane_addr + col, o);
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {  // this thread's 32 of the 128 output columns
+            uint32_t o[16];
+            const uint32_t col = kColO + (uint32_t)(32 * hf + 16 * hh);
+            tmem_ld16(tmem_base + lane_addr + col, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tmem_base + lane_addr + col, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tmem_base + lane_addr + col, o);
           }
           if (need) l_sum *= alpha;
         }
-        // P_g over the scores it came from: columns 8 hf .. 8 hf + 7 of the tile's buffer
-        tmem_st8(tmem_base + lane_addr + (uint32_t)((g % kSBufs) * kKeys + 8 * hf), pw);
+        // the weights rounded to bf16 (the PV's A operand); the row sum adds the rounded values
+        uint32_t pw[16];
+        float psum = 0.f;
+        if (!none) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(ex2_ftz(__uint_as_float(sv[2 * e]) - m_used),
+                                                            ex2_ftz(__uint_as_float(sv[2 * e + 1]) - m_used));
+            const float2 pr = __bfloat1622float2(pb);
+            psum += pr.x + pr.y;
+            pw[e] = *reinterpret_cast<const uint32_t*>(&pb);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pw[e] = 0u;
+        }
+        // P_g over the scores it came from: columns 16 hf .. 16 hf + 15 of the tile's buffer
+        tmem_st16(s_col + (uint32_t)(16 * hf), pw);
         tmem_wait_st();
         l_sum += psum;
-        fence_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar_p[g % kSBufs]));
         // (no wait for PV_{g-1} here: the rows wait for a PV only before a rescale of O and
-        // before the output; PV_t's barrier cannot complete its next phase, PV_{t+3}, before
-        // the rows have released P_{t+3}, so skipping the phases in between is safe)
+        // before the output; PV_t's barrier cannot complete its next phase, PV_{t+2}, before
+        // the rows have released P_{t+2}, so skipping the phases in between is safe)
       }
     };
 
@@ -830,7 +888,7 @@ int launch_g(const Args& a, cudaStream_t s, const char** why) {
 bool supported(const Args& a) {
   const uint64_t mem_rows = (uint64_t)a.B * a.L * 2 * a.H * a.M_max;
   const uint64_t loc_rows = (uint64_t)a.B * a.L * a.H * a.cap;
-  return mem_rows < (1ull << 31) && loc_rows + kKeys < (1ull << 31);
+  return mem_rows + kTile < (1ull << 31) && loc_rows + kTile < (1ull << 31);
 }
 
 int launch(const Args& a, cudaStream_t s, const char** why) {
