@@ -600,7 +600,7 @@ def time_sweep(dev, f8: bool):
         ws = torch.empty(msa.msa_route_topk_workspace_size(L, 1, Tq, H, C, n_docs, TOPK), dtype=torch.uint8,
                          device=dev)
         want = set(targets[:min(Tq, TOPK)].tolist())
-        row = {"T": Tq, "auto_path": "scan" if Tq <= 4 else ("tensor_e4m3" if f8 else "tensor_bf16")}
+        row = {"T": Tq, "auto_path": "scan" if Tq <= 4 else ("tensor_e4m3" if f8 and Tq >= 16 else "tensor_bf16")}
         paths = [("scan", msa.MSA_ROUTE_SCAN, None, 2, False)] if Tq <= 64 else []
         paths += [("tensor_bf16", msa.MSA_ROUTE_TENSOR, None, 2, False)]
         if f8:

@@ -83,7 +83,8 @@ msa_status msa_route_filter_keys(const void* kr_hat, int32_t n_layers, int64_t n
  *                    routing keys (msa_pool_blocks), 16-byte aligned.
  *   kr_f8            DEVICE, msa_route_filter_keys(kr_hat), or NULL.  Required by
  *                    MSA_ROUTE_TENSOR_F8; with MSA_ROUTE_AUTO its presence selects that path
- *                    for queries beyond the scan length.
+ *                    for queries beyond the scan length that average at least 16 tokens
+ *                    (shorter ones take the bf16 filter).
  *   doc_chunk_offsets DEVICE int64 [n_docs + 1], doc_chunk_offsets[n_docs] = n_chunks.
  *   head_dim = 128; n_kv_heads = 8 on the tensor-core path; n_q_heads % n_kv_heads = 0;
  *   1 <= top_k <= 64; 1 <= n_queries <= 256; n_kv_heads in {2, 4, 8, 16}; n_q_heads <= 64.

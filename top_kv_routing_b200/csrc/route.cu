@@ -1575,12 +1575,15 @@ msa_status route_impl(const QuerySrc& src, const int32_t* q_offsets_host, int32_
   const int H = n_kv_heads;
 
   // Path: the streaming scan while the query is a handful of tokens (those its tensor-core
-  // form takes), the tcgen05 filter GEMM beyond (on the E4M3 keys when the caller has them).
+  // form takes), the tcgen05 filter GEMM beyond: on the E4M3 keys when the caller has them
+  // and the queries average at least kF8MinTokens tokens (below that the E4M3 bound leaves
+  // most layers to the bf16 second pass, which then costs more than the bf16 filter alone).
+  constexpr int32_t kF8MinTokens = 16;
   int path = flags;
   if (path == MSA_ROUTE_AUTO)
     path = (T_total <= scan_mma_tokens(n_kv_heads) && !layer_mean)
                ? MSA_ROUTE_SCAN
-               : (kr_f8 ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
+               : (kr_f8 && T_total >= kF8MinTokens * n_queries ? MSA_ROUTE_TENSOR_F8 : MSA_ROUTE_TENSOR);
   if ((path == MSA_ROUTE_TENSOR || path == MSA_ROUTE_TENSOR_F8) && !route_tc::supported(H)) {
     if (flags != MSA_ROUTE_AUTO || layer_mean)
       return msa_fail(MSA_ERR_UNSUPPORTED, "tensor path needs n_kv_heads = 8");
