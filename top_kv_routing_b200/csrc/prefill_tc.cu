@@ -284,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_q = bars + 4 * kStages;  // a unit's queries in tensor memory (16 warps; a phase per unit)
   uint64_t* bar_s = bar_q + 1;           // [kSBufs] scores ready
   // weights ready (16 warps) and PV done, one of each per score buffer: tile g's phases are
-  // g / 3 of barrier g % 3, so neither side can complete a phase the other has not waited
-  // for yet (the MMA thread issues scores up to two tiles ahead)
+  // g / 2 of barrier g % 2, so neither side can complete a phase the other has not waited
+  // for yet (the MMA thread issues scores one tile ahead)
   uint64_t* bar_p = bar_s + kSBufs;      // [kSBufs]
   uint64_t* bar_pv = bar_p + kSBufs;     // [kSBufs]
   uint64_t* drain = bar_pv + kSBufs;
