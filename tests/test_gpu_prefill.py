@@ -105,6 +105,14 @@ def test_prefill_long_context(msa):
     _run(msa, case, [130])
 
 
+def test_prefill_partly_filled_tiles(msa):
+    # score tiles hold 128 keys: memory lengths 200 and 100 and local lengths 102..110 leave
+    # 65..127 valid keys in a tile (both 64-key boxes loaded, the rest masked and its value
+    # rows zeroed); 40 tokens at G = 4 span two units
+    case = Case(B=1, L=2, M_max=200, mem_len=[[200, 100]], len0=[70], cap=110, seed=23)
+    _run(msa, case, [40])
+
+
 @pytest.mark.parametrize("hq,h,T", [(8, 8, 70), (16, 8, 33), (64, 8, 9)])
 def test_prefill_group_sizes(msa, hq, h, T):
     # G = 1, 2, 8: 64, 32, 8 tokens per CTA, each with a ragged tail
